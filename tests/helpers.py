@@ -1,0 +1,34 @@
+"""Shared test helpers: build MXFP4 layers from seeded draws through the oracle quantiser."""
+from __future__ import annotations
+
+import numpy as np
+
+import synth
+from oracle import moe, mxfp4
+
+
+def quantized_layer_np(w: synth.Workload, layer: int = 0, seed: int = 0, tokens=None):
+    """Host draw of one layer, quantised by the oracle.  Returns (x_bits or None, LayerWeights, raw)."""
+    raw = synth.layer_inputs_np(w, layer=layer, seed=seed, tokens=tokens)
+    q = {k: [mxfp4.quantize(a) for a in raw[k]] for k in ("gate", "up", "down")}
+    lw = moe.LayerWeights(
+        gate_codes=[c for c, _ in q["gate"]], gate_scales=[s for _, s in q["gate"]],
+        up_codes=[c for c, _ in q["up"]], up_scales=[s for _, s in q["up"]],
+        down_codes=[c for c, _ in q["down"]], down_scales=[s for _, s in q["down"]],
+        router_w=raw["router_w"], router_b=raw["router_b"])
+    return raw.get("x"), lw, raw
+
+
+def x_values(bits: np.ndarray) -> np.ndarray:
+    return mxfp4.bf16_to_f64(bits)
+
+
+def tolerance_ok(got: np.ndarray, ref: np.ndarray, rel=8e-3, rms_frac=1e-3):
+    """Elementwise |got-ref| <= rel*|ref| + rms_frac*rms(ref); returns (ok, worst ratio)."""
+    ref = np.asarray(ref, np.float64)
+    got = np.asarray(got, np.float64)
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    bound = rel * np.abs(ref) + rms_frac * rms
+    err = np.abs(got - ref)
+    ratio = float((err / np.maximum(bound, 1e-300)).max()) if ref.size else 0.0
+    return bool((err <= bound).all()), ratio
