@@ -1,0 +1,451 @@
+#!/usr/bin/env python
+"""Benchmark of the decode-time MXFP4 MoE expert layer (one verify block per GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--tokens T]
+
+A step is one pass of the whole hot path -- router, permutation, gate/up
+projection + SwiGLU, down projection, weighted combine -- over one token block
+(one ``moe_forward`` call, a single engine launch).  Default workload: the
+single-sequence decode verify step, T=9 tokens, H=4096, I=1536, E=128, top-8,
+MXFP4 expert weights drawn N(0, 0.02) and quantised on the device, activations
+N(0, 1).  Each step routes a different seeded token block (8 blocks in
+rotation), and the ~0.5 GB of expert weights one step streams exceeds the
+126 MB L2, so no L2 flush is inserted between steps.
+
+Under torchrun each rank runs the same layer on its own token blocks (independent
+verify steps: weak scaling, no collective on the data path); the timed region is
+bracketed by a barrier and device synchronisation, and the slowest rank's time
+is reported.  ``--impl reference`` times the fp64 CPU oracle on a bounded sample
+of the same workload on this host's cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "MoE layer µs + MXFP4 weight-stream HBM GB/s (% of peak) at T=9; tokens/s"
+PROFILE = os.path.join(ROOT, "profiles", "engine_decode_t9_h4096_e128.md")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="decode_t9_h4096_e128", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=None, help="override T (sweep workload)")
+    ap.add_argument("--batches", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    return ap.parse_args()
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "mxfp4_moe_expert_router_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current source."""
+    try:
+        txt = open(PROFILE).read()
+    except OSError:
+        return None
+    kv = {}
+    for ln in txt.splitlines():
+        if ln.startswith("- ") and ":" in ln:
+            k, v = ln[2:].split(":", 1)
+            kv[k.strip()] = v.strip().strip("`")
+    if kv.get("source_sha256_16") != source_digest():
+        return None
+    try:
+        return float(kv["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling of one GPU while the timed region runs."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.proc = None
+        self.path = os.path.join("/tmp", f"moe_clocks_{os.getpid()}.csv")
+        if uuid is None:
+            return
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={uuid}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in open(self.path):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---- workload construction ---------------------------------------------------------------------
+
+def build_layer(mx, w: synth.Workload, layer: int, seed: int):
+    """Draw and quantise one layer on the device with the library's own quantiser."""
+    import torch
+    H, I, E = w.hidden, w.inter, w.experts
+    u8 = dict(dtype=torch.uint8, device="cuda")
+    gc, uc = torch.empty((E, I, H // 2), **u8), torch.empty((E, I, H // 2), **u8)
+    gs, us = torch.empty((E, I, H // 32), **u8), torch.empty((E, I, H // 32), **u8)
+    dc, ds = torch.empty((E, H, I // 2), **u8), torch.empty((E, H, I // 32), **u8)
+    stream = mx._stream()
+    for e in range(E):
+        for kind, c, s in (("gate", gc, gs), ("up", uc, us), ("down", dc, ds)):
+            wt = synth.expert_torch(w, layer, e, kind, seed=seed)
+            st = mx.lib.mxfp4_quantize(mx._ptr(wt), wt.shape[0], wt.shape[1], mx._ptr(c[e]),
+                                       mx._ptr(s[e]), stream)
+            if st != 0:
+                raise mx.MoeError(st, "mxfp4_quantize")
+    dense = synth.layer_inputs_torch(w, layer=layer, seed=seed)
+    return mx.LayerMX(gc, gs, uc, us, dc, ds, dense["router_w"].contiguous(), dense["router_b"])
+
+
+def token_blocks(w: synth.Workload, T: int, n: int, rank: int):
+    import torch
+    return [synth.draw_torch(1000 + rank * 64 + b, 0, "x", -1, (T, w.hidden), 1.0) for b in range(n)]
+
+
+def algorithmic_bytes(w: synth.Workload, T: int, hit: int) -> float:
+    """MXFP4 bytes of the hit experts + fp32 router weights + bf16 x and y, per layer."""
+    return hit * 3 * w.hidden * w.inter * 0.53125 + 4.0 * w.experts * w.hidden + 4.0 * T * w.hidden
+
+
+# ---- the CPU oracle as baseline / reference arm --------------------------------------------------
+
+def oracle_sample(w: synth.Workload, T: int, layer_dev, x_dev, budget_s: float):
+    """Time the oracle on a bounded sample of one layer; returns (layer seconds estimate, info).
+
+    Untimed: regenerate the hit experts' bf16 weights (same device generator as
+    the GPU path), copy them to the host and quantise them with the oracle.
+    Timed: oracle routing of the whole block, then dequantisation + SwiGLU FFN +
+    weighting of as many hit experts (in expert order) as fit in ``budget_s``.
+    The layer time is extrapolated by the fraction of hit experts done.
+    """
+    import torch
+    from oracle import moe, mxfp4
+    xb = x_dev.view(torch.int16).cpu().numpy().view(np.uint16)
+    x = mxfp4.bf16_to_f64(xb)
+    rw = layer_dev.router_w.cpu().numpy()
+    rb = None if layer_dev.router_b is None else layer_dev.router_b.cpu().numpy()
+    t0 = time.perf_counter()
+    idx, wts, _ = moe.route(x, rw, rb, w.top_k)
+    counts, offsets, perm, inv = moe.permute(idx, w.experts)
+    t_route = time.perf_counter() - t0
+    hit = [int(e) for e in np.nonzero(counts)[0]]
+    t_ffn, done = 0.0, 0
+    flat_w = wts.reshape(-1)
+    for e in hit:
+        q = {}
+        for kind in ("gate", "up", "down"):
+            bits = synth.expert_torch(w, 0, e, kind).view(torch.int16).cpu().numpy().view(np.uint16)
+            q[kind] = mxfp4.quantize(bits)
+        t1 = time.perf_counter()
+        seg = perm[offsets[e]:offsets[e + 1]]
+        wg = mxfp4.dequantize(*q["gate"])
+        wu = mxfp4.dequantize(*q["up"])
+        wd = mxfp4.dequantize(*q["down"])
+        _ = moe.expert_ffn(x[seg // w.top_k], wg, wu, wd) * flat_w[seg][:, None]
+        t_ffn += time.perf_counter() - t1
+        done += 1
+        if t_ffn + t_route >= budget_s:
+            break
+    layer_s = t_route + t_ffn * len(hit) / done
+    return layer_s, {"experts_timed": done, "experts_hit": len(hit), "route_s": t_route,
+                     "ffn_s_timed": t_ffn}
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ---- main ------------------------------------------------------------------------------------------
+
+def main():
+    args = parse_args()
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = synth.WORKLOADS[args.workload]
+    T = args.tokens or (9 if args.workload.startswith("sweep") else w.tokens)
+    w = w.with_tokens(max(T, w.tokens)) if args.workload.startswith("sweep") else w
+
+    if args.impl == "reference":
+        return run_reference(args, w, T, rank, world)
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    import mxfp4_moe_expert_router_b200 as mx
+
+    layers = [build_layer(mx, w, l, seed=0) for l in range(w.layers)]
+    m = mx.Moe(w.hidden, w.inter, w.experts, w.top_k, T, layers)
+    xs = token_blocks(w, T, args.batches, rank)
+    hits = []
+    for x in xs:
+        r = m.moe_route(x, layer=0)
+        hits.append(int((r["counts"] > 0).sum().item()))
+    m.moe_status()
+    y = torch.empty((T, w.hidden), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    sp = mx._stream(stream)
+    xptr = [mx._ptr(x) for x in xs]
+    yptr = mx._ptr(y)
+
+    def step(i):
+        st = mx.lib.moe_forward(m.handle, xptr[i % len(xptr)], T, yptr, None, sp)
+        if st != 0:
+            raise mx.MoeError(st, "moe_forward")
+
+    for i in range(args.warmup):
+        step(i)
+    m.moe_status()
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid if rank == 0 else None)
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    m.moe_status()
+    ms_total = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms_total], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    tokens_per_s = world * T * args.steps / (ms_total / 1e3)
+    mean_hit = float(np.mean([hits[i % len(hits)] for i in range(args.steps)]))
+    alg_bytes = algorithmic_bytes(w, T, mean_hit) * w.layers if w.layers == 1 else None
+    # the chain workload's later layers route on the previous layer's output: count them
+    if alg_bytes is None:
+        alg_bytes = float(np.mean([sum(algorithmic_bytes(w, T, h) for h in chain_hits(m, mx, w, T, x))
+                                   for x in xs[:2]]))
+    peak, peak_kind = measured_peaks()
+    achieved = alg_bytes / (ms_step * 1e-3) / 1e9
+    traffic = profile_traffic()
+
+    # end-to-end: the same metric through the public host-buffer entry point
+    e2e = None
+    if not args.no_e2e:
+        xh = [x.cpu().pin_memory() for x in xs]
+        yh = torch.empty((T, w.hidden), dtype=torch.bfloat16).pin_memory()
+        n_e2e = args.e2e_steps or max(1, min(args.steps, 500))
+        for i in range(min(3, n_e2e)):
+            m.moe_forward_host(xh[i % len(xh)], yh)
+        if world > 1:
+            dist.barrier()
+        t0 = time.perf_counter()
+        for i in range(n_e2e):
+            m.moe_forward_host(xh[i % len(xh)], yh)
+        el = time.perf_counter() - t0
+        if world > 1:
+            t = torch.tensor([el], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            el = float(t.item())
+        e2e = {"value": world * T * n_e2e / el, "unit": "tokens/s", "steps": n_e2e,
+               "h2d_bytes_per_step": T * w.hidden * 2, "d2h_bytes_per_step": T * w.hidden * 2}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        layer_s, info = oracle_sample(w, T, layers[0], xs[0], budget_s=15.0)
+        cpu = {"value": T / layer_s if w.layers == 1 else T / (layer_s * w.layers),
+               "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"fp64 numpy oracle, layer 0, token block 0: routing of all {T} tokens + "
+                         f"{info['experts_timed']} of {info['experts_hit']} hit experts "
+                         f"(dequantise + SwiGLU FFN), extrapolated to all hit experts"
+                         + (f" and {w.layers} layers" if w.layers > 1 else ""),
+               "layer_s_estimate": layer_s}
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "mxfp4-w/fp32-acc",
+            "data": "synthetic (seeded N(0,0.02) expert weights quantised to MXFP4, N(0,1) bf16 tokens)",
+            "config": {"workload": w.name if not args.workload.startswith("sweep") else f"{w.name}_t{T}",
+                       "hidden": w.hidden, "inter": w.inter, "experts": w.experts, "top_k": w.top_k,
+                       "tokens_per_gpu": T, "layers": w.layers, "token_blocks": len(xs),
+                       "mean_experts_hit": mean_hit,
+                       "l2": "no flush: ~%.0f MB of expert weights streamed per step > 126 MB L2"
+                             % (alg_bytes / 1e6),
+                       "parallelism": f"replicas x{world} (independent verify blocks)"},
+            "layer_us": ms_step * 1e3 / w.layers,
+            "weight_stream_gbs": achieved,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_source": peak_kind,
+                         "algorithmic_bytes_per_launch": alg_bytes,
+                         "traffic": traffic, "kernel": "engine_kernel"},
+            "gpu_launches": args.steps,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "clocks": clk,
+        }
+        print(json.dumps(out), flush=True)
+    m.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def chain_hits(m, mx, w, T, x):
+    """Experts hit per layer of the chain on token block x (routes each layer's real input)."""
+    import torch
+    io = torch.empty((w.layers + 1, T, w.hidden), dtype=torch.bfloat16, device="cuda")
+    m.moe_forward(x, layer_io=io)
+    hits = []
+    for l in range(w.layers):
+        r = m.moe_route(io[l].contiguous(), layer=l)
+        hits.append(int((r["counts"] > 0).sum().item()))
+    return hits
+
+
+def run_reference(args, w, T, rank, world):
+    """The fp64 CPU oracle on this host's cores, rank 0 only; each step a bounded sample."""
+    if rank != 0:
+        return
+    import torch
+    have_cuda = torch.cuda.is_available()
+    dev = "cuda" if have_cuda else "cpu"
+    from oracle import moe, mxfp4
+    # inputs: same recipe as the GPU arm (device draws when a GPU is present)
+    x = synth.draw_torch(1000, 0, "x", -1, (T, w.hidden), 1.0, device=dev)
+    xb = x.view(torch.int16).cpu().numpy().view(np.uint16)
+    xv = mxfp4.bf16_to_f64(xb)
+    dense = synth.layer_inputs_torch(w, 0, 0, tokens=T, device=dev)
+    rw = dense["router_w"].cpu().numpy()
+    rb = None if dense["router_b"] is None else dense["router_b"].cpu().numpy()
+    idx, wts, _ = moe.route(xv, rw, rb, w.top_k)
+    counts, offsets, perm, inv = moe.permute(idx, w.experts)
+    hit = [int(e) for e in np.nonzero(counts)[0]]
+    # per-step sample: a slice of R rows of each projection of one hit expert
+    q = {}
+    e0 = hit[0]
+    for kind in ("gate", "up", "down"):
+        bits = synth.expert_torch(w, 0, e0, kind, device=dev).view(torch.int16).cpu().numpy().view(np.uint16)
+        q[kind] = mxfp4.quantize(bits)
+    seg = perm[offsets[e0]:offsets[e0 + 1]]
+    xr = xv[seg // w.top_k]
+
+    def expert_slice(frac):
+        ri, rh = max(1, int(w.inter * frac)), max(1, int(w.hidden * frac))
+        wg = mxfp4.dequantize(q["gate"][0][:ri], q["gate"][1][:ri])
+        wu = mxfp4.dequantize(q["up"][0][:ri], q["up"][1][:ri])
+        a = moe.silu(xr @ wg.T) * (xr @ wu.T)
+        full_a = np.zeros((xr.shape[0], w.inter))
+        full_a[:, :ri] = a
+        wd = mxfp4.dequantize(q["down"][0][:rh], q["down"][1][:rh])
+        return full_a @ wd.T
+
+    t0 = time.perf_counter()
+    expert_slice(1.0)
+    t_expert = time.perf_counter() - t0
+    budget = 90.0
+    frac = min(1.0, max(1.0 / 64, budget / max(1, args.steps + args.warmup) / max(t_expert, 1e-6)))
+    for _ in range(args.warmup):
+        expert_slice(frac)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        expert_slice(frac)
+    el = time.perf_counter() - t0
+    layer_s = (el / args.steps) / frac * len(hit) * w.layers
+    value = T / layer_s
+    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": layer_s * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "impl": "reference",
+           "config": {"workload": w.name, "hidden": w.hidden, "inter": w.inter, "experts": w.experts,
+                      "top_k": w.top_k, "tokens_per_gpu": T, "layers": w.layers},
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                            "sample": f"each step: dequantise + SwiGLU FFN of {frac:.3f} of the rows of one "
+                                      f"hit expert's projections; layer time extrapolated by rows and "
+                                      f"by {len(hit)} hit experts"},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

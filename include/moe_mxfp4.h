@@ -1,0 +1,181 @@
+/*
+ * moe_mxfp4.h -- C ABI of the decode-time MoE expert feed-forward with MXFP4
+ * expert weights (B200 / sm_100a).
+ *
+ * What it computes.  One MoE layer per call of the expert weights stored in
+ * MXFP4 (4 bits per expert parameter; the MiMo-V2.5-Pro-UltraSpeed / TileRT
+ * pages: bjdmk.com.cn news, section "极致协同，通向千速之路", and the yifor
+ * blog digest "Xiaomi MiMo and TileRT Push a 1-Trillion-Parameter Model Past
+ * 1000 Tokens Per Second on Commodity GPUs", section "三層協同設計"), applied to
+ * the small token block of a speculative-decoding verify step (draft block
+ * size 8, so about 9 tokens per sequence: bjdmk.com.cn news, same section).
+ * The pages give no formula; the library takes the plain MoE reading:
+ *
+ *   logits = x Wr^T + b                      (fp64 accumulation, see moe_route)
+ *   idx    = the top_k experts by logit, descending, ties to the lower index
+ *   w      = softmax(logits)[idx] / sum      (renormalised over the top_k)
+ *   y_t    = sum_slot w_slot * Wd_e (silu(Wg_e x_t) * (Wu_e x_t)),  e = idx[t][slot]
+ *
+ * with Wg, Wu, Wd dequantised exactly from MXFP4 and fp32 accumulation.  With
+ * num_layers > 1 the layers run back to back in one launch, each layer's bf16
+ * output going through RMSNorm (unit gamma, eps = cfg.rms_eps, no residual)
+ * and bf16 rounding to become the next layer's input.  The pages put a
+ * persistent engine kernel around this (TileRT blog "Breaking 1000 TPS",
+ * section "第一次跃迁：Execution Model Revolution"): moe_forward is one
+ * cooperative launch of such a kernel.
+ *
+ * MXFP4 (OCP Microscaling v1.0): 32-element blocks along the contraction
+ * dimension K; each element an E2M1 code (bit 3 sign, bits 2..0 index into
+ * {0, 0.5, 1, 1.5, 2, 3, 4, 6}), element 2j in the LOW nibble of byte j; one
+ * E8M0 scale byte per block, value 2^(byte-127), byte 255 = NaN.
+ *
+ * Conventions for every entry point below.
+ *  - Pointers named *_host are host memory; every other pointer is DEVICE
+ *    memory of the current CUDA device, row-major and contiguous, 16-byte
+ *    aligned.  The caller keeps ownership of everything it passes.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Device work
+ *    is enqueued asynchronously on it; only moe_status, moe_forward_host and
+ *    moe_mxfp4_create (which waits for its repack) synchronise.
+ *  - Return value: moe_status_t (0 = MOE_OK).  Argument errors are detected on
+ *    the host before any work is enqueued.  Errors detected on the device
+ *    (a bounded wait that ran out) are recorded in the handle and reported by
+ *    the next moe_status call.  No entry point aborts, throws or prints.
+ */
+#ifndef MOE_MXFP4_H
+#define MOE_MXFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,       /* null pointer, size out of range, misaligned pointer */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2, /* a shape the kernels do not tile (see moe_mxfp4_create) */
+  MOE_ERR_OOM = 3,               /* device allocation failed in moe_mxfp4_create */
+  MOE_ERR_CUDA = 4,              /* a CUDA runtime call or launch failed */
+  MOE_ERR_TIMEOUT = 5,           /* a device-side wait exceeded its bound (reported by moe_status) */
+  MOE_ERR_DEVICE = 6             /* no usable device, or the engine cannot be co-resident */
+} moe_status_t;
+
+typedef struct moe_mxfp4 moe_mxfp4_t; /* opaque handle */
+
+typedef struct {
+  int32_t hidden;      /* H: multiple of 128, at most 8192 */
+  int32_t inter;       /* I: expert intermediate size, multiple of 128 */
+  int32_t num_experts; /* E: 1 .. 512 */
+  int32_t top_k;       /* k: 1 .. min(E, 32) */
+  int32_t max_tokens;  /* largest T any call will pass, >= 1 */
+  int32_t num_layers;  /* 1 .. 16 layers chained inside one moe_forward */
+  float rms_eps;       /* RMSNorm epsilon between chained layers (e.g. 1e-6) */
+} moe_config_t;
+
+/*
+ * mxfp4_quantize -- MXFP4-quantise bf16 weights w_bf16 [rows][K] (K % 32 == 0).
+ * Per 32-element block along K: s = max(floor(log2 amax) - 2, -127), scale
+ * byte s + 127; each code is the input's sign bit and the nearest E2M1
+ * magnitude of |w| / 2^s (ties to the even code, saturating at 6).  A block
+ * holding an Inf or NaN gets scale byte 255 and all-zero codes.
+ * Output codes [rows][K/2] (element 2j in the low nibble), scales [rows][K/32].
+ * rows == 0 is a no-op.  Errors: MOE_ERR_INVALID_ARG for null pointers with
+ * rows > 0, rows < 0, K <= 0 or K % 32 != 0; MOE_ERR_CUDA if the launch fails.
+ */
+MOE_API int32_t mxfp4_quantize(const void* w_bf16, int64_t rows, int64_t K, uint8_t* codes,
+                       uint8_t* scales, void* stream);
+
+/*
+ * moe_mxfp4_create -- build a handle that owns device copies of num_layers
+ * MoE layers, repacked for the weight stream, plus all workspace for calls
+ * with up to cfg->max_tokens tokens.
+ * Per layer l (host arrays of num_layers DEVICE pointers):
+ *   gate_codes[l], up_codes[l]   [E][I][H/2],  gate_scales[l], up_scales[l] [E][I][H/32]
+ *   down_codes[l]                [E][H][I/2],  down_scales[l]               [E][H][I/32]
+ *   router_w[l]                  [E][H] fp32;  router_bias == NULL or router_bias[l] == NULL
+ *                                              means no bias, else [E] fp32.
+ * The inputs are read on `stream`; the call synchronises `stream` before it
+ * returns, after which the caller may free them.  *out is set to NULL on error.
+ * Errors: MOE_ERR_INVALID_ARG (null pointers, cfg fields out of range, device
+ * pointers not 16-byte aligned), MOE_ERR_UNSUPPORTED_SHAPE (H or I not a
+ * multiple of 128, H > 8192, E > 512, top_k > 32), MOE_ERR_OOM, MOE_ERR_CUDA,
+ * MOE_ERR_DEVICE (no device, or the engine kernel does not fit on an SM).
+ */
+MOE_API int32_t moe_mxfp4_create(const moe_config_t* cfg,
+                         const uint8_t* const* gate_codes, const uint8_t* const* gate_scales,
+                         const uint8_t* const* up_codes, const uint8_t* const* up_scales,
+                         const uint8_t* const* down_codes, const uint8_t* const* down_scales,
+                         const float* const* router_w, const float* const* router_bias,
+                         void* stream, moe_mxfp4_t** out);
+
+/*
+ * moe_route -- routing and permutation of layer `layer` for x_bf16 [T][H]:
+ *   topk_idx [T][k] int32   experts in descending-logit order (ties: lower index)
+ *   topk_w   [T][k] fp32    softmax over all E, renormalised over the k
+ *   counts   [E]    int32   pairs routed to each expert
+ *   offsets  [E+1]  int32   exclusive prefix sum of counts
+ *   perm     [T*k]  int32   pair id p = t*k + slot at each permuted position;
+ *                           each expert's segment is in ascending p
+ *   inv_perm [T*k]  int32   position of each pair id
+ * Logits are accumulated in fp64 from exact bf16 x fp32 products, so the
+ * selection agrees with an exact computation except on logit gaps below about
+ * 1e-10.  T == 0 is a no-op.  Errors: MOE_ERR_INVALID_ARG (null handle or
+ * pointers, layer out of range, T < 0 or T > max_tokens), MOE_ERR_CUDA.
+ */
+MOE_API int32_t moe_route(moe_mxfp4_t* h, int32_t layer, const void* x_bf16, int32_t T,
+                  int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
+                  int32_t* perm, int32_t* inv_perm, void* stream);
+
+/*
+ * moe_forward -- y_bf16 [T][H] = the chain of num_layers MoE layers on
+ * x_bf16 [T][H], in ONE cooperative launch on `stream`.  layer_io_bf16 is
+ * NULL or a [num_layers+1][T][H] bf16 buffer that receives every layer's
+ * input (slot l) and the final output (slot num_layers).  x and y may not
+ * overlap.  T == 0 is a no-op.  Errors: MOE_ERR_INVALID_ARG, MOE_ERR_CUDA;
+ * device-side timeouts are reported by the next moe_status.
+ */
+MOE_API int32_t moe_forward(moe_mxfp4_t* h, const void* x_bf16, int32_t T, void* y_bf16,
+                    void* layer_io_bf16, void* stream);
+
+/*
+ * moe_forward_host -- moe_forward with HOST input and output: copies
+ * x_host [T][H] bf16 to the handle's device staging buffer, runs the layers,
+ * copies y back to y_host [T][H] and synchronises `stream`.  Pinned host
+ * memory gives asynchronous copies; pageable memory works too.  Returns the
+ * first error, device-side errors included.
+ */
+MOE_API int32_t moe_forward_host(moe_mxfp4_t* h, const void* x_host, int32_t T, void* y_host,
+                         void* stream);
+
+/*
+ * moe_status -- synchronise `stream`, then return and clear the device-side
+ * status of the handle: MOE_OK, or MOE_ERR_TIMEOUT if a bounded wait inside
+ * the engine expired (the handle's wait state is reset, so it stays usable).
+ * MOE_ERR_CUDA if the synchronisation itself fails.
+ */
+MOE_API int32_t moe_status(moe_mxfp4_t* h, void* stream);
+
+/* moe_set_timeout_ns -- bound of every device-side wait (default 2 s; env MOE_TIMEOUT_NS). */
+MOE_API int32_t moe_set_timeout_ns(moe_mxfp4_t* h, uint64_t ns);
+
+/* moe_engine_grid -- CTAs of one engine launch (one per SM on B200), or 0 for a NULL handle. */
+MOE_API int32_t moe_engine_grid(const moe_mxfp4_t* h);
+
+/* moe_mxfp4_destroy -- free every device allocation of the handle (NULL is a no-op).
+ * Work already enqueued on the handle must have finished. */
+MOE_API void moe_mxfp4_destroy(moe_mxfp4_t* h);
+
+/* moe_status_str -- static English text for a status code. */
+MOE_API const char* moe_status_str(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_MXFP4_H */

@@ -1,0 +1,196 @@
+"""Python binding of the MXFP4 MoE expert feed-forward C ABI (``include/moe_mxfp4.h``).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libmoe_mxfp4.so``.  PyTorch supplies device memory and streams.
+Importing this package fails loudly when the library has not been built
+(``python mxfp4_moe_expert_router_b200/build.py``); there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe_mxfp4.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_OOM, MOE_ERR_CUDA, \
+    MOE_ERR_TIMEOUT, MOE_ERR_DEVICE = range(7)
+
+EXPORTS = ("mxfp4_quantize", "moe_mxfp4_create", "moe_route", "moe_forward", "moe_forward_host",
+           "moe_status", "moe_set_timeout_ns", "moe_engine_grid", "moe_mxfp4_destroy",
+           "moe_status_str")
+
+
+class MoeConfig(ctypes.Structure):
+    """Mirror of ``moe_config_t``."""
+    _fields_ = [("hidden", ctypes.c_int32), ("inter", ctypes.c_int32),
+                ("num_experts", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("max_tokens", ctypes.c_int32), ("num_layers", ctypes.c_int32),
+                ("rms_eps", ctypes.c_float)]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_str(status)} ({status})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python mxfp4_moe_expert_router_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64
+    pp = ctypes.POINTER(ctypes.c_void_p)
+    sig = {
+        "mxfp4_quantize": (i32, [vp, i64, i64, vp, vp, vp]),
+        "moe_mxfp4_create": (i32, [ctypes.POINTER(MoeConfig), pp, pp, pp, pp, pp, pp, pp, pp, vp,
+                                   ctypes.POINTER(vp)]),
+        "moe_route": (i32, [vp, i32, vp, i32, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_forward": (i32, [vp, vp, i32, vp, vp, vp]),
+        "moe_forward_host": (i32, [vp, vp, i32, vp, vp]),
+        "moe_status": (i32, [vp, vp]),
+        "moe_set_timeout_ns": (i32, [vp, u64]),
+        "moe_engine_grid": (i32, [vp]),
+        "moe_mxfp4_destroy": (None, [vp]),
+        "moe_status_str": (ctypes.c_char_p, [i32]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def status_str(status: int) -> str:
+    return lib.moe_status_str(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+def _stream(stream=None):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def mxfp4_quantize(w, stream=None):
+    """bf16 ``w`` [rows][K] (CUDA) -> (codes uint8 [rows][K/2], scales uint8 [rows][K/32])."""
+    import torch
+    assert w.dtype == torch.bfloat16 and w.is_cuda and w.dim() == 2 and w.is_contiguous()
+    rows, K = w.shape
+    codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((rows, K // 32), dtype=torch.uint8, device=w.device)
+    _check(lib.mxfp4_quantize(_ptr(w), rows, K, _ptr(codes), _ptr(scales), _stream(stream)),
+           "mxfp4_quantize")
+    return codes, scales
+
+
+@dataclass
+class LayerMX:
+    """One layer's canonical MXFP4 tensors on the device (see ``moe_mxfp4_create``)."""
+    gate_codes: object
+    gate_scales: object
+    up_codes: object
+    up_scales: object
+    down_codes: object
+    down_scales: object
+    router_w: object
+    router_b: object = None
+
+
+class Moe:
+    """Owner of a ``moe_mxfp4_t`` handle."""
+
+    def __init__(self, hidden, inter, num_experts, top_k, max_tokens, layers, rms_eps=1e-6,
+                 stream=None):
+        self.cfg = MoeConfig(hidden, inter, num_experts, top_k, max_tokens, len(layers), rms_eps)
+        self.handle = ctypes.c_void_p(0)
+        n = len(layers)
+
+        def arr(get):
+            a = (ctypes.c_void_p * n)()
+            for i, lw in enumerate(layers):
+                v = get(lw)
+                a[i] = v.data_ptr() if v is not None else 0
+            return ctypes.cast(a, ctypes.POINTER(ctypes.c_void_p)), a
+
+        keep = [arr(lambda l, f=f: getattr(l, f)) for f in
+                ("gate_codes", "gate_scales", "up_codes", "up_scales", "down_codes",
+                 "down_scales", "router_w", "router_b")]
+        _check(lib.moe_mxfp4_create(ctypes.byref(self.cfg), *[k[0] for k in keep], _stream(stream),
+                                    ctypes.byref(self.handle)), "moe_mxfp4_create")
+
+    # -- the C entry points, same names -------------------------------------------------------
+    def moe_route(self, x, layer=0, stream=None):
+        import torch
+        T = x.shape[0]
+        K, E = self.cfg.top_k, self.cfg.num_experts
+        dev = x.device
+        out = dict(topk_idx=torch.empty((T, K), dtype=torch.int32, device=dev),
+                   topk_w=torch.empty((T, K), dtype=torch.float32, device=dev),
+                   counts=torch.empty((E,), dtype=torch.int32, device=dev),
+                   offsets=torch.empty((E + 1,), dtype=torch.int32, device=dev),
+                   perm=torch.empty((T * K,), dtype=torch.int32, device=dev),
+                   inv_perm=torch.empty((T * K,), dtype=torch.int32, device=dev))
+        _check(lib.moe_route(self.handle, layer, _ptr(x), T, *[_ptr(out[k]) for k in
+                             ("topk_idx", "topk_w", "counts", "offsets", "perm", "inv_perm")],
+                             _stream(stream)), "moe_route")
+        return out
+
+    def moe_forward(self, x, y=None, layer_io=None, stream=None):
+        import torch
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty((T, self.cfg.hidden), dtype=torch.bfloat16, device=x.device)
+        _check(lib.moe_forward(self.handle, _ptr(x), T, _ptr(y), _ptr(layer_io), _stream(stream)),
+               "moe_forward")
+        return y
+
+    def moe_forward_host(self, x_host, y_host=None, stream=None):
+        import torch
+        T = x_host.shape[0]
+        if y_host is None:
+            y_host = torch.empty((T, self.cfg.hidden), dtype=torch.bfloat16, pin_memory=True)
+        _check(lib.moe_forward_host(self.handle, _ptr(x_host), T, _ptr(y_host), _stream(stream)),
+               "moe_forward_host")
+        return y_host
+
+    def moe_status(self, stream=None):
+        _check(lib.moe_status(self.handle, _stream(stream)), "moe_status")
+
+    def moe_set_timeout_ns(self, ns: int):
+        _check(lib.moe_set_timeout_ns(self.handle, int(ns)), "moe_set_timeout_ns")
+
+    @property
+    def grid(self) -> int:
+        return lib.moe_engine_grid(self.handle)
+
+    def moe_mxfp4_destroy(self):
+        if self.handle and self.handle.value:
+            lib.moe_mxfp4_destroy(self.handle)
+            self.handle = ctypes.c_void_p(0)
+
+    close = moe_mxfp4_destroy
+
+    def __del__(self):
+        try:
+            self.moe_mxfp4_destroy()
+        except Exception:
+            pass
+
+
+def moe_mxfp4_create(hidden, inter, num_experts, top_k, max_tokens, layers, rms_eps=1e-6,
+                     stream=None) -> Moe:
+    return Moe(hidden, inter, num_experts, top_k, max_tokens, layers, rms_eps, stream)

@@ -1,0 +1,279 @@
+// C-ABI of the MXFP4 MoE expert feed-forward: argument validation, the handle
+// (repacked weights + workspace), and the launches.  Declarations and the
+// contract of every entry point are in include/moe_mxfp4.h.
+#include "moe_mxfp4.h"
+
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "engine.cuh"
+
+using namespace moe;
+
+struct moe_mxfp4 {
+  moe_config_t cfg{};
+  int device = 0;
+  int grid = 0;
+  uint64_t timeout_ns = 2000000000ull;
+  int umax = 0;
+  uint8_t* w_gu[MAX_LAYERS] = {};
+  uint8_t* w_d[MAX_LAYERS] = {};
+  float* router_w[MAX_LAYERS] = {};
+  float* router_b[MAX_LAYERS] = {};
+  double* logits = nullptr;
+  float* xf = nullptr;
+  __nv_bfloat16* xnext = nullptr;
+  int32_t *idx = nullptr, *counts = nullptr, *offsets = nullptr, *perm = nullptr, *inv = nullptr,
+          *tokpos = nullptr, *units = nullptr, *n_units = nullptr;
+  float *wts = nullptr, *wpos = nullptr, *abuf = nullptr, *ypair = nullptr;
+  uint32_t* sync = nullptr;
+  __nv_bfloat16 *x_stage = nullptr, *y_stage = nullptr;
+  std::vector<void*> allocs;
+};
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <class T>
+bool dalloc(moe_mxfp4* h, T** out, size_t bytes) {
+  void* p = nullptr;
+  if (cudaMalloc(&p, bytes < 16 ? 16 : bytes) != cudaSuccess) { *out = nullptr; return false; }
+  h->allocs.push_back(p);
+  *out = static_cast<T*>(p);
+  return true;
+}
+
+void free_all(moe_mxfp4* h) {
+  for (void* p : h->allocs) cudaFree(p);
+  h->allocs.clear();
+}
+
+size_t stage_bytes_gu(const moe_config_t& c) {
+  return (size_t)c.num_experts * (c.inter / GU_ROWS) * (c.hidden / KC) * STAGE_W_BYTES;
+}
+size_t stage_bytes_d(const moe_config_t& c) {
+  return (size_t)c.num_experts * (c.hidden / ROWS) * (c.inter / KC) * STAGE_W_BYTES;
+}
+
+int32_t validate_cfg(const moe_config_t* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->hidden <= 0 || c->inter <= 0 || c->num_experts <= 0 || c->top_k <= 0 ||
+      c->max_tokens <= 0 || c->num_layers <= 0 || c->top_k > c->num_experts ||
+      !(c->rms_eps >= 0.f))
+    return MOE_ERR_INVALID_ARG;
+  if (c->hidden % KC || c->inter % KC || c->hidden > 8192 || c->num_experts > MAX_EXPERTS ||
+      c->top_k > 32 || c->num_layers > MAX_LAYERS)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((int64_t)c->max_tokens * c->top_k > (int64_t)1 << 28) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+EngineParams base_params(const moe_mxfp4* h, int T) {
+  EngineParams p{};
+  p.H = h->cfg.hidden; p.I = h->cfg.inter; p.E = h->cfg.num_experts; p.K = h->cfg.top_k;
+  p.T = T; p.TK = T * h->cfg.top_k; p.L = h->cfg.num_layers;
+  p.rms_eps = h->cfg.rms_eps;
+  p.timeout_ns = h->timeout_ns;
+  for (int l = 0; l < h->cfg.num_layers; ++l)
+    p.layers[l] = LayerPtrs{h->w_gu[l], h->w_d[l], h->router_w[l], h->router_b[l]};
+  p.logits = h->logits; p.xf = h->xf; p.xnext = h->xnext;
+  p.idx = h->idx; p.wts = h->wts; p.counts = h->counts; p.offsets = h->offsets;
+  p.perm = h->perm; p.inv = h->inv; p.tokpos = h->tokpos; p.wpos = h->wpos;
+  p.units = h->units; p.n_units = h->n_units; p.abuf = h->abuf; p.ypair = h->ypair;
+  p.sync = h->sync;
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_str(int32_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_ERR_OOM: return "device out of memory";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_DEVICE: return "no usable device";
+    default: return "unknown status";
+  }
+}
+
+int32_t mxfp4_quantize(const void* w_bf16, int64_t rows, int64_t K, uint8_t* codes,
+                       uint8_t* scales, void* stream) {
+  if (rows < 0 || K <= 0 || K % 32) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!w_bf16 || !codes || !scales || !aligned16(w_bf16) || !aligned16(codes))
+    return MOE_ERR_INVALID_ARG;
+  return quantize_launch(w_bf16, rows, K, codes, scales, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int32_t moe_mxfp4_create(const moe_config_t* cfg, const uint8_t* const* gate_codes,
+                         const uint8_t* const* gate_scales, const uint8_t* const* up_codes,
+                         const uint8_t* const* up_scales, const uint8_t* const* down_codes,
+                         const uint8_t* const* down_scales, const float* const* router_w,
+                         const float* const* router_bias, void* stream, moe_mxfp4_t** out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  int32_t st = validate_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (!gate_codes || !gate_scales || !up_codes || !up_scales || !down_codes || !down_scales ||
+      !router_w)
+    return MOE_ERR_INVALID_ARG;
+  const int L = cfg->num_layers;
+  for (int l = 0; l < L; ++l) {
+    if (!gate_codes[l] || !gate_scales[l] || !up_codes[l] || !up_scales[l] || !down_codes[l] ||
+        !down_scales[l] || !router_w[l])
+      return MOE_ERR_INVALID_ARG;
+    if (!aligned16(gate_codes[l]) || !aligned16(up_codes[l]) || !aligned16(down_codes[l]) ||
+        !aligned16(router_w[l]))
+      return MOE_ERR_INVALID_ARG;
+  }
+  int dev = 0, ndev = 0, major = 0, minor = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) { cudaGetLastError(); return MOE_ERR_DEVICE; }
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_DEVICE;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0) return MOE_ERR_DEVICE;  // built for sm_100a only
+
+  moe_mxfp4* h = new (std::nothrow) moe_mxfp4();
+  if (!h) return MOE_ERR_OOM;
+  h->cfg = *cfg;
+  h->device = dev;
+  if (const char* env = std::getenv("MOE_TIMEOUT_NS")) {
+    const unsigned long long v = std::strtoull(env, nullptr, 10);
+    if (v > 0) h->timeout_ns = v;
+  }
+  int gerr = 0;
+  const int maxg = engine_max_grid(dev, &gerr);
+  int sms = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (gerr || maxg < 1 || sms < 1) { delete h; return MOE_ERR_DEVICE; }
+  h->grid = maxg < sms ? maxg : sms;
+
+  const int H = cfg->hidden, I = cfg->inter, E = cfg->num_experts, K = cfg->top_k;
+  const int64_t Tm = cfg->max_tokens, TKm = Tm * K;
+  h->umax = (int)((E < TKm ? E : TKm) + TKm / NT_MAX + 1);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  bool ok = true;
+  for (int l = 0; l < L && ok; ++l) {
+    ok = dalloc(h, &h->w_gu[l], stage_bytes_gu(*cfg)) && dalloc(h, &h->w_d[l], stage_bytes_d(*cfg)) &&
+         dalloc(h, &h->router_w[l], (size_t)E * H * 4);
+    if (ok && router_bias && router_bias[l]) ok = dalloc(h, &h->router_b[l], (size_t)E * 4);
+  }
+  ok = ok && dalloc(h, &h->logits, (size_t)Tm * E * 8) && dalloc(h, &h->xf, (size_t)Tm * H * 4) &&
+       dalloc(h, &h->xnext, (size_t)Tm * H * 2) && dalloc(h, &h->idx, (size_t)TKm * 4) &&
+       dalloc(h, &h->wts, (size_t)TKm * 4) && dalloc(h, &h->counts, (size_t)E * 4) &&
+       dalloc(h, &h->offsets, (size_t)(E + 1) * 4) && dalloc(h, &h->perm, (size_t)TKm * 4) &&
+       dalloc(h, &h->inv, (size_t)TKm * 4) && dalloc(h, &h->tokpos, (size_t)TKm * 4) &&
+       dalloc(h, &h->wpos, (size_t)TKm * 4) && dalloc(h, &h->units, (size_t)h->umax * 16) &&
+       dalloc(h, &h->n_units, 16) && dalloc(h, &h->abuf, (size_t)I * TKm * 4) &&
+       dalloc(h, &h->ypair, (size_t)TKm * H * 4) &&
+       dalloc(h, &h->sync, (size_t)(SY_READY + h->umax) * 4) &&
+       dalloc(h, &h->x_stage, (size_t)Tm * H * 2) && dalloc(h, &h->y_stage, (size_t)Tm * H * 2);
+  if (!ok) { free_all(h); delete h; cudaGetLastError(); return MOE_ERR_OOM; }
+
+  cudaError_t e = cudaMemsetAsync(h->sync, 0, (size_t)(SY_READY + h->umax) * 4, s);
+  for (int l = 0; l < L && e == cudaSuccess; ++l) {
+    e = repack_gu_launch(gate_codes[l], gate_scales[l], up_codes[l], up_scales[l], E, I, H,
+                         h->w_gu[l], s);
+    if (e == cudaSuccess) e = repack_d_launch(down_codes[l], down_scales[l], E, H, I, h->w_d[l], s);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(h->router_w[l], router_w[l], (size_t)E * H * 4, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess && h->router_b[l])
+      e = cudaMemcpyAsync(h->router_b[l], router_bias[l], (size_t)E * 4, cudaMemcpyDeviceToDevice, s);
+  }
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) { free_all(h); delete h; cudaGetLastError(); return MOE_ERR_CUDA; }
+  *out = h;
+  return MOE_OK;
+}
+
+int32_t moe_route(moe_mxfp4_t* h, int32_t layer, const void* x_bf16, int32_t T,
+                  int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
+                  int32_t* perm, int32_t* inv_perm, void* stream) {
+  if (!h || layer < 0 || layer >= h->cfg.num_layers || T < 0 || T > h->cfg.max_tokens)
+    return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x_bf16 || !topk_idx || !topk_w || !counts || !offsets || !perm || !inv_perm ||
+      !aligned16(x_bf16))
+    return MOE_ERR_INVALID_ARG;
+  EngineParams p = base_params(h, T);
+  p.L = 1;
+  p.layers[0] = p.layers[layer];
+  p.route_only = 1;
+  p.x_in = static_cast<const __nv_bfloat16*>(x_bf16);
+  p.idx = topk_idx; p.wts = topk_w; p.counts = counts; p.offsets = offsets; p.perm = perm;
+  p.inv = inv_perm;
+  return engine_launch(p, h->grid, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK
+                                                                                     : MOE_ERR_CUDA;
+}
+
+int32_t moe_forward(moe_mxfp4_t* h, const void* x_bf16, int32_t T, void* y_bf16,
+                    void* layer_io_bf16, void* stream) {
+  if (!h || T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x_bf16 || !y_bf16 || !aligned16(x_bf16) || !aligned16(y_bf16) ||
+      (layer_io_bf16 && !aligned16(layer_io_bf16)))
+    return MOE_ERR_INVALID_ARG;
+  const size_t bytes = (size_t)T * h->cfg.hidden * 2;
+  const char* xa = static_cast<const char*>(x_bf16);
+  const char* ya = static_cast<const char*>(y_bf16);
+  if (xa < ya + bytes && ya < xa + bytes) return MOE_ERR_INVALID_ARG;
+  EngineParams p = base_params(h, T);
+  p.x_in = static_cast<const __nv_bfloat16*>(x_bf16);
+  p.y_out = static_cast<__nv_bfloat16*>(y_bf16);
+  p.layer_io = static_cast<__nv_bfloat16*>(layer_io_bf16);
+  return engine_launch(p, h->grid, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK
+                                                                                     : MOE_ERR_CUDA;
+}
+
+int32_t moe_status(moe_mxfp4_t* h, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t words[SY_READY] = {};
+  if (cudaMemcpy(words, h->sync, sizeof(words), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (words[SY_ERROR] == DEV_OK) return MOE_OK;
+  if (cudaMemset(h->sync, 0, sizeof(words)) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_ERR_TIMEOUT;
+}
+
+int32_t moe_forward_host(moe_mxfp4_t* h, const void* x_host, int32_t T, void* y_host,
+                         void* stream) {
+  if (!h || T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x_host || !y_host) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t)T * h->cfg.hidden * 2;
+  if (cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  int32_t st = moe_forward(h, h->x_stage, T, h->y_stage, nullptr, stream);
+  if (st != MOE_OK) return st;
+  if (cudaMemcpyAsync(y_host, h->y_stage, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return moe_status(h, stream);
+}
+
+int32_t moe_set_timeout_ns(moe_mxfp4_t* h, uint64_t ns) {
+  if (!h || ns == 0) return MOE_ERR_INVALID_ARG;
+  h->timeout_ns = ns;
+  return MOE_OK;
+}
+
+int32_t moe_engine_grid(const moe_mxfp4_t* h) { return h ? h->grid : 0; }
+
+void moe_mxfp4_destroy(moe_mxfp4_t* h) {
+  if (!h) return;
+  free_all(h);
+  delete h;
+}
+
+}  // extern "C"

@@ -1,6 +1,9 @@
 """Shared test helpers: build MXFP4 layers from seeded draws through the oracle quantiser."""
 from __future__ import annotations
 
+import importlib.util
+import os
+
 import numpy as np
 
 import synth
@@ -32,3 +35,13 @@ def tolerance_ok(got: np.ndarray, ref: np.ndarray, rel=8e-3, rms_frac=1e-3):
     err = np.abs(got - ref)
     ratio = float((err / np.maximum(bound, 1e-300)).max()) if ref.size else 0.0
     return bool((err <= bound).all()), ratio
+
+
+def build_library():
+    """Compile libmoe_mxfp4.so if stale, without importing the binding package."""
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                        "mxfp4_moe_expert_router_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_moe_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()

@@ -1,0 +1,212 @@
+"""GPU path vs the fp64 oracle through the C ABI: quantiser, routing, forward.
+
+Bit-exact: MXFP4 codes/scales, top-k indices (outside counted near ties),
+counts/offsets/perm/inv.  Routing weights within 1e-5.  bf16 outputs within
+|err| <= 8e-3*|ref| + 1e-3*rms(ref): bf16 output rounding alone is up to
+2^-9 = 1.95e-3 relative, fp32 accumulation over K <= 8192 terms adds ~1e-6
+relative, and the 1e-3*rms floor absorbs absolute error on outputs near zero.
+"""
+import numpy as np
+import pytest
+
+import synth
+from oracle import moe, mxfp4
+from tests.helpers import quantized_layer_np, x_values
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def m():
+    from tests.gpu_helpers import mx
+    return mx()
+
+
+def _q_gpu(m, bits):
+    from tests.gpu_helpers import bf16_dev
+    c, s = m.mxfp4_quantize(bf16_dev(bits))
+    return c.cpu().numpy(), s.cpu().numpy()
+
+
+def test_quantize_every_bf16_pattern(m):
+    bits = np.zeros((65536, 32), np.uint16)
+    bits[:, 0] = np.arange(65536)
+    bits[:, 1] = np.arange(65536)[::-1]
+    c, s = _q_gpu(m, bits)
+    rc, rs = mxfp4.quantize(bits)
+    assert (s == rs).all() and (c == rc).all()
+
+
+@pytest.mark.parametrize("amax", [1.0, 6.0 * 2.0 ** 10, 1.5 * 2.0 ** -120, 2.0 ** -125, 3.0e38])
+def test_quantize_all_patterns_under_fixed_max(m, amax):
+    ab = int(np.array([amax], np.float32).view(np.uint32)[0] >> 16)
+    bits = np.zeros((65536, 32), np.uint16)
+    bits[:, 5] = ab
+    bits[:, 6] = np.arange(65536)
+    fin = ((bits[:, 6] >> 7) & 0xFF) != 0xFF
+    vals = np.abs(mxfp4.bf16_to_f64(bits[:, 6]))
+    keep = fin & (vals <= mxfp4.bf16_to_f64(np.array([ab], np.uint16))[0])
+    bits = bits[keep]
+    c, s = _q_gpu(m, bits)
+    rc, rs = mxfp4.quantize(bits)
+    assert (s == rs).all() and (c == rc).all()
+
+
+@pytest.mark.parametrize("shape", [(1, 32), (3, 96), (256, 7168), (2048, 128)])
+def test_quantize_random_weights(m, shape):
+    rng = np.random.default_rng(shape[0] * 7 + shape[1])
+    w = (rng.standard_normal(shape) * 0.02).astype(np.float32)
+    w.reshape(-1)[:: max(1, w.size // 7)] *= 1e-30  # a few subnormal-range elements
+    bits = synth.bf16_bits_from_f32(w)
+    if shape[0] > 2:
+        bits[1, :32] = 0x7F80  # +inf block
+        bits[2, :32] = 0x8000  # all -0 block
+    c, s = _q_gpu(m, bits)
+    rc, rs = mxfp4.quantize(bits)
+    assert (s == rs).all() and (c == rc).all()
+
+
+SHAPES = {
+    # name: (H, I, E, k, T) -- several tiles and ragged segments; small (T*k<=256) and large paths
+    "tiny": (256, 128, 8, 2, 9),
+    "ragged_small": (512, 256, 16, 4, 37),
+    "ragged_large": (384, 256, 16, 4, 80),
+    "one_token": (256, 128, 8, 2, 1),
+    "all_experts": (256, 128, 4, 4, 9),
+    "top1": (256, 256, 8, 1, 17),
+    "many_tokens_one_expert": (256, 128, 2, 1, 40),
+}
+
+
+def _workload(name, zipf=None):
+    H, I, E, k, T = SHAPES[name]
+    return synth.Workload(name, H, I, E, k, T, zipf_alpha=zipf, device_draw=False)
+
+
+@pytest.mark.parametrize("name", list(SHAPES))
+def test_route_matches_oracle(m, name):
+    from tests.gpu_helpers import bf16_dev, check_route, make_moe
+    w = _workload(name, zipf=1.2 if name == "ragged_small" else None)
+    xb, lw, _ = quantized_layer_np(w, seed=11)
+    mo = make_moe(w, [lw])
+    out = mo.moe_route(bf16_dev(xb))
+    mo.moe_status()
+    assert check_route(out, x_values(xb), lw, w.top_k) == 0
+
+
+@pytest.mark.parametrize("name", list(SHAPES))
+def test_forward_matches_oracle(m, name):
+    from tests.gpu_helpers import bf16_dev, check_forward, make_moe
+    w = _workload(name)
+    xb, lw, _ = quantized_layer_np(w, seed=12)
+    mo = make_moe(w, [lw])
+    y = mo.moe_forward(bf16_dev(xb))
+    mo.moe_status()
+    check_forward(y, x_values(xb), lw, w.top_k)
+
+
+def test_forward_with_router_bias(m):
+    from tests.gpu_helpers import bf16_dev, check_forward, make_moe
+    w = _workload("ragged_large", zipf=1.2)
+    xb, lw, _ = quantized_layer_np(w, seed=13)
+    mo = make_moe(w, [lw])
+    check_forward(mo.moe_forward(bf16_dev(xb)), x_values(xb), lw, w.top_k)
+
+
+def test_tokens_fewer_than_max_and_empty(m):
+    from tests.gpu_helpers import bf16_dev, check_forward, make_moe
+    import torch
+    w = _workload("ragged_small")
+    xb, lw, _ = quantized_layer_np(w, seed=14)
+    mo = make_moe(w, [lw], max_tokens=64)
+    for T in (37, 5, 1):
+        y = mo.moe_forward(bf16_dev(xb[:T]))
+        check_forward(y, x_values(xb[:T]), lw, w.top_k)
+    y0 = mo.moe_forward(torch.empty((0, w.hidden), dtype=torch.bfloat16, device="cuda"))
+    assert y0.shape == (0, w.hidden)
+    mo.moe_status()
+    with pytest.raises(m.MoeError):
+        mo.moe_forward(bf16_dev(np.zeros((65, w.hidden), np.uint16)))
+
+
+def test_zero_input_gives_zero_output(m):
+    from tests.gpu_helpers import bf16_dev, bf16_host_bits, make_moe
+    w = _workload("ragged_small")
+    _, lw, _ = quantized_layer_np(w, seed=15)
+    mo = make_moe(w, [lw])
+    y = mo.moe_forward(bf16_dev(np.zeros((w.tokens, w.hidden), np.uint16)))
+    assert (x_values(bf16_host_bits(y)) == 0).all()
+
+
+def test_down_scale_increment_doubles_output_exactly(m):
+    from tests.gpu_helpers import bf16_dev, bf16_host_bits, make_moe
+    w = _workload("ragged_small")
+    xb, lw, _ = quantized_layer_np(w, seed=16)
+    lw2 = moe.LayerWeights(lw.gate_codes, lw.gate_scales, lw.up_codes, lw.up_scales,
+                           lw.down_codes, [s + 1 for s in lw.down_scales], lw.router_w, lw.router_b)
+    y1 = x_values(bf16_host_bits(make_moe(w, [lw]).moe_forward(bf16_dev(xb))))
+    y2 = x_values(bf16_host_bits(make_moe(w, [lw2]).moe_forward(bf16_dev(xb))))
+    assert (y2 == 2 * y1).all()
+
+
+def test_token_permutation_equivariance_and_determinism(m):
+    from tests.gpu_helpers import bf16_dev, bf16_host_bits, make_moe
+    w = _workload("ragged_large")
+    xb, lw, _ = quantized_layer_np(w, seed=17)
+    mo = make_moe(w, [lw])
+    perm = np.random.default_rng(0).permutation(w.tokens)
+    y = bf16_host_bits(mo.moe_forward(bf16_dev(xb)))
+    y_again = bf16_host_bits(mo.moe_forward(bf16_dev(xb)))
+    yp = bf16_host_bits(mo.moe_forward(bf16_dev(xb[perm])))
+    assert (y == y_again).all()
+    assert (yp == y[perm]).all()
+
+
+def test_forward_host_matches_device(m):
+    import torch
+    from tests.gpu_helpers import bf16_dev, bf16_host_bits, make_moe
+    w = _workload("tiny")
+    xb, lw, _ = quantized_layer_np(w, seed=18)
+    mo = make_moe(w, [lw])
+    y = bf16_host_bits(mo.moe_forward(bf16_dev(xb)))
+    xh = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = mo.moe_forward_host(xh)
+    assert (bf16_host_bits(yh) == y).all()
+
+
+def test_chain_teacher_forced(m):
+    """3 chained layers in one launch; each layer checked on the GPU's own bf16 input."""
+    import torch
+    from tests.gpu_helpers import bf16_dev, bf16_host_bits, make_moe
+    from tests.helpers import tolerance_ok
+    w = synth.Workload("chain", 512, 256, 16, 4, 9, layers=3, zipf_alpha=1.2, device_draw=False)
+    lws, xb = [], None
+    for l in range(3):
+        xl, lw, _ = quantized_layer_np(w, layer=l, seed=19)
+        lws.append(lw)
+        xb = xl if l == 0 else xb
+    mo = make_moe(w, lws)
+    io = torch.empty((4, w.tokens, w.hidden), dtype=torch.bfloat16, device="cuda")
+    y = mo.moe_forward(bf16_dev(xb), layer_io=io)
+    mo.moe_status()
+    io_h = x_values(bf16_host_bits(io))
+    assert (bf16_host_bits(io[0]) == xb).all()
+    assert (bf16_host_bits(io[3]) == bf16_host_bits(y)).all()
+    for l in range(3):
+        ref_y = moe.moe_layer(io_h[l], lws[l], w.top_k)["y"]
+        if l < 2:
+            ok, ratio = tolerance_ok(io_h[l + 1], moe.rmsnorm(ref_y))
+        else:
+            ok, ratio = tolerance_ok(io_h[3], ref_y)
+        assert ok, (l, ratio)
+
+
+def test_status_reports_ok_and_handle_reusable(m):
+    from tests.gpu_helpers import bf16_dev, make_moe
+    w = _workload("tiny")
+    xb, lw, _ = quantized_layer_np(w, seed=20)
+    mo = make_moe(w, [lw])
+    for _ in range(3):
+        mo.moe_forward(bf16_dev(xb))
+    mo.moe_status()
+    assert mo.grid > 0
