@@ -209,7 +209,7 @@ def oracle_sample(w: synth.Workload, T: int, layer_dev, x_dev, budget_s: float):
         _ = moe.expert_ffn(x[seg // w.top_k], wg, wu, wd) * flat_w[seg][:, None]
         t_ffn += time.perf_counter() - t1
         done += 1
-        if t_ffn + t_route >= budget_s:
+        if t_ffn + t_route >= budget_s or done >= 16:
             break
     layer_s = t_route + t_ffn * len(hit) / done
     return layer_s, {"experts_timed": done, "experts_hit": len(hit), "route_s": t_route,
@@ -332,7 +332,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        layer_s, info = oracle_sample(w, T, layers[0], xs[0], budget_s=15.0)
+        layer_s, info = oracle_sample(w, T, layers[0], xs[0], budget_s=6.0)
         cpu = {"value": T / layer_s if w.layers == 1 else T / (layer_s * w.layers),
                "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                "sample": f"fp64 numpy oracle, layer 0, token block 0: routing of all {T} tokens + "

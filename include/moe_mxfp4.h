@@ -172,6 +172,34 @@ MOE_API int32_t moe_engine_grid(const moe_mxfp4_t* h);
  * Work already enqueued on the handle must have finished. */
 MOE_API void moe_mxfp4_destroy(moe_mxfp4_t* h);
 
+/*
+ * moe_route_static -- moe_route without a handle and without any device
+ * allocation.  No counterpart on the pages: it exists for callers that cannot
+ * call cudaMalloc (a caching allocator that already owns the free memory, a
+ * process whose memory budget was reserved up front, a serving path where
+ * allocation is forbidden) but need the router.  Same outputs and output
+ * layouts as moe_route, for router_w [num_experts][hidden] fp32 and
+ * router_bias [num_experts] fp32 or NULL, both DEVICE pointers.
+ * Working memory: one static device array of MOE_ROUTE_STATIC_SCRATCH_BYTES
+ * that every device using the library holds until the process exits.  The
+ * first call on a device resolves that array's device address (and sets the
+ * kernel's shared-memory limit); make that first call before any stream
+ * capture.  All calls share the array: calls whose kernels overlap on the GPU
+ * race and give wrong outputs, so serialise them.  The call clears the words
+ * that must start at zero itself.  Sizes whose working memory exceeds the
+ * array (roughly T*(8*num_experts + 4*hidden) bytes) return
+ * MOE_ERR_UNSUPPORTED_SHAPE; hidden must be a multiple of 128 (at most 8192),
+ * num_experts <= 512, top_k <= min(num_experts, 32).  T == 0 is a no-op.
+ * There is no status query: a device-side wait that times out leaves the
+ * outputs undefined.
+ */
+#define MOE_ROUTE_STATIC_SCRATCH_BYTES (8u << 20)
+MOE_API int32_t moe_route_static(const void* x_bf16, int32_t T, int32_t hidden,
+                                 const float* router_w, const float* router_bias,
+                                 int32_t num_experts, int32_t top_k, int32_t* topk_idx,
+                                 float* topk_w, int32_t* counts, int32_t* offsets, int32_t* perm,
+                                 int32_t* inv_perm, void* stream);
+
 /* moe_status_str -- static English text for a status code. */
 MOE_API const char* moe_status_str(int32_t status);
 

@@ -19,7 +19,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_OOM, MOE_ERR_CUD
 
 EXPORTS = ("mxfp4_quantize", "moe_mxfp4_create", "moe_route", "moe_forward", "moe_forward_host",
            "moe_status", "moe_set_timeout_ns", "moe_engine_grid", "moe_mxfp4_destroy",
-           "moe_status_str")
+           "moe_status_str", "moe_route_static")
 
 
 class MoeConfig(ctypes.Structure):
@@ -55,6 +55,7 @@ def _load():
         "moe_engine_grid": (i32, [vp]),
         "moe_mxfp4_destroy": (None, [vp]),
         "moe_status_str": (ctypes.c_char_p, [i32]),
+        "moe_route_static": (i32, [vp, i32, i32, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -189,6 +190,29 @@ class Moe:
             self.moe_mxfp4_destroy()
         except Exception:
             pass
+
+
+def moe_route_static(x, router_w, router_b, top_k, stream=None):
+    """Routing without a handle or any device allocation (see ``moe_route_static`` in the header).
+
+    ``x`` bf16 [T][H], ``router_w`` fp32 [E][H], ``router_b`` fp32 [E] or None, all CUDA.
+    Returns the same dict as ``Moe.moe_route``.
+    """
+    import torch
+    T, H = x.shape
+    E = router_w.shape[0]
+    dev = x.device
+    out = dict(topk_idx=torch.empty((T, top_k), dtype=torch.int32, device=dev),
+               topk_w=torch.empty((T, top_k), dtype=torch.float32, device=dev),
+               counts=torch.empty((E,), dtype=torch.int32, device=dev),
+               offsets=torch.empty((E + 1,), dtype=torch.int32, device=dev),
+               perm=torch.empty((T * top_k,), dtype=torch.int32, device=dev),
+               inv_perm=torch.empty((T * top_k,), dtype=torch.int32, device=dev))
+    _check(lib.moe_route_static(_ptr(x), T, H, _ptr(router_w), _ptr(router_b), E, top_k,
+                                *[_ptr(out[k]) for k in ("topk_idx", "topk_w", "counts", "offsets",
+                                                         "perm", "inv_perm")], _stream(stream)),
+           "moe_route_static")
+    return out
 
 
 def moe_mxfp4_create(hidden, inter, num_experts, top_k, max_tokens, layers, rms_eps=1e-6,
