@@ -292,6 +292,7 @@ def main():
         dist.barrier()
     clk = clocks.stop()
     m.moe_status()
+    phases = m.moe_phase_ns()  # the last timed step, CTA 0's view
     ms_total = ev0.elapsed_time(ev1)
     if world > 1:
         t = torch.tensor([ms_total], device="cuda")
@@ -361,6 +362,8 @@ def main():
                          "algorithmic_bytes_per_launch": alg_bytes,
                          "traffic": traffic, "kernel": "engine_kernel"},
             "gpu_launches": args.steps,
+            "phase_us_last_step": {k: round(v / 1e3, 2) for k, v in
+                                   zip(("prepare", "route", "stream", "combine"), phases[:4])},
             "e2e": e2e,
             "cpu_baseline": cpu,
             "clocks": clk,

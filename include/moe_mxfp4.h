@@ -162,6 +162,15 @@ MOE_API int32_t moe_forward_host(moe_mxfp4_t* h, const void* x_host, int32_t T, 
  */
 MOE_API int32_t moe_status(moe_mxfp4_t* h, void* stream);
 
+/*
+ * moe_phase_ns -- tracing: synchronise `stream`, then write to the HOST array
+ * ns_out up to max_n durations (ns, %globaltimer of CTA 0) of the last
+ * moe_forward of the handle, four per layer: activation preparation + router
+ * logits, routing + permutation, the MXFP4 weight stream, combine (+ RMSNorm).
+ * Values of a launch that stopped early are unspecified.
+ */
+MOE_API int32_t moe_phase_ns(moe_mxfp4_t* h, uint64_t* ns_out, int32_t max_n, void* stream);
+
 /* moe_set_timeout_ns -- bound of every device-side wait (default 2 s; env MOE_TIMEOUT_NS). */
 MOE_API int32_t moe_set_timeout_ns(moe_mxfp4_t* h, uint64_t ns);
 

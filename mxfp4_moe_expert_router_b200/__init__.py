@@ -19,7 +19,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_OOM, MOE_ERR_CUD
 
 EXPORTS = ("mxfp4_quantize", "moe_mxfp4_create", "moe_route", "moe_forward", "moe_forward_host",
            "moe_status", "moe_set_timeout_ns", "moe_engine_grid", "moe_mxfp4_destroy",
-           "moe_status_str", "moe_route_static")
+           "moe_status_str", "moe_route_static", "moe_phase_ns")
 
 
 class MoeConfig(ctypes.Structure):
@@ -55,6 +55,7 @@ def _load():
         "moe_engine_grid": (i32, [vp]),
         "moe_mxfp4_destroy": (None, [vp]),
         "moe_status_str": (ctypes.c_char_p, [i32]),
+        "moe_phase_ns": (i32, [vp, ctypes.POINTER(ctypes.c_uint64), i32, vp]),
         "moe_route_static": (i32, [vp, i32, i32, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
@@ -170,6 +171,13 @@ class Moe:
 
     def moe_status(self, stream=None):
         _check(lib.moe_status(self.handle, _stream(stream)), "moe_status")
+
+    def moe_phase_ns(self, stream=None):
+        """Durations (ns) of the last forward's phases: 4 per layer (prepare, route, stream, combine)."""
+        n = self.cfg.num_layers * 4
+        arr = (ctypes.c_uint64 * n)()
+        _check(lib.moe_phase_ns(self.handle, arr, n, _stream(stream)), "moe_phase_ns")
+        return [int(v) for v in arr]
 
     def moe_set_timeout_ns(self, ns: int):
         _check(lib.moe_set_timeout_ns(self.handle, int(ns)), "moe_set_timeout_ns")

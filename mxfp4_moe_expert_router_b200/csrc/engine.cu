@@ -1,21 +1,34 @@
 // Persistent MXFP4 MoE engine: one cooperative launch runs, per layer,
-//   A  router logits (fp64 accumulation) and fp32 copy of the activations
+//   A  router partial logits (fp64 accumulation), per-token f16 activations
 //   B  top-k + renormalised weights, stable per-expert permutation, unit table
-//   C  the MXFP4 weight stream: gate/up projection + SwiGLU, then down
-//      projection x routing weight, as warp jobs fed by bulk copies
+//   C  the MXFP4 weight stream on tensor cores: gate/up projection + SwiGLU,
+//      then down projection x routing weight
 //   D  weighted combine to bf16 (+ RMSNorm into the next layer's input)
 // separated by bounded grid barriers.  The design follows the TileRT pages'
-// execution model: a resident engine kernel with continuous prefetch through
-// shared memory while the current tile computes, a tile-level pipeline and
+// execution model -- a resident engine kernel that keeps prefetching through
+// shared memory while the current tile computes, a tile-level pipeline, and
 // warp-specialised roles (TileRT blog "Breaking 1000 TPS", section
 // "第一次跃迁：Execution Model Revolution"; bjdmk.com.cn news, section
-// "极致协同，通向千速之路", on the persistent engine kernel), applied to the
+// "极致协同，通向千速之路", on the persistent engine kernel) -- applied to the
 // MoE expert layer whose routing is the runtime dynamism (HyperAI salon
 // transcript, section "Achieving maximum speed improvement ...").
 //
-// Every wait (grid barrier, mbarrier, per-unit readiness) is bounded by
-// p.timeout_ns of %globaltimer; on expiry the kernel records a status code in
-// sync[SY_ERROR], drains its own copies in flight and returns.
+// Weight stream (phase C).  Work is cut into CTA jobs of 64 weight rows x the
+// whole contraction dimension.  Warp NCW is the producer: it takes jobs from a
+// global counter, publishes them in a shared-memory job queue and streams each
+// job's K chunks (one 4352-byte MXFP4 stage + the matching activation slices)
+// into a ring of NSLOT slots with 1-D bulk copies (full/empty mbarriers).
+// Warps 0..NCW-1 consume chunk c of every job in warp c % NCW: E2M1 bytes are
+// turned into f16 A fragments in registers, the tokens form the N side of
+// mma.m16n8k16 (fp32 accumulate), and each MX block's E8M0 scale multiplies its
+// block partial in fp32.  The per-warp partial sums meet in shared memory
+// behind a named barrier and are reduced in warp order (deterministic), then
+// one warp per token (gate/up) or per pair (down) runs the epilogue.
+//
+// Every wait (grid barrier, mbarrier, job queue, per-unit readiness) is bounded
+// by p.timeout_ns of %globaltimer; on expiry the kernel records a status code
+// in sync[SY_ERROR], stops issuing work, lets every copy in flight land and
+// returns.
 #include <math.h>
 #include <cuda_fp16.h>
 
@@ -26,8 +39,15 @@ namespace moe {
 namespace {
 
 constexpr uint32_t FULL = 0xFFFFFFFFu;
-constexpr int WARP_BYTES = RING_BYTES + NBAR * 8 + JQ * 4;
 constexpr int SMALL_UNITS = 256 + SMALL_PAIRS / NT_MAX;
+
+struct JobEntry {
+  int32_t flag;  // queue index + 1 once the entry is written
+  int32_t job;   // -1: no more jobs in this phase
+  int32_t s0;    // stage sequence number of chunk 0
+  int32_t nc;    // chunks (stages)
+  int32_t unit, rb, isD, e, pos0, nt, pad0, pad1;
+};
 
 struct alignas(16) CtaTables {
   int32_t units[SMALL_UNITS * 4];  // first: read as int4
@@ -42,18 +62,25 @@ struct alignas(16) CtaTables {
   float red[WARPS];
   int32_t n_units;
 };
-constexpr size_t SMEM_BYTES = (size_t)WARPS * WARP_BYTES + sizeof(CtaTables);
 
-__device__ __forceinline__ uint8_t* warp_ring(uint8_t* smem, int w) { return smem + (size_t)w * WARP_BYTES; }
-__device__ __forceinline__ uint64_t* warp_bars(uint8_t* smem, int w) {
-  return reinterpret_cast<uint64_t*>(smem + (size_t)w * WARP_BYTES + RING_BYTES);
-}
-__device__ __forceinline__ int32_t* warp_jq(uint8_t* smem, int w) {
-  return reinterpret_cast<int32_t*>(smem + (size_t)w * WARP_BYTES + RING_BYTES + NBAR * 8);
-}
-__device__ __forceinline__ CtaTables& tables(uint8_t* smem) {
-  return *reinterpret_cast<CtaTables*>(smem + (size_t)WARPS * WARP_BYTES);
-}
+constexpr size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
+constexpr size_t OFF_RING = 0;
+constexpr size_t OFF_FULL = OFF_RING + (size_t)NSLOT * SLOT_BYTES;
+constexpr size_t OFF_EMPTY = OFF_FULL + NSLOT * 8;
+constexpr size_t OFF_JQ = align16(OFF_EMPTY + NSLOT * 8);
+constexpr size_t OFF_PART = align16(OFF_JQ + JQ * sizeof(JobEntry));
+constexpr size_t PART_BUF = (size_t)NCW * PART_COLS * PART_LD;  // floats per buffer
+constexpr size_t OFF_TABLES = align16(OFF_PART + 2 * PART_BUF * 4);
+constexpr size_t SMEM_BYTES = OFF_TABLES + sizeof(CtaTables);
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert((size_t)WARPS * MAX_EXPERTS * 4 <= (size_t)NSLOT * SLOT_BYTES, "routing scratch in ring");
+
+__device__ __forceinline__ uint8_t* ring_slot(uint8_t* smem, int s) { return smem + OFF_RING + (size_t)s * SLOT_BYTES; }
+__device__ __forceinline__ uint64_t* full_bar(uint8_t* smem, int s) { return reinterpret_cast<uint64_t*>(smem + OFF_FULL) + s; }
+__device__ __forceinline__ uint64_t* empty_bar(uint8_t* smem, int s) { return reinterpret_cast<uint64_t*>(smem + OFF_EMPTY) + s; }
+__device__ __forceinline__ JobEntry* job_queue(uint8_t* smem) { return reinterpret_cast<JobEntry*>(smem + OFF_JQ); }
+__device__ __forceinline__ float* part_buf(uint8_t* smem, int b) { return reinterpret_cast<float*>(smem + OFF_PART) + b * PART_BUF; }
+__device__ __forceinline__ CtaTables& tables(uint8_t* smem) { return *reinterpret_cast<CtaTables*>(smem + OFF_TABLES); }
 
 __device__ __forceinline__ void set_error(uint32_t* sync, uint32_t code, uint32_t info) {
   if (atomicCAS(sync + SY_ERROR, 0u, code) == 0u) atomicExch(sync + SY_ERRINFO, info);
@@ -91,53 +118,116 @@ __device__ bool grid_barrier(uint32_t* sync, uint64_t timeout_ns, uint32_t where
   return __syncthreads_and(ok) != 0;
 }
 
-// ---- phase A: router logits (fp64) ---------------------------------------------------
-// logits[t][e] = sum_h x[t][h] * Wr[e][h] + b[e]; bf16*fp32 products are exact
-// in fp64 and the sums are fp64, so top-k decisions match an fp64 reference
-// except on gaps below ~1e-10.
-__device__ void phase_logits(const EngineParams& p, const LayerPtrs& lp, const __nv_bfloat16* x,
-                             int layer) {
+// Bounded wait on an mbarrier phase; false on timeout or a recorded error.
+__device__ bool wait_mbar(uint64_t* bar, uint32_t parity, uint32_t* sync, uint64_t timeout_ns,
+                          uint32_t code, uint32_t info) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t spins = 0;
+  while (!mbar_try_wait(bar, parity)) {
+    if ((++spins & 63u) == 0u) {
+      if (error_set(sync)) return false;
+      if (globaltimer_ns() - t0 > timeout_ns) { set_error(sync, code, info); return false; }
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ float pow2f(int e) {  // 2^e for e in [-126, 127]
+  return __uint_as_float((uint32_t)(e + 127) << 23);
+}
+
+// ---- phase A: activations in f16 fragments, router partial logits -----------------------
+// Each token's x is scaled by 2^-px so that max|x| lies in [2^14, 2^15); then
+// every bf16 value is exact in f16 unless it is below max|x| * 2^-28.  The
+// 32-element blocks are stored in the mma B-fragment order (see chunk_mma).
+__device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const __nv_bfloat16* x,
+                              int layer) {
   const int T = p.T, H = p.H, E = p.E;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t gt = (int64_t)blockIdx.x * THREADS + threadIdx.x;
   const int64_t gs = (int64_t)gridDim.x * THREADS;
-  // fp32 activations for the weight stream; optional dump of the layer input
-  const int64_t n2 = (int64_t)T * H / 2;
-  const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(x);
-  float2* xf2 = reinterpret_cast<float2*>(p.xf);
-  __nv_bfloat162* dump = p.layer_io ? reinterpret_cast<__nv_bfloat162*>(p.layer_io + (int64_t)layer * T * H) : nullptr;
-  for (int64_t i = gt; i < n2; i += gs) {
-    const __nv_bfloat162 v = x2[i];
-    xf2[i] = __bfloat1622float2(v);
-    if (dump) dump[i] = v;
+  const int64_t wg = (int64_t)blockIdx.x * WARPS + warp, ws = (int64_t)gridDim.x * WARPS;
+  for (int64_t t = wg; t < T; t += ws) {
+    const __nv_bfloat16* xr = x + t * H;
+    float m = 0.f;
+    for (int h = lane * 8; h < H; h += 256) {
+      const uint4 v = *reinterpret_cast<const uint4*>(xr + h);
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        m = fmaxf(m, fabsf(__uint_as_float(u[i] << 16)));
+        m = fmaxf(m, fabsf(__uint_as_float(u[i] & 0xFFFF0000u)));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+    const int eb = (int)((__float_as_uint(m) >> 23) & 0xFF);
+    int px = m > 0.f ? eb - 127 - 14 : 0;
+    px = max(px, -126);
+    const float inv = pow2f(-px);
+    if (lane == 0) p.pxf[t] = pow2f(px);
+    for (int b = lane; b < H / 32; b += 32) {
+      const uint4* src = reinterpret_cast<const uint4*>(xr + b * 32);
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 q = src[i];
+        const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          v[i * 8 + 2 * k] = __uint_as_float(u[k] << 16) * inv;
+          v[i * 8 + 2 * k + 1] = __uint_as_float(u[k] & 0xFFFF0000u) * inv;
+        }
+      }
+      uint4* dst = reinterpret_cast<uint4*>(p.xh + (t * H + b * 32) * 2);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        __half2 h0 = __floats2half2_rn(v[2 * c], v[2 * c + 1]);
+        __half2 h1 = __floats2half2_rn(v[2 * c + 8], v[2 * c + 9]);
+        __half2 h2 = __floats2half2_rn(v[16 + 2 * c], v[17 + 2 * c]);
+        __half2 h3 = __floats2half2_rn(v[24 + 2 * c], v[25 + 2 * c]);
+        dst[c] = make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                            *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
+      }
+    }
+  }
+  if (p.layer_io) {
+    const int64_t n8 = (int64_t)T * H / 8;
+    const uint4* s8 = reinterpret_cast<const uint4*>(x);
+    uint4* d8 = reinterpret_cast<uint4*>(p.layer_io + (int64_t)layer * T * H);
+    for (int64_t i = gt; i < n8; i += gs) d8[i] = s8[i];
   }
   // per-layer resets of the stream's counters (used only after the next barrier)
   const int umax = min(E, p.TK) + p.TK / NT_MAX + 1;
   if (gt == 0) p.sync[SY_JOBS] = 0u;
   for (int64_t u = gt; u < umax; u += gs) p.sync[SY_READY + u] = 0u;
 
+  // partial logits[hs][t][e] = sum over the hs-th H part of x[t][h] * Wr[e][h];
+  // bf16 * fp32 products are exact in fp64 and the sums are fp64
+  const int HS = p.HS, hpart = H / HS;
   const int nchunk = (T + 7) / 8;
-  const int64_t njobs = (int64_t)E * nchunk;
-  const int64_t wg = (int64_t)blockIdx.x * WARPS + warp, ws = (int64_t)gridDim.x * WARPS;
+  const int64_t njobs = (int64_t)E * HS * nchunk;
   for (int64_t job = wg; job < njobs; job += ws) {
-    const int e = (int)(job % E), t0 = (int)(job / E) * 8;
+    const int e = (int)(job % E);
+    const int hs = (int)((job / E) % HS);
+    const int t0 = (int)(job / ((int64_t)E * HS)) * 8;
     const int nt = min(8, T - t0);
     double acc[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[j] = 0.0;
-    const float4* wr = reinterpret_cast<const float4*>(lp.router_w + (int64_t)e * H);
-    for (int h4 = lane; h4 < H / 4; h4 += 32) {
+    const float4* wr = reinterpret_cast<const float4*>(lp.router_w + (int64_t)e * H + hs * hpart);
+#pragma unroll 2
+    for (int h4 = lane; h4 < hpart / 4; h4 += 32) {
       const float4 w4 = __ldg(wr + h4);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         if (j < nt) {
-          const uint2 xb = *reinterpret_cast<const uint2*>(x + (int64_t)(t0 + j) * H + h4 * 4);
-          const float x0 = __uint_as_float(xb.x << 16), x1 = __uint_as_float(xb.x & 0xFFFF0000u);
-          const float x2v = __uint_as_float(xb.y << 16), x3 = __uint_as_float(xb.y & 0xFFFF0000u);
-          acc[j] = fma((double)x0, (double)w4.x, acc[j]);
-          acc[j] = fma((double)x1, (double)w4.y, acc[j]);
-          acc[j] = fma((double)x2v, (double)w4.z, acc[j]);
-          acc[j] = fma((double)x3, (double)w4.w, acc[j]);
+          const uint2 xb = *reinterpret_cast<const uint2*>(x + (int64_t)(t0 + j) * H + hs * hpart + h4 * 4);
+          acc[j] = fma((double)__uint_as_float(xb.x << 16), (double)w4.x, acc[j]);
+          acc[j] = fma((double)__uint_as_float(xb.x & 0xFFFF0000u), (double)w4.y, acc[j]);
+          acc[j] = fma((double)__uint_as_float(xb.y << 16), (double)w4.z, acc[j]);
+          acc[j] = fma((double)__uint_as_float(xb.y & 0xFFFF0000u), (double)w4.w, acc[j]);
         }
       }
     }
@@ -147,10 +237,9 @@ __device__ void phase_logits(const EngineParams& p, const LayerPtrs& lp, const _
       for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(FULL, acc[j], o);
     }
     if (lane == 0) {
-      const double b = lp.router_b ? (double)lp.router_b[e] : 0.0;
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        if (j < nt) p.logits[(int64_t)(t0 + j) * E + e] = acc[j] + b;
+        if (j < nt) p.logits[((int64_t)hs * T + t0 + j) * E + e] = acc[j];
     }
   }
 }
@@ -165,16 +254,26 @@ __device__ __forceinline__ double key_value(uint64_t k) {
   return __longlong_as_double((long long)b);
 }
 
-// One warp: the K largest logits of a row (descending, ties to the lower
-// expert), weights exp(l - lmax) / sum over the K.  Lane r < K writes slot r.
-__device__ void topk_row(const double* lg, int E, int K, int32_t* out_idx, float* out_w) {
+// One warp: logits of token t (partials summed in order, plus bias), the K
+// largest (descending, ties to the lower expert), weights exp(l - lmax) / sum
+// over the K.  Lane r < K writes slot r.
+__device__ void topk_row(const EngineParams& p, const float* bias, int t, int32_t* out_idx,
+                         float* out_w) {
   const int lane = threadIdx.x & 31;
+  const int E = p.E, K = p.K;
   constexpr int PER = MAX_EXPERTS / 32;
   uint64_t key[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int e = lane + 32 * i;
-    key[i] = e < E ? order_key(lg[e]) : 0ull;
+    if (e < E) {
+      double l = 0.0;
+      for (int hs = 0; hs < p.HS; ++hs) l += p.logits[((int64_t)hs * p.T + t) * E + e];
+      if (bias) l += (double)bias[e];
+      key[i] = order_key(l);
+    } else {
+      key[i] = 0ull;
+    }
   }
   uint32_t taken = 0;
   int my_e = -1;
@@ -204,9 +303,9 @@ __device__ void topk_row(const double* lg, int E, int K, int32_t* out_idx, float
   if (lane < K) { out_idx[lane] = my_e; out_w[lane] = (float)(ex / sum); }
 }
 
-// Exclusive scan of n <= 512 ints in shared memory by warp 0 (in place);
-// returns the total through *total.
-__device__ void warp0_exclusive_scan(int32_t* a, int n, int32_t* total) {
+// Exclusive scan of n <= 512 ints in shared memory by one warp (in place);
+// the total goes to *total.
+__device__ void warp_exclusive_scan(int32_t* a, int n, int32_t* total) {
   const int lane = threadIdx.x & 31;
   constexpr int PER = 16;
   int32_t v[PER];
@@ -235,16 +334,15 @@ __device__ void warp0_exclusive_scan(int32_t* a, int n, int32_t* total) {
 
 // Small T*K: every CTA routes all tokens itself (no barrier); CTA 0 also writes
 // the maps to global memory.
-__device__ void phase_route_small(const EngineParams& p, uint8_t* smem) {
+__device__ void phase_route_small(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem) {
   CtaTables& tb = tables(smem);
   const int T = p.T, E = p.E, K = p.K, TK = p.TK;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int t = warp; t < T; t += WARPS) topk_row(p.logits + (int64_t)t * E, E, K, tb.idx + t * K, tb.w + t * K);
-  // per-warp histograms (scratch in warp 0's ring, unused until phase C)
-  int32_t* hist = reinterpret_cast<int32_t*>(warp_ring(smem, 0));  // [WARPS][E]
+  for (int t = warp; t < T; t += WARPS) topk_row(p, lp.router_b, t, tb.idx + t * K, tb.w + t * K);
+  int32_t* hist = reinterpret_cast<int32_t*>(ring_slot(smem, 0));  // [WARPS][E] scratch
   for (int i = threadIdx.x; i < WARPS * E; i += THREADS) hist[i] = 0;
   __syncthreads();
-  const int pr = threadIdx.x;  // TK <= SMALL_PAIRS == THREADS: one pair per thread
+  const int pr = threadIdx.x;  // TK <= SMALL_PAIRS <= THREADS: one pair per thread
   const bool valid = pr < TK;
   const int e = valid ? tb.idx[pr] : -1 - lane;
   const uint32_t peers = __match_any_sync(FULL, e);
@@ -258,7 +356,7 @@ __device__ void phase_route_small(const EngineParams& p, uint8_t* smem) {
     tb.offsets[x] = c;
   }
   __syncthreads();
-  if (warp == 0) warp0_exclusive_scan(tb.offsets, E, tb.offsets + E);
+  if (warp == 0) warp_exclusive_scan(tb.offsets, E, tb.offsets + E);
   __syncthreads();
   if (valid) {
     int32_t before = 0;
@@ -269,12 +367,11 @@ __device__ void phase_route_small(const EngineParams& p, uint8_t* smem) {
     tb.tokpos[pos] = pr / K;
     tb.wpos[pos] = tb.w[pr];
   }
-  // units: ceil(count/NT_MAX) per hit expert, in expert order
-  int32_t* ubase = hist;  // reuse scratch after the pass above
+  int32_t* ubase = hist;
   __syncthreads();
   for (int x = threadIdx.x; x < E; x += THREADS) ubase[x] = (tb.counts[x] + NT_MAX - 1) / NT_MAX;
   __syncthreads();
-  if (warp == 0) warp0_exclusive_scan(ubase, E, &tb.n_units);
+  if (warp == 0) warp_exclusive_scan(ubase, E, &tb.n_units);
   __syncthreads();
   for (int x = threadIdx.x; x < E; x += THREADS) {
     const int c = tb.counts[x];
@@ -294,11 +391,11 @@ __device__ void phase_route_small(const EngineParams& p, uint8_t* smem) {
 }
 
 // Large T*K, step 1: top-k of every token, distributed over all warps.
-__device__ void phase_topk_large(const EngineParams& p) {
+__device__ void phase_topk_large(const EngineParams& p, const LayerPtrs& lp) {
   const int warp = threadIdx.x >> 5;
   const int64_t wg = (int64_t)blockIdx.x * WARPS + warp, ws = (int64_t)gridDim.x * WARPS;
   for (int64_t t = wg; t < p.T; t += ws)
-    topk_row(p.logits + t * p.E, p.E, p.K, p.idx + t * p.K, p.wts + t * p.K);
+    topk_row(p, lp.router_b, (int)t, p.idx + t * p.K, p.wts + t * p.K);
 }
 
 // Large T*K, step 2: counts/offsets in every CTA (shared-memory histogram),
@@ -313,13 +410,13 @@ __device__ void phase_permute_large(const EngineParams& p, uint8_t* smem) {
   __syncthreads();
   for (int i = threadIdx.x; i < E; i += THREADS) tb.offsets[i] = tb.counts[i];
   __syncthreads();
-  if (warp == 0) warp0_exclusive_scan(tb.offsets, E, tb.offsets + E);
+  if (warp == 0) warp_exclusive_scan(tb.offsets, E, tb.offsets + E);
   __syncthreads();
   if (blockIdx.x == 0) {
-    int32_t* ubase = reinterpret_cast<int32_t*>(warp_ring(smem, 0));
+    int32_t* ubase = reinterpret_cast<int32_t*>(ring_slot(smem, 0));
     for (int x = threadIdx.x; x < E; x += THREADS) ubase[x] = (tb.counts[x] + NT_MAX - 1) / NT_MAX;
     __syncthreads();
-    if (warp == 0) warp0_exclusive_scan(ubase, E, &tb.n_units);
+    if (warp == 0) warp_exclusive_scan(ubase, E, &tb.n_units);
     __syncthreads();
     for (int x = threadIdx.x; x < E; x += THREADS) {
       const int c = tb.counts[x];
@@ -348,236 +445,306 @@ __device__ void phase_permute_large(const EngineParams& p, uint8_t* smem) {
   }
 }
 
-// ---- phase C: the MXFP4 weight stream ------------------------------------------------------
-__device__ __forceinline__ float e8m0_to_f32(uint32_t b) {
-  if (b == 0u) return __uint_as_float(0x00400000u);  // 2^-127
-  if (b == 255u) return __uint_as_float(0x7FC00000u);
-  return __uint_as_float(b << 23);
+// ---- phase C: the MXFP4 weight stream on tensor cores --------------------------------------
+// E8M0 byte B of a word -> 2^(byte-127) as fp32; byte 0 gives 2^-127 exactly,
+// byte 255 gives +inf (its blocks hold zero codes, so the product is NaN).
+template <int B>
+__device__ __forceinline__ float e8m0_byte(uint32_t w) {
+  uint32_t bits;
+  if constexpr (B == 3) bits = (w >> 1) & 0x7F800000u;
+  else bits = (w << (23 - 8 * B)) & 0x7F800000u;
+  return __uint_as_float(max(bits, 0x00400000u));
 }
 
-// acc[j] += sum over this stage's KC elements of W[row][k] * x_j[k] for the
-// lane's row; weights decoded E2M1 -> f16x2 -> fp32 pairs, packed fp32 FMA,
-// one MX block at a time, scaled by its E8M0 factor.
-template <int NT>
-__device__ __forceinline__ void stage_dot(const uint8_t* st, int lane, float (&acc)[NT_MAX]) {
-  const uint32_t sc4 = *reinterpret_cast<const uint32_t*>(st + STAGE_CODE_BYTES + lane * KB);
-  const float* xs = reinterpret_cast<const float*>(st + STAGE_W_BYTES);
+// One K chunk (4 MX blocks) of a 64-row job for this warp:
+//   acc[t][n][i] += sum over blocks b of 2^s(row, b) [* 2^q(col, b)] * (A_b B_b)
+// A = the chunk's E2M1 codes of tile t as f16 fragments, B = activation
+// fragments of n-tile n.  Gate/up: columns are tokens (x in f16, scaled per
+// token).  Down: columns are (pair, hi/lo) halves of the SwiGLU output, scaled
+// per (pair, block) by 2^q.
+template <int NTILE, bool ISD>
+__device__ __forceinline__ void chunk_mma(const uint8_t* st, int lane, int nt, float (&acc)[4][2][4]) {
+  const int g = lane >> 2, c = lane & 3;
+  uint32_t sw0[4], sw1[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    sw0[t] = *reinterpret_cast<const uint32_t*>(st + STAGE_CODE_BYTES + (t * 16 + g) * KB);
+    sw1[t] = *reinterpret_cast<const uint32_t*>(st + STAGE_CODE_BYTES + (t * 16 + g + 8) * KB);
+  }
+  const uint8_t* act = st + STAGE_W_BYTES;
+  const uint8_t* bptr[NTILE];
+  const int8_t* qptr[NTILE];
+#pragma unroll
+  for (int n = 0; n < NTILE; ++n) {
+    if (!ISD) {
+      const int jb = g < nt ? g : 0;
+      bptr[n] = act + jb * XH_SLOT + c * 16;
+      qptr[n] = nullptr;
+    } else {
+      int pj = n * 4 + (g >> 1);
+      pj = pj < nt ? pj : 0;
+      bptr[n] = act + pj * A16_CHUNK_BYTES + A16_HDR + (g & 1) * 64 + c * 16;
+      int qj = n * 4 + c;
+      qj = qj < nt ? qj : 0;
+      qptr[n] = reinterpret_cast<const int8_t*>(act + qj * A16_CHUNK_BYTES);
+    }
+  }
 #pragma unroll
   for (int b = 0; b < KB; ++b) {
-    const uint4 q = *reinterpret_cast<const uint4*>(st + b * (ROWS * 16) + lane * 16);
-    const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
-    f32x2 part[NT];
+    const uint4 qa = *reinterpret_cast<const uint4*>(st + ((b * 2 + 0) * 32 + lane) * 16);
+    const uint4 qb = *reinterpret_cast<const uint4*>(st + ((b * 2 + 1) * 32 + lane) * 16);
+    uint4 bf[NTILE];
+    float qf[NTILE];
 #pragma unroll
-    for (int j = 0; j < NT; ++j) part[j] = {0.f, 0.f};
+    for (int n = 0; n < NTILE; ++n) {
+      bf[n] = *reinterpret_cast<const uint4*>(bptr[n] + b * (ISD ? 128 : 64));
+      qf[n] = ISD ? pow2f((int)qptr[n][b]) : 1.f;
+    }
+    const uint32_t wd[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
+    for (int t = 0; t < 4; ++t) {
+      uint32_t a0[4], a1[4];
+      e2m1x8_to_f16x2x4(wd[2 * t], a0);
+      e2m1x8_to_f16x2x4(wd[2 * t + 1], a1);
+      float f0, f1;
+      if (b == 0) { f0 = e8m0_byte<0>(sw0[t]); f1 = e8m0_byte<0>(sw1[t]); }
+      else if (b == 1) { f0 = e8m0_byte<1>(sw0[t]); f1 = e8m0_byte<1>(sw1[t]); }
+      else if (b == 2) { f0 = e8m0_byte<2>(sw0[t]); f1 = e8m0_byte<2>(sw1[t]); }
+      else { f0 = e8m0_byte<3>(sw0[t]); f1 = e8m0_byte<3>(sw1[t]); }
 #pragma unroll
-      for (int hb = 0; hb < 2; ++hb) {  // two bytes (four codes) per step
-        const uint32_t h0 = e2m1x2_to_f16x2(qw[m] >> (16 * hb));
-        const uint32_t h1 = e2m1x2_to_f16x2(qw[m] >> (16 * hb + 8));
-        const float2 w0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
-        const float2 w1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
-        const int k = b * 32 + m * 8 + hb * 4;
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          const float4 xv = *reinterpret_cast<const float4*>(xs + j * KC + k);
-          ffma2(part[j], {w0.x, w0.y}, {xv.x, xv.y});
-          ffma2(part[j], {w1.x, w1.y}, {xv.z, xv.w});
-        }
+      for (int n = 0; n < NTILE; ++n) {
+        float ct[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_f16_16816(ct, a0, bf[n].x, bf[n].y);
+        mma_f16_16816(ct, a1, bf[n].z, bf[n].w);
+        const float g0 = ISD ? f0 * qf[n] : f0, g1 = ISD ? f1 * qf[n] : f1;
+        acc[t][n][0] = fmaf(ct[0], g0, acc[t][n][0]);
+        acc[t][n][1] = fmaf(ct[1], g0, acc[t][n][1]);
+        acc[t][n][2] = fmaf(ct[2], g1, acc[t][n][2]);
+        acc[t][n][3] = fmaf(ct[3], g1, acc[t][n][3]);
       }
     }
-    const float sc = e8m0_to_f32((sc4 >> (8 * b)) & 0xFFu);
-#pragma unroll
-    for (int j = 0; j < NT; ++j) acc[j] = fmaf(part[j].x + part[j].y, sc, acc[j]);
   }
 }
 
-__device__ __forceinline__ void stage_dot_nt(int nt, const uint8_t* st, int lane, float (&acc)[NT_MAX]) {
-  switch (nt) {
-    case 1: stage_dot<1>(st, lane, acc); break;
-    case 2: stage_dot<2>(st, lane, acc); break;
-    case 3: stage_dot<3>(st, lane, acc); break;
-    case 4: stage_dot<4>(st, lane, acc); break;
-    case 5: stage_dot<5>(st, lane, acc); break;
-    case 6: stage_dot<6>(st, lane, acc); break;
-    case 7: stage_dot<7>(st, lane, acc); break;
-    default: stage_dot<8>(st, lane, acc); break;
-  }
-}
-
-struct Job {
-  int unit, rb, isD, e, pos0, nt, nc;
+struct StreamCtx {
+  const int32_t* units;
+  const int32_t* tokpos;
+  const float* wpos;
+  int n_units;
 };
 
-__device__ __forceinline__ Job decode_job(const EngineParams& p, const int32_t* units, int64_t j,
-                                          int64_t n_gu, int gub, int db) {
-  Job jb;
-  int64_t u;
-  if (j < n_gu) { u = j / gub; jb.rb = (int)(j % gub); jb.isD = 0; jb.nc = p.H / KC; }
-  else { const int64_t jj = j - n_gu; u = jj / db; jb.rb = (int)(jj % db); jb.isD = 1; jb.nc = p.I / KC; }
-  jb.unit = (int)u;
-  const int4 ur = *reinterpret_cast<const int4*>(units + u * 4);
-  jb.e = ur.x; jb.pos0 = ur.y; jb.nt = ur.z;
-  return jb;
-}
-
-__device__ __forceinline__ uint32_t ring_place(uint32_t v, uint32_t size) {
-  const uint32_t off = v % RING_BYTES;
-  return off + size > (uint32_t)RING_BYTES ? v + (RING_BYTES - off) : v;
-}
-
-// Runs this warp's share of the gate/up and down jobs.  Returns false on timeout.
-__device__ bool phase_stream(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem,
-                             const int32_t* units, int n_units, const int32_t* tokpos,
-                             const float* wpos, uint32_t& seq_base) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint8_t* ring = warp_ring(smem, warp);
-  uint64_t* bars = warp_bars(smem, warp);
-  int32_t* jq = warp_jq(smem, warp);
-  const int gub = p.I / GU_ROWS, db = p.H / ROWS;
-  const int64_t n_gu = (int64_t)n_units * gub, n_all = n_gu + (int64_t)n_units * db;
+// Producer warp: jobs -> queue entries -> stages into the ring.
+__device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem,
+                                const StreamCtx& cx, uint32_t& seq, int32_t& qk) {
+  const int lane = threadIdx.x & 31;
+  JobEntry* jq = job_queue(smem);
   uint32_t* ready = p.sync + SY_READY;
-
-  // producer state (warp-uniform except tok)
-  bool fetch_done = false, have_pjob = false, p_ready = true;
-  Job pj{};
-  int p_c = 0, tok = 0;
-  uint32_t p_v = 0, p_seq = seq_base, p_nj = 0;
-  // consumer state
-  Job cj{};
-  int c_c = 0;
-  uint32_t c_v = 0, c_seq = seq_base, c_nj = 0;
-  float acc[NT_MAX];
+  const int gub = p.I / (STAGE_ROWS / 2), db = p.H / STAGE_ROWS;
+  const int64_t n_gu = (int64_t)cx.n_units * gub, n_all = n_gu + (int64_t)cx.n_units * db;
+  const int nc_gu = p.H / KC, nc_d = p.I / KC;
+  const uint32_t seq_start = seq;
   bool ok = true;
   fence_proxy_async_global();
-  fence_proxy_async_smem();  // the ring held routing scratch written by generic stores
-
+  long long next = 0;
+  if (lane == 0) next = atomicAdd(p.sync + SY_JOBS, 1u);
   for (;;) {
-    // ---- issue as many stages as the ring allows
-    for (;;) {
-      if (!have_pjob) {
-        if (fetch_done) break;
-        int64_t j = 0;
-        if (lane == 0) j = atomicAdd(p.sync + SY_JOBS, 1u);
-        j = __shfl_sync(FULL, (long long)j, 0);
-        if (j >= n_all) { fetch_done = true; break; }
-        pj = decode_job(p, units, j, n_gu, gub, db);
-        if (lane == 0) jq[p_nj % JQ] = (int32_t)j;
-        ++p_nj;
-        p_c = 0;
-        have_pjob = true;
-        p_ready = !pj.isD;
-        if (!pj.isD && lane < pj.nt) tok = tokpos[pj.pos0 + lane];
-      }
-      if (!p_ready) {
-        if (ld_acquire_u32(ready + pj.unit) < (uint32_t)gub) break;
-        p_ready = true;
-        fence_proxy_async_global();
-      }
-      const uint32_t size = STAGE_W_BYTES + pj.nt * X_SLICE_BYTES;
-      const uint32_t start = ring_place(p_v, size);
-      if (p_seq - c_seq >= (uint32_t)NBAR || start + size - c_v > (uint32_t)RING_BYTES) break;
-      uint8_t* dst = ring + (start % RING_BYTES);
-      uint64_t* bar = bars + (p_seq % NBAR);
+    const int64_t j = __shfl_sync(FULL, next, 0);
+    if (j >= n_all || !ok || error_set(p.sync)) {
       if (lane == 0) {
-        mbar_arrive_expect_tx(bar, size);
-        const uint8_t* wsrc = pj.isD
-            ? lp.w_d + (((int64_t)pj.e * db + pj.rb) * pj.nc + p_c) * STAGE_W_BYTES
-            : lp.w_gu + (((int64_t)pj.e * gub + pj.rb) * pj.nc + p_c) * STAGE_W_BYTES;
-        bulk_g2s(dst, wsrc, STAGE_W_BYTES, bar);
-        if (pj.isD)
-          bulk_g2s(dst + STAGE_W_BYTES, p.abuf + ((int64_t)p_c * p.TK + pj.pos0) * KC,
-                   pj.nt * X_SLICE_BYTES, bar);
+        JobEntry* en = jq + (qk % JQ);
+        en->job = -1; en->s0 = (int32_t)seq; en->nc = 0;
+        __threadfence_block();
+        *reinterpret_cast<volatile int32_t*>(&en->flag) = qk + 1;
       }
-      __syncwarp();
-      if (!pj.isD && lane < pj.nt)
-        bulk_g2s(dst + STAGE_W_BYTES + lane * X_SLICE_BYTES, p.xf + (int64_t)tok * p.H + p_c * KC,
-                 X_SLICE_BYTES, bar);
-      p_v = start + size;
-      ++p_seq;
-      if (++p_c == pj.nc) have_pjob = false;
+      ++qk;
+      break;
     }
-
-    if (c_seq == p_seq) {  // nothing in flight
-      if (!have_pjob && fetch_done) break;
-      if (have_pjob && !p_ready) {  // wait for this unit's gate/up jobs (bounded)
+    if (lane == 0) next = atomicAdd(p.sync + SY_JOBS, 1u);  // prefetch the following job
+    const bool isD = j >= n_gu;
+    const int64_t jj = isD ? j - n_gu : j;
+    const int per = isD ? db : gub;
+    const int u = (int)(jj / per), rb = (int)(jj % per);
+    const int4 ur = *reinterpret_cast<const int4*>(cx.units + (int64_t)u * 4);
+    const int e = ur.x, pos0 = ur.y, nt = ur.z;
+    const int nc = isD ? nc_d : nc_gu;
+    if (lane == 0) {
+      JobEntry* en = jq + (qk % JQ);
+      en->job = (int32_t)j; en->s0 = (int32_t)seq; en->nc = nc; en->unit = u; en->rb = rb;
+      en->isD = isD; en->e = e; en->pos0 = pos0; en->nt = nt;
+      __threadfence_block();
+      *reinterpret_cast<volatile int32_t*>(&en->flag) = qk + 1;
+    }
+    ++qk;
+    if (isD) {  // the down stages read this unit's SwiGLU output: wait for its gate/up jobs
+      const uint32_t need = (uint32_t)(gub * nt);
+      if (ld_acquire_u32(ready + u) < need) {
         const uint64_t t0 = globaltimer_ns();
         uint32_t spins = 0;
-        while (ld_acquire_u32(ready + pj.unit) < (uint32_t)gub) {
+        while (ld_acquire_u32(ready + u) < need) {
           if ((++spins & 15u) == 0u) {
             if (error_set(p.sync)) { ok = false; break; }
-            if (globaltimer_ns() - t0 > p.timeout_ns) { set_error(p.sync, DEV_TIMEOUT_READY, pj.unit); ok = false; break; }
+            if (globaltimer_ns() - t0 > p.timeout_ns) { set_error(p.sync, DEV_TIMEOUT_READY, u); ok = false; break; }
           }
-          __nanosleep(128);
+          __nanosleep(100);
         }
-        if (!ok) break;
       }
-      continue;
+      fence_proxy_async_global();
     }
+    int tok = 0;
+    if (!isD && lane < nt) tok = cx.tokpos[pos0 + lane];
+    const uint8_t* wbase = isD ? lp.w_d + ((int64_t)e * db + rb) * nc * STAGE_W_BYTES
+                               : lp.w_gu + ((int64_t)e * gub + rb) * nc * STAGE_W_BYTES;
+    const uint32_t bytes = STAGE_W_BYTES + nt * (isD ? A16_CHUNK_BYTES : XH_CHUNK_BYTES);
+    for (int c = 0; c < nc && ok; ++c) {
+      const int slot = (int)(seq % NSLOT);
+      if (seq >= (uint32_t)NSLOT &&
+          !wait_mbar(empty_bar(smem, slot), ((seq / NSLOT) + 1) & 1u, p.sync, p.timeout_ns,
+                     DEV_TIMEOUT_PIPE, seq)) {
+        ok = false;
+        break;
+      }
+      uint8_t* dst = ring_slot(smem, slot);
+      uint64_t* fb = full_bar(smem, slot);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(fb, bytes);
+        bulk_g2s(dst, wbase + (int64_t)c * STAGE_W_BYTES, STAGE_W_BYTES, fb);
+        if (isD)
+          bulk_g2s(dst + STAGE_W_BYTES, p.a16 + ((int64_t)c * p.TK + pos0) * A16_CHUNK_BYTES,
+                   nt * A16_CHUNK_BYTES, fb);
+      }
+      __syncwarp();
+      if (!isD && lane < nt)
+        bulk_g2s(dst + STAGE_W_BYTES + lane * XH_SLOT, p.xh + ((int64_t)tok * p.H + c * KC) * 2,
+                 XH_CHUNK_BYTES, fb);
+      ++seq;
+    }
+  }
+  // let every issued copy land before the ring is reused or the CTA exits
+  const uint32_t issued = seq - seq_start;
+  const uint32_t n = issued < (uint32_t)NSLOT ? issued : (uint32_t)NSLOT;
+  for (uint32_t s = seq - n; s != seq; ++s) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(full_bar(smem, (int)(s % NSLOT)), (s / NSLOT) & 1u)) {
+      if (globaltimer_ns() - t0 > p.timeout_ns) break;
+    }
+  }
+}
 
-    // ---- consume the oldest stage
-    if (c_c == 0) {
-      const int64_t j = jq[c_nj % JQ];
-      cj = decode_job(p, units, j, n_gu, gub, db);
-#pragma unroll
-      for (int i = 0; i < NT_MAX; ++i) acc[i] = 0.f;
-    }
-    const uint32_t size = STAGE_W_BYTES + cj.nt * X_SLICE_BYTES;
-    const uint32_t start = ring_place(c_v, size);
-    uint64_t* bar = bars + (c_seq % NBAR);
-    const uint32_t parity = (c_seq / NBAR) & 1u;
-    if (!mbar_try_wait(bar, parity)) {
+// Consumer warps: chunks of every job, partial sums, reduction, epilogues.
+__device__ void stream_consumer(const EngineParams& p, uint8_t* smem, const StreamCtx& cx,
+                                int32_t& qk) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int g = lane >> 2, c = lane & 3;
+  JobEntry* jq = job_queue(smem);
+  uint32_t* ready = p.sync + SY_READY;
+  bool poison = false;
+  for (;;) {
+    JobEntry* en = jq + (qk % JQ);
+    // the producer publishes the entry (bounded wait; the producer's own waits
+    // are bounded by the same timeout, after which it publishes an end entry)
+    if (*reinterpret_cast<volatile int32_t*>(&en->flag) != qk + 1) {
       const uint64_t t0 = globaltimer_ns();
-      uint32_t spins = 0;
-      while (!mbar_try_wait(bar, parity)) {
-        if ((++spins & 63u) == 0u) {
-          if (error_set(p.sync)) { ok = false; break; }
-          if (globaltimer_ns() - t0 > p.timeout_ns) { set_error(p.sync, DEV_TIMEOUT_PIPE, c_seq); ok = false; break; }
-        }
+      while (*reinterpret_cast<volatile int32_t*>(&en->flag) != qk + 1) {
+        if (globaltimer_ns() - t0 > 2 * p.timeout_ns) { set_error(p.sync, DEV_TIMEOUT_QUEUE, qk); return; }
+        __nanosleep(32);
       }
-      if (!ok) break;
     }
-    stage_dot_nt(cj.nt, ring + (start % RING_BYTES), lane, acc);
-    __syncwarp();
-    c_v = start + size;
-    ++c_seq;
-    if (++c_c == cj.nc) {
-      c_c = 0;
-      ++c_nj;
-      if (!cj.isD) {  // SwiGLU epilogue: lanes 0-15 gate rows, 16-31 the same up rows
-        float u[NT_MAX];
+    const int job = *reinterpret_cast<volatile int32_t*>(&en->job);
+    if (job < 0) { ++qk; break; }
+    const int s0 = en->s0, nc = en->nc, u = en->unit, rb = en->rb, isD = en->isD;
+    const int pos0 = en->pos0, nt = en->nt;
+    const int buf = qk & 1;
+    float acc[4][2][4];
 #pragma unroll
-        for (int j = 0; j < NT_MAX; ++j) u[j] = __shfl_down_sync(FULL, acc[j], 16);
-        if (lane < 16) {
-          const int i = cj.rb * GU_ROWS + lane;
-          float* dst = p.abuf + ((int64_t)(i / KC) * p.TK + cj.pos0) * KC + (i % KC);
+    for (int t = 0; t < 4; ++t)
 #pragma unroll
-          for (int j = 0; j < NT_MAX; ++j) {
-            if (j < cj.nt) {
-              const float g = acc[j];
-              dst[(int64_t)j * KC] = g / (1.0f + expf(-g)) * u[j];
-            }
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[t][n][i] = 0.f;
+    for (int cc = w; cc < nc; cc += NCW) {
+      const uint32_t s = (uint32_t)s0 + cc;
+      const int slot = (int)(s % NSLOT);
+      if (!poison &&
+          !wait_mbar(full_bar(smem, slot), (s / NSLOT) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, s))
+        poison = true;
+      if (!poison) {
+        const uint8_t* st = ring_slot(smem, slot);
+        if (!isD) chunk_mma<1, false>(st, lane, nt, acc);
+        else if (nt <= 4) chunk_mma<1, true>(st, lane, nt, acc);
+        else chunk_mma<2, true>(st, lane, nt, acc);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar(smem, slot));
+    }
+    // deposit this warp's partial sums: part[w][col][row]
+    float* pb = part_buf(smem, buf) + (size_t)w * PART_COLS * PART_LD;
+    if (w < nc) {
+      const int ntile = isD && nt > 4 ? 2 : 1;
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+          if (n < ntile) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              pb[(n * 8 + 2 * c + (i & 1)) * PART_LD + t * 16 + g + (i >> 1) * 8] = acc[t][n][i];
           }
         }
+    }
+    named_barrier(1 + buf, NCW * 32);
+    const int nw = nc < NCW ? nc : NCW;
+    const float* pall = part_buf(smem, buf);
+    if (!poison && w < nt) {
+      if (!isD) {  // gate/up epilogue: token column w, lane = intermediate row i0 + lane
+        const int j = w;
+        const float px = p.pxf[cx.tokpos[pos0 + j]];
+        float gs = 0.f, us = 0.f;
+        for (int ww = 0; ww < nw; ++ww) {
+          gs += pall[((size_t)ww * PART_COLS + j) * PART_LD + lane];
+          us += pall[((size_t)ww * PART_COLS + j) * PART_LD + 32 + lane];
+        }
+        const float gv = gs * px, uv = us * px;
+        const float a = gv / (1.0f + expf(-gv)) * uv;
+        float am = fabsf(a);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(FULL, am, o));
+        const int eb = (int)((__float_as_uint(am) >> 23) & 0xFF);
+        int q = am > 0.f ? eb - 127 - 14 : 0;
+        q = max(q, -126);
+        const float v = a * pow2f(-q);
+        const __half hi = __float2half_rn(v);
+        const __half lo = __float2half_rn(v - __half2float(hi));
+        const int i0 = rb * (STAGE_ROWS / 2);
+        uint8_t* base = p.a16 + ((int64_t)(i0 / KC) * p.TK + pos0 + j) * A16_CHUNK_BYTES;
+        const int bi = (i0 % KC) / 32;
+        const int kk = lane & 15;
+        const int off = A16_HDR + bi * 128 + ((kk & 7) >> 1) * 16 +
+                        ((lane >> 4) * 4 + ((kk >> 3) << 1) + (kk & 1)) * 2;
+        *reinterpret_cast<__half*>(base + off) = hi;
+        *reinterpret_cast<__half*>(base + off + 64) = lo;
+        if (lane == 0) base[bi] = (uint8_t)(int8_t)q;
         __threadfence();
         __syncwarp();
-        if (lane == 0) red_release_add_u32(ready + cj.unit, 1u);
-      } else {  // down epilogue: weighted pair output rows
-        const int h = cj.rb * ROWS + lane;
+        if (lane == 0) red_release_add_u32(ready + u, 1u);
+      } else {  // down epilogue: pair w, lane = rows h0 + lane and h0 + 32 + lane
+        const int j = w;
+        const int col = (j >> 2) * 8 + 2 * (j & 3);
+        const float wp = cx.wpos[pos0 + j];
+        const int h0 = rb * STAGE_ROWS;
 #pragma unroll
-        for (int j = 0; j < NT_MAX; ++j)
-          if (j < cj.nt) p.ypair[(int64_t)(cj.pos0 + j) * p.H + h] = wpos[cj.pos0 + j] * acc[j];
+        for (int r2 = 0; r2 < 2; ++r2) {
+          const int r = lane + 32 * r2;
+          float y = 0.f;
+          for (int ww = 0; ww < nw; ++ww) {
+            const float* pw = pall + (size_t)ww * PART_COLS * PART_LD;
+            y += pw[col * PART_LD + r] + pw[(col + 1) * PART_LD + r];
+          }
+          p.ypair[(int64_t)(pos0 + j) * p.H + h0 + r] = y * wp;
+        }
       }
     }
+    ++qk;
   }
-  if (!ok) {  // drain this warp's copies still in flight (bounded) before leaving
-    const uint64_t t0 = globaltimer_ns();
-    while (c_seq != p_seq && globaltimer_ns() - t0 < p.timeout_ns) {
-      if (mbar_try_wait(bars + (c_seq % NBAR), (c_seq / NBAR) & 1u)) ++c_seq;
-    }
-  }
-  seq_base = p_seq;  // keep barrier phases consistent across layers
-  return ok;
 }
 
 // ---- phase D: combine (+ RMSNorm) ------------------------------------------------------------
@@ -616,7 +783,7 @@ __device__ void phase_combine_out(const EngineParams& p, const int32_t* inv) {
 __device__ void phase_combine_rmsnorm(const EngineParams& p, const int32_t* inv, uint8_t* smem) {
   CtaTables& tb = tables(smem);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int MAXV = 8;  // float4 per thread: H <= 8 * 4 * THREADS = 8192
+  constexpr int MAXV = (8192 / 4 + THREADS - 1) / THREADS;
   for (int t = blockIdx.x; t < p.T; t += gridDim.x) {
     float4 yv[MAXV];
     float ss = 0.f;
@@ -655,46 +822,59 @@ __device__ void phase_combine_rmsnorm(const EngineParams& p, const int32_t* inv,
 
 __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (lane == 0) {
-    uint64_t* bars = warp_bars(smem, warp);
-    for (int i = 0; i < NBAR; ++i) mbar_init(bars + i, 1);
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NSLOT; ++i) {
+      mbar_init(full_bar(smem, i), 1);
+      mbar_init(empty_bar(smem, i), 1);
+    }
     fence_mbar_init();
   }
+  for (int i = threadIdx.x; i < JQ; i += THREADS) job_queue(smem)[i].flag = 0;
   __syncthreads();
-  uint32_t seq = 0;
+  const bool stamp = p.stamps != nullptr && blockIdx.x == 0 && threadIdx.x == 0;
+  if (stamp) p.stamps[0] = globaltimer_ns();
+  uint32_t seq = 0;   // stage sequence (producer), continues across layers
+  int32_t qk = 0;     // job queue position, continues across layers
   const bool small = p.TK <= SMALL_PAIRS;
   CtaTables& tb = tables(smem);
   for (int layer = 0; layer < p.L; ++layer) {
     const LayerPtrs& lp = p.layers[layer];
     const __nv_bfloat16* x = layer == 0 ? p.x_in : p.xnext;
-    phase_logits(p, lp, x, layer);
+    uint64_t* st = stamp ? p.stamps + 1 + layer * STAMPS_PER_LAYER : nullptr;
+    phase_prepare(p, lp, x, layer);
     if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 1)) return;
-    const int32_t *units, *tokpos, *inv;
-    const float* wpos;
-    int n_units;
+    if (st) st[0] = globaltimer_ns();
+    StreamCtx cx;
+    const int32_t* inv;
     if (small) {
-      phase_route_small(p, smem);
-      units = tb.units; tokpos = tb.tokpos; wpos = tb.wpos; inv = tb.inv; n_units = tb.n_units;
+      phase_route_small(p, lp, smem);
+      cx = StreamCtx{tb.units, tb.tokpos, tb.wpos, tb.n_units};
+      inv = tb.inv;
       if (p.route_only) return;
     } else {
-      phase_topk_large(p);
+      phase_topk_large(p, lp);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 2)) return;
       phase_permute_large(p, smem);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 3)) return;
       if (p.route_only) return;
-      units = p.units; tokpos = p.tokpos; wpos = p.wpos; inv = p.inv; n_units = *p.n_units;
+      cx = StreamCtx{p.units, p.tokpos, p.wpos, *p.n_units};
+      inv = p.inv;
     }
+    if (st) st[1] = globaltimer_ns();
+    fence_proxy_async_smem();  // the ring held routing scratch written by generic stores
     __syncthreads();
-    const bool ok = phase_stream(p, lp, smem, units, n_units, tokpos, wpos, seq);
-    if (!ok) set_error(p.sync, DEV_TIMEOUT_PIPE, 0xFFFFFFFFu);  // no-op if already set
+    if (warp == NCW) stream_producer(p, lp, smem, cx, seq, qk);
+    else stream_consumer(p, smem, cx, qk);
     if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 4)) return;
+    if (st) st[2] = globaltimer_ns();
     if (layer + 1 < p.L) {
       phase_combine_rmsnorm(p, inv, smem);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 5)) return;
     } else {
       phase_combine_out(p, inv);
     }
+    if (st) st[3] = globaltimer_ns();
   }
 }
 

@@ -8,29 +8,37 @@
 namespace moe {
 
 // ---- streaming layout -------------------------------------------------------------
-// One pipeline stage covers KC elements of the contraction dimension for 32
-// weight rows: the codes of 4 MX blocks laid out [block][row][16 B], then the
-// 32 rows' 4 scale bytes [row][4 B].  A gate/up stage holds 16 gate rows
-// (lanes 0-15) then the same 16 up rows (lanes 16-31); a down stage holds 32
-// consecutive rows of Wd.  Stages of one (expert, row block) are contiguous
-// over the K chunks, so a warp streams one contiguous byte range per job.
-constexpr int KC = 128;                          // K elements per stage
-constexpr int KB = KC / 32;                      // MX blocks per stage
-constexpr int ROWS = 32;                         // weight rows per stage (= lanes)
-constexpr int STAGE_CODE_BYTES = ROWS * KC / 2;  // 2048
-constexpr int STAGE_W_BYTES = STAGE_CODE_BYTES + ROWS * KB;  // 2176
-constexpr int GU_ROWS = 16;                      // gate (and up) rows per gate/up job
-constexpr int NT_MAX = 8;                        // tokens per job (a "unit" of a segment)
-constexpr int X_SLICE_BYTES = KC * 4;            // one token's fp32 activations per stage
+// The weight stream is cut into jobs of 64 weight rows x the whole contraction
+// dimension: a gate/up job holds 32 gate rows and the same 32 up rows of one
+// expert (one 32-row block of the intermediate dimension), a down job 64 rows
+// of Wd.  A job is streamed in stages of KC = 128 K elements (four MX blocks);
+// the stage layout (see quantize.cu) is the mma.m16n8k16 A-fragment order, so
+// a lane turns its 16 bytes per half-stage straight into f16 fragments.
+constexpr int KC = 128;                                  // K elements per stage
+constexpr int KB = KC / 32;                              // MX blocks per stage
+constexpr int STAGE_ROWS = 64;                           // weight rows per stage
+constexpr int STAGE_CODE_BYTES = STAGE_ROWS * KC / 2;    // 4096
+constexpr int STAGE_W_BYTES = STAGE_CODE_BYTES + STAGE_ROWS * KB;  // 4352
+constexpr int NT_MAX = 8;                                // tokens per unit (one MMA n-tile)
+// activations of one stage, per token (gate/up) or per (token, expert) pair (down)
+constexpr int XH_CHUNK_BYTES = KC * 2;                   // f16 x, fragment order
+constexpr int XH_SLOT = XH_CHUNK_BYTES + 64;             // padded: conflict-free fragment loads
+constexpr int A16_HDR = 16;                              // 4 block exponents q, padded
+constexpr int A16_CHUNK_BYTES = A16_HDR + KC * 2 * 2;    // hi and lo f16 halves: 528
+constexpr int SLOT_BYTES = STAGE_W_BYTES + NT_MAX * A16_CHUNK_BYTES;  // 8576
+constexpr int MAX_HSPLIT = 8;                            // router dot products split along H
 
 constexpr int MAX_LAYERS = 16;
 constexpr int MAX_EXPERTS = 512;
-constexpr int THREADS = 256;                     // 8 warps per CTA
-constexpr int WARPS = THREADS / 32;
-constexpr int RING_BYTES = 24576;                // per-warp stage ring
-constexpr int NBAR = 16;                         // stages in flight per warp (max)
-constexpr int JQ = 32;                           // per-warp job queue entries
-constexpr int SMALL_PAIRS = 256;                 // T*k up to this: routing done per CTA
+constexpr int NCW = 8;                                   // consumer (MMA) warps per CTA
+constexpr int WARPS = NCW + 1;                           // + one producer warp
+constexpr int THREADS = WARPS * 32;
+constexpr int NSLOT = 15;                                // stage ring slots per CTA
+constexpr int JQ = 32;                                   // job queue entries per CTA
+constexpr int PART_LD = 68;                              // partial-sum column stride (floats)
+constexpr int PART_COLS = 16;                            // up to two n-tiles
+constexpr int SMALL_PAIRS = 256;                         // T*k up to this: routing done per CTA
+constexpr int STAMPS_PER_LAYER = 4;                      // prepared, routed, streamed, combined
 
 // sync word layout (uint32)
 enum : int {
@@ -40,17 +48,25 @@ enum : int {
 // device-side error codes (status word)
 enum : uint32_t {
   DEV_OK = 0, DEV_TIMEOUT_BARRIER = 1, DEV_TIMEOUT_PIPE = 2, DEV_TIMEOUT_READY = 3,
+  DEV_TIMEOUT_QUEUE = 4,
 };
 
+// Router split of H: about 1024 elements per part, each part a multiple of KC.
+inline int router_hsplit(int H) {
+  int hs = H % 1024 == 0 ? H / 1024 : 1;
+  return hs > MAX_HSPLIT ? (H % (MAX_HSPLIT * KC) == 0 ? MAX_HSPLIT : 1) : hs;
+}
+
 struct LayerPtrs {
-  const uint8_t* w_gu;  // gate/up stages  [E][I/16][H/KC][STAGE_W_BYTES]
-  const uint8_t* w_d;   // down stages     [E][H/32][I/KC][STAGE_W_BYTES]
+  const uint8_t* w_gu;  // gate/up stages  [E][I/32][H/KC][STAGE_W_BYTES]
+  const uint8_t* w_d;   // down stages     [E][H/64][I/KC][STAGE_W_BYTES]
   const float* router_w;  // [E][H]
   const float* router_b;  // [E] or null
 };
 
 struct EngineParams {
   int H, I, E, K, T, TK, L;  // hidden, inter, experts, top_k, tokens, T*K, layers to run
+  int HS;                    // router H split (H/HS a multiple of KC)
   int route_only;            // 1: stop after routing of layer 0, export maps
   float rms_eps;
   uint64_t timeout_ns;
@@ -59,8 +75,9 @@ struct EngineParams {
   __nv_bfloat16* y_out;       // [T][H] (null in route-only mode)
   __nv_bfloat16* layer_io;    // null or [L+1][T][H]
   // workspace (handle-owned)
-  double* logits;             // [T][E]
-  float* xf;                  // [T][H]
+  double* logits;             // [HS][T][E] partial logits
+  uint8_t* xh;                // [T][H] f16, fragment order within 32-blocks
+  float* pxf;                 // [T] power-of-two scale of each token's xh
   __nv_bfloat16* xnext;       // [T][H]
   int32_t* idx;               // [TK]
   float* wts;                 // [TK]
@@ -72,11 +89,10 @@ struct EngineParams {
   float* wpos;                // [TK] routing weight of each permuted position
   int32_t* units;             // [Umax][4] (expert, pos0, nt, 0)
   int32_t* n_units;           // [1]
-  float* abuf;                // [I/KC][TK][KC]
+  uint8_t* a16;               // [I/KC][TK][A16_CHUNK_BYTES]  SwiGLU output, hi/lo f16
   float* ypair;               // [TK][H]
   uint32_t* sync;             // see SY_*
-  // route-only exports (device, caller-owned)
-  int32_t* o_idx; float* o_w; int32_t* o_counts; int32_t* o_offsets; int32_t* o_perm; int32_t* o_inv;
+  uint64_t* stamps;           // null or [1 + MAX_LAYERS * STAMPS_PER_LAYER] %globaltimer ns (CTA 0)
 };
 
 size_t engine_smem_bytes();

@@ -23,12 +23,15 @@ struct moe_mxfp4 {
   float* router_w[MAX_LAYERS] = {};
   float* router_b[MAX_LAYERS] = {};
   double* logits = nullptr;
-  float* xf = nullptr;
+  uint8_t* xh = nullptr;
+  float* pxf = nullptr;
+  uint8_t* a16 = nullptr;
   __nv_bfloat16* xnext = nullptr;
   int32_t *idx = nullptr, *counts = nullptr, *offsets = nullptr, *perm = nullptr, *inv = nullptr,
           *tokpos = nullptr, *units = nullptr, *n_units = nullptr;
-  float *wts = nullptr, *wpos = nullptr, *abuf = nullptr, *ypair = nullptr;
+  float *wts = nullptr, *wpos = nullptr, *ypair = nullptr;
   uint32_t* sync = nullptr;
+  uint64_t* stamps = nullptr;
   __nv_bfloat16 *x_stage = nullptr, *y_stage = nullptr;
   std::vector<void*> allocs;
 };
@@ -52,10 +55,10 @@ void free_all(moe_mxfp4* h) {
 }
 
 size_t stage_bytes_gu(const moe_config_t& c) {
-  return (size_t)c.num_experts * (c.inter / GU_ROWS) * (c.hidden / KC) * STAGE_W_BYTES;
+  return (size_t)c.num_experts * (c.inter / (STAGE_ROWS / 2)) * (c.hidden / KC) * STAGE_W_BYTES;
 }
 size_t stage_bytes_d(const moe_config_t& c) {
-  return (size_t)c.num_experts * (c.hidden / ROWS) * (c.inter / KC) * STAGE_W_BYTES;
+  return (size_t)c.num_experts * (c.hidden / STAGE_ROWS) * (c.inter / KC) * STAGE_W_BYTES;
 }
 
 int32_t validate_cfg(const moe_config_t* c) {
@@ -76,14 +79,16 @@ EngineParams base_params(const moe_mxfp4* h, int T) {
   p.H = h->cfg.hidden; p.I = h->cfg.inter; p.E = h->cfg.num_experts; p.K = h->cfg.top_k;
   p.T = T; p.TK = T * h->cfg.top_k; p.L = h->cfg.num_layers;
   p.rms_eps = h->cfg.rms_eps;
+  p.HS = router_hsplit(h->cfg.hidden);
   p.timeout_ns = h->timeout_ns;
   for (int l = 0; l < h->cfg.num_layers; ++l)
     p.layers[l] = LayerPtrs{h->w_gu[l], h->w_d[l], h->router_w[l], h->router_b[l]};
-  p.logits = h->logits; p.xf = h->xf; p.xnext = h->xnext;
+  p.logits = h->logits; p.xh = h->xh; p.pxf = h->pxf; p.xnext = h->xnext;
   p.idx = h->idx; p.wts = h->wts; p.counts = h->counts; p.offsets = h->offsets;
   p.perm = h->perm; p.inv = h->inv; p.tokpos = h->tokpos; p.wpos = h->wpos;
-  p.units = h->units; p.n_units = h->n_units; p.abuf = h->abuf; p.ypair = h->ypair;
+  p.units = h->units; p.n_units = h->n_units; p.a16 = h->a16; p.ypair = h->ypair;
   p.sync = h->sync;
+  p.stamps = h->stamps;
   return p;
 }
 
@@ -167,15 +172,19 @@ int32_t moe_mxfp4_create(const moe_config_t* cfg, const uint8_t* const* gate_cod
          dalloc(h, &h->router_w[l], (size_t)E * H * 4);
     if (ok && router_bias && router_bias[l]) ok = dalloc(h, &h->router_b[l], (size_t)E * 4);
   }
-  ok = ok && dalloc(h, &h->logits, (size_t)Tm * E * 8) && dalloc(h, &h->xf, (size_t)Tm * H * 4) &&
+  const int HS = router_hsplit(H);
+  ok = ok && dalloc(h, &h->logits, (size_t)HS * Tm * E * 8) && dalloc(h, &h->xh, (size_t)Tm * H * 2) &&
+       dalloc(h, &h->pxf, (size_t)Tm * 4) &&
        dalloc(h, &h->xnext, (size_t)Tm * H * 2) && dalloc(h, &h->idx, (size_t)TKm * 4) &&
        dalloc(h, &h->wts, (size_t)TKm * 4) && dalloc(h, &h->counts, (size_t)E * 4) &&
        dalloc(h, &h->offsets, (size_t)(E + 1) * 4) && dalloc(h, &h->perm, (size_t)TKm * 4) &&
        dalloc(h, &h->inv, (size_t)TKm * 4) && dalloc(h, &h->tokpos, (size_t)TKm * 4) &&
        dalloc(h, &h->wpos, (size_t)TKm * 4) && dalloc(h, &h->units, (size_t)h->umax * 16) &&
-       dalloc(h, &h->n_units, 16) && dalloc(h, &h->abuf, (size_t)I * TKm * 4) &&
+       dalloc(h, &h->n_units, 16) &&
+       dalloc(h, &h->a16, (size_t)(I / KC) * TKm * A16_CHUNK_BYTES) &&
        dalloc(h, &h->ypair, (size_t)TKm * H * 4) &&
        dalloc(h, &h->sync, (size_t)(SY_READY + h->umax) * 4) &&
+       dalloc(h, &h->stamps, (size_t)(1 + MAX_LAYERS * STAMPS_PER_LAYER) * 8) &&
        dalloc(h, &h->x_stage, (size_t)Tm * H * 2) && dalloc(h, &h->y_stage, (size_t)Tm * H * 2);
   if (!ok) { free_all(h); delete h; cudaGetLastError(); return MOE_ERR_OOM; }
 
@@ -260,6 +269,17 @@ int32_t moe_forward_host(moe_mxfp4_t* h, const void* x_host, int32_t T, void* y_
   if (cudaMemcpyAsync(y_host, h->y_stage, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   return moe_status(h, stream);
+}
+
+int32_t moe_phase_ns(moe_mxfp4_t* h, uint64_t* ns_out, int32_t max_n, void* stream) {
+  if (!h || !ns_out || max_n < 0) return MOE_ERR_INVALID_ARG;
+  const int n = h->cfg.num_layers * STAMPS_PER_LAYER;
+  uint64_t raw[1 + MAX_LAYERS * STAMPS_PER_LAYER];
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess ||
+      cudaMemcpy(raw, h->stamps, (size_t)(1 + n) * 8, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  for (int i = 0; i < n && i < max_n; ++i) ns_out[i] = raw[i + 1] - raw[i];
+  return MOE_OK;
 }
 
 int32_t moe_set_timeout_ns(moe_mxfp4_t* h, uint64_t ns) {

@@ -37,7 +37,7 @@ int g_grid[kMaxDevices] = {};
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Layout {
-  size_t logits, xf, units, n_units, tokpos, wpos, sync, total;
+  size_t logits, xh, pxf, units, n_units, tokpos, wpos, sync, total;
   int umax;
 };
 
@@ -48,8 +48,9 @@ Layout layout_for(int T, int H, int E, int K) {
   l.umax = (int)((E < TK ? E : TK) + TK / NT_MAX + 1);
   size_t o = 0;
   l.sync = o;    o = align256(o + (size_t)(SY_READY + l.umax) * 4);
-  l.logits = o;  o = align256(o + (size_t)T * E * 8);
-  l.xf = o;      o = align256(o + (size_t)T * H * 4);
+  l.logits = o;  o = align256(o + (size_t)router_hsplit(H) * T * E * 8);
+  l.xh = o;      o = align256(o + (size_t)T * H * 2);
+  l.pxf = o;     o = align256(o + (size_t)T * 4);
   l.units = o;   o = align256(o + (size_t)l.umax * 16);
   l.n_units = o; o = align256(o + 16);
   l.tokpos = o;  o = align256(o + (size_t)TK * 4);
@@ -116,6 +117,7 @@ extern "C" MOE_API int32_t moe_route_static(const void* x_bf16, int32_t T, int32
   unsigned char* s = static_cast<unsigned char*>(base);
   EngineParams p{};
   p.H = hidden; p.I = KC; p.E = num_experts; p.K = top_k; p.T = T; p.TK = T * top_k; p.L = 1;
+  p.HS = router_hsplit(hidden);
   p.route_only = 1;
   p.timeout_ns = 2000000000ull;
   if (const char* env = std::getenv("MOE_TIMEOUT_NS")) {
@@ -125,7 +127,8 @@ extern "C" MOE_API int32_t moe_route_static(const void* x_bf16, int32_t T, int32
   p.layers[0] = LayerPtrs{nullptr, nullptr, router_w, router_bias};
   p.x_in = static_cast<const __nv_bfloat16*>(x_bf16);
   p.logits = reinterpret_cast<double*>(s + lay.logits);
-  p.xf = reinterpret_cast<float*>(s + lay.xf);
+  p.xh = s + lay.xh;
+  p.pxf = reinterpret_cast<float*>(s + lay.pxf);
   p.units = reinterpret_cast<int32_t*>(s + lay.units);
   p.n_units = reinterpret_cast<int32_t*>(s + lay.n_units);
   p.tokpos = reinterpret_cast<int32_t*>(s + lay.tokpos);
