@@ -171,6 +171,19 @@ MOE_API int32_t moe_status(moe_mxfp4_t* h, void* stream);
  */
 MOE_API int32_t moe_phase_ns(moe_mxfp4_t* h, uint64_t* ns_out, int32_t max_n, void* stream);
 
+/*
+ * moe_stream_profile -- tracing of the weight stream: synchronise `stream`,
+ * copy up to max_n counters accumulated since the previous call to the HOST
+ * array out (may be NULL when max_n == 0), reset them, and switch counting on
+ * (enable != 0) or off for the following launches.  Counters, in SM clock
+ * cycles summed over CTAs and warps: producer waiting for free ring slots,
+ * producer waiting for gate/up completion, producer total, stages issued;
+ * consumers waiting for data, in MMA chunks, at the per-job barrier, in
+ * epilogues, waiting for the job queue, consumer total, jobs.
+ */
+MOE_API int32_t moe_stream_profile(moe_mxfp4_t* h, int32_t enable, uint64_t* out, int32_t max_n,
+                                   void* stream);
+
 /* moe_set_timeout_ns -- bound of every device-side wait (default 2 s; env MOE_TIMEOUT_NS). */
 MOE_API int32_t moe_set_timeout_ns(moe_mxfp4_t* h, uint64_t ns);
 

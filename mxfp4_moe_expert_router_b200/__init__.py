@@ -19,7 +19,8 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_OOM, MOE_ERR_CUD
 
 EXPORTS = ("mxfp4_quantize", "moe_mxfp4_create", "moe_route", "moe_forward", "moe_forward_host",
            "moe_status", "moe_set_timeout_ns", "moe_engine_grid", "moe_mxfp4_destroy",
-           "moe_status_str", "moe_route_static", "moe_phase_ns")
+           "moe_status_str", "moe_route_static", "moe_phase_ns",
+           "moe_stream_profile")
 
 
 class MoeConfig(ctypes.Structure):
@@ -55,6 +56,7 @@ def _load():
         "moe_engine_grid": (i32, [vp]),
         "moe_mxfp4_destroy": (None, [vp]),
         "moe_status_str": (ctypes.c_char_p, [i32]),
+        "moe_stream_profile": (i32, [vp, i32, ctypes.POINTER(ctypes.c_uint64), i32, vp]),
         "moe_phase_ns": (i32, [vp, ctypes.POINTER(ctypes.c_uint64), i32, vp]),
         "moe_route_static": (i32, [vp, i32, i32, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, vp]),
     }
@@ -178,6 +180,18 @@ class Moe:
         arr = (ctypes.c_uint64 * n)()
         _check(lib.moe_phase_ns(self.handle, arr, n, _stream(stream)), "moe_phase_ns")
         return [int(v) for v in arr]
+
+    PROFILE_KEYS = ("prod_wait_empty", "prod_wait_ready", "prod_total", "stages",
+                    "cons_wait_full", "cons_mma", "cons_barrier", "cons_epilogue", "cons_queue",
+                    "cons_total", "jobs")
+
+    def moe_stream_profile(self, enable=True, stream=None):
+        """Counters since the previous call (dict), then counting switched on/off."""
+        n = len(self.PROFILE_KEYS)
+        arr = (ctypes.c_uint64 * n)()
+        _check(lib.moe_stream_profile(self.handle, int(bool(enable)), arr, n, _stream(stream)),
+               "moe_stream_profile")
+        return dict(zip(self.PROFILE_KEYS, (int(v) for v in arr)))
 
     def moe_set_timeout_ns(self, ns: int):
         _check(lib.moe_set_timeout_ns(self.handle, int(ns)), "moe_set_timeout_ns")

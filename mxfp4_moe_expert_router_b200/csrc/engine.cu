@@ -40,6 +40,7 @@ namespace {
 
 constexpr uint32_t FULL = 0xFFFFFFFFu;
 constexpr int SMALL_UNITS = 256 + SMALL_PAIRS / NT_MAX;
+constexpr int SMALL_DUNITS = 256 + SMALL_PAIRS / ND_MAX;
 
 struct JobEntry {
   int32_t flag;  // queue index + 1 once the entry is written
@@ -51,6 +52,7 @@ struct JobEntry {
 
 struct alignas(16) CtaTables {
   int32_t units[SMALL_UNITS * 4];  // first: read as int4
+  int32_t dunits[SMALL_DUNITS * 4];
   int32_t idx[SMALL_PAIRS];
   float w[SMALL_PAIRS];
   int32_t perm[SMALL_PAIRS];
@@ -60,7 +62,7 @@ struct alignas(16) CtaTables {
   int32_t counts[MAX_EXPERTS];
   int32_t offsets[MAX_EXPERTS + 1];
   float red[WARPS];
-  int32_t n_units;
+  int32_t n_units, n_dunits;
 };
 
 constexpr size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
@@ -199,7 +201,7 @@ __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const 
     for (int64_t i = gt; i < n8; i += gs) d8[i] = s8[i];
   }
   // per-layer resets of the stream's counters (used only after the next barrier)
-  const int umax = min(E, p.TK) + p.TK / NT_MAX + 1;
+  const int umax = max_units(E, p.TK);
   if (gt == 0) p.sync[SY_JOBS] = 0u;
   for (int64_t u = gt; u < umax; u += gs) p.sync[SY_READY + u] = 0u;
 
@@ -217,7 +219,7 @@ __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const 
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[j] = 0.0;
     const float4* wr = reinterpret_cast<const float4*>(lp.router_w + (int64_t)e * H + hs * hpart);
-#pragma unroll 2
+#pragma unroll 4
     for (int h4 = lane; h4 < hpart / 4; h4 += 32) {
       const float4 w4 = __ldg(wr + h4);
 #pragma unroll
@@ -267,8 +269,13 @@ __device__ void topk_row(const EngineParams& p, const float* bias, int t, int32_
   for (int i = 0; i < PER; ++i) {
     const int e = lane + 32 * i;
     if (e < E) {
+      double part[MAX_HSPLIT];
+#pragma unroll
+      for (int hs = 0; hs < MAX_HSPLIT; ++hs)
+        part[hs] = hs < p.HS ? p.logits[((int64_t)hs * p.T + t) * E + e] : 0.0;
       double l = 0.0;
-      for (int hs = 0; hs < p.HS; ++hs) l += p.logits[((int64_t)hs * p.T + t) * E + e];
+#pragma unroll
+      for (int hs = 0; hs < MAX_HSPLIT; ++hs) l += part[hs];
       if (bias) l += (double)bias[e];
       key[i] = order_key(l);
     } else {
@@ -332,6 +339,36 @@ __device__ void warp_exclusive_scan(int32_t* a, int n, int32_t* total) {
   if (lane == 31) *total = incl;
 }
 
+// Unit tables from per-expert counts/offsets: gate/up units of <= NT_MAX
+// consecutive positions of one expert's segment, down units of <= ND_MAX
+// (each inside one gate/up unit).  scratch: 2*E ints.
+__device__ void build_units(const int32_t* counts, const int32_t* offsets, int E, int32_t* scratch,
+                            int32_t* units, int32_t* dunits, int32_t* n_units, int32_t* n_dunits) {
+  const int warp = threadIdx.x >> 5;
+  int32_t* ubase = scratch;
+  int32_t* dbase = scratch + E;
+  for (int x = threadIdx.x; x < E; x += THREADS) {
+    ubase[x] = (counts[x] + NT_MAX - 1) / NT_MAX;
+    dbase[x] = (counts[x] + ND_MAX - 1) / ND_MAX;
+  }
+  __syncthreads();
+  if (warp == 0) warp_exclusive_scan(ubase, E, n_units);
+  if (warp == 1) warp_exclusive_scan(dbase, E, n_dunits);
+  __syncthreads();
+  for (int x = threadIdx.x; x < E; x += THREADS) {
+    const int c = counts[x];
+    for (int s = 0; s * NT_MAX < c; ++s) {
+      int32_t* u = units + (int64_t)(ubase[x] + s) * 4;
+      u[0] = x; u[1] = offsets[x] + s * NT_MAX; u[2] = min(NT_MAX, c - s * NT_MAX); u[3] = 0;
+    }
+    for (int s = 0; s * ND_MAX < c; ++s) {
+      int32_t* u = dunits + (int64_t)(dbase[x] + s) * 4;
+      u[0] = x; u[1] = offsets[x] + s * ND_MAX; u[2] = min(ND_MAX, c - s * ND_MAX);
+      u[3] = ubase[x] + (s * ND_MAX) / NT_MAX;
+    }
+  }
+}
+
 // Small T*K: every CTA routes all tokens itself (no barrier); CTA 0 also writes
 // the maps to global memory.
 __device__ void phase_route_small(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem) {
@@ -367,19 +404,8 @@ __device__ void phase_route_small(const EngineParams& p, const LayerPtrs& lp, ui
     tb.tokpos[pos] = pr / K;
     tb.wpos[pos] = tb.w[pr];
   }
-  int32_t* ubase = hist;
   __syncthreads();
-  for (int x = threadIdx.x; x < E; x += THREADS) ubase[x] = (tb.counts[x] + NT_MAX - 1) / NT_MAX;
-  __syncthreads();
-  if (warp == 0) warp_exclusive_scan(ubase, E, &tb.n_units);
-  __syncthreads();
-  for (int x = threadIdx.x; x < E; x += THREADS) {
-    const int c = tb.counts[x];
-    for (int s = 0; s * NT_MAX < c; ++s) {
-      int32_t* u = tb.units + (ubase[x] + s) * 4;
-      u[0] = x; u[1] = tb.offsets[x] + s * NT_MAX; u[2] = min(NT_MAX, c - s * NT_MAX); u[3] = 0;
-    }
-  }
+  build_units(tb.counts, tb.offsets, E, hist, tb.units, tb.dunits, &tb.n_units, &tb.n_dunits);
   __syncthreads();
   if (blockIdx.x == 0) {
     for (int i = threadIdx.x; i < TK; i += THREADS) {
@@ -413,21 +439,11 @@ __device__ void phase_permute_large(const EngineParams& p, uint8_t* smem) {
   if (warp == 0) warp_exclusive_scan(tb.offsets, E, tb.offsets + E);
   __syncthreads();
   if (blockIdx.x == 0) {
-    int32_t* ubase = reinterpret_cast<int32_t*>(ring_slot(smem, 0));
-    for (int x = threadIdx.x; x < E; x += THREADS) ubase[x] = (tb.counts[x] + NT_MAX - 1) / NT_MAX;
-    __syncthreads();
-    if (warp == 0) warp_exclusive_scan(ubase, E, &tb.n_units);
-    __syncthreads();
-    for (int x = threadIdx.x; x < E; x += THREADS) {
-      const int c = tb.counts[x];
-      for (int s = 0; s * NT_MAX < c; ++s) {
-        int32_t* u = p.units + (int64_t)(ubase[x] + s) * 4;
-        u[0] = x; u[1] = tb.offsets[x] + s * NT_MAX; u[2] = min(NT_MAX, c - s * NT_MAX); u[3] = 0;
-      }
-    }
+    int32_t* scratch = reinterpret_cast<int32_t*>(ring_slot(smem, 0));
+    build_units(tb.counts, tb.offsets, E, scratch, p.units, p.dunits, &tb.n_units, &tb.n_dunits);
     for (int i = threadIdx.x; i < E; i += THREADS) p.counts[i] = tb.counts[i];
     for (int i = threadIdx.x; i <= E; i += THREADS) p.offsets[i] = tb.offsets[i];
-    if (threadIdx.x == 0) *p.n_units = tb.n_units;
+    if (threadIdx.x == 0) { p.n_units[0] = tb.n_units; p.n_units[1] = tb.n_dunits; }
   }
   const int64_t wg = (int64_t)blockIdx.x * WARPS + warp, ws = (int64_t)gridDim.x * WARPS;
   for (int64_t x = wg; x < E; x += ws) {
@@ -457,13 +473,14 @@ __device__ __forceinline__ float e8m0_byte(uint32_t w) {
 }
 
 // One K chunk (4 MX blocks) of a 64-row job for this warp:
-//   acc[t][n][i] += sum over blocks b of 2^s(row, b) [* 2^q(col, b)] * (A_b B_b)
-// A = the chunk's E2M1 codes of tile t as f16 fragments, B = activation
-// fragments of n-tile n.  Gate/up: columns are tokens (x in f16, scaled per
-// token).  Down: columns are (pair, hi/lo) halves of the SwiGLU output, scaled
-// per (pair, block) by 2^q.
-template <int NTILE, bool ISD>
-__device__ __forceinline__ void chunk_mma(const uint8_t* st, int lane, int nt, float (&acc)[4][2][4]) {
+//   acc[t][i] += sum over blocks b of 2^s(row, b) [* 2^q(col, b)] * (A_b B_b)
+// A = the chunk's E2M1 codes of tile t as f16 fragments, B = the activation
+// fragments.  Gate/up: the 8 columns are tokens (x in f16, scaled per token).
+// Down: columns 2j, 2j+1 are the hi and lo f16 halves of pair j's SwiGLU
+// output, scaled per (pair, block) by 2^q.  Columns beyond nt read slot 0 and
+// are ignored.
+template <bool ISD>
+__device__ __forceinline__ void chunk_mma(const uint8_t* st, int lane, int nt, float (&acc)[4][4]) {
   const int g = lane >> 2, c = lane & 3;
   uint32_t sw0[4], sw1[4];
 #pragma unroll
@@ -472,78 +489,69 @@ __device__ __forceinline__ void chunk_mma(const uint8_t* st, int lane, int nt, f
     sw1[t] = *reinterpret_cast<const uint32_t*>(st + STAGE_CODE_BYTES + (t * 16 + g + 8) * KB);
   }
   const uint8_t* act = st + STAGE_W_BYTES;
-  const uint8_t* bptr[NTILE];
-  const int8_t* qptr[NTILE];
-#pragma unroll
-  for (int n = 0; n < NTILE; ++n) {
-    if (!ISD) {
-      const int jb = g < nt ? g : 0;
-      bptr[n] = act + jb * XH_SLOT + c * 16;
-      qptr[n] = nullptr;
-    } else {
-      int pj = n * 4 + (g >> 1);
-      pj = pj < nt ? pj : 0;
-      bptr[n] = act + pj * A16_CHUNK_BYTES + A16_HDR + (g & 1) * 64 + c * 16;
-      int qj = n * 4 + c;
-      qj = qj < nt ? qj : 0;
-      qptr[n] = reinterpret_cast<const int8_t*>(act + qj * A16_CHUNK_BYTES);
-    }
+  const uint8_t* bptr;
+  const int8_t* qptr = nullptr;
+  if (!ISD) {
+    const int jb = g < nt ? g : 0;
+    bptr = act + jb * XH_SLOT + c * 16;
+  } else {
+    const int pj = (g >> 1) < nt ? (g >> 1) : 0;
+    bptr = act + pj * A16_CHUNK_BYTES + A16_HDR + (g & 1) * 64 + c * 16;
+    qptr = reinterpret_cast<const int8_t*>(act + (c < nt ? c : 0) * A16_CHUNK_BYTES);
   }
 #pragma unroll
   for (int b = 0; b < KB; ++b) {
     const uint4 qa = *reinterpret_cast<const uint4*>(st + ((b * 2 + 0) * 32 + lane) * 16);
     const uint4 qb = *reinterpret_cast<const uint4*>(st + ((b * 2 + 1) * 32 + lane) * 16);
-    uint4 bf[NTILE];
-    float qf[NTILE];
-#pragma unroll
-    for (int n = 0; n < NTILE; ++n) {
-      bf[n] = *reinterpret_cast<const uint4*>(bptr[n] + b * (ISD ? 128 : 64));
-      qf[n] = ISD ? pow2f((int)qptr[n][b]) : 1.f;
-    }
+    const uint4 bf = *reinterpret_cast<const uint4*>(bptr + b * (ISD ? 128 : 64));
+    const float qf = ISD ? pow2f((int)qptr[b]) : 1.f;
     const uint32_t wd[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       uint32_t a0[4], a1[4];
       e2m1x8_to_f16x2x4(wd[2 * t], a0);
       e2m1x8_to_f16x2x4(wd[2 * t + 1], a1);
+      float ct[4] = {0.f, 0.f, 0.f, 0.f};
+      mma_f16_16816(ct, a0, bf.x, bf.y);
+      mma_f16_16816(ct, a1, bf.z, bf.w);
       float f0, f1;
       if (b == 0) { f0 = e8m0_byte<0>(sw0[t]); f1 = e8m0_byte<0>(sw1[t]); }
       else if (b == 1) { f0 = e8m0_byte<1>(sw0[t]); f1 = e8m0_byte<1>(sw1[t]); }
       else if (b == 2) { f0 = e8m0_byte<2>(sw0[t]); f1 = e8m0_byte<2>(sw1[t]); }
       else { f0 = e8m0_byte<3>(sw0[t]); f1 = e8m0_byte<3>(sw1[t]); }
-#pragma unroll
-      for (int n = 0; n < NTILE; ++n) {
-        float ct[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_f16_16816(ct, a0, bf[n].x, bf[n].y);
-        mma_f16_16816(ct, a1, bf[n].z, bf[n].w);
-        const float g0 = ISD ? f0 * qf[n] : f0, g1 = ISD ? f1 * qf[n] : f1;
-        acc[t][n][0] = fmaf(ct[0], g0, acc[t][n][0]);
-        acc[t][n][1] = fmaf(ct[1], g0, acc[t][n][1]);
-        acc[t][n][2] = fmaf(ct[2], g1, acc[t][n][2]);
-        acc[t][n][3] = fmaf(ct[3], g1, acc[t][n][3]);
-      }
+      if (ISD) { f0 *= qf; f1 *= qf; }
+      acc[t][0] = fmaf(ct[0], f0, acc[t][0]);
+      acc[t][1] = fmaf(ct[1], f0, acc[t][1]);
+      acc[t][2] = fmaf(ct[2], f1, acc[t][2]);
+      acc[t][3] = fmaf(ct[3], f1, acc[t][3]);
     }
   }
 }
 
 struct StreamCtx {
-  const int32_t* units;
+  const int32_t* units;   // gate/up units
+  const int32_t* dunits;  // down units
   const int32_t* tokpos;
   const float* wpos;
-  int n_units;
+  int n_units, n_dunits;
 };
 
-// Producer warp: jobs -> queue entries -> stages into the ring.
+// Producer warp: jobs -> queue entries -> stages into the ring.  Gate/up jobs
+// (unit, 32-row block of I) come first in unit order, then down jobs (down
+// unit, 64-row block of H); a down job waits until its gate/up unit's
+// SwiGLU output is complete.
 __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem,
                                 const StreamCtx& cx, uint32_t& seq, int32_t& qk) {
   const int lane = threadIdx.x & 31;
   JobEntry* jq = job_queue(smem);
   uint32_t* ready = p.sync + SY_READY;
   const int gub = p.I / (STAGE_ROWS / 2), db = p.H / STAGE_ROWS;
-  const int64_t n_gu = (int64_t)cx.n_units * gub, n_all = n_gu + (int64_t)cx.n_units * db;
+  const int64_t n_gu = (int64_t)cx.n_units * gub, n_all = n_gu + (int64_t)cx.n_dunits * db;
   const int nc_gu = p.H / KC, nc_d = p.I / KC;
   const uint32_t seq_start = seq;
   bool ok = true;
+  unsigned long long t_empty = 0, t_ready = 0;
+  const unsigned long long t_begin = clock64();
   fence_proxy_async_global();
   long long next = 0;
   if (lane == 0) next = atomicAdd(p.sync + SY_JOBS, 1u);
@@ -564,7 +572,7 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
     const int64_t jj = isD ? j - n_gu : j;
     const int per = isD ? db : gub;
     const int u = (int)(jj / per), rb = (int)(jj % per);
-    const int4 ur = *reinterpret_cast<const int4*>(cx.units + (int64_t)u * 4);
+    const int4 ur = *reinterpret_cast<const int4*>((isD ? cx.dunits : cx.units) + (int64_t)u * 4);
     const int e = ur.x, pos0 = ur.y, nt = ur.z;
     const int nc = isD ? nc_d : nc_gu;
     if (lane == 0) {
@@ -575,20 +583,23 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
       *reinterpret_cast<volatile int32_t*>(&en->flag) = qk + 1;
     }
     ++qk;
-    if (isD) {  // the down stages read this unit's SwiGLU output: wait for its gate/up jobs
-      const uint32_t need = (uint32_t)(gub * nt);
-      if (ld_acquire_u32(ready + u) < need) {
+    if (isD) {  // the down stages read the SwiGLU output: wait for the gate/up unit
+      const int gu = ur.w;
+      const uint32_t need = (uint32_t)gub * (uint32_t)cx.units[(int64_t)gu * 4 + 2];
+      const unsigned long long tr0 = clock64();
+      if (ld_acquire_u32(ready + gu) < need) {
         const uint64_t t0 = globaltimer_ns();
         uint32_t spins = 0;
-        while (ld_acquire_u32(ready + u) < need) {
+        while (ld_acquire_u32(ready + gu) < need) {
           if ((++spins & 15u) == 0u) {
             if (error_set(p.sync)) { ok = false; break; }
-            if (globaltimer_ns() - t0 > p.timeout_ns) { set_error(p.sync, DEV_TIMEOUT_READY, u); ok = false; break; }
+            if (globaltimer_ns() - t0 > p.timeout_ns) { set_error(p.sync, DEV_TIMEOUT_READY, gu); ok = false; break; }
           }
           __nanosleep(100);
         }
       }
       fence_proxy_async_global();
+      t_ready += clock64() - tr0;
     }
     int tok = 0;
     if (!isD && lane < nt) tok = cx.tokpos[pos0 + lane];
@@ -597,12 +608,14 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
     const uint32_t bytes = STAGE_W_BYTES + nt * (isD ? A16_CHUNK_BYTES : XH_CHUNK_BYTES);
     for (int c = 0; c < nc && ok; ++c) {
       const int slot = (int)(seq % NSLOT);
+      const unsigned long long te0 = clock64();
       if (seq >= (uint32_t)NSLOT &&
           !wait_mbar(empty_bar(smem, slot), ((seq / NSLOT) + 1) & 1u, p.sync, p.timeout_ns,
                      DEV_TIMEOUT_PIPE, seq)) {
         ok = false;
         break;
       }
+      t_empty += clock64() - te0;
       uint8_t* dst = ring_slot(smem, slot);
       uint64_t* fb = full_bar(smem, slot);
       if (lane == 0) {
@@ -618,6 +631,12 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
                  XH_CHUNK_BYTES, fb);
       ++seq;
     }
+  }
+  if (p.prof && lane == 0) {
+    atomicAdd(p.prof + PF_PROD_EMPTY, t_empty);
+    atomicAdd(p.prof + PF_PROD_READY, t_ready);
+    atomicAdd(p.prof + PF_PROD_TOTAL, clock64() - t_begin);
+    atomicAdd(p.prof + PF_STAGES, (unsigned long long)(seq - seq_start));
   }
   // let every issued copy land before the ring is reused or the CTA exits
   const uint32_t issued = seq - seq_start;
@@ -638,8 +657,11 @@ __device__ void stream_consumer(const EngineParams& p, uint8_t* smem, const Stre
   JobEntry* jq = job_queue(smem);
   uint32_t* ready = p.sync + SY_READY;
   bool poison = false;
+  unsigned long long t_full = 0, t_mma = 0, t_bar = 0, t_epi = 0, t_queue = 0, n_jobs = 0;
+  const unsigned long long t_begin = clock64();
   for (;;) {
     JobEntry* en = jq + (qk % JQ);
+    const unsigned long long tq0 = clock64();
     // the producer publishes the entry (bounded wait; the producer's own waits
     // are bounded by the same timeout, after which it publishes an end entry)
     if (*reinterpret_cast<volatile int32_t*>(&en->flag) != qk + 1) {
@@ -650,53 +672,53 @@ __device__ void stream_consumer(const EngineParams& p, uint8_t* smem, const Stre
       }
     }
     const int job = *reinterpret_cast<volatile int32_t*>(&en->job);
+    t_queue += clock64() - tq0;
     if (job < 0) { ++qk; break; }
+    ++n_jobs;
     const int s0 = en->s0, nc = en->nc, u = en->unit, rb = en->rb, isD = en->isD;
     const int pos0 = en->pos0, nt = en->nt;
     const int buf = qk & 1;
-    float acc[4][2][4];
+    float acc[4][4];
 #pragma unroll
     for (int t = 0; t < 4; ++t)
 #pragma unroll
-      for (int n = 0; n < 2; ++n)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[t][n][i] = 0.f;
+      for (int i = 0; i < 4; ++i) acc[t][i] = 0.f;
     for (int cc = w; cc < nc; cc += NCW) {
       const uint32_t s = (uint32_t)s0 + cc;
       const int slot = (int)(s % NSLOT);
+      const unsigned long long tf0 = clock64();
       if (!poison &&
           !wait_mbar(full_bar(smem, slot), (s / NSLOT) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, s))
         poison = true;
+      const unsigned long long tm0 = clock64();
+      t_full += tm0 - tf0;
       if (!poison) {
         const uint8_t* st = ring_slot(smem, slot);
-        if (!isD) chunk_mma<1, false>(st, lane, nt, acc);
-        else if (nt <= 4) chunk_mma<1, true>(st, lane, nt, acc);
-        else chunk_mma<2, true>(st, lane, nt, acc);
+        if (!isD) chunk_mma<false>(st, lane, nt, acc);
+        else chunk_mma<true>(st, lane, nt, acc);
       }
+      t_mma += clock64() - tm0;
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar(smem, slot));
     }
     // deposit this warp's partial sums: part[w][col][row]
     float* pb = part_buf(smem, buf) + (size_t)w * PART_COLS * PART_LD;
     if (w < nc) {
-      const int ntile = isD && nt > 4 ? 2 : 1;
 #pragma unroll
       for (int t = 0; t < 4; ++t)
 #pragma unroll
-        for (int n = 0; n < 2; ++n) {
-          if (n < ntile) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              pb[(n * 8 + 2 * c + (i & 1)) * PART_LD + t * 16 + g + (i >> 1) * 8] = acc[t][n][i];
-          }
-        }
+        for (int i = 0; i < 4; ++i) pb[(2 * c + (i & 1)) * PART_LD + t * 16 + g + (i >> 1) * 8] = acc[t][i];
     }
+    const unsigned long long tb0 = clock64();
     named_barrier(1 + buf, NCW * 32);
+    const unsigned long long te0 = clock64();
+    t_bar += te0 - tb0;
     const int nw = nc < NCW ? nc : NCW;
     const float* pall = part_buf(smem, buf);
-    if (!poison && w < nt) {
-      if (!isD) {  // gate/up epilogue: token column w, lane = intermediate row i0 + lane
-        const int j = w;
+    // the epilogue of column j runs on warp (j + qk) % NCW: the duty rotates
+    const int j = (w + NCW - (qk % NCW)) % NCW;
+    if (!poison && j < nt) {
+      if (!isD) {  // gate/up epilogue: token column j, lane = intermediate row i0 + lane
         const float px = p.pxf[cx.tokpos[pos0 + j]];
         float gs = 0.f, us = 0.f;
         for (int ww = 0; ww < nw; ++ww) {
@@ -723,12 +745,12 @@ __device__ void stream_consumer(const EngineParams& p, uint8_t* smem, const Stre
         *reinterpret_cast<__half*>(base + off) = hi;
         *reinterpret_cast<__half*>(base + off + 64) = lo;
         if (lane == 0) base[bi] = (uint8_t)(int8_t)q;
-        __threadfence();
         __syncwarp();
-        if (lane == 0) red_release_add_u32(ready + u, 1u);
-      } else {  // down epilogue: pair w, lane = rows h0 + lane and h0 + 32 + lane
-        const int j = w;
-        const int col = (j >> 2) * 8 + 2 * (j & 3);
+        if (lane == 0) {
+          __threadfence();
+          red_release_add_u32(ready + u, 1u);
+        }
+      } else {  // down epilogue: pair j, lane = rows h0 + lane and h0 + 32 + lane
         const float wp = cx.wpos[pos0 + j];
         const int h0 = rb * STAGE_ROWS;
 #pragma unroll
@@ -737,13 +759,23 @@ __device__ void stream_consumer(const EngineParams& p, uint8_t* smem, const Stre
           float y = 0.f;
           for (int ww = 0; ww < nw; ++ww) {
             const float* pw = pall + (size_t)ww * PART_COLS * PART_LD;
-            y += pw[col * PART_LD + r] + pw[(col + 1) * PART_LD + r];
+            y += pw[(2 * j) * PART_LD + r] + pw[(2 * j + 1) * PART_LD + r];
           }
           p.ypair[(int64_t)(pos0 + j) * p.H + h0 + r] = y * wp;
         }
       }
     }
+    t_epi += clock64() - te0;
     ++qk;
+  }
+  if (p.prof && lane == 0) {
+    atomicAdd(p.prof + PF_CONS_FULL, t_full);
+    atomicAdd(p.prof + PF_CONS_MMA, t_mma);
+    atomicAdd(p.prof + PF_CONS_BAR, t_bar);
+    atomicAdd(p.prof + PF_CONS_EPI, t_epi);
+    atomicAdd(p.prof + PF_CONS_QUEUE, t_queue);
+    atomicAdd(p.prof + PF_CONS_TOTAL, clock64() - t_begin);
+    atomicAdd(p.prof + PF_JOBS, n_jobs);
   }
 }
 
@@ -849,7 +881,7 @@ __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p
     const int32_t* inv;
     if (small) {
       phase_route_small(p, lp, smem);
-      cx = StreamCtx{tb.units, tb.tokpos, tb.wpos, tb.n_units};
+      cx = StreamCtx{tb.units, tb.dunits, tb.tokpos, tb.wpos, tb.n_units, tb.n_dunits};
       inv = tb.inv;
       if (p.route_only) return;
     } else {
@@ -858,7 +890,7 @@ __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p
       phase_permute_large(p, smem);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 3)) return;
       if (p.route_only) return;
-      cx = StreamCtx{p.units, p.tokpos, p.wpos, *p.n_units};
+      cx = StreamCtx{p.units, p.dunits, p.tokpos, p.wpos, p.n_units[0], p.n_units[1]};
       inv = p.inv;
     }
     if (st) st[1] = globaltimer_ns();

@@ -19,13 +19,16 @@ constexpr int KB = KC / 32;                              // MX blocks per stage
 constexpr int STAGE_ROWS = 64;                           // weight rows per stage
 constexpr int STAGE_CODE_BYTES = STAGE_ROWS * KC / 2;    // 4096
 constexpr int STAGE_W_BYTES = STAGE_CODE_BYTES + STAGE_ROWS * KB;  // 4352
-constexpr int NT_MAX = 8;                                // tokens per unit (one MMA n-tile)
+constexpr int NT_MAX = 8;                                // tokens per gate/up unit (one MMA n-tile)
+constexpr int ND_MAX = 4;                                // pairs per down unit (hi+lo: one n-tile)
 // activations of one stage, per token (gate/up) or per (token, expert) pair (down)
 constexpr int XH_CHUNK_BYTES = KC * 2;                   // f16 x, fragment order
 constexpr int XH_SLOT = XH_CHUNK_BYTES + 64;             // padded: conflict-free fragment loads
 constexpr int A16_HDR = 16;                              // 4 block exponents q, padded
 constexpr int A16_CHUNK_BYTES = A16_HDR + KC * 2 * 2;    // hi and lo f16 halves: 528
-constexpr int SLOT_BYTES = STAGE_W_BYTES + NT_MAX * A16_CHUNK_BYTES;  // 8576
+constexpr int SLOT_ACT_BYTES = NT_MAX * XH_SLOT > ND_MAX * A16_CHUNK_BYTES ? NT_MAX * XH_SLOT
+                                                                          : ND_MAX * A16_CHUNK_BYTES;
+constexpr int SLOT_BYTES = STAGE_W_BYTES + SLOT_ACT_BYTES;  // 6912
 constexpr int MAX_HSPLIT = 8;                            // router dot products split along H
 
 constexpr int MAX_LAYERS = 16;
@@ -33,10 +36,10 @@ constexpr int MAX_EXPERTS = 512;
 constexpr int NCW = 8;                                   // consumer (MMA) warps per CTA
 constexpr int WARPS = NCW + 1;                           // + one producer warp
 constexpr int THREADS = WARPS * 32;
-constexpr int NSLOT = 15;                                // stage ring slots per CTA
+constexpr int NSLOT = 25;                                // stage ring slots per CTA
 constexpr int JQ = 32;                                   // job queue entries per CTA
 constexpr int PART_LD = 68;                              // partial-sum column stride (floats)
-constexpr int PART_COLS = 16;                            // up to two n-tiles
+constexpr int PART_COLS = 8;                             // one n-tile
 constexpr int SMALL_PAIRS = 256;                         // T*k up to this: routing done per CTA
 constexpr int STAMPS_PER_LAYER = 4;                      // prepared, routed, streamed, combined
 
@@ -50,6 +53,10 @@ enum : uint32_t {
   DEV_OK = 0, DEV_TIMEOUT_BARRIER = 1, DEV_TIMEOUT_PIPE = 2, DEV_TIMEOUT_READY = 3,
   DEV_TIMEOUT_QUEUE = 4,
 };
+
+// Upper bounds of the unit tables for T*K pairs over E experts.
+__host__ __device__ inline int max_units(int E, int64_t TK) { return (int)((E < TK ? E : TK) + TK / NT_MAX + 1); }
+__host__ __device__ inline int max_dunits(int E, int64_t TK) { return (int)((E < TK ? E : TK) + TK / ND_MAX + 1); }
 
 // Router split of H: about 1024 elements per part, each part a multiple of KC.
 inline int router_hsplit(int H) {
@@ -87,12 +94,21 @@ struct EngineParams {
   int32_t* inv;               // [TK]
   int32_t* tokpos;            // [TK] token of each permuted position
   float* wpos;                // [TK] routing weight of each permuted position
-  int32_t* units;             // [Umax][4] (expert, pos0, nt, 0)
-  int32_t* n_units;           // [1]
+  int32_t* units;             // [Umax][4] gate/up units (expert, pos0, nt <= 8, 0)
+  int32_t* dunits;            // [Dmax][4] down units (expert, pos0, nt <= 4, gate/up unit)
+  int32_t* n_units;           // [2] gate/up units, down units
   uint8_t* a16;               // [I/KC][TK][A16_CHUNK_BYTES]  SwiGLU output, hi/lo f16
   float* ypair;               // [TK][H]
   uint32_t* sync;             // see SY_*
   uint64_t* stamps;           // null or [1 + MAX_LAYERS * STAMPS_PER_LAYER] %globaltimer ns (CTA 0)
+  unsigned long long* prof;   // null or [PROF_COUNTERS] summed SM-clock cycles (stream phase)
+};
+
+// stream-phase profile counters (cycles summed over CTAs / warps)
+enum : int {
+  PF_PROD_EMPTY = 0, PF_PROD_READY, PF_PROD_TOTAL, PF_STAGES,
+  PF_CONS_FULL, PF_CONS_MMA, PF_CONS_BAR, PF_CONS_EPI, PF_CONS_QUEUE, PF_CONS_TOTAL, PF_JOBS,
+  PROF_COUNTERS
 };
 
 size_t engine_smem_bytes();

@@ -28,10 +28,12 @@ struct moe_mxfp4 {
   uint8_t* a16 = nullptr;
   __nv_bfloat16* xnext = nullptr;
   int32_t *idx = nullptr, *counts = nullptr, *offsets = nullptr, *perm = nullptr, *inv = nullptr,
-          *tokpos = nullptr, *units = nullptr, *n_units = nullptr;
+          *tokpos = nullptr, *units = nullptr, *dunits = nullptr, *n_units = nullptr;
   float *wts = nullptr, *wpos = nullptr, *ypair = nullptr;
   uint32_t* sync = nullptr;
   uint64_t* stamps = nullptr;
+  unsigned long long* prof = nullptr;
+  bool profiling = false;
   __nv_bfloat16 *x_stage = nullptr, *y_stage = nullptr;
   std::vector<void*> allocs;
 };
@@ -86,9 +88,11 @@ EngineParams base_params(const moe_mxfp4* h, int T) {
   p.logits = h->logits; p.xh = h->xh; p.pxf = h->pxf; p.xnext = h->xnext;
   p.idx = h->idx; p.wts = h->wts; p.counts = h->counts; p.offsets = h->offsets;
   p.perm = h->perm; p.inv = h->inv; p.tokpos = h->tokpos; p.wpos = h->wpos;
-  p.units = h->units; p.n_units = h->n_units; p.a16 = h->a16; p.ypair = h->ypair;
+  p.units = h->units; p.dunits = h->dunits; p.n_units = h->n_units; p.a16 = h->a16;
+  p.ypair = h->ypair;
   p.sync = h->sync;
   p.stamps = h->stamps;
+  p.prof = h->profiling ? h->prof : nullptr;
   return p;
 }
 
@@ -164,7 +168,8 @@ int32_t moe_mxfp4_create(const moe_config_t* cfg, const uint8_t* const* gate_cod
 
   const int H = cfg->hidden, I = cfg->inter, E = cfg->num_experts, K = cfg->top_k;
   const int64_t Tm = cfg->max_tokens, TKm = Tm * K;
-  h->umax = (int)((E < TKm ? E : TKm) + TKm / NT_MAX + 1);
+  h->umax = max_units(E, TKm);
+  const int dmax = max_dunits(E, TKm);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   bool ok = true;
   for (int l = 0; l < L && ok; ++l) {
@@ -180,11 +185,13 @@ int32_t moe_mxfp4_create(const moe_config_t* cfg, const uint8_t* const* gate_cod
        dalloc(h, &h->offsets, (size_t)(E + 1) * 4) && dalloc(h, &h->perm, (size_t)TKm * 4) &&
        dalloc(h, &h->inv, (size_t)TKm * 4) && dalloc(h, &h->tokpos, (size_t)TKm * 4) &&
        dalloc(h, &h->wpos, (size_t)TKm * 4) && dalloc(h, &h->units, (size_t)h->umax * 16) &&
+       dalloc(h, &h->dunits, (size_t)dmax * 16) &&
        dalloc(h, &h->n_units, 16) &&
        dalloc(h, &h->a16, (size_t)(I / KC) * TKm * A16_CHUNK_BYTES) &&
        dalloc(h, &h->ypair, (size_t)TKm * H * 4) &&
        dalloc(h, &h->sync, (size_t)(SY_READY + h->umax) * 4) &&
        dalloc(h, &h->stamps, (size_t)(1 + MAX_LAYERS * STAMPS_PER_LAYER) * 8) &&
+       dalloc(h, &h->prof, (size_t)PROF_COUNTERS * 8) &&
        dalloc(h, &h->x_stage, (size_t)Tm * H * 2) && dalloc(h, &h->y_stage, (size_t)Tm * H * 2);
   if (!ok) { free_all(h); delete h; cudaGetLastError(); return MOE_ERR_OOM; }
 
@@ -279,6 +286,21 @@ int32_t moe_phase_ns(moe_mxfp4_t* h, uint64_t* ns_out, int32_t max_n, void* stre
       cudaMemcpy(raw, h->stamps, (size_t)(1 + n) * 8, cudaMemcpyDeviceToHost) != cudaSuccess)
     return MOE_ERR_CUDA;
   for (int i = 0; i < n && i < max_n; ++i) ns_out[i] = raw[i + 1] - raw[i];
+  return MOE_OK;
+}
+
+int32_t moe_stream_profile(moe_mxfp4_t* h, int32_t enable, uint64_t* out, int32_t max_n,
+                           void* stream) {
+  if (!h || max_n < 0 || (max_n > 0 && !out)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (max_n > 0) {
+    uint64_t raw[PROF_COUNTERS];
+    if (cudaMemcpy(raw, h->prof, sizeof(raw), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    for (int i = 0; i < PROF_COUNTERS && i < max_n; ++i) out[i] = raw[i];
+  }
+  if (cudaMemset(h->prof, 0, (size_t)PROF_COUNTERS * 8) != cudaSuccess) return MOE_ERR_CUDA;
+  h->profiling = enable != 0;
   return MOE_OK;
 }
 

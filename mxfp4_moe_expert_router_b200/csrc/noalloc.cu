@@ -37,7 +37,7 @@ int g_grid[kMaxDevices] = {};
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Layout {
-  size_t logits, xh, pxf, units, n_units, tokpos, wpos, sync, total;
+  size_t logits, xh, pxf, units, dunits, n_units, tokpos, wpos, sync, total;
   int umax;
 };
 
@@ -45,13 +45,14 @@ struct Layout {
 Layout layout_for(int T, int H, int E, int K) {
   Layout l{};
   const int64_t TK = (int64_t)T * K;
-  l.umax = (int)((E < TK ? E : TK) + TK / NT_MAX + 1);
+  l.umax = max_units(E, TK);
   size_t o = 0;
   l.sync = o;    o = align256(o + (size_t)(SY_READY + l.umax) * 4);
   l.logits = o;  o = align256(o + (size_t)router_hsplit(H) * T * E * 8);
   l.xh = o;      o = align256(o + (size_t)T * H * 2);
   l.pxf = o;     o = align256(o + (size_t)T * 4);
   l.units = o;   o = align256(o + (size_t)l.umax * 16);
+  l.dunits = o;  o = align256(o + (size_t)max_dunits(E, TK) * 16);
   l.n_units = o; o = align256(o + 16);
   l.tokpos = o;  o = align256(o + (size_t)TK * 4);
   l.wpos = o;    o = align256(o + (size_t)TK * 4);
@@ -130,6 +131,7 @@ extern "C" MOE_API int32_t moe_route_static(const void* x_bf16, int32_t T, int32
   p.xh = s + lay.xh;
   p.pxf = reinterpret_cast<float*>(s + lay.pxf);
   p.units = reinterpret_cast<int32_t*>(s + lay.units);
+  p.dunits = reinterpret_cast<int32_t*>(s + lay.dunits);
   p.n_units = reinterpret_cast<int32_t*>(s + lay.n_units);
   p.tokpos = reinterpret_cast<int32_t*>(s + lay.tokpos);
   p.wpos = reinterpret_cast<float*>(s + lay.wpos);
