@@ -363,7 +363,8 @@ def main():
                          "traffic": traffic, "kernel": "engine_kernel"},
             "gpu_launches": args.steps,
             "phase_us_last_step": {k: round(v / 1e3, 2) for k, v in
-                                   zip(("prepare", "route", "stream", "combine"), phases[:4])},
+                                   zip(("convert_x", "router_logits", "grid_wait", "topk", "permute", "stream",
+                                       "combine"), phases[:7])},
             "e2e": e2e,
             "cpu_baseline": cpu,
             "clocks": clk,

@@ -175,8 +175,9 @@ class Moe:
         _check(lib.moe_status(self.handle, _stream(stream)), "moe_status")
 
     def moe_phase_ns(self, stream=None):
-        """Durations (ns) of the last forward's phases: 4 per layer (prepare, route, stream, combine)."""
-        n = self.cfg.num_layers * 4
+        """Durations (ns) of the last forward's phases, 7 per layer: x conversion and
+        router logits (CTA 0), grid wait, top-k, permute, stream, combine."""
+        n = self.cfg.num_layers * 7
         arr = (ctypes.c_uint64 * n)()
         _check(lib.moe_phase_ns(self.handle, arr, n, _stream(stream)), "moe_phase_ns")
         return [int(v) for v in arr]

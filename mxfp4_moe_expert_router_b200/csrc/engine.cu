@@ -59,6 +59,7 @@ struct alignas(16) CtaTables {
   int32_t inv[SMALL_PAIRS];
   int32_t tokpos[SMALL_PAIRS];
   float wpos[SMALL_PAIRS];
+  float pxf[SMALL_PAIRS];
   int32_t counts[MAX_EXPERTS];
   int32_t offsets[MAX_EXPERTS + 1];
   float red[WARPS];
@@ -135,6 +136,8 @@ __device__ bool wait_mbar(uint64_t* bar, uint32_t parity, uint32_t* sync, uint64
   return true;
 }
 
+__device__ __forceinline__ unsigned long long pclock(bool on) { return on ? clock64() : 0ull; }
+
 __device__ __forceinline__ float pow2f(int e) {  // 2^e for e in [-126, 127]
   return __uint_as_float((uint32_t)(e + 127) << 23);
 }
@@ -144,16 +147,18 @@ __device__ __forceinline__ float pow2f(int e) {  // 2^e for e in [-126, 127]
 // every bf16 value is exact in f16 unless it is below max|x| * 2^-28.  The
 // 32-element blocks are stored in the mma B-fragment order (see chunk_mma).
 __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const __nv_bfloat16* x,
-                              int layer) {
+                              int layer, uint8_t* smem, uint64_t* stamp) {
   const int T = p.T, H = p.H, E = p.E;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t gt = (int64_t)blockIdx.x * THREADS + threadIdx.x;
   const int64_t gs = (int64_t)gridDim.x * THREADS;
   const int64_t wg = (int64_t)blockIdx.x * WARPS + warp, ws = (int64_t)gridDim.x * WARPS;
-  for (int64_t t = wg; t < T; t += ws) {
+  // one CTA per token: CTA-wide max, then every thread converts whole blocks
+  float* red = tables(smem).red;
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
     const __nv_bfloat16* xr = x + t * H;
     float m = 0.f;
-    for (int h = lane * 8; h < H; h += 256) {
+    for (int h = threadIdx.x * 8; h < H; h += THREADS * 8) {
       const uint4 v = *reinterpret_cast<const uint4*>(xr + h);
       const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -164,12 +169,17 @@ __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const 
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+    __syncthreads();
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+#pragma unroll
+    for (int w2 = 0; w2 < WARPS; ++w2) m = fmaxf(m, red[w2]);
     const int eb = (int)((__float_as_uint(m) >> 23) & 0xFF);
     int px = m > 0.f ? eb - 127 - 14 : 0;
     px = max(px, -126);
     const float inv = pow2f(-px);
-    if (lane == 0) p.pxf[t] = pow2f(px);
-    for (int b = lane; b < H / 32; b += 32) {
+    if (threadIdx.x == 0) p.pxf[t] = pow2f(px);
+    for (int b = threadIdx.x; b < H / 32; b += THREADS) {
       const uint4* src = reinterpret_cast<const uint4*>(xr + b * 32);
       float v[32];
 #pragma unroll
@@ -194,6 +204,7 @@ __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const 
       }
     }
   }
+  if (stamp) stamp[0] = globaltimer_ns();
   if (p.layer_io) {
     const int64_t n8 = (int64_t)T * H / 8;
     const uint4* s8 = reinterpret_cast<const uint4*>(x);
@@ -206,7 +217,17 @@ __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const 
   for (int64_t u = gt; u < umax; u += gs) p.sync[SY_READY + u] = 0u;
 
   // partial logits[hs][t][e] = sum over the hs-th H part of x[t][h] * Wr[e][h];
-  // bf16 * fp32 products are exact in fp64 and the sums are fp64
+  // bf16 * fp32 products are exact in fp64 and the sums are fp64.  A token
+  // block that fits in the (idle) stage ring is staged there first, so that
+  // only the router weights come from L2.
+  const __nv_bfloat16* xr = x;
+  if ((int64_t)T * H * 2 <= (int64_t)NSLOT * SLOT_BYTES) {
+    uint4* d = reinterpret_cast<uint4*>(ring_slot(smem, 0));
+    const uint4* s8 = reinterpret_cast<const uint4*>(x);
+    for (int64_t i = threadIdx.x; i < (int64_t)T * H / 8; i += THREADS) d[i] = s8[i];
+    __syncthreads();
+    xr = reinterpret_cast<const __nv_bfloat16*>(ring_slot(smem, 0));
+  }
   const int HS = p.HS, hpart = H / HS;
   const int nchunk = (T + 7) / 8;
   const int64_t njobs = (int64_t)E * HS * nchunk;
@@ -219,13 +240,13 @@ __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const 
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[j] = 0.0;
     const float4* wr = reinterpret_cast<const float4*>(lp.router_w + (int64_t)e * H + hs * hpart);
-#pragma unroll 4
+#pragma unroll 8
     for (int h4 = lane; h4 < hpart / 4; h4 += 32) {
       const float4 w4 = __ldg(wr + h4);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         if (j < nt) {
-          const uint2 xb = *reinterpret_cast<const uint2*>(x + (int64_t)(t0 + j) * H + hs * hpart + h4 * 4);
+          const uint2 xb = *reinterpret_cast<const uint2*>(xr + (int64_t)(t0 + j) * H + hs * hpart + h4 * 4);
           acc[j] = fma((double)__uint_as_float(xb.x << 16), (double)w4.x, acc[j]);
           acc[j] = fma((double)__uint_as_float(xb.x & 0xFFFF0000u), (double)w4.y, acc[j]);
           acc[j] = fma((double)__uint_as_float(xb.y << 16), (double)w4.z, acc[j]);
@@ -244,6 +265,7 @@ __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const 
         if (j < nt) p.logits[((int64_t)hs * T + t0 + j) * E + e] = acc[j];
     }
   }
+  if (stamp) stamp[1] = globaltimer_ns();
 }
 
 // ---- phase B: top-k, weights, permutation ------------------------------------------------
@@ -258,16 +280,21 @@ __device__ __forceinline__ double key_value(uint64_t k) {
 
 // One warp: logits of token t (partials summed in order, plus bias), the K
 // largest (descending, ties to the lower expert), weights exp(l - lmax) / sum
-// over the K.  Lane r < K writes slot r.
-__device__ void topk_row(const EngineParams& p, const float* bias, int t, int32_t* out_idx,
-                         float* out_w) {
+// over the K.  Lane r < K writes slot r.  Each lane holds experts lane + 32 i
+// (i < PER) as order-preserving 64-bit keys, sorts them once (descending, the
+// lower expert first on equal keys), and each of the K rounds takes the
+// warp-wide maximum of the lanes' heads; the winning lane drops its head.
+template <int PER>
+__device__ void topk_row_n(const EngineParams& p, const float* bias, int t, int32_t* out_idx,
+                           float* out_w) {
   const int lane = threadIdx.x & 31;
   const int E = p.E, K = p.K;
-  constexpr int PER = MAX_EXPERTS / 32;
   uint64_t key[PER];
+  int ix[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int e = lane + 32 * i;
+    ix[i] = i;
     if (e < E) {
       double part[MAX_HSPLIT];
 #pragma unroll
@@ -282,23 +309,33 @@ __device__ void topk_row(const EngineParams& p, const float* bias, int t, int32_
       key[i] = 0ull;
     }
   }
-  uint32_t taken = 0;
+  // odd-even transposition sort, descending; on equal keys the lower index first
+#pragma unroll
+  for (int r = 0; r < PER; ++r) {
+#pragma unroll
+    for (int i = r & 1; i + 1 < PER; i += 2) {
+      const bool sw = key[i + 1] > key[i] || (key[i + 1] == key[i] && ix[i + 1] < ix[i]);
+      const uint64_t k0 = key[i], k1 = key[i + 1];
+      const int i0 = ix[i], i1 = ix[i + 1];
+      key[i] = sw ? k1 : k0; key[i + 1] = sw ? k0 : k1;
+      ix[i] = sw ? i1 : i0; ix[i + 1] = sw ? i0 : i1;
+    }
+  }
   int my_e = -1;
   double my_l = 0.0, lmax = 0.0;
   for (int r = 0; r < K; ++r) {
-    uint64_t best = 0;
-    int bi = -1;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u) && (bi < 0 || key[i] > best)) { best = key[i]; bi = i; }
-    }
-    const uint32_t hi = __reduce_max_sync(FULL, bi >= 0 ? (uint32_t)(best >> 32) : 0u);
-    const uint32_t lo = __reduce_max_sync(FULL, (bi >= 0 && (uint32_t)(best >> 32) == hi) ? (uint32_t)best : 0u);
+    const uint64_t best = key[0];
+    const uint32_t hi = __reduce_max_sync(FULL, (uint32_t)(best >> 32));
+    const uint32_t lo = __reduce_max_sync(FULL, (uint32_t)(best >> 32) == hi ? (uint32_t)best : 0u);
     const uint64_t top = ((uint64_t)hi << 32) | lo;
-    const uint32_t m = __reduce_max_sync(FULL, (bi >= 0 && best == top) ? (65536u - (uint32_t)(lane + 32 * bi)) : 0u);
+    const int ehead = lane + 32 * ix[0];
+    const uint32_t m = __reduce_max_sync(FULL, best == top ? (65536u - (uint32_t)ehead) : 0u);
     const int esel = (int)(65536u - m);
-    if ((esel & 31) == lane) taken |= 1u << (esel >> 5);
+    if (esel == ehead) {  // the winning lane drops its head
+#pragma unroll
+      for (int i = 0; i + 1 < PER; ++i) { key[i] = key[i + 1]; ix[i] = ix[i + 1]; }
+      key[PER - 1] = 0ull;
+    }
     const double v = key_value(top);
     if (r == 0) lmax = v;
     if (lane == r) { my_e = esel; my_l = v; }
@@ -308,6 +345,13 @@ __device__ void topk_row(const EngineParams& p, const float* bias, int t, int32_
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(FULL, sum, o);
   if (lane < K) { out_idx[lane] = my_e; out_w[lane] = (float)(ex / sum); }
+}
+
+__device__ __forceinline__ void topk_row(const EngineParams& p, const float* bias, int t,
+                                         int32_t* out_idx, float* out_w) {
+  if (p.E <= 128) topk_row_n<4>(p, bias, t, out_idx, out_w);
+  else if (p.E <= 256) topk_row_n<8>(p, bias, t, out_idx, out_w);
+  else topk_row_n<16>(p, bias, t, out_idx, out_w);
 }
 
 // Exclusive scan of n <= 512 ints in shared memory by one warp (in place);
@@ -371,11 +415,14 @@ __device__ void build_units(const int32_t* counts, const int32_t* offsets, int E
 
 // Small T*K: every CTA routes all tokens itself (no barrier); CTA 0 also writes
 // the maps to global memory.
-__device__ void phase_route_small(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem) {
+__device__ void phase_route_small(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem,
+                                  uint64_t* stamp) {
   CtaTables& tb = tables(smem);
   const int T = p.T, E = p.E, K = p.K, TK = p.TK;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int t = warp; t < T; t += WARPS) topk_row(p, lp.router_b, t, tb.idx + t * K, tb.w + t * K);
+  for (int t = threadIdx.x; t < T; t += THREADS) tb.pxf[t] = p.pxf[t];
+  if (stamp) *stamp = globaltimer_ns();
   int32_t* hist = reinterpret_cast<int32_t*>(ring_slot(smem, 0));  // [WARPS][E] scratch
   for (int i = threadIdx.x; i < WARPS * E; i += THREADS) hist[i] = 0;
   __syncthreads();
@@ -474,37 +521,27 @@ __device__ __forceinline__ float e8m0_byte(uint32_t w) {
 
 // One K chunk (4 MX blocks) of a 64-row job for this warp:
 //   acc[t][i] += sum over blocks b of 2^s(row, b) [* 2^q(col, b)] * (A_b B_b)
-// A = the chunk's E2M1 codes of tile t as f16 fragments, B = the activation
-// fragments.  Gate/up: the 8 columns are tokens (x in f16, scaled per token).
-// Down: columns 2j, 2j+1 are the hi and lo f16 halves of pair j's SwiGLU
-// output, scaled per (pair, block) by 2^q.  Columns beyond nt read slot 0 and
-// are ignored.
+// A = the chunk's E2M1 codes of tile t as f16 fragments (from the ring slot
+// st), B = the lane's activation fragments bfr[b] (loaded by the caller).
+// Gate/up: the 8 columns are tokens (x in f16, scaled per token).  Down:
+// columns 2j, 2j+1 are the hi and lo f16 halves of pair j's SwiGLU output,
+// scaled per (pair, block) by 2^q, q4 holding this lane's pair's 4 exponents.
 template <bool ISD>
-__device__ __forceinline__ void chunk_mma(const uint8_t* st, int lane, int nt, float (&acc)[4][4]) {
-  const int g = lane >> 2, c = lane & 3;
+__device__ __forceinline__ void chunk_mma(const uint8_t* st, int lane, const uint4 (&bfr)[KB],
+                                          uint32_t q4, float (&acc)[4][4]) {
+  const int g = lane >> 2;
   uint32_t sw0[4], sw1[4];
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
     sw0[t] = *reinterpret_cast<const uint32_t*>(st + STAGE_CODE_BYTES + (t * 16 + g) * KB);
     sw1[t] = *reinterpret_cast<const uint32_t*>(st + STAGE_CODE_BYTES + (t * 16 + g + 8) * KB);
   }
-  const uint8_t* act = st + STAGE_W_BYTES;
-  const uint8_t* bptr;
-  const int8_t* qptr = nullptr;
-  if (!ISD) {
-    const int jb = g < nt ? g : 0;
-    bptr = act + jb * XH_SLOT + c * 16;
-  } else {
-    const int pj = (g >> 1) < nt ? (g >> 1) : 0;
-    bptr = act + pj * A16_CHUNK_BYTES + A16_HDR + (g & 1) * 64 + c * 16;
-    qptr = reinterpret_cast<const int8_t*>(act + (c < nt ? c : 0) * A16_CHUNK_BYTES);
-  }
 #pragma unroll
   for (int b = 0; b < KB; ++b) {
     const uint4 qa = *reinterpret_cast<const uint4*>(st + ((b * 2 + 0) * 32 + lane) * 16);
     const uint4 qb = *reinterpret_cast<const uint4*>(st + ((b * 2 + 1) * 32 + lane) * 16);
-    const uint4 bf = *reinterpret_cast<const uint4*>(bptr + b * (ISD ? 128 : 64));
-    const float qf = ISD ? pow2f((int)qptr[b]) : 1.f;
+    const uint4 bf = bfr[b];
+    const float qf = ISD ? pow2f((int)(int8_t)((q4 >> (8 * b)) & 0xFFu)) : 1.f;
     const uint32_t wd[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
@@ -533,6 +570,7 @@ struct StreamCtx {
   const int32_t* dunits;  // down units
   const int32_t* tokpos;
   const float* wpos;
+  const float* pxf;       // per-token activation scale 2^px
   int n_units, n_dunits;
 };
 
@@ -557,7 +595,7 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
   if (lane == 0) next = atomicAdd(p.sync + SY_JOBS, 1u);
   for (;;) {
     const int64_t j = __shfl_sync(FULL, next, 0);
-    if (j >= n_all || !ok || error_set(p.sync)) {
+    if (j >= n_all || !ok) {
       if (lane == 0) {
         JobEntry* en = jq + (qk % JQ);
         en->job = -1; en->s0 = (int32_t)seq; en->nc = 0;
@@ -575,14 +613,6 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
     const int4 ur = *reinterpret_cast<const int4*>((isD ? cx.dunits : cx.units) + (int64_t)u * 4);
     const int e = ur.x, pos0 = ur.y, nt = ur.z;
     const int nc = isD ? nc_d : nc_gu;
-    if (lane == 0) {
-      JobEntry* en = jq + (qk % JQ);
-      en->job = (int32_t)j; en->s0 = (int32_t)seq; en->nc = nc; en->unit = u; en->rb = rb;
-      en->isD = isD; en->e = e; en->pos0 = pos0; en->nt = nt;
-      __threadfence_block();
-      *reinterpret_cast<volatile int32_t*>(&en->flag) = qk + 1;
-    }
-    ++qk;
     if (isD) {  // the down stages read the SwiGLU output: wait for the gate/up unit
       const int gu = ur.w;
       const uint32_t need = (uint32_t)gub * (uint32_t)cx.units[(int64_t)gu * 4 + 2];
@@ -598,38 +628,41 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
           __nanosleep(100);
         }
       }
-      fence_proxy_async_global();
       t_ready += clock64() - tr0;
+      if (!ok) continue;  // publishes the end entry
     }
-    int tok = 0;
-    if (!isD && lane < nt) tok = cx.tokpos[pos0 + lane];
+    // publish the job (after the readiness acquire, so the consumers' reads of
+    // the SwiGLU output are ordered after it)
+    if (lane == 0) {
+      JobEntry* en = jq + (qk % JQ);
+      en->job = (int32_t)j; en->s0 = (int32_t)seq; en->nc = nc; en->unit = u; en->rb = rb;
+      en->isD = isD; en->e = e; en->pos0 = pos0; en->nt = nt;
+      __threadfence_block();
+      *reinterpret_cast<volatile int32_t*>(&en->flag) = qk + 1;
+    }
+    ++qk;
     const uint8_t* wbase = isD ? lp.w_d + ((int64_t)e * db + rb) * nc * STAGE_W_BYTES
                                : lp.w_gu + ((int64_t)e * gub + rb) * nc * STAGE_W_BYTES;
-    const uint32_t bytes = STAGE_W_BYTES + nt * (isD ? A16_CHUNK_BYTES : XH_CHUNK_BYTES);
-    for (int c = 0; c < nc && ok; ++c) {
-      const int slot = (int)(seq % NSLOT);
+    // Stages are issued in batches: successive 1-D bulk copies issued by one
+    // warp instruction each are serialised, while the copies of one
+    // instruction (one per lane) proceed in parallel.
+    for (int c0 = 0; c0 < nc && ok; c0 += PRODUCER_BATCH) {
+      const int nb = min(PRODUCER_BATCH, nc - c0);
       const unsigned long long te0 = clock64();
-      if (seq >= (uint32_t)NSLOT &&
-          !wait_mbar(empty_bar(smem, slot), ((seq / NSLOT) + 1) & 1u, p.sync, p.timeout_ns,
-                     DEV_TIMEOUT_PIPE, seq)) {
-        ok = false;
-        break;
-      }
+      bool bad = false;
+      const uint32_t s = seq + lane;
+      const int slot = (int)(s % NSLOT);
+      if (lane < nb && s >= (uint32_t)NSLOT)  // wait until the slot is free
+        bad = !wait_mbar(empty_bar(smem, slot), ((s / NSLOT) + 1) & 1u, p.sync, p.timeout_ns,
+                         DEV_TIMEOUT_PIPE, s);
+      if (__any_sync(FULL, bad)) { ok = false; break; }
       t_empty += clock64() - te0;
-      uint8_t* dst = ring_slot(smem, slot);
-      uint64_t* fb = full_bar(smem, slot);
-      if (lane == 0) {
-        mbar_arrive_expect_tx(fb, bytes);
-        bulk_g2s(dst, wbase + (int64_t)c * STAGE_W_BYTES, STAGE_W_BYTES, fb);
-        if (isD)
-          bulk_g2s(dst + STAGE_W_BYTES, p.a16 + ((int64_t)c * p.TK + pos0) * A16_CHUNK_BYTES,
-                   nt * A16_CHUNK_BYTES, fb);
+      if (lane < nb) {
+        mbar_arrive_expect_tx(full_bar(smem, slot), STAGE_W_BYTES);
+        bulk_g2s(ring_slot(smem, slot), wbase + (int64_t)(c0 + lane) * STAGE_W_BYTES, STAGE_W_BYTES,
+                 full_bar(smem, slot));
       }
-      __syncwarp();
-      if (!isD && lane < nt)
-        bulk_g2s(dst + STAGE_W_BYTES + lane * XH_SLOT, p.xh + ((int64_t)tok * p.H + c * KC) * 2,
-                 XH_CHUNK_BYTES, fb);
-      ++seq;
+      seq += nb;
     }
   }
   if (p.prof && lane == 0) {
@@ -657,14 +690,30 @@ __device__ void stream_consumer(const EngineParams& p, uint8_t* smem, const Stre
   JobEntry* jq = job_queue(smem);
   uint32_t* ready = p.sync + SY_READY;
   bool poison = false;
+  const bool prof = p.prof != nullptr;
   unsigned long long t_full = 0, t_mma = 0, t_bar = 0, t_epi = 0, t_queue = 0, n_jobs = 0;
-  const unsigned long long t_begin = clock64();
+  const unsigned long long t_begin = pclock(prof);
+  // A gate/up epilogue's readiness signal (release fence + counter add) is
+  // deferred until after this warp's next chunk, when its stores have landed
+  // and the fence is cheap; it is flushed at once whenever the warp would wait
+  // for the producer (which may itself wait for that signal).
+  int pend_u = -1;
+  auto flush_ready = [&]() {
+    if (pend_u >= 0) {
+      if (lane == 0) {
+        __threadfence();
+        red_release_add_u32(ready + pend_u, 1u);
+      }
+      pend_u = -1;
+    }
+  };
   for (;;) {
     JobEntry* en = jq + (qk % JQ);
-    const unsigned long long tq0 = clock64();
+    const unsigned long long tq0 = pclock(prof);
     // the producer publishes the entry (bounded wait; the producer's own waits
     // are bounded by the same timeout, after which it publishes an end entry)
     if (*reinterpret_cast<volatile int32_t*>(&en->flag) != qk + 1) {
+      flush_ready();
       const uint64_t t0 = globaltimer_ns();
       while (*reinterpret_cast<volatile int32_t*>(&en->flag) != qk + 1) {
         if (globaltimer_ns() - t0 > 2 * p.timeout_ns) { set_error(p.sync, DEV_TIMEOUT_QUEUE, qk); return; }
@@ -672,34 +721,75 @@ __device__ void stream_consumer(const EngineParams& p, uint8_t* smem, const Stre
       }
     }
     const int job = *reinterpret_cast<volatile int32_t*>(&en->job);
-    t_queue += clock64() - tq0;
+    t_queue += pclock(prof) - tq0;
     if (job < 0) { ++qk; break; }
     ++n_jobs;
     const int s0 = en->s0, nc = en->nc, u = en->unit, rb = en->rb, isD = en->isD;
     const int pos0 = en->pos0, nt = en->nt;
     const int buf = qk & 1;
+    // order the reads of activations (written by other CTAs, seen through the
+    // producer's acquire) after the queue entry
+    __threadfence_block();
+    // this lane's activation fragments: base address of chunk 0 and the step
+    // between K chunks.  Gate/up: column g is token g (columns >= nt repeat
+    // token 0 and are ignored).  Down: column g is the hi (g even) or lo half
+    // of pair g/2, and the lane's output pair c supplies the block exponents.
+    const uint8_t* fbase;
+    const uint8_t* qbase = nullptr;
+    int64_t cstep;
+    int bstep;
+    if (!isD) {
+      const int tok = cx.tokpos[pos0 + (g < nt ? g : 0)];
+      fbase = p.xh + (int64_t)tok * p.H * 2 + c * 16;
+      cstep = (int64_t)KC * 2;
+      bstep = 64;
+    } else {
+      const int pj = (g >> 1) < nt ? (g >> 1) : 0;
+      fbase = p.a16 + (int64_t)(pos0 + pj) * A16_CHUNK_BYTES + A16_HDR + (g & 1) * 64 + c * 16;
+      qbase = p.a16 + (int64_t)(pos0 + (c < nt ? c : 0)) * A16_CHUNK_BYTES;
+      cstep = (int64_t)p.TK * A16_CHUNK_BYTES;
+      bstep = 128;
+    }
     float acc[4][4];
 #pragma unroll
     for (int t = 0; t < 4; ++t)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[t][i] = 0.f;
+    uint4 fcur[KB];
+    uint32_t qcur = 0;
+    if (w < nc) {
+#pragma unroll
+      for (int b = 0; b < KB; ++b) fcur[b] = ld_cg_v4(fbase + w * cstep + b * bstep);
+      if (isD) qcur = ld_cg_u32(qbase + w * cstep);
+    }
     for (int cc = w; cc < nc; cc += NCW) {
+      // fetch the next chunk's fragments while this one computes
+      uint4 fnext[KB];
+      uint32_t qnext = 0;
+      const int cn = cc + NCW < nc ? cc + NCW : cc;
+#pragma unroll
+      for (int b = 0; b < KB; ++b) fnext[b] = ld_cg_v4(fbase + cn * cstep + b * bstep);
+      if (isD) qnext = ld_cg_u32(qbase + cn * cstep);
       const uint32_t s = (uint32_t)s0 + cc;
       const int slot = (int)(s % NSLOT);
-      const unsigned long long tf0 = clock64();
+      const unsigned long long tf0 = pclock(prof);
       if (!poison &&
           !wait_mbar(full_bar(smem, slot), (s / NSLOT) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, s))
         poison = true;
-      const unsigned long long tm0 = clock64();
+      const unsigned long long tm0 = pclock(prof);
       t_full += tm0 - tf0;
       if (!poison) {
         const uint8_t* st = ring_slot(smem, slot);
-        if (!isD) chunk_mma<false>(st, lane, nt, acc);
-        else chunk_mma<true>(st, lane, nt, acc);
+        if (!isD) chunk_mma<false>(st, lane, fcur, 0u, acc);
+        else chunk_mma<true>(st, lane, fcur, qcur, acc);
       }
-      t_mma += clock64() - tm0;
+      t_mma += pclock(prof) - tm0;
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar(smem, slot));
+      flush_ready();
+#pragma unroll
+      for (int b = 0; b < KB; ++b) fcur[b] = fnext[b];
+      qcur = qnext;
     }
     // deposit this warp's partial sums: part[w][col][row]
     float* pb = part_buf(smem, buf) + (size_t)w * PART_COLS * PART_LD;
@@ -709,9 +799,9 @@ __device__ void stream_consumer(const EngineParams& p, uint8_t* smem, const Stre
 #pragma unroll
         for (int i = 0; i < 4; ++i) pb[(2 * c + (i & 1)) * PART_LD + t * 16 + g + (i >> 1) * 8] = acc[t][i];
     }
-    const unsigned long long tb0 = clock64();
+    const unsigned long long tb0 = pclock(prof);
     named_barrier(1 + buf, NCW * 32);
-    const unsigned long long te0 = clock64();
+    const unsigned long long te0 = pclock(prof);
     t_bar += te0 - tb0;
     const int nw = nc < NCW ? nc : NCW;
     const float* pall = part_buf(smem, buf);
@@ -719,7 +809,7 @@ __device__ void stream_consumer(const EngineParams& p, uint8_t* smem, const Stre
     const int j = (w + NCW - (qk % NCW)) % NCW;
     if (!poison && j < nt) {
       if (!isD) {  // gate/up epilogue: token column j, lane = intermediate row i0 + lane
-        const float px = p.pxf[cx.tokpos[pos0 + j]];
+        const float px = cx.pxf[cx.tokpos[pos0 + j]];
         float gs = 0.f, us = 0.f;
         for (int ww = 0; ww < nw; ++ww) {
           gs += pall[((size_t)ww * PART_COLS + j) * PART_LD + lane];
@@ -746,10 +836,8 @@ __device__ void stream_consumer(const EngineParams& p, uint8_t* smem, const Stre
         *reinterpret_cast<__half*>(base + off + 64) = lo;
         if (lane == 0) base[bi] = (uint8_t)(int8_t)q;
         __syncwarp();
-        if (lane == 0) {
-          __threadfence();
-          red_release_add_u32(ready + u, 1u);
-        }
+        flush_ready();  // a previous job's signal, if still pending
+        pend_u = u;
       } else {  // down epilogue: pair j, lane = rows h0 + lane and h0 + 32 + lane
         const float wp = cx.wpos[pos0 + j];
         const int h0 = rb * STAGE_ROWS;
@@ -765,16 +853,17 @@ __device__ void stream_consumer(const EngineParams& p, uint8_t* smem, const Stre
         }
       }
     }
-    t_epi += clock64() - te0;
+    t_epi += pclock(prof) - te0;
     ++qk;
   }
+  flush_ready();
   if (p.prof && lane == 0) {
     atomicAdd(p.prof + PF_CONS_FULL, t_full);
     atomicAdd(p.prof + PF_CONS_MMA, t_mma);
     atomicAdd(p.prof + PF_CONS_BAR, t_bar);
     atomicAdd(p.prof + PF_CONS_EPI, t_epi);
     atomicAdd(p.prof + PF_CONS_QUEUE, t_queue);
-    atomicAdd(p.prof + PF_CONS_TOTAL, clock64() - t_begin);
+    atomicAdd(p.prof + PF_CONS_TOTAL, pclock(prof) - t_begin);
     atomicAdd(p.prof + PF_JOBS, n_jobs);
   }
 }
@@ -874,39 +963,40 @@ __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p
     const LayerPtrs& lp = p.layers[layer];
     const __nv_bfloat16* x = layer == 0 ? p.x_in : p.xnext;
     uint64_t* st = stamp ? p.stamps + 1 + layer * STAMPS_PER_LAYER : nullptr;
-    phase_prepare(p, lp, x, layer);
+    phase_prepare(p, lp, x, layer, smem, st);
     if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 1)) return;
-    if (st) st[0] = globaltimer_ns();
+    if (st) st[2] = globaltimer_ns();
     StreamCtx cx;
     const int32_t* inv;
     if (small) {
-      phase_route_small(p, lp, smem);
-      cx = StreamCtx{tb.units, tb.dunits, tb.tokpos, tb.wpos, tb.n_units, tb.n_dunits};
+      phase_route_small(p, lp, smem, st ? st + 3 : nullptr);
+      cx = StreamCtx{tb.units, tb.dunits, tb.tokpos, tb.wpos, tb.pxf, tb.n_units, tb.n_dunits};
       inv = tb.inv;
       if (p.route_only) return;
     } else {
       phase_topk_large(p, lp);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 2)) return;
+      if (st) st[3] = globaltimer_ns();
       phase_permute_large(p, smem);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 3)) return;
       if (p.route_only) return;
-      cx = StreamCtx{p.units, p.dunits, p.tokpos, p.wpos, p.n_units[0], p.n_units[1]};
+      cx = StreamCtx{p.units, p.dunits, p.tokpos, p.wpos, p.pxf, p.n_units[0], p.n_units[1]};
       inv = p.inv;
     }
-    if (st) st[1] = globaltimer_ns();
+    if (st) st[4] = globaltimer_ns();
     fence_proxy_async_smem();  // the ring held routing scratch written by generic stores
     __syncthreads();
     if (warp == NCW) stream_producer(p, lp, smem, cx, seq, qk);
     else stream_consumer(p, smem, cx, qk);
     if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 4)) return;
-    if (st) st[2] = globaltimer_ns();
+    if (st) st[5] = globaltimer_ns();
     if (layer + 1 < p.L) {
       phase_combine_rmsnorm(p, inv, smem);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 5)) return;
     } else {
       phase_combine_out(p, inv);
     }
-    if (st) st[3] = globaltimer_ns();
+    if (st) st[6] = globaltimer_ns();
   }
 }
 

@@ -21,14 +21,13 @@ constexpr int STAGE_CODE_BYTES = STAGE_ROWS * KC / 2;    // 4096
 constexpr int STAGE_W_BYTES = STAGE_CODE_BYTES + STAGE_ROWS * KB;  // 4352
 constexpr int NT_MAX = 8;                                // tokens per gate/up unit (one MMA n-tile)
 constexpr int ND_MAX = 4;                                // pairs per down unit (hi+lo: one n-tile)
-// activations of one stage, per token (gate/up) or per (token, expert) pair (down)
-constexpr int XH_CHUNK_BYTES = KC * 2;                   // f16 x, fragment order
-constexpr int XH_SLOT = XH_CHUNK_BYTES + 64;             // padded: conflict-free fragment loads
-constexpr int A16_HDR = 16;                              // 4 block exponents q, padded
-constexpr int A16_CHUNK_BYTES = A16_HDR + KC * 2 * 2;    // hi and lo f16 halves: 528
-constexpr int SLOT_ACT_BYTES = NT_MAX * XH_SLOT > ND_MAX * A16_CHUNK_BYTES ? NT_MAX * XH_SLOT
-                                                                          : ND_MAX * A16_CHUNK_BYTES;
-constexpr int SLOT_BYTES = STAGE_W_BYTES + SLOT_ACT_BYTES;  // 6912
+// activations of one K chunk, per (token, expert) pair of the down projection:
+// 4 block exponents q (padded to 16 bytes), then the hi and lo f16 halves of
+// the SwiGLU output in fragment order.  Consumer lanes read activation
+// fragments straight from L2; the ring carries weight stages only.
+constexpr int A16_HDR = 16;
+constexpr int A16_CHUNK_BYTES = A16_HDR + KC * 2 * 2;    // 528
+constexpr int SLOT_BYTES = STAGE_W_BYTES;                // 4352
 constexpr int MAX_HSPLIT = 8;                            // router dot products split along H
 
 constexpr int MAX_LAYERS = 16;
@@ -36,12 +35,13 @@ constexpr int MAX_EXPERTS = 512;
 constexpr int NCW = 8;                                   // consumer (MMA) warps per CTA
 constexpr int WARPS = NCW + 1;                           // + one producer warp
 constexpr int THREADS = WARPS * 32;
-constexpr int NSLOT = 25;                                // stage ring slots per CTA
+constexpr int NSLOT = 40;                                // stage ring slots per CTA
+constexpr int PRODUCER_BATCH = 16;                       // stages per bulk-copy instruction
 constexpr int JQ = 32;                                   // job queue entries per CTA
 constexpr int PART_LD = 68;                              // partial-sum column stride (floats)
 constexpr int PART_COLS = 8;                             // one n-tile
 constexpr int SMALL_PAIRS = 256;                         // T*k up to this: routing done per CTA
-constexpr int STAMPS_PER_LAYER = 4;                      // prepared, routed, streamed, combined
+constexpr int STAMPS_PER_LAYER = 7;  // x converted, logits (CTA 0), prepared, top-k, routed, streamed, combined
 
 // sync word layout (uint32)
 enum : int {

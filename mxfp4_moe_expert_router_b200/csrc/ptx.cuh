@@ -94,6 +94,19 @@ __device__ __forceinline__ uint32_t ld_volatile_u32(const uint32_t* p) {
   return v;
 }
 
+// ---- L2-coherent loads (bypass L1: data written by other CTAs in this launch) ---------
+__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_cg_u32(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
 // ---- E2M1 / packed fp32 ----------------------------------------------------------
 // Two E2M1 codes (low nibble first) -> f16x2 {lo, hi}; exact.
 __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte_in_low8) {
