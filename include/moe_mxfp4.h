@@ -177,10 +177,11 @@ MOE_API int32_t moe_phase_ns(moe_mxfp4_t* h, uint64_t* ns_out, int32_t max_n, vo
  * copy up to max_n counters accumulated since the previous call to the HOST
  * array out (may be NULL when max_n == 0), reset them, and switch counting on
  * (enable != 0) or off for the following launches.  Counters, in SM clock
- * cycles summed over CTAs and warps: producer waiting for free ring slots,
- * producer waiting for gate/up completion, producer total, stages issued;
- * consumers waiting for data, in MMA chunks, at the per-job barrier, in
- * epilogues, waiting for the job queue, consumer total, jobs.
+ * cycles summed over CTAs (and over the 8 epilogue warps for the epilogue
+ * ones): producer waiting for free ring slots, producer waiting for gate/up
+ * completion, producer total, stages issued; MMA issuer waiting for stage
+ * data, issuing (scale copies + MMAs), waiting for a free accumulator;
+ * epilogue waiting for accumulators, epilogue work, epilogue total; jobs.
  */
 MOE_API int32_t moe_stream_profile(moe_mxfp4_t* h, int32_t enable, uint64_t* out, int32_t max_n,
                                    void* stream);

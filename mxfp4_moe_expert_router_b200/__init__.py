@@ -183,8 +183,8 @@ class Moe:
         return [int(v) for v in arr]
 
     PROFILE_KEYS = ("prod_wait_empty", "prod_wait_ready", "prod_total", "stages",
-                    "cons_wait_full", "cons_mma", "cons_barrier", "cons_epilogue", "cons_queue",
-                    "cons_total", "jobs")
+                    "mma_wait_full", "mma_issue", "mma_wait_acc", "epi_wait_acc", "epi_work",
+                    "epi_total", "jobs")
 
     def moe_stream_profile(self, enable=True, stream=None):
         """Counters since the previous call (dict), then counting switched on/off."""

@@ -13,22 +13,32 @@
 // MoE expert layer whose routing is the runtime dynamism (HyperAI salon
 // transcript, section "Achieving maximum speed improvement ...").
 //
-// Weight stream (phase C).  Work is cut into CTA jobs of 64 weight rows x the
-// whole contraction dimension.  Warp NCW is the producer: it takes jobs from a
-// global counter, publishes them in a shared-memory job queue and streams each
-// job's K chunks (one 4352-byte MXFP4 stage + the matching activation slices)
-// into a ring of NSLOT slots with 1-D bulk copies (full/empty mbarriers).
-// Warps 0..NCW-1 consume chunk c of every job in warp c % NCW: E2M1 bytes are
-// turned into f16 A fragments in registers, the tokens form the N side of
-// mma.m16n8k16 (fp32 accumulate), and each MX block's E8M0 scale multiplies its
-// block partial in fp32.  The per-warp partial sums meet in shared memory
-// behind a named barrier and are reduced in warp order (deterministic), then
-// one warp per token (gate/up) or per pair (down) runs the epilogue.
+// Weight stream (phase C).  Work is cut into CTA jobs of 128 weight rows x the
+// whole contraction dimension (see engine.cuh).  Warp 0 is the producer: it
+// takes jobs from a global counter, publishes them in a shared-memory job
+// queue and streams each job's K stages -- an 8704-byte MXFP4 weight stage
+// plus the E2M1 term images of the unit's activations -- into a ring of NSLOT
+// slots with 1-D bulk copies (full/empty mbarriers).  One thread of warp 1
+// issues the fifth-generation tensor-core MMAs: per stage it copies the
+// weight and activation E8M0 scales into tensor memory and runs two
+// block-scaled kind::mxf4 MMAs (M = 128, K = 64, N = 8 columns per token or
+// pair) accumulating in tensor memory; a commit frees the ring slot when they
+// complete, and a commit at the job's end hands the accumulator buffer to the
+// epilogue.  Warps 4..11 (two groups of four, one warp per 32-lane
+// sub-partition of tensor memory) run the epilogues of alternate jobs: sum the
+// 8 term columns, SwiGLU and the term expansion of its output (gate/up), or
+// scale by the routing weight (down).  No CUDA core touches a weight.
+//
+// Activations as E2M1 terms.  The MMA multiplies E2M1 by E2M1, so a value v of
+// a 32-element block with amax A is written as v = sum_k c_k 2^s_k, c_k E2M1,
+// s_0 = ceil(log2(A / 6)), s_k = s_0 + 1 - 3k (k >= 1): each term rounds the
+// remaining residual to nearest, exactly, and the residual after NTERM = 8
+// terms is below 2^(s_0 - 21) <= A * 2^-21 -- beneath the fp32 accumulation.
 //
 // Every wait (grid barrier, mbarrier, job queue, per-unit readiness) is bounded
 // by p.timeout_ns of %globaltimer; on expiry the kernel records a status code
-// in sync[SY_ERROR], stops issuing work, lets every copy in flight land and
-// returns.
+// in sync[SY_ERROR], stops issuing work, lets every copy and MMA in flight
+// complete, frees its tensor memory and returns.
 #include <math.h>
 #include <cuda_fp16.h>
 
@@ -45,9 +55,11 @@ constexpr int SMALL_DUNITS = 256 + SMALL_PAIRS / ND_MAX;
 struct JobEntry {
   int32_t flag;  // queue index + 1 once the entry is written
   int32_t job;   // -1: no more jobs in this phase
-  int32_t s0;    // stage sequence number of chunk 0
-  int32_t nc;    // chunks (stages)
-  int32_t unit, rb, isD, e, pos0, nt, pad0, pad1;
+  int32_t s0;    // stage sequence number of stage 0
+  int32_t nc;    // stages
+  int32_t unit, rb, isD, e, pos0, nt;
+  int32_t wj;    // work index (per CTA): accumulator buffer wj % NACC, epilogue group wj % 2
+  int32_t pad;
 };
 
 struct alignas(16) CtaTables {
@@ -59,7 +71,6 @@ struct alignas(16) CtaTables {
   int32_t inv[SMALL_PAIRS];
   int32_t tokpos[SMALL_PAIRS];
   float wpos[SMALL_PAIRS];
-  float pxf[SMALL_PAIRS];
   int32_t counts[MAX_EXPERTS];
   int32_t offsets[MAX_EXPERTS + 1];
   float red[WARPS];
@@ -67,22 +78,42 @@ struct alignas(16) CtaTables {
 };
 
 constexpr size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
+constexpr size_t RING_BYTES = (size_t)NPIPE * NSLOT * SLOT_BYTES;   // all pipelines' rings
 constexpr size_t OFF_RING = 0;
-constexpr size_t OFF_FULL = OFF_RING + (size_t)NSLOT * SLOT_BYTES;
-constexpr size_t OFF_EMPTY = OFF_FULL + NSLOT * 8;
-constexpr size_t OFF_JQ = align16(OFF_EMPTY + NSLOT * 8);
-constexpr size_t OFF_PART = align16(OFF_JQ + JQ * sizeof(JobEntry));
-constexpr size_t PART_BUF = (size_t)NCW * PART_COLS * PART_LD;  // floats per buffer
-constexpr size_t OFF_TABLES = align16(OFF_PART + 2 * PART_BUF * 4);
+constexpr size_t OFF_FULL = OFF_RING + RING_BYTES;                  // [NPIPE][NSLOT]
+constexpr size_t OFF_EMPTY = OFF_FULL + NPIPE * NSLOT * 8;          // [NPIPE][NSLOT]
+constexpr size_t OFF_ACCF = OFF_EMPTY + NPIPE * NSLOT * 8;          // [NPIPE][NACC]
+constexpr size_t OFF_ACCE = OFF_ACCF + NPIPE * NACC * 8;            // [NPIPE][NACC]
+constexpr size_t OFF_XBAR = OFF_ACCE + NPIPE * NACC * 8;            // [NPIPE][2] amax exchange
+constexpr size_t OFF_DRAIN = OFF_XBAR + NPIPE * 2 * 8;              // [NPIPE]
+constexpr size_t OFF_TMEMBASE = OFF_DRAIN + NPIPE * 8;
+constexpr size_t OFF_JQ = align16(OFF_TMEMBASE + 8);                // [NPIPE][JQ]
+constexpr size_t OFF_XCH = align16(OFF_JQ + NPIPE * JQ * sizeof(JobEntry));  // [NPIPE][2][NT_MAX][4] floats
+constexpr size_t OFF_TABLES = align16(OFF_XCH + NPIPE * 2 * NT_MAX * 4 * 4);
 constexpr size_t SMEM_BYTES = OFF_TABLES + sizeof(CtaTables);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert((size_t)WARPS * MAX_EXPERTS * 4 <= (size_t)NSLOT * SLOT_BYTES, "routing scratch in ring");
+static_assert((size_t)WARPS * MAX_EXPERTS * 4 <= RING_BYTES, "routing scratch in ring");
+static_assert(SLOT_BYTES % 16 == 0 && STAGE_A_BYTES % 16 == 0 && IMG_BYTES % 16 == 0, "bulk-copy alignment");
+// tensor memory: pipeline p's accumulators, then its scale-factor buffers
+__host__ __device__ constexpr uint32_t tm_acc(int pipe, int b) { return (uint32_t)(pipe * NACC + b) * ACC_COLS; }
+__host__ __device__ constexpr uint32_t tm_sf(int pipe, int i) {
+  return (uint32_t)(NPIPE * NACC * ACC_COLS + (pipe * NSF + i) * SF_COLS);
+}
 
-__device__ __forceinline__ uint8_t* ring_slot(uint8_t* smem, int s) { return smem + OFF_RING + (size_t)s * SLOT_BYTES; }
-__device__ __forceinline__ uint64_t* full_bar(uint8_t* smem, int s) { return reinterpret_cast<uint64_t*>(smem + OFF_FULL) + s; }
-__device__ __forceinline__ uint64_t* empty_bar(uint8_t* smem, int s) { return reinterpret_cast<uint64_t*>(smem + OFF_EMPTY) + s; }
-__device__ __forceinline__ JobEntry* job_queue(uint8_t* smem) { return reinterpret_cast<JobEntry*>(smem + OFF_JQ); }
-__device__ __forceinline__ float* part_buf(uint8_t* smem, int b) { return reinterpret_cast<float*>(smem + OFF_PART) + b * PART_BUF; }
+__device__ __forceinline__ uint8_t* ring_slot(uint8_t* smem, int pipe, int s) {
+  return smem + OFF_RING + ((size_t)pipe * NSLOT + s) * SLOT_BYTES;
+}
+__device__ __forceinline__ uint64_t* full_bar(uint8_t* smem, int pipe, int s) { return reinterpret_cast<uint64_t*>(smem + OFF_FULL) + pipe * NSLOT + s; }
+__device__ __forceinline__ uint64_t* empty_bar(uint8_t* smem, int pipe, int s) { return reinterpret_cast<uint64_t*>(smem + OFF_EMPTY) + pipe * NSLOT + s; }
+__device__ __forceinline__ uint64_t* accf_bar(uint8_t* smem, int pipe, int b) { return reinterpret_cast<uint64_t*>(smem + OFF_ACCF) + pipe * NACC + b; }
+__device__ __forceinline__ uint64_t* acce_bar(uint8_t* smem, int pipe, int b) { return reinterpret_cast<uint64_t*>(smem + OFF_ACCE) + pipe * NACC + b; }
+__device__ __forceinline__ uint64_t* xch_bar(uint8_t* smem, int pipe, int i) { return reinterpret_cast<uint64_t*>(smem + OFF_XBAR) + pipe * 2 + i; }
+__device__ __forceinline__ uint64_t* drain_bar(uint8_t* smem, int pipe) { return reinterpret_cast<uint64_t*>(smem + OFF_DRAIN) + pipe; }
+__device__ __forceinline__ uint32_t* tmem_base_word(uint8_t* smem) { return reinterpret_cast<uint32_t*>(smem + OFF_TMEMBASE); }
+__device__ __forceinline__ JobEntry* job_queue(uint8_t* smem, int pipe) { return reinterpret_cast<JobEntry*>(smem + OFF_JQ) + pipe * JQ; }
+__device__ __forceinline__ float* xch_buf(uint8_t* smem, int pipe, int i) {
+  return reinterpret_cast<float*>(smem + OFF_XCH) + (pipe * 2 + i) * NT_MAX * 4;
+}
 __device__ __forceinline__ CtaTables& tables(uint8_t* smem) { return *reinterpret_cast<CtaTables*>(smem + OFF_TABLES); }
 
 __device__ __forceinline__ void set_error(uint32_t* sync, uint32_t code, uint32_t info) {
@@ -142,10 +173,61 @@ __device__ __forceinline__ float pow2f(int e) {  // 2^e for e in [-126, 127]
   return __uint_as_float((uint32_t)(e + 127) << 23);
 }
 
-// ---- phase A: activations in f16 fragments, router partial logits -----------------------
-// Each token's x is scaled by 2^-px so that max|x| lies in [2^14, 2^15); then
-// every bf16 value is exact in f16 unless it is below max|x| * 2^-28.  The
-// 32-element blocks are stored in the mma B-fragment order (see chunk_mma).
+// ---- E2M1 term expansion of activations ----------------------------------------------------
+// Exponent of term 0 for a block with amax A > 0: the least s with A <= 6 * 2^s
+// (A = m 2^E, m in [1, 2): s = E - 2 if m <= 1.5, else E - 1), kept in
+// [-126, 126] so that every term exponent has an E8M0 byte in [1, 253].
+__device__ __forceinline__ int term0_exp(float amax) {
+  const uint32_t u = __float_as_uint(amax);
+  const int E = (int)((u >> 23) & 0xFF) - 127;
+  if (E < -126) return -126;  // zero or subnormal amax
+  const int s = (u & 0x7FFFFFu) <= 0x400000u ? E - 2 : E - 1;
+  return min(max(s, -126), 126);
+}
+__device__ __forceinline__ int term_exp(int s0, int k) { return max(k == 0 ? s0 : s0 + 1 - 3 * k, -126); }
+
+// E2M1 value of a code (low nibble), exact.
+__device__ __forceinline__ float e2m1_value(uint32_t code) {
+  return __half2float(__ushort_as_half((uint16_t)(e2m1x2_to_f16x2(code) & 0xFFFFu)));
+}
+
+// The NTERM E2M1 codes c_k of v = sum_k c_k 2^s_k (+ a residual below
+// 2^(s_0 - 21)); code k in bits 4k..4k+3.  Each step rounds the current
+// residual r to the nearest E2M1 multiple of 2^s_k and subtracts it exactly.
+__device__ __forceinline__ uint32_t e2m1_terms(float v, int s0) {
+  uint32_t w = 0;
+  float r = v;
+#pragma unroll
+  for (int k = 0; k < NTERM; ++k) {
+    const int sk = term_exp(s0, k);
+    const uint32_t c = f32x2_to_e2m1x2(0.f, r * pow2f(-sk)) & 0xFu;
+    r = fmaf(-e2m1_value(c), pow2f(sk), r);
+    w |= c << (4 * k);
+  }
+  return w;
+}
+
+// Warp transpose of term codes: lane i holds the NTERM codes of element i of
+// `n` consecutive elements (n = 16 or 32); lane o receives the 32-bit word of
+// term o / (n / 8) covering elements 8 (o % (n / 8)) .. +7 (element 8q + j at
+// bits 4j, so the word is little-endian bytes of packed E2M1 pairs).
+template <int NEL>
+__device__ __forceinline__ uint32_t term_word(uint32_t codes, int lane) {
+  constexpr int WPT = NEL / 8;  // words per term
+  const int k = (lane / WPT) % NTERM, q = lane % WPT;
+  uint32_t out = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t v = __shfl_sync(FULL, codes, 8 * q + j);
+    out |= ((v >> (4 * k)) & 0xFu) << (4 * j);
+  }
+  return out;
+}
+
+// ---- phase A: activation term images, router partial logits --------------------------------
+// x[t] (bf16) -> xt[stage][t]: per 32-element block one warp expands the values
+// into NTERM E2M1 terms (codes at the MMA's B-operand rows, scales at the
+// scale-factor rows of the image).
 __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const __nv_bfloat16* x,
                               int layer, uint8_t* smem, uint64_t* stamp) {
   const int T = p.T, H = p.H, E = p.E;
@@ -153,56 +235,20 @@ __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const 
   const int64_t gt = (int64_t)blockIdx.x * THREADS + threadIdx.x;
   const int64_t gs = (int64_t)gridDim.x * THREADS;
   const int64_t wg = (int64_t)blockIdx.x * WARPS + warp, ws = (int64_t)gridDim.x * WARPS;
-  // one CTA per token: CTA-wide max, then every thread converts whole blocks
-  float* red = tables(smem).red;
-  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-    const __nv_bfloat16* xr = x + t * H;
-    float m = 0.f;
-    for (int h = threadIdx.x * 8; h < H; h += THREADS * 8) {
-      const uint4 v = *reinterpret_cast<const uint4*>(xr + h);
-      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  const int nblk = H / 32;
+  const int64_t ntask = p.route_only ? 0 : (int64_t)T * nblk;  // routing alone needs no images
+  for (int64_t task = wg; task < ntask; task += ws) {
+    const int t = (int)(task / nblk), gb = (int)(task % nblk);
+    const float v = __bfloat162float(x[(int64_t)t * H + gb * 32 + lane]);
+    float am = fabsf(v);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        m = fmaxf(m, fabsf(__uint_as_float(u[i] << 16)));
-        m = fmaxf(m, fabsf(__uint_as_float(u[i] & 0xFFFF0000u)));
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
-    __syncthreads();
-    if (lane == 0) red[warp] = m;
-    __syncthreads();
-#pragma unroll
-    for (int w2 = 0; w2 < WARPS; ++w2) m = fmaxf(m, red[w2]);
-    const int eb = (int)((__float_as_uint(m) >> 23) & 0xFF);
-    int px = m > 0.f ? eb - 127 - 14 : 0;
-    px = max(px, -126);
-    const float inv = pow2f(-px);
-    if (threadIdx.x == 0) p.pxf[t] = pow2f(px);
-    for (int b = threadIdx.x; b < H / 32; b += THREADS) {
-      const uint4* src = reinterpret_cast<const uint4*>(xr + b * 32);
-      float v[32];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 q = src[i];
-        const uint32_t u[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          v[i * 8 + 2 * k] = __uint_as_float(u[k] << 16) * inv;
-          v[i * 8 + 2 * k + 1] = __uint_as_float(u[k] & 0xFFFF0000u) * inv;
-        }
-      }
-      uint4* dst = reinterpret_cast<uint4*>(p.xh + (t * H + b * 32) * 2);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        __half2 h0 = __floats2half2_rn(v[2 * c], v[2 * c + 1]);
-        __half2 h1 = __floats2half2_rn(v[2 * c + 8], v[2 * c + 9]);
-        __half2 h2 = __floats2half2_rn(v[16 + 2 * c], v[17 + 2 * c]);
-        __half2 h3 = __floats2half2_rn(v[24 + 2 * c], v[25 + 2 * c]);
-        dst[c] = make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
-                            *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
-      }
-    }
+    for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(FULL, am, o));
+    const int s0 = term0_exp(am);
+    const uint32_t word = term_word<32>(e2m1_terms(v, s0), lane);
+    const int b = gb % KB, kk = b >> 1, kc = b & 1;
+    uint8_t* img = p.xt + ((int64_t)(gb / KB) * T + t) * IMG_BYTES;
+    *reinterpret_cast<uint32_t*>(img + kk * 256 + kc * 128 + (lane >> 2) * 16 + (lane & 3) * 4) = word;
+    if (lane < NTERM) img[IMG_CODE_BYTES + lane * 16 + b] = (uint8_t)(term_exp(s0, lane) + 127);
   }
   if (stamp) stamp[0] = globaltimer_ns();
   if (p.layer_io) {
@@ -221,12 +267,12 @@ __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const 
   // block that fits in the (idle) stage ring is staged there first, so that
   // only the router weights come from L2.
   const __nv_bfloat16* xr = x;
-  if ((int64_t)T * H * 2 <= (int64_t)NSLOT * SLOT_BYTES) {
-    uint4* d = reinterpret_cast<uint4*>(ring_slot(smem, 0));
+  if ((int64_t)T * H * 2 <= (int64_t)RING_BYTES) {
+    uint4* d = reinterpret_cast<uint4*>(ring_slot(smem, 0, 0));
     const uint4* s8 = reinterpret_cast<const uint4*>(x);
     for (int64_t i = threadIdx.x; i < (int64_t)T * H / 8; i += THREADS) d[i] = s8[i];
     __syncthreads();
-    xr = reinterpret_cast<const __nv_bfloat16*>(ring_slot(smem, 0));
+    xr = reinterpret_cast<const __nv_bfloat16*>(ring_slot(smem, 0, 0));
   }
   const int HS = p.HS, hpart = H / HS;
   const int nchunk = (T + 7) / 8;
@@ -421,9 +467,8 @@ __device__ void phase_route_small(const EngineParams& p, const LayerPtrs& lp, ui
   const int T = p.T, E = p.E, K = p.K, TK = p.TK;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int t = warp; t < T; t += WARPS) topk_row(p, lp.router_b, t, tb.idx + t * K, tb.w + t * K);
-  for (int t = threadIdx.x; t < T; t += THREADS) tb.pxf[t] = p.pxf[t];
   if (stamp) *stamp = globaltimer_ns();
-  int32_t* hist = reinterpret_cast<int32_t*>(ring_slot(smem, 0));  // [WARPS][E] scratch
+  int32_t* hist = reinterpret_cast<int32_t*>(ring_slot(smem, 0, 0));  // [WARPS][E] scratch
   for (int i = threadIdx.x; i < WARPS * E; i += THREADS) hist[i] = 0;
   __syncthreads();
   const int pr = threadIdx.x;  // TK <= SMALL_PAIRS <= THREADS: one pair per thread
@@ -486,7 +531,7 @@ __device__ void phase_permute_large(const EngineParams& p, uint8_t* smem) {
   if (warp == 0) warp_exclusive_scan(tb.offsets, E, tb.offsets + E);
   __syncthreads();
   if (blockIdx.x == 0) {
-    int32_t* scratch = reinterpret_cast<int32_t*>(ring_slot(smem, 0));
+    int32_t* scratch = reinterpret_cast<int32_t*>(ring_slot(smem, 0, 0));
     build_units(tb.counts, tb.offsets, E, scratch, p.units, p.dunits, &tb.n_units, &tb.n_dunits);
     for (int i = threadIdx.x; i < E; i += THREADS) p.counts[i] = tb.counts[i];
     for (int i = threadIdx.x; i <= E; i += THREADS) p.offsets[i] = tb.offsets[i];
@@ -509,84 +554,54 @@ __device__ void phase_permute_large(const EngineParams& p, uint8_t* smem) {
 }
 
 // ---- phase C: the MXFP4 weight stream on tensor cores --------------------------------------
-// E8M0 byte B of a word -> 2^(byte-127) as fp32; byte 0 gives 2^-127 exactly,
-// byte 255 gives +inf (its blocks hold zero codes, so the product is NaN).
-template <int B>
-__device__ __forceinline__ float e8m0_byte(uint32_t w) {
-  uint32_t bits;
-  if constexpr (B == 3) bits = (w >> 1) & 0x7F800000u;
-  else bits = (w << (23 - 8 * B)) & 0x7F800000u;
-  return __uint_as_float(max(bits, 0x00400000u));
-}
-
-// One K chunk (4 MX blocks) of a 64-row job for this warp:
-//   acc[t][i] += sum over blocks b of 2^s(row, b) [* 2^q(col, b)] * (A_b B_b)
-// A = the chunk's E2M1 codes of tile t as f16 fragments (from the ring slot
-// st), B = the lane's activation fragments bfr[b] (loaded by the caller).
-// Gate/up: the 8 columns are tokens (x in f16, scaled per token).  Down:
-// columns 2j, 2j+1 are the hi and lo f16 halves of pair j's SwiGLU output,
-// scaled per (pair, block) by 2^q, q4 holding this lane's pair's 4 exponents.
-template <bool ISD>
-__device__ __forceinline__ void chunk_mma(const uint8_t* st, int lane, const uint4 (&bfr)[KB],
-                                          uint32_t q4, float (&acc)[4][4]) {
-  const int g = lane >> 2;
-  uint32_t sw0[4], sw1[4];
-#pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    sw0[t] = *reinterpret_cast<const uint32_t*>(st + STAGE_CODE_BYTES + (t * 16 + g) * KB);
-    sw1[t] = *reinterpret_cast<const uint32_t*>(st + STAGE_CODE_BYTES + (t * 16 + g + 8) * KB);
-  }
-#pragma unroll
-  for (int b = 0; b < KB; ++b) {
-    const uint4 qa = *reinterpret_cast<const uint4*>(st + ((b * 2 + 0) * 32 + lane) * 16);
-    const uint4 qb = *reinterpret_cast<const uint4*>(st + ((b * 2 + 1) * 32 + lane) * 16);
-    const uint4 bf = bfr[b];
-    const float qf = ISD ? pow2f((int)(int8_t)((q4 >> (8 * b)) & 0xFFu)) : 1.f;
-    const uint32_t wd[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      uint32_t a0[4], a1[4];
-      e2m1x8_to_f16x2x4(wd[2 * t], a0);
-      e2m1x8_to_f16x2x4(wd[2 * t + 1], a1);
-      float ct[4] = {0.f, 0.f, 0.f, 0.f};
-      mma_f16_16816(ct, a0, bf.x, bf.y);
-      mma_f16_16816(ct, a1, bf.z, bf.w);
-      float f0, f1;
-      if (b == 0) { f0 = e8m0_byte<0>(sw0[t]); f1 = e8m0_byte<0>(sw1[t]); }
-      else if (b == 1) { f0 = e8m0_byte<1>(sw0[t]); f1 = e8m0_byte<1>(sw1[t]); }
-      else if (b == 2) { f0 = e8m0_byte<2>(sw0[t]); f1 = e8m0_byte<2>(sw1[t]); }
-      else { f0 = e8m0_byte<3>(sw0[t]); f1 = e8m0_byte<3>(sw1[t]); }
-      if (ISD) { f0 *= qf; f1 *= qf; }
-      acc[t][0] = fmaf(ct[0], f0, acc[t][0]);
-      acc[t][1] = fmaf(ct[1], f0, acc[t][1]);
-      acc[t][2] = fmaf(ct[2], f1, acc[t][2]);
-      acc[t][3] = fmaf(ct[3], f1, acc[t][3]);
-    }
-  }
-}
-
 struct StreamCtx {
   const int32_t* units;   // gate/up units
   const int32_t* dunits;  // down units
   const int32_t* tokpos;
   const float* wpos;
-  const float* pxf;       // per-token activation scale 2^px
   int n_units, n_dunits;
 };
 
+// Per-thread pipeline positions, continued across layers.
+struct RoleState {
+  uint32_t seq = 0;  // producer: stage sequence number
+  int32_t qk = 0;    // job queue position (every role reads every entry)
+  int32_t wj = 0;    // producer: next work index
+  uint32_t sfc = 0;  // MMA issuer: scale-factor buffer counter
+  uint32_t gcount = 0;  // epilogue warp: gate/up jobs done (amax exchange buffer and phase)
+};
+
+// Bounded wait for queue entry qk; false on timeout or a recorded error.
+__device__ bool wait_entry(const EngineParams& p, JobEntry* en, int32_t qk) {
+  if (*reinterpret_cast<volatile int32_t*>(&en->flag) == qk + 1) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t spins = 0;
+  while (*reinterpret_cast<volatile int32_t*>(&en->flag) != qk + 1) {
+    if ((++spins & 15u) == 0u) {
+      if (error_set(p.sync)) return false;
+      if (globaltimer_ns() - t0 > 2 * p.timeout_ns) { set_error(p.sync, DEV_TIMEOUT_QUEUE, qk); return false; }
+    }
+    __nanosleep(32);
+  }
+  return true;
+}
+
 // Producer warp: jobs -> queue entries -> stages into the ring.  Gate/up jobs
-// (unit, 32-row block of I) come first in unit order, then down jobs (down
-// unit, 64-row block of H); a down job waits until its gate/up unit's
-// SwiGLU output is complete.
+// (unit, 64-row block of I) come first in unit order, then down jobs (down
+// unit, 128-row block of H); a down job waits until its gate/up unit's SwiGLU
+// term images are complete.  A stage is the job's weight stage plus one term
+// image per token (gate/up, from xt) or the unit's consecutive pair images
+// (down, from aimg).
 __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem,
-                                const StreamCtx& cx, uint32_t& seq, int32_t& qk) {
+                                const StreamCtx& cx, int pipe, RoleState& rs) {
   const int lane = threadIdx.x & 31;
-  JobEntry* jq = job_queue(smem);
+  JobEntry* jq = job_queue(smem, pipe);
   uint32_t* ready = p.sync + SY_READY;
-  const int gub = p.I / (STAGE_ROWS / 2), db = p.H / STAGE_ROWS;
+  const int gub = p.I / GU_I_ROWS, db = p.H / JOB_ROWS;
   const int64_t n_gu = (int64_t)cx.n_units * gub, n_all = n_gu + (int64_t)cx.n_dunits * db;
-  const int nc_gu = p.H / KC, nc_d = p.I / KC;
-  const uint32_t seq_start = seq;
+  const int nc_gu = p.H / KS, nc_d = p.I / KS;
+  const uint32_t need = (uint32_t)gub * 4u;  // readiness signals per gate/up unit: 4 warps per job
+  const uint32_t seq_start = rs.seq;
   bool ok = true;
   unsigned long long t_empty = 0, t_ready = 0;
   const unsigned long long t_begin = clock64();
@@ -597,12 +612,12 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
     const int64_t j = __shfl_sync(FULL, next, 0);
     if (j >= n_all || !ok) {
       if (lane == 0) {
-        JobEntry* en = jq + (qk % JQ);
-        en->job = -1; en->s0 = (int32_t)seq; en->nc = 0;
+        JobEntry* en = jq + (rs.qk % JQ);
+        en->job = -1; en->s0 = (int32_t)rs.seq; en->nc = 0;
         __threadfence_block();
-        *reinterpret_cast<volatile int32_t*>(&en->flag) = qk + 1;
+        *reinterpret_cast<volatile int32_t*>(&en->flag) = rs.qk + 1;
       }
-      ++qk;
+      ++rs.qk;
       break;
     }
     if (lane == 0) next = atomicAdd(p.sync + SY_JOBS, 1u);  // prefetch the following job
@@ -613,9 +628,8 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
     const int4 ur = *reinterpret_cast<const int4*>((isD ? cx.dunits : cx.units) + (int64_t)u * 4);
     const int e = ur.x, pos0 = ur.y, nt = ur.z;
     const int nc = isD ? nc_d : nc_gu;
-    if (isD) {  // the down stages read the SwiGLU output: wait for the gate/up unit
+    if (isD) {  // the down stages read the SwiGLU term images: wait for the gate/up unit
       const int gu = ur.w;
-      const uint32_t need = (uint32_t)gub * (uint32_t)cx.units[(int64_t)gu * 4 + 2];
       const unsigned long long tr0 = clock64();
       if (ld_acquire_u32(ready + gu) < need) {
         const uint64_t t0 = globaltimer_ns();
@@ -630,241 +644,255 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
       }
       t_ready += clock64() - tr0;
       if (!ok) continue;  // publishes the end entry
+      fence_proxy_async_global();  // the images were written by generic stores of other CTAs
     }
-    // publish the job (after the readiness acquire, so the consumers' reads of
-    // the SwiGLU output are ordered after it)
     if (lane == 0) {
-      JobEntry* en = jq + (qk % JQ);
-      en->job = (int32_t)j; en->s0 = (int32_t)seq; en->nc = nc; en->unit = u; en->rb = rb;
-      en->isD = isD; en->e = e; en->pos0 = pos0; en->nt = nt;
+      JobEntry* en = jq + (rs.qk % JQ);
+      en->job = (int32_t)j; en->s0 = (int32_t)rs.seq; en->nc = nc; en->unit = u; en->rb = rb;
+      en->isD = isD; en->e = e; en->pos0 = pos0; en->nt = nt; en->wj = rs.wj;
       __threadfence_block();
-      *reinterpret_cast<volatile int32_t*>(&en->flag) = qk + 1;
+      *reinterpret_cast<volatile int32_t*>(&en->flag) = rs.qk + 1;
     }
-    ++qk;
-    const uint8_t* wbase = isD ? lp.w_d + ((int64_t)e * db + rb) * nc * STAGE_W_BYTES
-                               : lp.w_gu + ((int64_t)e * gub + rb) * nc * STAGE_W_BYTES;
-    // Stages are issued in batches: successive 1-D bulk copies issued by one
-    // warp instruction each are serialised, while the copies of one
-    // instruction (one per lane) proceed in parallel.
-    for (int c0 = 0; c0 < nc && ok; c0 += PRODUCER_BATCH) {
+    ++rs.qk;
+    ++rs.wj;
+    const uint8_t* wbase = isD ? lp.w_d + ((int64_t)e * db + rb) * nc * STAGE_A_BYTES
+                               : lp.w_gu + ((int64_t)e * gub + rb) * nc * STAGE_A_BYTES;
+    const int tok = (!isD && lane < nt) ? cx.tokpos[pos0 + lane] : 0;
+    const uint32_t stage_bytes = STAGE_A_BYTES + (uint32_t)nt * IMG_BYTES;
+    // Stages are issued in batches, one stage per lane: successive 1-D bulk
+    // copies issued by one warp instruction each are serialised, while the
+    // copies of one instruction proceed in parallel.  A batch is the run of
+    // consecutive stages whose slots are already free (non-blocking test), so
+    // the ring refills as soon as the MMAs release slots and the batch grows
+    // whenever the producer falls behind.
+    int c0 = 0;
+    while (c0 < nc && ok) {
       const int nb = min(PRODUCER_BATCH, nc - c0);
-      const unsigned long long te0 = clock64();
-      bool bad = false;
-      const uint32_t s = seq + lane;
+      const uint32_t s = rs.seq + lane;
       const int slot = (int)(s % NSLOT);
-      if (lane < nb && s >= (uint32_t)NSLOT)  // wait until the slot is free
-        bad = !wait_mbar(empty_bar(smem, slot), ((s / NSLOT) + 1) & 1u, p.sync, p.timeout_ns,
-                         DEV_TIMEOUT_PIPE, s);
-      if (__any_sync(FULL, bad)) { ok = false; break; }
-      t_empty += clock64() - te0;
-      if (lane < nb) {
-        mbar_arrive_expect_tx(full_bar(smem, slot), STAGE_W_BYTES);
-        bulk_g2s(ring_slot(smem, slot), wbase + (int64_t)(c0 + lane) * STAGE_W_BYTES, STAGE_W_BYTES,
-                 full_bar(smem, slot));
+      const uint32_t par = ((s / NSLOT) + 1) & 1u;  // completion of the slot's previous use
+      const bool fr = lane < nb && (s < (uint32_t)NSLOT || mbar_test_wait(empty_bar(smem, pipe, slot), par));
+      const int k = __ffs(~__ballot_sync(FULL, fr)) - 1;  // leading run of free slots
+      if (k == 0) {
+        const unsigned long long te0 = clock64();
+        bool bad = false;
+        if (lane == 0) bad = !wait_mbar(empty_bar(smem, pipe, slot), par, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, s);
+        t_empty += clock64() - te0;
+        if (__any_sync(FULL, bad)) ok = false;
+        continue;
       }
-      seq += nb;
+      uint8_t* dst = ring_slot(smem, pipe, slot);
+      uint64_t* fb = full_bar(smem, pipe, slot);
+      const int c = c0 + lane;
+      if (lane < k) {
+        mbar_arrive_expect_tx(fb, stage_bytes);
+        bulk_g2s(dst, wbase + (int64_t)c * STAGE_A_BYTES, STAGE_A_BYTES, fb);
+        if (isD)
+          bulk_g2s(dst + STAGE_A_BYTES, p.aimg + ((int64_t)c * p.TK + pos0) * IMG_BYTES,
+                   (uint32_t)nt * IMG_BYTES, fb);
+      }
+      if (!isD) {
+        for (int tl = 0; tl < nt; ++tl) {
+          const int tk = __shfl_sync(FULL, tok, tl);
+          if (lane < k)
+            bulk_g2s(dst + STAGE_A_BYTES + tl * IMG_BYTES, p.xt + ((int64_t)c * p.T + tk) * IMG_BYTES,
+                     IMG_BYTES, fb);
+        }
+      }
+      rs.seq += k;
+      c0 += k;
     }
   }
   if (p.prof && lane == 0) {
     atomicAdd(p.prof + PF_PROD_EMPTY, t_empty);
     atomicAdd(p.prof + PF_PROD_READY, t_ready);
     atomicAdd(p.prof + PF_PROD_TOTAL, clock64() - t_begin);
-    atomicAdd(p.prof + PF_STAGES, (unsigned long long)(seq - seq_start));
+    atomicAdd(p.prof + PF_STAGES, (unsigned long long)(rs.seq - seq_start));
   }
   // let every issued copy land before the ring is reused or the CTA exits
-  const uint32_t issued = seq - seq_start;
+  const uint32_t issued = rs.seq - seq_start;
   const uint32_t n = issued < (uint32_t)NSLOT ? issued : (uint32_t)NSLOT;
-  for (uint32_t s = seq - n; s != seq; ++s) {
+  for (uint32_t s = rs.seq - n; s != rs.seq; ++s) {
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(full_bar(smem, (int)(s % NSLOT)), (s / NSLOT) & 1u)) {
+    while (!mbar_try_wait(full_bar(smem, pipe, (int)(s % NSLOT)), (s / NSLOT) & 1u)) {
       if (globaltimer_ns() - t0 > p.timeout_ns) break;
     }
   }
 }
 
-// Consumer warps: chunks of every job, partial sums, reduction, epilogues.
-__device__ void stream_consumer(const EngineParams& p, uint8_t* smem, const StreamCtx& cx,
-                                int32_t& qk) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int g = lane >> 2, c = lane & 3;
-  JobEntry* jq = job_queue(smem);
-  uint32_t* ready = p.sync + SY_READY;
-  bool poison = false;
+// MMA issuer (one thread): per stage, the weight and activation scale factors
+// go to tensor memory and two block-scaled MMAs (K = 64 each, N = 8 columns
+// per token or pair) accumulate into the job's tensor-memory buffer; the slot
+// is released by a commit when they complete.
+__device__ void stream_mma(const EngineParams& p, uint8_t* smem, uint32_t tmem, int pipe, RoleState& rs) {
+  JobEntry* jq = job_queue(smem, pipe);
+  const uint32_t ring0 = smem_u32(ring_slot(smem, pipe, 0));
   const bool prof = p.prof != nullptr;
-  unsigned long long t_full = 0, t_mma = 0, t_bar = 0, t_epi = 0, t_queue = 0, n_jobs = 0;
-  const unsigned long long t_begin = pclock(prof);
-  // A gate/up epilogue's readiness signal (release fence + counter add) is
-  // deferred until after this warp's next chunk, when its stores have landed
-  // and the fence is cheap; it is flushed at once whenever the warp would wait
-  // for the producer (which may itself wait for that signal).
-  int pend_u = -1;
-  auto flush_ready = [&]() {
-    if (pend_u >= 0) {
-      if (lane == 0) {
-        __threadfence();
-        red_release_add_u32(ready + pend_u, 1u);
-      }
-      pend_u = -1;
-    }
-  };
+  unsigned long long t_full = 0, t_issue = 0, t_acc = 0;
+  bool ok = true;
   for (;;) {
-    JobEntry* en = jq + (qk % JQ);
-    const unsigned long long tq0 = pclock(prof);
-    // the producer publishes the entry (bounded wait; the producer's own waits
-    // are bounded by the same timeout, after which it publishes an end entry)
-    if (*reinterpret_cast<volatile int32_t*>(&en->flag) != qk + 1) {
-      flush_ready();
-      const uint64_t t0 = globaltimer_ns();
-      while (*reinterpret_cast<volatile int32_t*>(&en->flag) != qk + 1) {
-        if (globaltimer_ns() - t0 > 2 * p.timeout_ns) { set_error(p.sync, DEV_TIMEOUT_QUEUE, qk); return; }
-        __nanosleep(32);
-      }
-    }
+    JobEntry* en = jq + (rs.qk % JQ);
+    if (!wait_entry(p, en, rs.qk)) return;
     const int job = *reinterpret_cast<volatile int32_t*>(&en->job);
-    t_queue += pclock(prof) - tq0;
-    if (job < 0) { ++qk; break; }
-    ++n_jobs;
-    const int s0 = en->s0, nc = en->nc, u = en->unit, rb = en->rb, isD = en->isD;
-    const int pos0 = en->pos0, nt = en->nt;
-    const int buf = qk & 1;
-    // order the reads of activations (written by other CTAs, seen through the
-    // producer's acquire) after the queue entry
-    __threadfence_block();
-    // this lane's activation fragments: base address of chunk 0 and the step
-    // between K chunks.  Gate/up: column g is token g (columns >= nt repeat
-    // token 0 and are ignored).  Down: column g is the hi (g even) or lo half
-    // of pair g/2, and the lane's output pair c supplies the block exponents.
-    const uint8_t* fbase;
-    const uint8_t* qbase = nullptr;
-    int64_t cstep;
-    int bstep;
-    if (!isD) {
-      const int tok = cx.tokpos[pos0 + (g < nt ? g : 0)];
-      fbase = p.xh + (int64_t)tok * p.H * 2 + c * 16;
-      cstep = (int64_t)KC * 2;
-      bstep = 64;
-    } else {
-      const int pj = (g >> 1) < nt ? (g >> 1) : 0;
-      fbase = p.a16 + (int64_t)(pos0 + pj) * A16_CHUNK_BYTES + A16_HDR + (g & 1) * 64 + c * 16;
-      qbase = p.a16 + (int64_t)(pos0 + (c < nt ? c : 0)) * A16_CHUNK_BYTES;
-      cstep = (int64_t)p.TK * A16_CHUNK_BYTES;
-      bstep = 128;
+    if (job < 0) { ++rs.qk; break; }
+    const int s0 = en->s0, nc = en->nc, nt = en->nt, wj = en->wj;
+    ++rs.qk;
+    if (!ok) continue;
+    const int b = wj % NACC;
+    const uint32_t use = (uint32_t)(wj / NACC);
+    const unsigned long long ta0 = pclock(prof);
+    if (use > 0 &&
+        !wait_mbar(acce_bar(smem, pipe, b), (use - 1) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, wj)) {
+      ok = false;
+      continue;
     }
-    float acc[4][4];
-#pragma unroll
-    for (int t = 0; t < 4; ++t)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[t][i] = 0.f;
-    uint4 fcur[KB];
-    uint32_t qcur = 0;
-    if (w < nc) {
-#pragma unroll
-      for (int b = 0; b < KB; ++b) fcur[b] = ld_cg_v4(fbase + w * cstep + b * bstep);
-      if (isD) qcur = ld_cg_u32(qbase + w * cstep);
-    }
-    for (int cc = w; cc < nc; cc += NCW) {
-      // fetch the next chunk's fragments while this one computes
-      uint4 fnext[KB];
-      uint32_t qnext = 0;
-      const int cn = cc + NCW < nc ? cc + NCW : cc;
-#pragma unroll
-      for (int b = 0; b < KB; ++b) fnext[b] = ld_cg_v4(fbase + cn * cstep + b * bstep);
-      if (isD) qnext = ld_cg_u32(qbase + cn * cstep);
-      const uint32_t s = (uint32_t)s0 + cc;
+    t_acc += pclock(prof) - ta0;
+    tc_fence_after();
+    const uint32_t tacc = tmem + tm_acc(pipe, b);
+    const uint32_t idesc0 = mxf4_idesc(nt * NTERM, 0u), idesc1 = mxf4_idesc(nt * NTERM, 2u);
+    for (int c = 0; c < nc; ++c) {
+      const uint32_t s = (uint32_t)s0 + c;
       const int slot = (int)(s % NSLOT);
       const unsigned long long tf0 = pclock(prof);
-      if (!poison &&
-          !wait_mbar(full_bar(smem, slot), (s / NSLOT) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, s))
-        poison = true;
+      if (!wait_mbar(full_bar(smem, pipe, slot), (s / NSLOT) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, s)) {
+        ok = false;
+        break;
+      }
       const unsigned long long tm0 = pclock(prof);
       t_full += tm0 - tf0;
-      if (!poison) {
-        const uint8_t* st = ring_slot(smem, slot);
-        if (!isD) chunk_mma<false>(st, lane, fcur, 0u, acc);
-        else chunk_mma<true>(st, lane, fcur, qcur, acc);
-      }
-      t_mma += pclock(prof) - tm0;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty_bar(smem, slot));
-      flush_ready();
-#pragma unroll
-      for (int b = 0; b < KB; ++b) fcur[b] = fnext[b];
-      qcur = qnext;
+      const uint32_t sa = ring0 + (uint32_t)slot * SLOT_BYTES, sb = sa + STAGE_A_BYTES;
+      const uint32_t tsf = tmem + tm_sf(pipe, (int)(rs.sfc++ % NSF));
+      tmem_cp_sf(tsf, smem_desc(sa + STAGE_CODE_BYTES, 0, 128));
+      tmem_cp_sf(tsf + 4, smem_desc(sb + IMG_CODE_BYTES, 0, IMG_BYTES));
+      mma_mxf4(tacc, smem_desc(sa, 128, 256), smem_desc(sb, 128, IMG_BYTES), idesc0, tsf, tsf + 4,
+               c > 0 ? 1u : 0u);
+      mma_mxf4(tacc, smem_desc(sa + 4096, 128, 256), smem_desc(sb + 256, 128, IMG_BYTES), idesc1,
+               tsf | (2u << 30), (tsf + 4) | (2u << 30), 1u);
+      tc_commit(empty_bar(smem, pipe, slot));
+      t_issue += pclock(prof) - tm0;
     }
-    // deposit this warp's partial sums: part[w][col][row]
-    float* pb = part_buf(smem, buf) + (size_t)w * PART_COLS * PART_LD;
-    if (w < nc) {
-#pragma unroll
-      for (int t = 0; t < 4; ++t)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) pb[(2 * c + (i & 1)) * PART_LD + t * 16 + g + (i >> 1) * 8] = acc[t][i];
-    }
-    const unsigned long long tb0 = pclock(prof);
-    named_barrier(1 + buf, NCW * 32);
-    const unsigned long long te0 = pclock(prof);
-    t_bar += te0 - tb0;
-    const int nw = nc < NCW ? nc : NCW;
-    const float* pall = part_buf(smem, buf);
-    // the epilogue of column j runs on warp (j + qk) % NCW: the duty rotates
-    const int j = (w + NCW - (qk % NCW)) % NCW;
-    if (!poison && j < nt) {
-      if (!isD) {  // gate/up epilogue: token column j, lane = intermediate row i0 + lane
-        const float px = cx.pxf[cx.tokpos[pos0 + j]];
-        float gs = 0.f, us = 0.f;
-        for (int ww = 0; ww < nw; ++ww) {
-          gs += pall[((size_t)ww * PART_COLS + j) * PART_LD + lane];
-          us += pall[((size_t)ww * PART_COLS + j) * PART_LD + 32 + lane];
-        }
-        const float gv = gs * px, uv = us * px;
-        const float a = gv / (1.0f + expf(-gv)) * uv;
-        float am = fabsf(a);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(FULL, am, o));
-        const int eb = (int)((__float_as_uint(am) >> 23) & 0xFF);
-        int q = am > 0.f ? eb - 127 - 14 : 0;
-        q = max(q, -126);
-        const float v = a * pow2f(-q);
-        const __half hi = __float2half_rn(v);
-        const __half lo = __float2half_rn(v - __half2float(hi));
-        const int i0 = rb * (STAGE_ROWS / 2);
-        uint8_t* base = p.a16 + ((int64_t)(i0 / KC) * p.TK + pos0 + j) * A16_CHUNK_BYTES;
-        const int bi = (i0 % KC) / 32;
-        const int kk = lane & 15;
-        const int off = A16_HDR + bi * 128 + ((kk & 7) >> 1) * 16 +
-                        ((lane >> 4) * 4 + ((kk >> 3) << 1) + (kk & 1)) * 2;
-        *reinterpret_cast<__half*>(base + off) = hi;
-        *reinterpret_cast<__half*>(base + off + 64) = lo;
-        if (lane == 0) base[bi] = (uint8_t)(int8_t)q;
-        __syncwarp();
-        flush_ready();  // a previous job's signal, if still pending
-        pend_u = u;
-      } else {  // down epilogue: pair j, lane = rows h0 + lane and h0 + 32 + lane
-        const float wp = cx.wpos[pos0 + j];
-        const int h0 = rb * STAGE_ROWS;
-#pragma unroll
-        for (int r2 = 0; r2 < 2; ++r2) {
-          const int r = lane + 32 * r2;
-          float y = 0.f;
-          for (int ww = 0; ww < nw; ++ww) {
-            const float* pw = pall + (size_t)ww * PART_COLS * PART_LD;
-            y += pw[(2 * j) * PART_LD + r] + pw[(2 * j + 1) * PART_LD + r];
-          }
-          p.ypair[(int64_t)(pos0 + j) * p.H + h0 + r] = y * wp;
-        }
-      }
-    }
-    t_epi += pclock(prof) - te0;
-    ++qk;
+    if (ok) tc_commit(accf_bar(smem, pipe, b));
   }
-  flush_ready();
-  if (p.prof && lane == 0) {
-    atomicAdd(p.prof + PF_CONS_FULL, t_full);
-    atomicAdd(p.prof + PF_CONS_MMA, t_mma);
-    atomicAdd(p.prof + PF_CONS_BAR, t_bar);
-    atomicAdd(p.prof + PF_CONS_EPI, t_epi);
-    atomicAdd(p.prof + PF_CONS_QUEUE, t_queue);
-    atomicAdd(p.prof + PF_CONS_TOTAL, pclock(prof) - t_begin);
-    atomicAdd(p.prof + PF_JOBS, n_jobs);
+  if (prof) {
+    atomicAdd(p.prof + PF_MMA_FULL, t_full);
+    atomicAdd(p.prof + PF_MMA_ISSUE, t_issue);
+    atomicAdd(p.prof + PF_MMA_ACC, t_acc);
+  }
+}
+
+// Epilogue of pipeline `pipe` (four warps, warp q = warp % 4 reading
+// tensor-memory lanes 32q..32q+31).
+//   gate/up: lane l of warp q holds gate (l < 16) or up (l >= 16) of
+//     intermediate row i0 + 16 q + l % 16 for every token column group;
+//     a = silu(g) u, then its E2M1 term image (block amax shared by warps q,
+//     q ^ 1 through shared memory) goes to aimg and the unit's readiness
+//     counter is incremented once per warp.
+//   down: row h0 + 32 q + l of every pair, times the routing weight -> ypair.
+__device__ void stream_epilogue(const EngineParams& p, uint8_t* smem, const StreamCtx& cx,
+                                uint32_t tmem, int pipe, RoleState& rs) {
+  const int lane = threadIdx.x & 31, q = (threadIdx.x >> 5) & 3;
+  JobEntry* jq = job_queue(smem, pipe);
+  uint32_t* ready = p.sync + SY_READY;
+  const bool prof = p.prof != nullptr;
+  unsigned long long t_wait = 0, t_work = 0, n_jobs = 0;
+  const unsigned long long t_begin = pclock(prof);
+  bool ok = true;
+  for (;;) {
+    JobEntry* en = jq + (rs.qk % JQ);
+    if (!wait_entry(p, en, rs.qk)) return;
+    const int job = *reinterpret_cast<volatile int32_t*>(&en->job);
+    if (job < 0) { ++rs.qk; break; }
+    const int wj = en->wj;
+    const int u = en->unit, rb = en->rb, isD = en->isD, pos0 = en->pos0, nt = en->nt;
+    ++rs.qk;
+    if (!ok) continue;
+    ++n_jobs;
+    const uint32_t gc = isD ? 0u : rs.gcount++;
+    const int b = wj % NACC;
+    const unsigned long long tw0 = pclock(prof);
+    if (!wait_mbar(accf_bar(smem, pipe, b), (uint32_t)(wj / NACC) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, wj)) {
+      ok = false;
+      continue;
+    }
+    const unsigned long long tk0 = pclock(prof);
+    t_wait += tk0 - tw0;
+    tc_fence_after();
+    const uint32_t tacc = tmem + ((uint32_t)(32 * q) << 16) + tm_acc(pipe, b);
+    if (!isD) {
+      float av[NT_MAX];
+      // block amax of warps q and q ^ 1 meet in shared memory; the exchange
+      // buffer alternates so that a warp one job ahead cannot overwrite it
+      const int xb = (int)(gc & 1u);
+      float* xc = xch_buf(smem, pipe, xb);
+#pragma unroll
+      for (int j = 0; j < NT_MAX; ++j) {
+        av[j] = 0.f;
+        if (j < nt) {
+          float v[NTERM];
+          tmem_ld8(tacc + j * NTERM, v);
+          float sum = v[NTERM - 1];
+#pragma unroll
+          for (int k = NTERM - 2; k >= 0; --k) sum += v[k];
+          const float other = __shfl_xor_sync(FULL, sum, 16);
+          const float g = lane < 16 ? sum : other, up = lane < 16 ? other : sum;
+          const float a = g / (1.0f + expf(-g)) * up;
+          av[j] = a;
+          float am = fabsf(a);
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(FULL, am, o));
+          if (lane == 0) xc[j * 4 + q] = am;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xch_bar(smem, pipe, xb));
+      if (!wait_mbar(xch_bar(smem, pipe, xb), (gc >> 1) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, wj)) {
+        ok = false;
+        continue;
+      }
+      const int i0 = rb * GU_I_ROWS, sD = i0 / KS, kk = (i0 % KS) / 64, kc = q >> 1;
+#pragma unroll
+      for (int j = 0; j < NT_MAX; ++j) {
+        if (j < nt) {
+          const int s0 = term0_exp(fmaxf(xc[j * 4 + q], xc[j * 4 + (q ^ 1)]));
+          const uint32_t word = term_word<16>(e2m1_terms(av[j], s0), lane);
+          uint8_t* img = p.aimg + ((int64_t)sD * p.TK + pos0 + j) * IMG_BYTES;
+          if (lane < 16)
+            *reinterpret_cast<uint32_t*>(img + kk * 256 + kc * 128 + (lane >> 1) * 16 + (q & 1) * 8 +
+                                         (lane & 1) * 4) = word;
+          if ((q & 1) == 0 && lane < NTERM)
+            img[IMG_CODE_BYTES + lane * 16 + 2 * kk + kc] = (uint8_t)(term_exp(s0, lane) + 127);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        fence_proxy_async_global();
+        __threadfence();
+        red_release_add_u32(ready + u, 1u);
+      }
+    } else {
+      const int h0 = rb * JOB_ROWS;
+#pragma unroll
+      for (int j = 0; j < ND_MAX; ++j) {
+        if (j < nt) {
+          float v[NTERM];
+          tmem_ld8(tacc + j * NTERM, v);
+          float sum = v[NTERM - 1];
+#pragma unroll
+          for (int k = NTERM - 2; k >= 0; --k) sum += v[k];
+          p.ypair[(int64_t)(pos0 + j) * p.H + h0 + 32 * q + lane] = sum * cx.wpos[pos0 + j];
+        }
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(acce_bar(smem, pipe, b));
+    t_work += pclock(prof) - tk0;
+  }
+  if (prof && lane == 0) {
+    atomicAdd(p.prof + PF_EPI_WAIT, t_wait);
+    atomicAdd(p.prof + PF_EPI_WORK, t_work);
+    atomicAdd(p.prof + PF_EPI_TOTAL, pclock(prof) - t_begin);
+    if (q == 0) atomicAdd(p.prof + PF_JOBS, n_jobs);
   }
 }
 
@@ -941,22 +969,11 @@ __device__ void phase_combine_rmsnorm(const EngineParams& p, const int32_t* inv,
   }
 }
 
-__global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int warp = threadIdx.x >> 5;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < NSLOT; ++i) {
-      mbar_init(full_bar(smem, i), 1);
-      mbar_init(empty_bar(smem, i), 1);
-    }
-    fence_mbar_init();
-  }
-  for (int i = threadIdx.x; i < JQ; i += THREADS) job_queue(smem)[i].flag = 0;
-  __syncthreads();
-  const bool stamp = p.stamps != nullptr && blockIdx.x == 0 && threadIdx.x == 0;
-  if (stamp) p.stamps[0] = globaltimer_ns();
-  uint32_t seq = 0;   // stage sequence (producer), continues across layers
-  int32_t qk = 0;     // job queue position, continues across layers
+// All layers; returns early (every thread of the CTA together) when a grid
+// barrier reports an error, or after routing in route-only mode.
+__device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, RoleState& rs,
+                           bool stamp) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool small = p.TK <= SMALL_PAIRS;
   CtaTables& tb = tables(smem);
   for (int layer = 0; layer < p.L; ++layer) {
@@ -970,7 +987,7 @@ __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p
     const int32_t* inv;
     if (small) {
       phase_route_small(p, lp, smem, st ? st + 3 : nullptr);
-      cx = StreamCtx{tb.units, tb.dunits, tb.tokpos, tb.wpos, tb.pxf, tb.n_units, tb.n_dunits};
+      cx = StreamCtx{tb.units, tb.dunits, tb.tokpos, tb.wpos, tb.n_units, tb.n_dunits};
       inv = tb.inv;
       if (p.route_only) return;
     } else {
@@ -980,14 +997,23 @@ __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p
       phase_permute_large(p, smem);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 3)) return;
       if (p.route_only) return;
-      cx = StreamCtx{p.units, p.dunits, p.tokpos, p.wpos, p.pxf, p.n_units[0], p.n_units[1]};
+      cx = StreamCtx{p.units, p.dunits, p.tokpos, p.wpos, p.n_units[0], p.n_units[1]};
       inv = p.inv;
     }
     if (st) st[4] = globaltimer_ns();
     fence_proxy_async_smem();  // the ring held routing scratch written by generic stores
     __syncthreads();
-    if (warp == NCW) stream_producer(p, lp, smem, cx, seq, qk);
-    else stream_consumer(p, smem, cx, qk);
+    if (warp < EPI_WARP0) {
+      const int pipe = warp >> 1;
+      if ((warp & 1) == 0) {
+        stream_producer(p, lp, smem, cx, pipe, rs);
+      } else {
+        if (lane == 0) stream_mma(p, smem, tmem, pipe, rs);
+        __syncwarp();
+      }
+    } else {
+      stream_epilogue(p, smem, cx, tmem, (warp - EPI_WARP0) / 4, rs);
+    }
     if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 4)) return;
     if (st) st[5] = globaltimer_ns();
     if (layer + 1 < p.L) {
@@ -997,6 +1023,56 @@ __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p
       phase_combine_out(p, inv);
     }
     if (st) st[6] = globaltimer_ns();
+  }
+}
+
+__global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int pp = 0; pp < NPIPE; ++pp) {
+      for (int i = 0; i < NSLOT; ++i) {
+        mbar_init(full_bar(smem, pp, i), 1);
+        mbar_init(empty_bar(smem, pp, i), 1);
+      }
+      for (int i = 0; i < NACC; ++i) {
+        mbar_init(accf_bar(smem, pp, i), 1);
+        mbar_init(acce_bar(smem, pp, i), 4);
+      }
+      for (int i = 0; i < 2; ++i) mbar_init(xch_bar(smem, pp, i), 4);
+      mbar_init(drain_bar(smem, pp), 1);
+    }
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < NPIPE * JQ; i += THREADS) job_queue(smem, 0)[i].flag = 0;
+  const bool use_tmem = !p.route_only;
+  if (use_tmem && warp == 1) {
+    tmem_alloc(tmem_base_word(smem), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = use_tmem ? *tmem_base_word(smem) : 0u;
+  const bool stamp = p.stamps != nullptr && blockIdx.x == 0 && threadIdx.x == 0;
+  if (stamp) p.stamps[0] = globaltimer_ns();
+  RoleState rs;
+  run_layers(p, smem, tmem, rs, stamp);
+  if (use_tmem) {
+    // free tensor memory only once every MMA this CTA issued has completed
+    if (warp < EPI_WARP0 && (warp & 1) && lane == 0) {
+      uint64_t* db = drain_bar(smem, warp >> 1);
+      tc_commit(db);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(db, 0u)) {
+        if (globaltimer_ns() - t0 > p.timeout_ns) { set_error(p.sync, DEV_TIMEOUT_PIPE, 0xFFFFu); break; }
+      }
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 

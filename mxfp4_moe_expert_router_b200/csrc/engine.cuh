@@ -8,39 +8,60 @@
 namespace moe {
 
 // ---- streaming layout -------------------------------------------------------------
-// The weight stream is cut into jobs of 64 weight rows x the whole contraction
-// dimension: a gate/up job holds 32 gate rows and the same 32 up rows of one
-// expert (one 32-row block of the intermediate dimension), a down job 64 rows
-// of Wd.  A job is streamed in stages of KC = 128 K elements (four MX blocks);
-// the stage layout (see quantize.cu) is the mma.m16n8k16 A-fragment order, so
-// a lane turns its 16 bytes per half-stage straight into f16 fragments.
-constexpr int KC = 128;                                  // K elements per stage
-constexpr int KB = KC / 32;                              // MX blocks per stage
-constexpr int STAGE_ROWS = 64;                           // weight rows per stage
-constexpr int STAGE_CODE_BYTES = STAGE_ROWS * KC / 2;    // 4096
-constexpr int STAGE_W_BYTES = STAGE_CODE_BYTES + STAGE_ROWS * KB;  // 4352
-constexpr int NT_MAX = 8;                                // tokens per gate/up unit (one MMA n-tile)
-constexpr int ND_MAX = 4;                                // pairs per down unit (hi+lo: one n-tile)
-// activations of one K chunk, per (token, expert) pair of the down projection:
-// 4 block exponents q (padded to 16 bytes), then the hi and lo f16 halves of
-// the SwiGLU output in fragment order.  Consumer lanes read activation
-// fragments straight from L2; the ring carries weight stages only.
-constexpr int A16_HDR = 16;
-constexpr int A16_CHUNK_BYTES = A16_HDR + KC * 2 * 2;    // 528
-constexpr int SLOT_BYTES = STAGE_W_BYTES;                // 4352
+// The weight stream is cut into jobs of 128 weight rows (the M of one
+// block-scaled tensor-core MMA) x the whole contraction dimension: a gate/up
+// job holds 64 gate rows and the same 64 up rows of one expert, a down job 128
+// rows of Wd.  A job is streamed in stages of KS = 128 K elements (four MX
+// blocks).  A stage is laid out exactly as the MMA reads it from shared
+// memory: E2M1 codes as K-major 8-row x 16-byte core matrices (two MMAs of
+// K = 64), then the E8M0 scales in the scale-factor copy layout (row m at byte
+// (m % 32) * 16 + (m / 32) * 4 + block).  Row m of a gate/up job is, with
+// q = m / 32 and l = m % 32, gate (l < 16) or up (l >= 16) of intermediate row
+// 16 q + (l % 16), so that both halves of a SwiGLU meet in one warp.
+constexpr int KS = 128;                                  // K elements per stage
+constexpr int KB = KS / 32;                              // MX blocks per stage
+constexpr int JOB_ROWS = 128;                            // weight rows per job
+constexpr int GU_I_ROWS = JOB_ROWS / 2;                  // intermediate rows per gate/up job
+constexpr int STAGE_CODE_BYTES = JOB_ROWS * KS / 2;      // 8192
+constexpr int STAGE_A_BYTES = STAGE_CODE_BYTES + JOB_ROWS * KB;  // 8704
+// Activations enter the MMA as B operands: each column group (a token of a
+// gate/up unit, a (token, expert) pair of a down unit) is 8 MMA columns, the
+// terms v = sum_k c_k 2^s_k (c_k E2M1, one E8M0 exponent per term and block)
+// of an exact E2M1 expansion.  Per stage and group: 8 rows x 64 bytes of codes
+// (two K = 64 halves of 2 x 16-byte chunks) and 8 rows x 16 bytes of scales
+// (bytes 0..3 = the four blocks, 4..15 zero).
+constexpr int NTERM = 8;
+constexpr int IMG_CODE_BYTES = NTERM * KS / 2;           // 512
+constexpr int IMG_BYTES = IMG_CODE_BYTES + NTERM * 16;   // 640
+constexpr int NT_MAX = 4;                                // tokens per gate/up unit (N <= 32)
+constexpr int ND_MAX = 4;                                // pairs per down unit
+constexpr int SLOT_BYTES = STAGE_A_BYTES + NT_MAX * IMG_BYTES;  // 11264
 constexpr int MAX_HSPLIT = 8;                            // router dot products split along H
 
 constexpr int MAX_LAYERS = 16;
 constexpr int MAX_EXPERTS = 512;
-constexpr int NCW = 8;                                   // consumer (MMA) warps per CTA
-constexpr int WARPS = NCW + 1;                           // + one producer warp
+// The weight stream runs as NPIPE independent pipelines per CTA, each with its
+// own job queue, stage ring, tensor-memory accumulators and roles: warp 2p is
+// pipeline p's producer, warp 2p + 1 its MMA issuer, warps 4 + 4p .. 7 + 4p its
+// epilogue (one warp per 32-lane tensor-memory sub-partition).  A single
+// thread issues tcgen05 instructions at a few hundred cycles per stage, so two
+// issuers are needed to keep up with HBM.
+constexpr int NPIPE = 2;
+constexpr int WARPS = 12;
 constexpr int THREADS = WARPS * 32;
-constexpr int NSLOT = 40;                                // stage ring slots per CTA
-constexpr int PRODUCER_BATCH = 16;                       // stages per bulk-copy instruction
-constexpr int JQ = 32;                                   // job queue entries per CTA
-constexpr int PART_LD = 68;                              // partial-sum column stride (floats)
-constexpr int PART_COLS = 8;                             // one n-tile
-constexpr int SMALL_PAIRS = 256;                         // T*k up to this: routing done per CTA
+constexpr int EPI_WARP0 = 4;
+constexpr int NSLOT = 9;                                 // stage ring slots per pipeline
+constexpr int PRODUCER_BATCH = 8;                        // most stages per bulk-copy round
+constexpr int JQ = 32;                                   // job queue entries per pipeline
+constexpr int NACC = 2;                                  // accumulator buffers per pipeline
+constexpr int ACC_COLS = NT_MAX * NTERM;                 // 32 columns per buffer
+constexpr int NSF = 4;                                   // scale-factor buffers per pipeline
+constexpr int SF_COLS = 8;                               // A (4 columns) + B (4 columns)
+constexpr int TMEM_COLS = 256;
+static_assert(NPIPE * (NACC * ACC_COLS + NSF * SF_COLS) <= TMEM_COLS, "tensor memory budget");
+// a batch's stages must occupy distinct slots whose previous use is already issued
+static_assert(PRODUCER_BATCH <= NSLOT && PRODUCER_BATCH < 32, "producer batch");
+constexpr int SMALL_PAIRS = 256;                         // T*K up to this: routing done per CTA
 constexpr int STAMPS_PER_LAYER = 7;  // x converted, logits (CTA 0), prepared, top-k, routed, streamed, combined
 
 // sync word layout (uint32)
@@ -58,22 +79,22 @@ enum : uint32_t {
 __host__ __device__ inline int max_units(int E, int64_t TK) { return (int)((E < TK ? E : TK) + TK / NT_MAX + 1); }
 __host__ __device__ inline int max_dunits(int E, int64_t TK) { return (int)((E < TK ? E : TK) + TK / ND_MAX + 1); }
 
-// Router split of H: about 1024 elements per part, each part a multiple of KC.
+// Router split of H: about 1024 elements per part, each part a multiple of KS.
 inline int router_hsplit(int H) {
   int hs = H % 1024 == 0 ? H / 1024 : 1;
-  return hs > MAX_HSPLIT ? (H % (MAX_HSPLIT * KC) == 0 ? MAX_HSPLIT : 1) : hs;
+  return hs > MAX_HSPLIT ? (H % (MAX_HSPLIT * KS) == 0 ? MAX_HSPLIT : 1) : hs;
 }
 
 struct LayerPtrs {
-  const uint8_t* w_gu;  // gate/up stages  [E][I/32][H/KC][STAGE_W_BYTES]
-  const uint8_t* w_d;   // down stages     [E][H/64][I/KC][STAGE_W_BYTES]
+  const uint8_t* w_gu;  // gate/up stages  [E][I/64][H/KS][STAGE_A_BYTES]
+  const uint8_t* w_d;   // down stages     [E][H/128][I/KS][STAGE_A_BYTES]
   const float* router_w;  // [E][H]
   const float* router_b;  // [E] or null
 };
 
 struct EngineParams {
   int H, I, E, K, T, TK, L;  // hidden, inter, experts, top_k, tokens, T*K, layers to run
-  int HS;                    // router H split (H/HS a multiple of KC)
+  int HS;                    // router H split (H/HS a multiple of KS)
   int route_only;            // 1: stop after routing of layer 0, export maps
   float rms_eps;
   uint64_t timeout_ns;
@@ -83,8 +104,7 @@ struct EngineParams {
   __nv_bfloat16* layer_io;    // null or [L+1][T][H]
   // workspace (handle-owned)
   double* logits;             // [HS][T][E] partial logits
-  uint8_t* xh;                // [T][H] f16, fragment order within 32-blocks
-  float* pxf;                 // [T] power-of-two scale of each token's xh
+  uint8_t* xt;                // [H/KS][T][IMG_BYTES] E2M1 term images of x
   __nv_bfloat16* xnext;       // [T][H]
   int32_t* idx;               // [TK]
   float* wts;                 // [TK]
@@ -94,20 +114,21 @@ struct EngineParams {
   int32_t* inv;               // [TK]
   int32_t* tokpos;            // [TK] token of each permuted position
   float* wpos;                // [TK] routing weight of each permuted position
-  int32_t* units;             // [Umax][4] gate/up units (expert, pos0, nt <= 8, 0)
-  int32_t* dunits;            // [Dmax][4] down units (expert, pos0, nt <= 4, gate/up unit)
+  int32_t* units;             // [Umax][4] gate/up units (expert, pos0, nt <= NT_MAX, 0)
+  int32_t* dunits;            // [Dmax][4] down units (expert, pos0, nt <= ND_MAX, gate/up unit)
   int32_t* n_units;           // [2] gate/up units, down units
-  uint8_t* a16;               // [I/KC][TK][A16_CHUNK_BYTES]  SwiGLU output, hi/lo f16
+  uint8_t* aimg;              // [I/KS][TK][IMG_BYTES] E2M1 term images of the SwiGLU output
   float* ypair;               // [TK][H]
   uint32_t* sync;             // see SY_*
   uint64_t* stamps;           // null or [1 + MAX_LAYERS * STAMPS_PER_LAYER] %globaltimer ns (CTA 0)
   unsigned long long* prof;   // null or [PROF_COUNTERS] summed SM-clock cycles (stream phase)
 };
 
-// stream-phase profile counters (cycles summed over CTAs / warps)
+// stream-phase profile counters (SM-clock cycles summed over CTAs; the
+// epilogue ones also over its 8 warps)
 enum : int {
   PF_PROD_EMPTY = 0, PF_PROD_READY, PF_PROD_TOTAL, PF_STAGES,
-  PF_CONS_FULL, PF_CONS_MMA, PF_CONS_BAR, PF_CONS_EPI, PF_CONS_QUEUE, PF_CONS_TOTAL, PF_JOBS,
+  PF_MMA_FULL, PF_MMA_ISSUE, PF_MMA_ACC, PF_EPI_WAIT, PF_EPI_WORK, PF_EPI_TOTAL, PF_JOBS,
   PROF_COUNTERS
 };
 
@@ -117,7 +138,8 @@ int engine_max_grid(int device, int* err);
 
 cudaError_t quantize_launch(const void* w, int64_t rows, int64_t K, uint8_t* codes,
                             uint8_t* scales, cudaStream_t s);
-// Repack canonical codes [E][N][K/2] + scales [E][N][K/32] into streaming stages.
+// Repack canonical codes [E][N][K/2] + scales [E][N][K/32] into streaming stages
+// (rows must be a multiple of 64 for gate/up, 128 for down; K a multiple of KS).
 cudaError_t repack_gu_launch(const uint8_t* gc, const uint8_t* gs, const uint8_t* uc,
                              const uint8_t* us, int E, int I, int H, uint8_t* out, cudaStream_t s);
 cudaError_t repack_d_launch(const uint8_t* dc, const uint8_t* ds, int E, int H, int I,

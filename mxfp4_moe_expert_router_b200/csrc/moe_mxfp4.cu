@@ -23,9 +23,8 @@ struct moe_mxfp4 {
   float* router_w[MAX_LAYERS] = {};
   float* router_b[MAX_LAYERS] = {};
   double* logits = nullptr;
-  uint8_t* xh = nullptr;
-  float* pxf = nullptr;
-  uint8_t* a16 = nullptr;
+  uint8_t* xt = nullptr;
+  uint8_t* aimg = nullptr;
   __nv_bfloat16* xnext = nullptr;
   int32_t *idx = nullptr, *counts = nullptr, *offsets = nullptr, *perm = nullptr, *inv = nullptr,
           *tokpos = nullptr, *units = nullptr, *dunits = nullptr, *n_units = nullptr;
@@ -57,10 +56,10 @@ void free_all(moe_mxfp4* h) {
 }
 
 size_t stage_bytes_gu(const moe_config_t& c) {
-  return (size_t)c.num_experts * (c.inter / (STAGE_ROWS / 2)) * (c.hidden / KC) * STAGE_W_BYTES;
+  return (size_t)c.num_experts * (c.inter / GU_I_ROWS) * (c.hidden / KS) * STAGE_A_BYTES;
 }
 size_t stage_bytes_d(const moe_config_t& c) {
-  return (size_t)c.num_experts * (c.hidden / STAGE_ROWS) * (c.inter / KC) * STAGE_W_BYTES;
+  return (size_t)c.num_experts * (c.hidden / JOB_ROWS) * (c.inter / KS) * STAGE_A_BYTES;
 }
 
 int32_t validate_cfg(const moe_config_t* c) {
@@ -69,7 +68,7 @@ int32_t validate_cfg(const moe_config_t* c) {
       c->max_tokens <= 0 || c->num_layers <= 0 || c->top_k > c->num_experts ||
       !(c->rms_eps >= 0.f))
     return MOE_ERR_INVALID_ARG;
-  if (c->hidden % KC || c->inter % KC || c->hidden > 8192 || c->num_experts > MAX_EXPERTS ||
+  if (c->hidden % KS || c->inter % KS || c->hidden > 8192 || c->num_experts > MAX_EXPERTS ||
       c->top_k > 32 || c->num_layers > MAX_LAYERS)
     return MOE_ERR_UNSUPPORTED_SHAPE;
   if ((int64_t)c->max_tokens * c->top_k > (int64_t)1 << 28) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -85,10 +84,10 @@ EngineParams base_params(const moe_mxfp4* h, int T) {
   p.timeout_ns = h->timeout_ns;
   for (int l = 0; l < h->cfg.num_layers; ++l)
     p.layers[l] = LayerPtrs{h->w_gu[l], h->w_d[l], h->router_w[l], h->router_b[l]};
-  p.logits = h->logits; p.xh = h->xh; p.pxf = h->pxf; p.xnext = h->xnext;
+  p.logits = h->logits; p.xt = h->xt; p.xnext = h->xnext;
   p.idx = h->idx; p.wts = h->wts; p.counts = h->counts; p.offsets = h->offsets;
   p.perm = h->perm; p.inv = h->inv; p.tokpos = h->tokpos; p.wpos = h->wpos;
-  p.units = h->units; p.dunits = h->dunits; p.n_units = h->n_units; p.a16 = h->a16;
+  p.units = h->units; p.dunits = h->dunits; p.n_units = h->n_units; p.aimg = h->aimg;
   p.ypair = h->ypair;
   p.sync = h->sync;
   p.stamps = h->stamps;
@@ -178,8 +177,7 @@ int32_t moe_mxfp4_create(const moe_config_t* cfg, const uint8_t* const* gate_cod
     if (ok && router_bias && router_bias[l]) ok = dalloc(h, &h->router_b[l], (size_t)E * 4);
   }
   const int HS = router_hsplit(H);
-  ok = ok && dalloc(h, &h->logits, (size_t)HS * Tm * E * 8) && dalloc(h, &h->xh, (size_t)Tm * H * 2) &&
-       dalloc(h, &h->pxf, (size_t)Tm * 4) &&
+  ok = ok && dalloc(h, &h->logits, (size_t)HS * Tm * E * 8) && dalloc(h, &h->xt, (size_t)(H / KS) * Tm * IMG_BYTES) &&
        dalloc(h, &h->xnext, (size_t)Tm * H * 2) && dalloc(h, &h->idx, (size_t)TKm * 4) &&
        dalloc(h, &h->wts, (size_t)TKm * 4) && dalloc(h, &h->counts, (size_t)E * 4) &&
        dalloc(h, &h->offsets, (size_t)(E + 1) * 4) && dalloc(h, &h->perm, (size_t)TKm * 4) &&
@@ -187,7 +185,7 @@ int32_t moe_mxfp4_create(const moe_config_t* cfg, const uint8_t* const* gate_cod
        dalloc(h, &h->wpos, (size_t)TKm * 4) && dalloc(h, &h->units, (size_t)h->umax * 16) &&
        dalloc(h, &h->dunits, (size_t)dmax * 16) &&
        dalloc(h, &h->n_units, 16) &&
-       dalloc(h, &h->a16, (size_t)(I / KC) * TKm * A16_CHUNK_BYTES) &&
+       dalloc(h, &h->aimg, (size_t)(I / KS) * TKm * IMG_BYTES) &&
        dalloc(h, &h->ypair, (size_t)TKm * H * 4) &&
        dalloc(h, &h->sync, (size_t)(SY_READY + h->umax) * 4) &&
        dalloc(h, &h->stamps, (size_t)(1 + MAX_LAYERS * STAMPS_PER_LAYER) * 8) &&
@@ -195,7 +193,11 @@ int32_t moe_mxfp4_create(const moe_config_t* cfg, const uint8_t* const* gate_cod
        dalloc(h, &h->x_stage, (size_t)Tm * H * 2) && dalloc(h, &h->y_stage, (size_t)Tm * H * 2);
   if (!ok) { free_all(h); delete h; cudaGetLastError(); return MOE_ERR_OOM; }
 
+  // term images: the scale rows' padding bytes 4..15 are read by the
+  // scale-factor copies and must stay zero; the kernels never write them
   cudaError_t e = cudaMemsetAsync(h->sync, 0, (size_t)(SY_READY + h->umax) * 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->xt, 0, (size_t)(H / KS) * Tm * IMG_BYTES, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->aimg, 0, (size_t)(I / KS) * TKm * IMG_BYTES, s);
   for (int l = 0; l < L && e == cudaSuccess; ++l) {
     e = repack_gu_launch(gate_codes[l], gate_scales[l], up_codes[l], up_scales[l], E, I, H,
                          h->w_gu[l], s);

@@ -8,7 +8,7 @@
 // moe_route needs a handle, and moe_mxfp4_create allocates.
 //
 // The working memory the routing kernel needs beyond its inputs and outputs
-// (fp64 logits, fp32 activations, the unit table, barrier and status words)
+// (fp64 partial logits, the unit table, barrier and status words)
 // lives in one file-scope __device__ array of MOE_ROUTE_STATIC_SCRATCH_BYTES.
 // Every device that loads this library holds that array until the process
 // exits.  All calls share it: two calls whose kernels overlap on the GPU (on
@@ -37,7 +37,7 @@ int g_grid[kMaxDevices] = {};
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Layout {
-  size_t logits, xh, pxf, units, dunits, n_units, tokpos, wpos, sync, total;
+  size_t logits, units, dunits, n_units, tokpos, wpos, sync, total;
   int umax;
 };
 
@@ -49,8 +49,6 @@ Layout layout_for(int T, int H, int E, int K) {
   size_t o = 0;
   l.sync = o;    o = align256(o + (size_t)(SY_READY + l.umax) * 4);
   l.logits = o;  o = align256(o + (size_t)router_hsplit(H) * T * E * 8);
-  l.xh = o;      o = align256(o + (size_t)T * H * 2);
-  l.pxf = o;     o = align256(o + (size_t)T * 4);
   l.units = o;   o = align256(o + (size_t)l.umax * 16);
   l.dunits = o;  o = align256(o + (size_t)max_dunits(E, TK) * 16);
   l.n_units = o; o = align256(o + 16);
@@ -96,7 +94,7 @@ extern "C" MOE_API int32_t moe_route_static(const void* x_bf16, int32_t T, int32
                                             int32_t* perm, int32_t* inv_perm, void* stream) {
   if (T < 0 || hidden <= 0 || num_experts <= 0 || top_k <= 0 || top_k > num_experts)
     return MOE_ERR_INVALID_ARG;
-  if (hidden % KC || hidden > 8192 || num_experts > MAX_EXPERTS || top_k > 32)
+  if (hidden % KS || hidden > 8192 || num_experts > MAX_EXPERTS || top_k > 32)
     return MOE_ERR_UNSUPPORTED_SHAPE;
   if (T == 0) return MOE_OK;
   if (!x_bf16 || !router_w || !topk_idx || !topk_w || !counts || !offsets || !perm || !inv_perm ||
@@ -117,7 +115,7 @@ extern "C" MOE_API int32_t moe_route_static(const void* x_bf16, int32_t T, int32
 
   unsigned char* s = static_cast<unsigned char*>(base);
   EngineParams p{};
-  p.H = hidden; p.I = KC; p.E = num_experts; p.K = top_k; p.T = T; p.TK = T * top_k; p.L = 1;
+  p.H = hidden; p.I = KS; p.E = num_experts; p.K = top_k; p.T = T; p.TK = T * top_k; p.L = 1;
   p.HS = router_hsplit(hidden);
   p.route_only = 1;
   p.timeout_ns = 2000000000ull;
@@ -128,8 +126,6 @@ extern "C" MOE_API int32_t moe_route_static(const void* x_bf16, int32_t T, int32
   p.layers[0] = LayerPtrs{nullptr, nullptr, router_w, router_bias};
   p.x_in = static_cast<const __nv_bfloat16*>(x_bf16);
   p.logits = reinterpret_cast<double*>(s + lay.logits);
-  p.xh = s + lay.xh;
-  p.pxf = reinterpret_cast<float*>(s + lay.pxf);
   p.units = reinterpret_cast<int32_t*>(s + lay.units);
   p.dunits = reinterpret_cast<int32_t*>(s + lay.dunits);
   p.n_units = reinterpret_cast<int32_t*>(s + lay.n_units);

@@ -1,7 +1,10 @@
 // Hand-written sm_100a PTX wrappers used by the MXFP4 MoE kernels:
 // mbarriers, 1-D bulk (TMA engine) copies global -> shared, proxy fences,
-// acquire/release accesses, the global nanosecond timer and the E2M1 and
-// packed-fp32 instructions.  No tensor-map or multicast copy is used anywhere.
+// acquire/release accesses, the global nanosecond timer, the E2M1
+// conversions and the fifth-generation tensor-core (tcgen05) instructions:
+// tensor-memory allocation, shared -> tensor memory copies of scale factors,
+// the block-scaled MXF4 MMA, commit to an mbarrier and tensor-memory loads.
+// No tensor-map or multicast copy is used anywhere.
 #pragma once
 #include <stdint.h>
 #include <cuda_bf16.h>
@@ -38,6 +41,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   asm volatile(
       "{\n .reg .pred p;\n"
       " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+// Non-blocking test of a phase.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
       " selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
   return ok != 0;
@@ -124,39 +138,92 @@ __device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float hi, float lo) {
   return r;
 }
 
-// Four E2M1 byte pairs of a word -> four f16x2 registers (A fragment a0..a3).
-__device__ __forceinline__ void e2m1x8_to_f16x2x4(uint32_t w, uint32_t (&a)[4]) {
-  asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %4;\n"
-      " cvt.rn.f16x2.e2m1x2 %0, b0;\n cvt.rn.f16x2.e2m1x2 %1, b1;\n"
-      " cvt.rn.f16x2.e2m1x2 %2, b2;\n cvt.rn.f16x2.e2m1x2 %3, b3;\n}\n"
-      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]) : "r"(w));
-}
-
-// D = A(16x16, f16, row) * B(16x8, f16, col) + C, fp32 accumulate.
-__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                              uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 // Named barrier among `count` threads (id 1..15; 0 is __syncthreads).
 __device__ __forceinline__ void named_barrier(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-struct f32x2 { float x, y; };
+// ---- tcgen05: tensor memory and the block-scaled MMA ---------------------------------
+// Tensor-memory addresses: bits 31..16 lane, 15..0 column (32-bit columns).  For
+// 8-bit scale factors, bits 31..30 of the address select the byte in a column.
 
-// d = a * b + c on pairs of fp32 lanes (sm_100 packed FMA).
-__device__ __forceinline__ void ffma2(f32x2& d, f32x2 a, f32x2 b) {
-  uint64_t A, B, D;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a.x), "f"(a.y));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(B) : "f"(b.x), "f"(b.y));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(D) : "f"(d.x), "f"(d.y));
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(D) : "l"(A), "l"(B));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(D));
+// Allocate `ncols` columns (a power of two >= 32); warp-wide.  The base address
+// is written to *dst (shared memory).
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+               ::"r"(smem_u32(dst)), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, K-major, no swizzle: 8-row x 16-byte core
+// matrices; `lbo` = byte step between the two 16-byte K chunks of an MMA,
+// `sbo` = byte step between 8-row groups.  Bits 46..47 = 1 (descriptor version).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+// 32 rows x 16 bytes of shared memory (four core matrices, `sdesc`) -> tensor
+// memory lanes 0..31, four columns from `taddr`, replicated into all four
+// 32-lane sub-partitions (the scale-factor layout of the block-scaled MMA).
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// Instruction descriptor of kind::mxf4 (E2M1 x E2M1, E8M0 scales per 32
+// elements), M = 128, K-major A and B, N columns; sf = byte of the scale
+// factor columns (0 or 2) used for this MMA's two K blocks.
+__device__ __forceinline__ uint32_t mxf4_idesc(int n, uint32_t sf) {
+  return (sf << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) |
+         ((uint32_t)(128 >> 4) << 24) | (sf << 29);
+}
+
+// D[128 x N] (+)= (A * 2^SFA) (B * 2^SFB)^T over K = 64, fp32 accumulate in
+// tensor memory; issued by one thread.
+__device__ __forceinline__ void mma_mxf4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t tsfa, uint32_t tsfb,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n}\n"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05 operation this thread issued so far
+// has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Eight consecutive columns of this warp's 32 lanes (one value per thread),
+// waited for inside the same statement so no use can be scheduled before the
+// load completes.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 }  // namespace moe

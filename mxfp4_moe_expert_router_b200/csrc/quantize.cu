@@ -66,75 +66,65 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restric
   scales[b] = static_cast<uint8_t>(sbyte);
 }
 
-// Streaming stages for the tensor-core weight stream.  A stage is 64 weight
-// rows (four 16-row MMA tiles t) x KC = 128 K elements (four MX blocks b).
-// Codes: [b][half][lane][16 B]; for lane (g = lane/4, c = lane%4) the 16 bytes
-// of half h hold tiles 2h and 2h+1, each as two k16 steps s of four bytes
-//   R[g][c + 8s], R[g+8][c + 8s], R[g][c + 4 + 8s], R[g+8][c + 4 + 8s]
-// where R[r][j] is byte j (elements 2j, 2j+1) of row r's 16-byte block chunk:
-// exactly the A-fragment registers a0..a3 of mma.m16n8k16 after E2M1 -> f16x2.
-// Scales: [row 64][b 4].  Gate/up stage rows: tile 0/1 = gate rows i0..i0+31,
-// tile 2/3 = up rows i0..i0+31 (i0 = 32 * row block); down stage rows:
-// h0 + 16 t + r (h0 = 64 * row block).
-__device__ __forceinline__ int64_t stage_src_row(int is_down, int e, int nrows, int rb, int t, int rr,
+// Streaming stages for the tensor-core weight stream.  A stage is JOB_ROWS =
+// 128 weight rows x KS = 128 K elements (four MX blocks), stored as the
+// block-scaled MMA reads it from shared memory:
+//   codes: byte kk * 4096 + (m / 8) * 256 + kc * 128 + (m % 8) * 16 + j holds
+//          elements 64 kk + 32 kc + 2 j (low nibble) and + 1 (high nibble) of
+//          row m -- a straight copy of 16-byte pieces of the canonical rows,
+//          whose nibble order is the MMA's;
+//   scales: byte 8192 + (m % 32) * 16 + (m / 32) * 4 + b = scale of block b.
+// Row m of a gate/up job (q = m / 32, l = m % 32) is gate (l < 16) or up
+// (l >= 16) row i0 + 16 q + (l % 16), i0 = 64 * job row block; row m of a
+// down job is hidden row h0 + m, h0 = 128 * job row block.
+__device__ __forceinline__ int64_t stage_src_row(int is_down, int e, int nrows, int rb, int m,
                                                  int* which) {
-  if (is_down) { *which = 0; return (int64_t)e * nrows + rb * STAGE_ROWS + t * 16 + rr; }
-  *which = t >= 2;  // 0 gate, 1 up
-  return (int64_t)e * nrows + rb * (STAGE_ROWS / 2) + (t & 1) * 16 + rr;
+  if (is_down) { *which = 0; return (int64_t)e * nrows + (int64_t)rb * JOB_ROWS + m; }
+  const int q = m >> 5, l = m & 31;
+  *which = l >= 16;  // 0 gate, 1 up
+  return (int64_t)e * nrows + (int64_t)rb * GU_I_ROWS + 16 * q + (l & 15);
 }
 
+// One thread per (stage, row m, 16-byte chunk): a 128-element row is 64 bytes,
+// four chunks (kk = chunk / 2, kc = chunk % 2).
 __global__ void repack_codes_kernel(const uint8_t* __restrict__ c0, const uint8_t* __restrict__ c1,
                                     int is_down, int E, int nrows, int K, uint8_t* __restrict__ out) {
-  const int nc = K / KC, nrb = is_down ? nrows / STAGE_ROWS : nrows / (STAGE_ROWS / 2);
-  const int64_t total = (int64_t)E * nrb * nc * KB * 2 * 32;
+  const int nc = K / KS, nrb = is_down ? nrows / JOB_ROWS : nrows / GU_I_ROWS;
+  const int64_t total = (int64_t)E * nrb * nc * JOB_ROWS * 4;
   const int64_t gidx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (gidx >= total) return;
-  const int lane = (int)(gidx % 32);
-  const int half = (int)((gidx / 32) % 2);
-  const int b = (int)((gidx / 64) % KB);
-  const int64_t st = gidx / (64 * KB);
-  const int c = (int)(st % nc);
-  const int rb = (int)((st / nc) % nrb);
-  const int e = (int)(st / ((int64_t)nc * nrb));
-  const int g = lane >> 2, cc = lane & 3;
-  const int kbg = c * KB + b;
-  uint32_t w[4];
-#pragma unroll
-  for (int tt = 0; tt < 2; ++tt) {
-    const int t = half * 2 + tt;
-    int which = 0;
-    const int64_t r0 = stage_src_row(is_down, e, nrows, rb, t, g, &which);
-    const int64_t r1 = stage_src_row(is_down, e, nrows, rb, t, g + 8, &which);
-    const uint8_t* src = which ? c1 : c0;
-    const uint8_t* p0 = src + r0 * (K / 2) + kbg * 16;
-    const uint8_t* p1 = src + r1 * (K / 2) + kbg * 16;
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      const uint32_t b0 = p0[cc + 8 * s], b1 = p1[cc + 8 * s];
-      const uint32_t b2 = p0[cc + 4 + 8 * s], b3 = p1[cc + 4 + 8 * s];
-      w[tt * 2 + s] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-    }
-  }
-  uint8_t* so = out + st * STAGE_W_BYTES + ((b * 2 + half) * 32 + lane) * 16;
-  *reinterpret_cast<uint4*>(so) = make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-__global__ void repack_scales_kernel(const uint8_t* __restrict__ s0, const uint8_t* __restrict__ s1,
-                                     int is_down, int E, int nrows, int K, uint8_t* __restrict__ out) {
-  const int nc = K / KC, nrb = is_down ? nrows / STAGE_ROWS : nrows / (STAGE_ROWS / 2);
-  const int64_t total = (int64_t)E * nrb * nc * STAGE_ROWS * KB;
-  const int64_t gidx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (gidx >= total) return;
-  const int b = (int)(gidx % KB);
-  const int r = (int)((gidx / KB) % STAGE_ROWS);
-  const int64_t st = gidx / (KB * STAGE_ROWS);
+  const int ch = (int)(gidx % 4);
+  const int m = (int)((gidx / 4) % JOB_ROWS);
+  const int64_t st = gidx / (4 * JOB_ROWS);
   const int c = (int)(st % nc);
   const int rb = (int)((st / nc) % nrb);
   const int e = (int)(st / ((int64_t)nc * nrb));
   int which = 0;
-  const int64_t row = stage_src_row(is_down, e, nrows, rb, r >> 4, r & 15, &which);
-  const uint8_t* src = which ? s1 : s0;
-  out[st * STAGE_W_BYTES + STAGE_CODE_BYTES + r * KB + b] = src[row * (K / 32) + c * KB + b];
+  const int64_t row = stage_src_row(is_down, e, nrows, rb, m, &which);
+  const uint8_t* src = (which ? c1 : c0) + row * (K / 2) + (int64_t)c * (KS / 2) + ch * 16;
+  const int kk = ch >> 1, kc = ch & 1;
+  uint8_t* dst = out + st * STAGE_A_BYTES + kk * 4096 + (m >> 3) * 256 + kc * 128 + (m & 7) * 16;
+  *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+}
+
+// One thread per (stage, row m): the row's four block scales.
+__global__ void repack_scales_kernel(const uint8_t* __restrict__ s0, const uint8_t* __restrict__ s1,
+                                     int is_down, int E, int nrows, int K, uint8_t* __restrict__ out) {
+  const int nc = K / KS, nrb = is_down ? nrows / JOB_ROWS : nrows / GU_I_ROWS;
+  const int64_t total = (int64_t)E * nrb * nc * JOB_ROWS;
+  const int64_t gidx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (gidx >= total) return;
+  const int m = (int)(gidx % JOB_ROWS);
+  const int64_t st = gidx / JOB_ROWS;
+  const int c = (int)(st % nc);
+  const int rb = (int)((st / nc) % nrb);
+  const int e = (int)(st / ((int64_t)nc * nrb));
+  int which = 0;
+  const int64_t row = stage_src_row(is_down, e, nrows, rb, m, &which);
+  const uint8_t* src = (which ? s1 : s0) + row * (K / 32) + (int64_t)c * KB;
+  uint8_t* dst = out + st * STAGE_A_BYTES + STAGE_CODE_BYTES + (m & 31) * 16 + (m >> 5) * 4;
+  *reinterpret_cast<uint32_t*>(dst) =
+      (uint32_t)src[0] | ((uint32_t)src[1] << 8) | ((uint32_t)src[2] << 16) | ((uint32_t)src[3] << 24);
 }
 
 }  // namespace
@@ -151,8 +141,8 @@ cudaError_t quantize_launch(const void* w, int64_t rows, int64_t K, uint8_t* cod
 
 cudaError_t repack_gu_launch(const uint8_t* gc, const uint8_t* gs, const uint8_t* uc,
                              const uint8_t* us, int E, int I, int H, uint8_t* out, cudaStream_t s) {
-  const int64_t stages = (int64_t)E * (I / (STAGE_ROWS / 2)) * (H / KC);
-  const int64_t n1 = stages * KB * 64, n2 = stages * STAGE_ROWS * KB;
+  const int64_t stages = (int64_t)E * (I / GU_I_ROWS) * (H / KS);
+  const int64_t n1 = stages * JOB_ROWS * 4, n2 = stages * JOB_ROWS;
   repack_codes_kernel<<<(unsigned)((n1 + 255) / 256), 256, 0, s>>>(gc, uc, 0, E, I, H, out);
   repack_scales_kernel<<<(unsigned)((n2 + 255) / 256), 256, 0, s>>>(gs, us, 0, E, I, H, out);
   return cudaGetLastError();
@@ -160,8 +150,8 @@ cudaError_t repack_gu_launch(const uint8_t* gc, const uint8_t* gs, const uint8_t
 
 cudaError_t repack_d_launch(const uint8_t* dc, const uint8_t* ds, int E, int H, int I,
                             uint8_t* out, cudaStream_t s) {
-  const int64_t stages = (int64_t)E * (H / STAGE_ROWS) * (I / KC);
-  const int64_t n1 = stages * KB * 64, n2 = stages * STAGE_ROWS * KB;
+  const int64_t stages = (int64_t)E * (H / JOB_ROWS) * (I / KS);
+  const int64_t n1 = stages * JOB_ROWS * 4, n2 = stages * JOB_ROWS;
   repack_codes_kernel<<<(unsigned)((n1 + 255) / 256), 256, 0, s>>>(dc, dc, 1, E, H, I, out);
   repack_scales_kernel<<<(unsigned)((n2 + 255) / 256), 256, 0, s>>>(ds, ds, 1, E, H, I, out);
   return cudaGetLastError();
