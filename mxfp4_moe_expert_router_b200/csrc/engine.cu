@@ -75,6 +75,7 @@ struct alignas(16) CtaTables {
   int32_t offsets[MAX_EXPERTS + 1];
   float red[WARPS];
   int32_t n_units, n_dunits;
+  int32_t last, gen;  // route barrier: this CTA arrived last; barrier generation
 };
 
 constexpr size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
@@ -92,7 +93,8 @@ constexpr size_t OFF_XCH = align16(OFF_JQ + NPIPE * JQ * sizeof(JobEntry));  // 
 constexpr size_t OFF_TABLES = align16(OFF_XCH + NPIPE * 2 * NT_MAX * 4 * 4);
 constexpr size_t SMEM_BYTES = OFF_TABLES + sizeof(CtaTables);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert((size_t)WARPS * MAX_EXPERTS * 4 <= RING_BYTES, "routing scratch in ring");
+static_assert((size_t)WARPS * MAX_EXPERTS * 8 <= RING_BYTES, "routing scratch in ring");
+static_assert((size_t)16 * (8192 / MAX_HSPLIT) * 8 <= RING_BYTES, "router x slice in ring");
 static_assert(SLOT_BYTES % 16 == 0 && STAGE_A_BYTES % 16 == 0 && IMG_BYTES % 16 == 0, "bulk-copy alignment");
 // tensor memory: pipeline p's accumulators, then its scale-factor buffers
 __host__ __device__ constexpr uint32_t tm_acc(int pipe, int b) { return (uint32_t)(pipe * NACC + b) * ACC_COLS; }
@@ -225,6 +227,52 @@ __device__ __forceinline__ uint32_t term_word(uint32_t codes, int lane) {
 }
 
 // ---- phase A: activation term images, router partial logits --------------------------------
+constexpr int RTC = 16;  // tokens per router chunk
+
+// Router work of this CTA: the H parts hs = hs0, hs0 + hstep, ... and, for
+// each, the experts e = e0, e0 + estep, ...  With at least HS CTAs every CTA
+// owns one part (the CTAs of part hs share its experts), so each converts a
+// single slice of x; with fewer CTAs a CTA owns whole parts.
+struct RouterWork { int hs0, hstep, e0, estep; };
+__device__ __forceinline__ RouterWork router_work(const EngineParams& p) {
+  const int g = (int)gridDim.x, c = (int)blockIdx.x;
+  if (g >= p.HS) {
+    const int hs = c % p.HS;
+    return RouterWork{hs, p.HS, c / p.HS, (g - hs + p.HS - 1) / p.HS};
+  }
+  return RouterWork{c, g, 0, 1};
+}
+
+// L2 prefetch of the router weight rows this CTA's dot products will read.
+__device__ void router_prefetch(const EngineParams& p, const LayerPtrs& lp) {
+  const RouterWork rw = router_work(p);
+  const int hpart = p.H / p.HS;
+#pragma unroll 1
+  for (int hs = rw.hs0; hs < p.HS; hs += rw.hstep) {
+    const int ne = (p.E - rw.e0 + rw.estep - 1) / rw.estep;
+#pragma unroll 1
+    for (int k = (int)threadIdx.x; k < ne; k += THREADS)
+      prefetch_l2_bulk(lp.router_w + (int64_t)(rw.e0 + k * rw.estep) * p.H + hs * hpart, (uint32_t)hpart * 4u);
+  }
+}
+
+// Sum over the warp of 16 values per lane, reduce-scatter order: afterwards
+// lane l holds the total of value l % 16 (16 double shuffles instead of 80).
+__device__ __forceinline__ double warp_sum16(double (&v)[RTC], int lane) {
+  static_assert(RTC == 16, "reduce-scatter written for 16 values");
+#pragma unroll
+  for (int st = 0; st < 4; ++st) {
+    const int n = 8 >> st;  // values kept after this step
+    const bool hi = (lane >> st) & 1;
+#pragma unroll
+    for (int k = 0; k < n; ++k) {
+      const double send = hi ? v[2 * k] : v[2 * k + 1];
+      const double keep = hi ? v[2 * k + 1] : v[2 * k];
+      v[k] = keep + __shfl_xor_sync(FULL, send, 1 << st);
+    }
+  }
+  return v[0] + __shfl_xor_sync(FULL, v[0], 16);
+}
 // x[t] (bf16) -> xt[stage][t]: per 32-element block one warp expands the values
 // into NTERM E2M1 terms (codes at the MMA's B-operand rows, scales at the
 // scale-factor rows of the image).
@@ -235,11 +283,12 @@ __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const 
   const int64_t gt = (int64_t)blockIdx.x * THREADS + threadIdx.x;
   const int64_t gs = (int64_t)gridDim.x * THREADS;
   const int64_t wg = (int64_t)blockIdx.x * WARPS + warp, ws = (int64_t)gridDim.x * WARPS;
+  router_prefetch(p, lp);
   const int nblk = H / 32;
   const int64_t ntask = p.route_only ? 0 : (int64_t)T * nblk;  // routing alone needs no images
   for (int64_t task = wg; task < ntask; task += ws) {
     const int t = (int)(task / nblk), gb = (int)(task % nblk);
-    const float v = __bfloat162float(x[(int64_t)t * H + gb * 32 + lane]);
+    const float v = __bfloat162float(__ldcg(x + (int64_t)t * H + gb * 32 + lane));
     float am = fabsf(v);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(FULL, am, o));
@@ -255,7 +304,7 @@ __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const 
     const int64_t n8 = (int64_t)T * H / 8;
     const uint4* s8 = reinterpret_cast<const uint4*>(x);
     uint4* d8 = reinterpret_cast<uint4*>(p.layer_io + (int64_t)layer * T * H);
-    for (int64_t i = gt; i < n8; i += gs) d8[i] = s8[i];
+    for (int64_t i = gt; i < n8; i += gs) d8[i] = __ldcg(s8 + i);
   }
   // per-layer resets of the stream's counters (used only after the next barrier)
   const int umax = max_units(E, p.TK);
@@ -263,52 +312,37 @@ __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const 
   for (int64_t u = gt; u < umax; u += gs) p.sync[SY_READY + u] = 0u;
 
   // partial logits[hs][t][e] = sum over the hs-th H part of x[t][h] * Wr[e][h];
-  // bf16 * fp32 products are exact in fp64 and the sums are fp64.  A token
-  // block that fits in the (idle) stage ring is staged there first, so that
-  // only the router weights come from L2.
-  const __nv_bfloat16* xr = x;
-  if ((int64_t)T * H * 2 <= (int64_t)RING_BYTES) {
-    uint4* d = reinterpret_cast<uint4*>(ring_slot(smem, 0, 0));
-    const uint4* s8 = reinterpret_cast<const uint4*>(x);
-    for (int64_t i = threadIdx.x; i < (int64_t)T * H / 8; i += THREADS) d[i] = s8[i];
-    __syncthreads();
-    xr = reinterpret_cast<const __nv_bfloat16*>(ring_slot(smem, 0, 0));
-  }
+  // bf16 * fp32 products are exact in fp64 and the sums are fp64.  The (hs, e)
+  // dot products are cut into one contiguous range per CTA (mostly a single
+  // hs), so that a CTA converts its slice of x to fp64 once, in shared
+  // memory, and every warp then runs one expert over all tokens of a chunk.
+  const RouterWork rw = router_work(p);
   const int HS = p.HS, hpart = H / HS;
-  const int nchunk = (T + 7) / 8;
-  const int64_t njobs = (int64_t)E * HS * nchunk;
-  for (int64_t job = wg; job < njobs; job += ws) {
-    const int e = (int)(job % E);
-    const int hs = (int)((job / E) % HS);
-    const int t0 = (int)(job / ((int64_t)E * HS)) * 8;
-    const int nt = min(8, T - t0);
-    double acc[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = 0.0;
-    const float4* wr = reinterpret_cast<const float4*>(lp.router_w + (int64_t)e * H + hs * hpart);
-#pragma unroll 8
-    for (int h4 = lane; h4 < hpart / 4; h4 += 32) {
-      const float4 w4 = __ldg(wr + h4);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j < nt) {
-          const uint2 xb = *reinterpret_cast<const uint2*>(xr + (int64_t)(t0 + j) * H + hs * hpart + h4 * 4);
-          acc[j] = fma((double)__uint_as_float(xb.x << 16), (double)w4.x, acc[j]);
-          acc[j] = fma((double)__uint_as_float(xb.x & 0xFFFF0000u), (double)w4.y, acc[j]);
-          acc[j] = fma((double)__uint_as_float(xb.y << 16), (double)w4.z, acc[j]);
-          acc[j] = fma((double)__uint_as_float(xb.y & 0xFFFF0000u), (double)w4.w, acc[j]);
-        }
+  double* xd = reinterpret_cast<double*>(ring_slot(smem, 0, 0));  // [RTC][hpart], idle ring
+  for (int hs = rw.hs0; hs < HS; hs += rw.hstep) {
+    for (int t0 = 0; t0 < T; t0 += RTC) {
+      const int nt = min(RTC, T - t0);
+      __syncthreads();  // the previous chunk's readers are done
+      for (int i = threadIdx.x; i < nt * hpart; i += THREADS) {
+        const int t = i / hpart, h = i - t * hpart;
+        xd[i] = (double)__bfloat162float(__ldcg(x + (int64_t)(t0 + t) * H + hs * hpart + h));
       }
-    }
+      __syncthreads();
+      for (int e = rw.e0 + warp * rw.estep; e < E; e += WARPS * rw.estep) {
+        const float* wr = lp.router_w + (int64_t)e * H + hs * hpart;
+        double acc[RTC];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < RTC; ++j) acc[j] = 0.0;
+#pragma unroll 4
+        for (int h = lane; h < hpart; h += 32) {
+          const double w = (double)__ldg(wr + h);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(FULL, acc[j], o);
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (j < nt) p.logits[((int64_t)hs * T + t0 + j) * E + e] = acc[j];
+          for (int j = 0; j < RTC; ++j)
+            if (j < nt) acc[j] = fma(xd[j * hpart + h], w, acc[j]);
+        }
+        const double v = warp_sum16(acc, lane);  // lane l (< 16) holds token t0 + l
+        if (lane < nt) p.logits[((int64_t)hs * T + t0 + lane) * E + e] = v;
+      }
     }
   }
   if (stamp) stamp[1] = globaltimer_ns();
@@ -326,62 +360,56 @@ __device__ __forceinline__ double key_value(uint64_t k) {
 
 // One warp: logits of token t (partials summed in order, plus bias), the K
 // largest (descending, ties to the lower expert), weights exp(l - lmax) / sum
-// over the K.  Lane r < K writes slot r.  Each lane holds experts lane + 32 i
-// (i < PER) as order-preserving 64-bit keys, sorts them once (descending, the
-// lower expert first on equal keys), and each of the K rounds takes the
-// warp-wide maximum of the lanes' heads; the winning lane drops its head.
-template <int PER>
-__device__ void topk_row_n(const EngineParams& p, const float* bias, int t, int32_t* out_idx,
-                           float* out_w) {
+// over the K.  Lane r < K writes slot r.  The token's keys (order-preserving
+// 64-bit images of the fp64 logits) sit in the warp's shared-memory row; each
+// of the K rounds takes every lane's best key, then the warp-wide maximum
+// (the lower expert on equal keys), and removes the winner.  Kept out of line
+// and without unrolled sorting networks: the code runs once per layer and its
+// instruction fetch, not its arithmetic, sets its latency.
+// (Scalar arguments: a reference to the kernel's parameter block would move
+// that block to local memory for the whole kernel.)
+__device__ __noinline__ void topk_row(const double* logits, int T, int E, int K, int HS,
+                                      const float* bias, int t, uint64_t* keys, int32_t* out_idx,
+                                      float* out_w) {
   const int lane = threadIdx.x & 31;
-  const int E = p.E, K = p.K;
-  uint64_t key[PER];
-  int ix[PER];
+  // all of a lane's partial loads in flight at once (four experts x MAX_HSPLIT parts)
+#pragma unroll 1
+  for (int e0 = lane; e0 < E; e0 += 128) {
+    double part[4][MAX_HSPLIT];
 #pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    const int e = lane + 32 * i;
-    ix[i] = i;
-    if (e < E) {
-      double part[MAX_HSPLIT];
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int hs = 0; hs < MAX_HSPLIT; ++hs)
-        part[hs] = hs < p.HS ? p.logits[((int64_t)hs * p.T + t) * E + e] : 0.0;
+      for (int hs = 0; hs < MAX_HSPLIT; ++hs) {
+        const int e = e0 + 32 * i;
+        part[i][hs] = (hs < HS && e < E) ? __ldcg(logits + ((int64_t)hs * T + t) * E + e) : 0.0;
+      }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = e0 + 32 * i;
       double l = 0.0;
 #pragma unroll
-      for (int hs = 0; hs < MAX_HSPLIT; ++hs) l += part[hs];
-      if (bias) l += (double)bias[e];
-      key[i] = order_key(l);
-    } else {
-      key[i] = 0ull;
+      for (int hs = 0; hs < MAX_HSPLIT; ++hs) l += part[i][hs];
+      if (e < E) keys[e] = order_key(bias ? l + (double)bias[e] : l);
     }
   }
-  // odd-even transposition sort, descending; on equal keys the lower index first
-#pragma unroll
-  for (int r = 0; r < PER; ++r) {
-#pragma unroll
-    for (int i = r & 1; i + 1 < PER; i += 2) {
-      const bool sw = key[i + 1] > key[i] || (key[i + 1] == key[i] && ix[i + 1] < ix[i]);
-      const uint64_t k0 = key[i], k1 = key[i + 1];
-      const int i0 = ix[i], i1 = ix[i + 1];
-      key[i] = sw ? k1 : k0; key[i + 1] = sw ? k0 : k1;
-      ix[i] = sw ? i1 : i0; ix[i + 1] = sw ? i0 : i1;
-    }
-  }
+  __syncwarp();
   int my_e = -1;
   double my_l = 0.0, lmax = 0.0;
+#pragma unroll 1
   for (int r = 0; r < K; ++r) {
-    const uint64_t best = key[0];
+    uint64_t best = 0ull;
+    int be = E;
+#pragma unroll 1
+    for (int e = lane; e < E; e += 32) {
+      const uint64_t k = keys[e];
+      if (k > best) { best = k; be = e; }  // ascending e: equal keys keep the lower expert
+    }
     const uint32_t hi = __reduce_max_sync(FULL, (uint32_t)(best >> 32));
     const uint32_t lo = __reduce_max_sync(FULL, (uint32_t)(best >> 32) == hi ? (uint32_t)best : 0u);
     const uint64_t top = ((uint64_t)hi << 32) | lo;
-    const int ehead = lane + 32 * ix[0];
-    const uint32_t m = __reduce_max_sync(FULL, best == top ? (65536u - (uint32_t)ehead) : 0u);
-    const int esel = (int)(65536u - m);
-    if (esel == ehead) {  // the winning lane drops its head
-#pragma unroll
-      for (int i = 0; i + 1 < PER; ++i) { key[i] = key[i + 1]; ix[i] = ix[i + 1]; }
-      key[PER - 1] = 0ull;
-    }
+    const int esel = (int)__reduce_min_sync(FULL, best == top ? (uint32_t)be : 0xFFFFFFFFu);
+    if (lane == (esel & 31)) keys[esel] = 0ull;
+    __syncwarp();
     const double v = key_value(top);
     if (r == 0) lmax = v;
     if (lane == r) { my_e = esel; my_l = v; }
@@ -393,16 +421,9 @@ __device__ void topk_row_n(const EngineParams& p, const float* bias, int t, int3
   if (lane < K) { out_idx[lane] = my_e; out_w[lane] = (float)(ex / sum); }
 }
 
-__device__ __forceinline__ void topk_row(const EngineParams& p, const float* bias, int t,
-                                         int32_t* out_idx, float* out_w) {
-  if (p.E <= 128) topk_row_n<4>(p, bias, t, out_idx, out_w);
-  else if (p.E <= 256) topk_row_n<8>(p, bias, t, out_idx, out_w);
-  else topk_row_n<16>(p, bias, t, out_idx, out_w);
-}
-
 // Exclusive scan of n <= 512 ints in shared memory by one warp (in place);
 // the total goes to *total.
-__device__ void warp_exclusive_scan(int32_t* a, int n, int32_t* total) {
+__device__ __noinline__ void warp_exclusive_scan(int32_t* a, int n, int32_t* total) {
   const int lane = threadIdx.x & 31;
   constexpr int PER = 16;
   int32_t v[PER];
@@ -432,7 +453,7 @@ __device__ void warp_exclusive_scan(int32_t* a, int n, int32_t* total) {
 // Unit tables from per-expert counts/offsets: gate/up units of <= NT_MAX
 // consecutive positions of one expert's segment, down units of <= ND_MAX
 // (each inside one gate/up unit).  scratch: 2*E ints.
-__device__ void build_units(const int32_t* counts, const int32_t* offsets, int E, int32_t* scratch,
+__device__ __noinline__ void build_units(const int32_t* counts, const int32_t* offsets, int E, int32_t* scratch,
                             int32_t* units, int32_t* dunits, int32_t* n_units, int32_t* n_dunits) {
   const int warp = threadIdx.x >> 5;
   int32_t* ubase = scratch;
@@ -466,7 +487,9 @@ __device__ void phase_route_small(const EngineParams& p, const LayerPtrs& lp, ui
   CtaTables& tb = tables(smem);
   const int T = p.T, E = p.E, K = p.K, TK = p.TK;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int t = warp; t < T; t += WARPS) topk_row(p, lp.router_b, t, tb.idx + t * K, tb.w + t * K);
+  uint64_t* keys = reinterpret_cast<uint64_t*>(ring_slot(smem, 0, 0)) + warp * MAX_EXPERTS;
+  for (int t = warp; t < T; t += WARPS) topk_row(p.logits, T, E, K, p.HS, lp.router_b, t, keys, tb.idx + t * K, tb.w + t * K);
+  __syncthreads();  // the key rows share the ring with the histogram below
   if (stamp) *stamp = globaltimer_ns();
   int32_t* hist = reinterpret_cast<int32_t*>(ring_slot(smem, 0, 0));  // [WARPS][E] scratch
   for (int i = threadIdx.x; i < WARPS * E; i += THREADS) hist[i] = 0;
@@ -499,21 +522,89 @@ __device__ void phase_route_small(const EngineParams& p, const LayerPtrs& lp, ui
   __syncthreads();
   build_units(tb.counts, tb.offsets, E, hist, tb.units, tb.dunits, &tb.n_units, &tb.n_dunits);
   __syncthreads();
-  if (blockIdx.x == 0) {
-    for (int i = threadIdx.x; i < TK; i += THREADS) {
-      p.idx[i] = tb.idx[i]; p.wts[i] = tb.w[i]; p.perm[i] = tb.perm[i]; p.inv[i] = tb.inv[i];
-    }
-    for (int i = threadIdx.x; i < E; i += THREADS) p.counts[i] = tb.counts[i];
-    for (int i = threadIdx.x; i <= E; i += THREADS) p.offsets[i] = tb.offsets[i];
+  // publish: the maps of the ABI and the stream's tables
+  for (int i = threadIdx.x; i < TK; i += THREADS) {
+    p.idx[i] = tb.idx[i]; p.wts[i] = tb.w[i]; p.perm[i] = tb.perm[i]; p.inv[i] = tb.inv[i];
+    p.tokpos[i] = tb.tokpos[i]; p.wpos[i] = tb.wpos[i];
   }
+  for (int i = threadIdx.x; i < E; i += THREADS) p.counts[i] = tb.counts[i];
+  for (int i = threadIdx.x; i <= E; i += THREADS) p.offsets[i] = tb.offsets[i];
+  for (int i = threadIdx.x; i < tb.n_units * 4; i += THREADS) p.units[i] = tb.units[i];
+  for (int i = threadIdx.x; i < tb.n_dunits * 4; i += THREADS) p.dunits[i] = tb.dunits[i];
+  if (threadIdx.x == 0) { p.n_units[0] = tb.n_units; p.n_units[1] = tb.n_dunits; }
+}
+
+// Small T*K: the grid barrier after the router phase.  The CTA that arrives
+// last computes the routing once (top-k, permutation, unit tables) and
+// publishes it before releasing the barrier; every other CTA then copies the
+// stream's tables (a few KB) into shared memory.  One CTA reading all partial
+// logits is much faster than every CTA reading them at once.  Bounded like
+// grid_barrier; false on timeout or a recorded error.
+__device__ bool route_barrier(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem, uint32_t where,
+                              uint64_t* stamp) {
+  CtaTables& tb = tables(smem);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t gen = ld_volatile_u32(p.sync + SY_BAR_GEN);
+    __threadfence();
+    const uint32_t prev = atomicAdd(p.sync + SY_BAR_COUNT, 1u);
+    __threadfence();
+    tb.last = prev == gridDim.x - 1;
+    tb.gen = (int32_t)gen;
+  }
+  __syncthreads();
+  int ok = 1;
+  if (tb.last) {
+    phase_route_small(p, lp, smem, stamp);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      atomicExch(p.sync + SY_BAR_COUNT, 0u);
+      __threadfence();
+      st_release_u32(p.sync + SY_BAR_GEN, (uint32_t)tb.gen + 1u);
+      if (error_set(p.sync)) ok = 0;
+    }
+    return __syncthreads_and(ok) != 0;
+  }
+  if (threadIdx.x == 0) {
+    const uint32_t gen = (uint32_t)tb.gen;
+    const uint64_t t0 = globaltimer_ns();
+    uint32_t spins = 0;
+    while (ld_acquire_u32(p.sync + SY_BAR_GEN) == gen) {
+      if ((++spins & 15u) == 0u) {
+        if (error_set(p.sync)) { ok = 0; break; }
+        if (globaltimer_ns() - t0 > p.timeout_ns) { set_error(p.sync, DEV_TIMEOUT_BARRIER, where); ok = 0; break; }
+      }
+      __nanosleep(32);
+    }
+    __threadfence();
+    if (ok && error_set(p.sync)) ok = 0;
+  }
+  if (!__syncthreads_and(ok)) return false;
+  if (stamp) stamp[0] = globaltimer_ns();
+  if (p.route_only) return true;
+  const int nu = ld_cg_u32(p.n_units), nd = ld_cg_u32(p.n_units + 1);
+  const uint4* su = reinterpret_cast<const uint4*>(p.units);
+  const uint4* sd = reinterpret_cast<const uint4*>(p.dunits);
+  for (int i = threadIdx.x; i < nu; i += THREADS) reinterpret_cast<uint4*>(tb.units)[i] = ld_cg_v4(su + i);
+  for (int i = threadIdx.x; i < nd; i += THREADS) reinterpret_cast<uint4*>(tb.dunits)[i] = ld_cg_v4(sd + i);
+  for (int i = threadIdx.x; i < p.TK; i += THREADS) {
+    tb.tokpos[i] = (int32_t)ld_cg_u32(p.tokpos + i);
+    tb.wpos[i] = __uint_as_float(ld_cg_u32(p.wpos + i));
+    tb.inv[i] = (int32_t)ld_cg_u32(p.inv + i);
+  }
+  if (threadIdx.x == 0) { tb.n_units = nu; tb.n_dunits = nd; }
+  __syncthreads();
+  return true;
 }
 
 // Large T*K, step 1: top-k of every token, distributed over all warps.
-__device__ void phase_topk_large(const EngineParams& p, const LayerPtrs& lp) {
+__device__ void phase_topk_large(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem) {
   const int warp = threadIdx.x >> 5;
   const int64_t wg = (int64_t)blockIdx.x * WARPS + warp, ws = (int64_t)gridDim.x * WARPS;
+  uint64_t* keys = reinterpret_cast<uint64_t*>(ring_slot(smem, 0, 0)) + warp * MAX_EXPERTS;
   for (int64_t t = wg; t < p.T; t += ws)
-    topk_row(p, lp.router_b, (int)t, p.idx + t * p.K, p.wts + t * p.K);
+    topk_row(p.logits, p.T, p.E, p.K, p.HS, lp.router_b, (int)t, keys, p.idx + t * p.K, p.wts + t * p.K);
 }
 
 // Large T*K, step 2: counts/offsets in every CTA (shared-memory histogram),
@@ -524,7 +615,7 @@ __device__ void phase_permute_large(const EngineParams& p, uint8_t* smem) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < E; i += THREADS) tb.counts[i] = 0;
   __syncthreads();
-  for (int i = threadIdx.x; i < TK; i += THREADS) atomicAdd(&tb.counts[p.idx[i]], 1);
+  for (int i = threadIdx.x; i < TK; i += THREADS) atomicAdd(&tb.counts[__ldcg(p.idx + i)], 1);
   __syncthreads();
   for (int i = threadIdx.x; i < E; i += THREADS) tb.offsets[i] = tb.counts[i];
   __syncthreads();
@@ -542,11 +633,11 @@ __device__ void phase_permute_large(const EngineParams& p, uint8_t* smem) {
     int run = tb.offsets[x];
     for (int base = 0; base < TK; base += 32) {
       const int pr = base + lane;
-      const bool hit = pr < TK && p.idx[pr] == (int)x;
+      const bool hit = pr < TK && __ldcg(p.idx + pr) == (int)x;
       const uint32_t b = __ballot_sync(FULL, hit);
       if (hit) {
         const int pos = run + __popc(b & ((1u << lane) - 1u));
-        p.perm[pos] = pr; p.inv[pr] = pos; p.tokpos[pos] = pr / K; p.wpos[pos] = p.wts[pr];
+        p.perm[pos] = pr; p.inv[pr] = pos; p.tokpos[pos] = pr / K; p.wpos[pos] = __ldcg(p.wts + pr);
       }
       run += __popc(b);
     }
@@ -560,7 +651,12 @@ struct StreamCtx {
   const int32_t* tokpos;
   const float* wpos;
   int n_units, n_dunits;
+  bool global;            // tables in global memory (written in this launch: read through L2)
 };
+
+// Table read: shared memory, or global memory bypassing the (non-coherent) L1.
+template <class V>
+__device__ __forceinline__ V ld_tab(const V* ptr, bool global) { return global ? __ldcg(ptr) : *ptr; }
 
 // Per-thread pipeline positions, continued across layers.
 struct RoleState {
@@ -606,8 +702,10 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
   unsigned long long t_empty = 0, t_ready = 0;
   const unsigned long long t_begin = clock64();
   fence_proxy_async_global();
-  long long next = 0;
-  if (lane == 0) next = atomicAdd(p.sync + SY_JOBS, 1u);
+  // the first job of every pipeline is static (no atomic round trip at the
+  // start of the stream); later jobs come from the global counter
+  const int64_t jbase = (int64_t)NPIPE * gridDim.x;
+  long long next = (int64_t)blockIdx.x + (int64_t)pipe * gridDim.x;
   for (;;) {
     const int64_t j = __shfl_sync(FULL, next, 0);
     if (j >= n_all || !ok) {
@@ -620,12 +718,12 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
       ++rs.qk;
       break;
     }
-    if (lane == 0) next = atomicAdd(p.sync + SY_JOBS, 1u);  // prefetch the following job
+    if (lane == 0) next = jbase + atomicAdd(p.sync + SY_JOBS, 1u);  // prefetch the following job
     const bool isD = j >= n_gu;
     const int64_t jj = isD ? j - n_gu : j;
     const int per = isD ? db : gub;
     const int u = (int)(jj / per), rb = (int)(jj % per);
-    const int4 ur = *reinterpret_cast<const int4*>((isD ? cx.dunits : cx.units) + (int64_t)u * 4);
+    const int4 ur = ld_tab(reinterpret_cast<const int4*>((isD ? cx.dunits : cx.units) + (int64_t)u * 4), cx.global);
     const int e = ur.x, pos0 = ur.y, nt = ur.z;
     const int nc = isD ? nc_d : nc_gu;
     if (isD) {  // the down stages read the SwiGLU term images: wait for the gate/up unit
@@ -657,7 +755,7 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
     ++rs.wj;
     const uint8_t* wbase = isD ? lp.w_d + ((int64_t)e * db + rb) * nc * STAGE_A_BYTES
                                : lp.w_gu + ((int64_t)e * gub + rb) * nc * STAGE_A_BYTES;
-    const int tok = (!isD && lane < nt) ? cx.tokpos[pos0 + lane] : 0;
+    const int tok = (!isD && lane < nt) ? ld_tab(cx.tokpos + pos0 + lane, cx.global) : 0;
     const uint32_t stage_bytes = STAGE_A_BYTES + (uint32_t)nt * IMG_BYTES;
     // Stages are issued in batches, one stage per lane: successive 1-D bulk
     // copies issued by one warp instruction each are serialised, while the
@@ -879,7 +977,7 @@ __device__ void stream_epilogue(const EngineParams& p, uint8_t* smem, const Stre
           float sum = v[NTERM - 1];
 #pragma unroll
           for (int k = NTERM - 2; k >= 0; --k) sum += v[k];
-          p.ypair[(int64_t)(pos0 + j) * p.H + h0 + 32 * q + lane] = sum * cx.wpos[pos0 + j];
+          p.ypair[(int64_t)(pos0 + j) * p.H + h0 + 32 * q + lane] = sum * ld_tab(cx.wpos + pos0 + j, cx.global);
         }
       }
     }
@@ -909,7 +1007,7 @@ __device__ __forceinline__ float4 combine4(const EngineParams& p, const int32_t*
   float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int slot = 0; slot < p.K; ++slot) {
     const int pos = inv[t * p.K + slot];
-    const float4 v = *reinterpret_cast<const float4*>(p.ypair + (int64_t)pos * p.H + h);
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(p.ypair + (int64_t)pos * p.H + h));
     s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
   }
   return s;
@@ -981,23 +1079,24 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
     const __nv_bfloat16* x = layer == 0 ? p.x_in : p.xnext;
     uint64_t* st = stamp ? p.stamps + 1 + layer * STAMPS_PER_LAYER : nullptr;
     phase_prepare(p, lp, x, layer, smem, st);
-    if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 1)) return;
-    if (st) st[2] = globaltimer_ns();
     StreamCtx cx;
     const int32_t* inv;
     if (small) {
-      phase_route_small(p, lp, smem, st ? st + 3 : nullptr);
-      cx = StreamCtx{tb.units, tb.dunits, tb.tokpos, tb.wpos, tb.n_units, tb.n_dunits};
-      inv = tb.inv;
+      if (!route_barrier(p, lp, smem, 10 * layer + 1, st ? st + 2 : nullptr)) return;
       if (p.route_only) return;
+      if (st) st[3] = globaltimer_ns();
+      cx = StreamCtx{tb.units, tb.dunits, tb.tokpos, tb.wpos, tb.n_units, tb.n_dunits, false};
+      inv = tb.inv;
     } else {
-      phase_topk_large(p, lp);
+      if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 1)) return;
+      if (st) st[2] = globaltimer_ns();
+      phase_topk_large(p, lp, smem);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 2)) return;
       if (st) st[3] = globaltimer_ns();
       phase_permute_large(p, smem);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 3)) return;
       if (p.route_only) return;
-      cx = StreamCtx{p.units, p.dunits, p.tokpos, p.wpos, p.n_units[0], p.n_units[1]};
+      cx = StreamCtx{p.units, p.dunits, p.tokpos, p.wpos, (int)ld_cg_u32(p.n_units), (int)ld_cg_u32(p.n_units + 1), true};
       inv = p.inv;
     }
     if (st) st[4] = globaltimer_ns();

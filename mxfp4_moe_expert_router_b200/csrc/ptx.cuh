@@ -78,6 +78,12 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src, uint32
       ::"r"(smem_u32(dst_smem)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 
+// Prefetch `bytes` of global memory into L2 (16-byte aligned address, size a
+// multiple of 16); no data is returned.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Order this thread's earlier generic-proxy global accesses with its later
 // async-proxy (bulk copy) accesses.
 __device__ __forceinline__ void fence_proxy_async_global() {
