@@ -162,9 +162,31 @@ def build_layer(mx, w: synth.Workload, layer: int, seed: int):
     return mx.LayerMX(gc, gs, uc, us, dc, ds, dense["router_w"].contiguous(), dense["router_b"])
 
 
+def token_block_ids(rank: int, n: int) -> list:
+    """Stream ids of the n token blocks rank `rank` runs: 64 ids per rank, disjoint across ranks
+    (every rank verifies its own blocks; nothing is exchanged on the data path)."""
+    if not 0 < n <= 64:
+        raise ValueError("1..64 token blocks per rank")
+    return [1000 + rank * 64 + b for b in range(n)]
+
+
 def token_blocks(w: synth.Workload, T: int, n: int, rank: int):
+    return [synth.draw_torch(i, 0, "x", -1, (T, w.hidden), 1.0) for i in token_block_ids(rank, n)]
+
+
+def max_over_ranks(value: float, dist=None, device="cpu") -> float:
+    """The slowest rank's time (identity with one rank or no process group)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
     import torch
-    return [synth.draw_torch(1000 + rank * 64 + b, 0, "x", -1, (T, w.hidden), 1.0) for b in range(n)]
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, T: int, steps: int, seconds: float) -> float:
+    """Whole-job throughput: every rank verifies T tokens per step."""
+    return world * T * steps / seconds
 
 
 def algorithmic_bytes(w: synth.Workload, T: int, hit: int) -> float:
@@ -293,13 +315,9 @@ def main():
     clk = clocks.stop()
     m.moe_status()
     phases = m.moe_phase_ns()  # the last timed step, CTA 0's view
-    ms_total = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms_total], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), dist if world > 1 else None, "cuda")
     ms_step = ms_total / args.steps
-    tokens_per_s = world * T * args.steps / (ms_total / 1e3)
+    tokens_per_s = job_tokens_per_s(world, T, args.steps, ms_total / 1e3)
     mean_hit = float(np.mean([hits[i % len(hits)] for i in range(args.steps)]))
     alg_bytes = algorithmic_bytes(w, T, mean_hit) * w.layers if w.layers == 1 else None
     # the chain workload's later layers route on the previous layer's output: count them
@@ -320,15 +338,15 @@ def main():
             m.moe_forward_host(xh[i % len(xh)], yh)
         if world > 1:
             dist.barrier()
-        t0 = time.perf_counter()
-        for i in range(n_e2e):
-            m.moe_forward_host(xh[i % len(xh)], yh)
-        el = time.perf_counter() - t0
-        if world > 1:
-            t = torch.tensor([el], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            el = float(t.item())
-        e2e = {"value": world * T * n_e2e / el, "unit": "tokens/s", "steps": n_e2e,
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n_e2e):  # each call: H2D of x, the layer, D2H of y, on this stream
+            m.moe_forward_host(xh[i % len(xh)], yh, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        el = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist if world > 1 else None, "cuda")
+        e2e = {"value": job_tokens_per_s(world, T, n_e2e, el), "unit": "tokens/s", "steps": n_e2e,
                "h2d_bytes_per_step": T * w.hidden * 2, "d2h_bytes_per_step": T * w.hidden * 2}
 
     cpu = None

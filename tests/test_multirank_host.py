@@ -1,0 +1,67 @@
+"""Host logic of the N > 1 bench path on CPU: two gloo ranks (no GPU).
+
+Each rank verifies its own token blocks (weak scaling, no collective on the data
+path); the only collective is the max over ranks of the timed region.
+"""
+import os
+import socket
+
+import pytest
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # rank r reports a distinct elapsed time; every rank must see the slowest
+        mine = 10.0 + 7.5 * rank
+        slowest = bench.max_over_ranks(mine, dist, "cpu")
+        ids = bench.token_block_ids(rank, 8)
+        dist.barrier()
+        out.put((rank, mine, slowest, ids))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_max_and_disjoint_blocks():
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    res.sort()
+    assert [r[2] for r in res] == [17.5, 17.5]           # both ranks see the slowest rank
+    ids0, ids1 = res[0][3], res[1][3]
+    assert len(set(ids0)) == 8 and not set(ids0) & set(ids1)  # each rank its own blocks
+
+
+def test_max_over_ranks_without_a_group_is_identity():
+    assert bench.max_over_ranks(3.25) == 3.25
+
+
+def test_job_throughput_counts_every_rank():
+    # 4 ranks x 9 tokens x 100 steps in 0.5 s
+    assert bench.job_tokens_per_s(4, 9, 100, 0.5) == pytest.approx(7200.0)
+    assert bench.job_tokens_per_s(1, 9, 100, 0.5) == pytest.approx(1800.0)
+
+
+def test_token_block_ids_bounds():
+    assert bench.token_block_ids(0, 1) == [1000]
+    assert bench.token_block_ids(3, 2) == [1192, 1193]
+    with pytest.raises(ValueError):
+        bench.token_block_ids(0, 65)
