@@ -319,23 +319,47 @@ __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const 
   const RouterWork rw = router_work(p);
   const int HS = p.HS, hpart = H / HS;
   double* xd = reinterpret_cast<double*>(ring_slot(smem, 0, 0));  // [RTC][hpart], idle ring
+  // this CTA's router weight slices (one per expert it owns) are staged in
+  // shared memory once and reused by every token chunk, when they fit
+  float* wsm = reinterpret_cast<float*>(xd + (size_t)RTC * hpart);
+  const int nexp = rw.e0 < E ? (E - rw.e0 + rw.estep - 1) / rw.estep : 0;
+  const bool wstaged = ((size_t)RTC * hpart * 8 + (size_t)nexp * hpart * 4) <= RING_BYTES;
   for (int hs = rw.hs0; hs < HS; hs += rw.hstep) {
+    if (wstaged) {
+      __syncthreads();  // the previous part's readers are done
+      const int hp4 = hpart / 4;
+      for (int i = threadIdx.x; i < nexp * hp4; i += THREADS) {
+        const int k = i / hp4, h4 = i - k * hp4;
+        reinterpret_cast<float4*>(wsm)[i] =
+            __ldg(reinterpret_cast<const float4*>(lp.router_w + (int64_t)(rw.e0 + k * rw.estep) * H + hs * hpart) + h4);
+      }
+    }
     for (int t0 = 0; t0 < T; t0 += RTC) {
       const int nt = min(RTC, T - t0);
       __syncthreads();  // the previous chunk's readers are done
-      for (int i = threadIdx.x; i < nt * hpart; i += THREADS) {
-        const int t = i / hpart, h = i - t * hpart;
-        xd[i] = (double)__bfloat162float(__ldcg(x + (int64_t)(t0 + t) * H + hs * hpart + h));
+      const int hp8 = hpart / 8;  // 8 bf16 per 16-byte load (H / HS is a multiple of 8)
+#pragma unroll 4
+      for (int i = threadIdx.x; i < nt * hp8; i += THREADS) {
+        const int t = i / hp8, h8 = i - t * hp8;
+        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(x + (int64_t)(t0 + t) * H + hs * hpart) + h8);
+        double* d = xd + (size_t)t * hpart + h8 * 8;
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          d[2 * q] = (double)__uint_as_float(u[q] << 16);
+          d[2 * q + 1] = (double)__uint_as_float(u[q] & 0xFFFF0000u);
+        }
       }
       __syncthreads();
-      for (int e = rw.e0 + warp * rw.estep; e < E; e += WARPS * rw.estep) {
-        const float* wr = lp.router_w + (int64_t)e * H + hs * hpart;
+      for (int k = warp; k < nexp; k += WARPS) {
+        const int e = rw.e0 + k * rw.estep;
+        const float* wr = wstaged ? wsm + (size_t)k * hpart : lp.router_w + (int64_t)e * H + hs * hpart;
         double acc[RTC];
 #pragma unroll
         for (int j = 0; j < RTC; ++j) acc[j] = 0.0;
 #pragma unroll 4
         for (int h = lane; h < hpart; h += 32) {
-          const double w = (double)__ldg(wr + h);
+          const double w = (double)wr[h];
 #pragma unroll
           for (int j = 0; j < RTC; ++j)
             if (j < nt) acc[j] = fma(xd[j * hpart + h], w, acc[j]);

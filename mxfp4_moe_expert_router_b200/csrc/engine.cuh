@@ -79,8 +79,8 @@ enum : uint32_t {
 __host__ __device__ inline int max_units(int E, int64_t TK) { return (int)((E < TK ? E : TK) + TK / NT_MAX + 1); }
 __host__ __device__ inline int max_dunits(int E, int64_t TK) { return (int)((E < TK ? E : TK) + TK / ND_MAX + 1); }
 
-// Router split of H into HS parts of H / HS elements (a multiple of 4).
-inline int router_hsplit(int H) { return H % (4 * MAX_HSPLIT) == 0 ? MAX_HSPLIT : 1; }
+// Router split of H into HS parts of H / HS elements (a multiple of 8).
+inline int router_hsplit(int H) { return H % (8 * MAX_HSPLIT) == 0 ? MAX_HSPLIT : 1; }
 
 struct LayerPtrs {
   const uint8_t* w_gu;  // gate/up stages  [E][I/64][H/KS][STAGE_A_BYTES]
@@ -91,7 +91,7 @@ struct LayerPtrs {
 
 struct EngineParams {
   int H, I, E, K, T, TK, L;  // hidden, inter, experts, top_k, tokens, T*K, layers to run
-  int HS;                    // router H split (H/HS a multiple of 4)
+  int HS;                    // router H split (H/HS a multiple of 8)
   int route_only;            // 1: stop after routing of layer 0, export maps
   float rms_eps;
   uint64_t timeout_ns;
