@@ -90,11 +90,14 @@ constexpr size_t OFF_DRAIN = OFF_XBAR + NPIPE * 2 * 8;              // [NPIPE]
 constexpr size_t OFF_TMEMBASE = OFF_DRAIN + NPIPE * 8;
 constexpr size_t OFF_JQ = align16(OFF_TMEMBASE + 8);                // [NPIPE][JQ]
 constexpr size_t OFF_XCH = align16(OFF_JQ + NPIPE * JQ * sizeof(JobEntry));  // [NPIPE][2][NT_MAX][4] floats
-constexpr size_t OFF_TABLES = align16(OFF_XCH + NPIPE * 2 * NT_MAX * 4 * 4);
+constexpr size_t XCH_FLOATS = (NPIPE * 2 * NT_MAX > 2 * LT_MAX ? NPIPE * 2 * NT_MAX : 2 * LT_MAX) * 4;
+constexpr size_t OFF_TABLES = align16(OFF_XCH + XCH_FLOATS * 4);
 constexpr size_t SMEM_BYTES = OFF_TABLES + sizeof(CtaTables);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert((size_t)WARPS * MAX_EXPERTS * 8 <= RING_BYTES, "routing scratch in ring");
 static_assert((size_t)16 * (8192 / MAX_HSPLIT) * 8 <= RING_BYTES, "router x slice in ring");
+static_assert((size_t)LT_NSLOT * LT_SLOT_BYTES <= RING_BYTES && LT_SLOT_BYTES % 16 == 0, "tile ring");
+static_assert(PRODUCER_BATCH <= LT_NSLOT, "producer batch (tiles)");
 static_assert(SLOT_BYTES % 16 == 0 && STAGE_A_BYTES % 16 == 0 && IMG_BYTES % 16 == 0, "bulk-copy alignment");
 // tensor memory: pipeline p's accumulators, then its scale-factor buffers
 __host__ __device__ constexpr uint32_t tm_acc(int pipe, int b) { return (uint32_t)(pipe * NACC + b) * ACC_COLS; }
@@ -478,13 +481,13 @@ __device__ __noinline__ void warp_exclusive_scan(int32_t* a, int n, int32_t* tot
 // consecutive positions of one expert's segment, down units of <= ND_MAX
 // (each inside one gate/up unit).  scratch: 2*E ints.
 __device__ __noinline__ void build_units(const int32_t* counts, const int32_t* offsets, int E, int32_t* scratch,
-                            int32_t* units, int32_t* dunits, int32_t* n_units, int32_t* n_dunits) {
+                            int32_t* units, int32_t* dunits, int32_t* n_units, int32_t* n_dunits, int us) {
   const int warp = threadIdx.x >> 5;
   int32_t* ubase = scratch;
   int32_t* dbase = scratch + E;
   for (int x = threadIdx.x; x < E; x += THREADS) {
-    ubase[x] = (counts[x] + NT_MAX - 1) / NT_MAX;
-    dbase[x] = (counts[x] + ND_MAX - 1) / ND_MAX;
+    ubase[x] = (counts[x] + us - 1) / us;
+    dbase[x] = (counts[x] + us - 1) / us;
   }
   __syncthreads();
   if (warp == 0) warp_exclusive_scan(ubase, E, n_units);
@@ -492,14 +495,14 @@ __device__ __noinline__ void build_units(const int32_t* counts, const int32_t* o
   __syncthreads();
   for (int x = threadIdx.x; x < E; x += THREADS) {
     const int c = counts[x];
-    for (int s = 0; s * NT_MAX < c; ++s) {
+    for (int s = 0; s * us < c; ++s) {
       int32_t* u = units + (int64_t)(ubase[x] + s) * 4;
-      u[0] = x; u[1] = offsets[x] + s * NT_MAX; u[2] = min(NT_MAX, c - s * NT_MAX); u[3] = 0;
+      u[0] = x; u[1] = offsets[x] + s * us; u[2] = min(us, c - s * us); u[3] = 0;
     }
-    for (int s = 0; s * ND_MAX < c; ++s) {
+    for (int s = 0; s * us < c; ++s) {  // down units are the gate/up units
       int32_t* u = dunits + (int64_t)(dbase[x] + s) * 4;
-      u[0] = x; u[1] = offsets[x] + s * ND_MAX; u[2] = min(ND_MAX, c - s * ND_MAX);
-      u[3] = ubase[x] + (s * ND_MAX) / NT_MAX;
+      u[0] = x; u[1] = offsets[x] + s * us; u[2] = min(us, c - s * us);
+      u[3] = ubase[x] + s;
     }
   }
 }
@@ -544,7 +547,7 @@ __device__ void phase_route_small(const EngineParams& p, const LayerPtrs& lp, ui
     tb.wpos[pos] = tb.w[pr];
   }
   __syncthreads();
-  build_units(tb.counts, tb.offsets, E, hist, tb.units, tb.dunits, &tb.n_units, &tb.n_dunits);
+  build_units(tb.counts, tb.offsets, E, hist, tb.units, tb.dunits, &tb.n_units, &tb.n_dunits, NT_MAX);
   __syncthreads();
   // publish: the maps of the ABI and the stream's tables
   for (int i = threadIdx.x; i < TK; i += THREADS) {
@@ -647,7 +650,8 @@ __device__ void phase_permute_large(const EngineParams& p, uint8_t* smem) {
   __syncthreads();
   if (blockIdx.x == 0) {
     int32_t* scratch = reinterpret_cast<int32_t*>(ring_slot(smem, 0, 0));
-    build_units(tb.counts, tb.offsets, E, scratch, p.units, p.dunits, &tb.n_units, &tb.n_dunits);
+    build_units(tb.counts, tb.offsets, E, scratch, p.units, p.dunits, &tb.n_units, &tb.n_dunits,
+                use_tiles(TK, E) ? LT_MAX : NT_MAX);
     for (int i = threadIdx.x; i < E; i += THREADS) p.counts[i] = tb.counts[i];
     for (int i = threadIdx.x; i <= E; i += THREADS) p.offsets[i] = tb.offsets[i];
     if (threadIdx.x == 0) { p.n_units[0] = tb.n_units; p.n_units[1] = tb.n_dunits; }
@@ -664,6 +668,47 @@ __device__ void phase_permute_large(const EngineParams& p, uint8_t* smem) {
         p.perm[pos] = pr; p.inv[pr] = pos; p.tokpos[pos] = pr / K; p.wpos[pos] = __ldcg(p.wts + pr);
       }
       run += __popc(b);
+    }
+  }
+}
+
+// Large T*K: the x term images of every tile, gathered from the per-token
+// images (codes as they are, scale words into the tile's scale-factor blocks).
+// A warp moves GATHER_PER positions of one (tile, stage) per round, all loads
+// first.
+constexpr int GATHER_PER = 4;
+__device__ void phase_tile_gather(const EngineParams& p) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ns = p.H / KS, nu = ld_cg_u32(p.n_units);
+  constexpr int NG = LT_MAX / GATHER_PER;
+  static_assert(LT_MAX % GATHER_PER == 0, "gather groups");
+  const int64_t ntask = (int64_t)nu * ns * NG;
+  for (int64_t task = (int64_t)blockIdx.x * WARPS + warp; task < ntask; task += (int64_t)gridDim.x * WARPS) {
+    const int g = (int)(task % NG);
+    const int64_t us = task / NG;  // tile * ns + stage
+    const int u = (int)(us / ns), st = (int)(us % ns);
+    const int4 ur = __ldcg(reinterpret_cast<const int4*>(p.units) + u);
+    const int n = min(GATHER_PER, ur.z - g * GATHER_PER);
+    if (n <= 0) continue;
+    uint4 c[GATHER_PER];
+    uint32_t sfw[GATHER_PER];
+#pragma unroll
+    for (int i = 0; i < GATHER_PER; ++i) {
+      if (i < n) {
+        const int tok = __ldcg(p.tokpos + ur.y + g * GATHER_PER + i);
+        const uint8_t* src = p.xt + ((int64_t)st * p.T + tok) * IMG_BYTES;
+        c[i] = __ldcg(reinterpret_cast<const uint4*>(src) + lane);
+        sfw[i] = __ldcg(reinterpret_cast<const uint32_t*>(src + IMG_CODE_BYTES + (lane & 7) * 16));
+      }
+    }
+    uint8_t* dst = p.xtl + us * LT_IMG_BYTES;
+#pragma unroll
+    for (int i = 0; i < GATHER_PER; ++i) {
+      if (i < n) {
+        const int tl = g * GATHER_PER + i;
+        reinterpret_cast<uint4*>(dst + lt_code_offset(tl))[lane] = c[i];
+        if (lane < NTERM) *reinterpret_cast<uint32_t*>(dst + lt_sf_offset(tl, lane, 0)) = sfw[i];
+      }
     }
   }
 }
@@ -712,8 +757,11 @@ __device__ bool wait_entry(const EngineParams& p, JobEntry* en, int32_t qk) {
 // term images are complete.  A stage is the job's weight stage plus one term
 // image per token (gate/up, from xt) or the unit's consecutive pair images
 // (down, from aimg).
+template <bool LT>
 __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem,
                                 const StreamCtx& cx, int pipe, RoleState& rs) {
+  constexpr int NS = LT ? LT_NSLOT : NSLOT;  // ring slots
+  constexpr int NP = LT ? 1 : NPIPE;         // pipelines per CTA
   const int lane = threadIdx.x & 31;
   JobEntry* jq = job_queue(smem, pipe);
   uint32_t* ready = p.sync + SY_READY;
@@ -728,7 +776,7 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
   fence_proxy_async_global();
   // the first job of every pipeline is static (no atomic round trip at the
   // start of the stream); later jobs come from the global counter
-  const int64_t jbase = (int64_t)NPIPE * gridDim.x;
+  const int64_t jbase = (int64_t)NP * gridDim.x;
   long long next = (int64_t)blockIdx.x + (int64_t)pipe * gridDim.x;
   for (;;) {
     const int64_t j = __shfl_sync(FULL, next, 0);
@@ -779,8 +827,9 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
     ++rs.wj;
     const uint8_t* wbase = isD ? lp.w_d + ((int64_t)e * db + rb) * nc * STAGE_A_BYTES
                                : lp.w_gu + ((int64_t)e * gub + rb) * nc * STAGE_A_BYTES;
-    const int tok = (!isD && lane < nt) ? ld_tab(cx.tokpos + pos0 + lane, cx.global) : 0;
-    const uint32_t stage_bytes = STAGE_A_BYTES + (uint32_t)nt * IMG_BYTES;
+    const int tok = (!LT && !isD && lane < nt) ? ld_tab(cx.tokpos + pos0 + lane, cx.global) : 0;
+    const uint32_t bbytes = LT ? (uint32_t)(LT_SF_BYTES + nt * IMG_CODE_BYTES) : (uint32_t)nt * IMG_BYTES;
+    const uint32_t stage_bytes = STAGE_A_BYTES + bbytes;
     // Stages are issued in batches, one stage per lane: successive 1-D bulk
     // copies issued by one warp instruction each are serialised, while the
     // copies of one instruction proceed in parallel.  A batch is the run of
@@ -791,9 +840,9 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
     while (c0 < nc && ok) {
       const int nb = min(PRODUCER_BATCH, nc - c0);
       const uint32_t s = rs.seq + lane;
-      const int slot = (int)(s % NSLOT);
-      const uint32_t par = ((s / NSLOT) + 1) & 1u;  // completion of the slot's previous use
-      const bool fr = lane < nb && (s < (uint32_t)NSLOT || mbar_test_wait(empty_bar(smem, pipe, slot), par));
+      const int slot = (int)(s % NS);
+      const uint32_t par = ((s / NS) + 1) & 1u;  // completion of the slot's previous use
+      const bool fr = lane < nb && (s < (uint32_t)NS || mbar_test_wait(empty_bar(smem, pipe, slot), par));
       const int k = __ffs(~__ballot_sync(FULL, fr)) - 1;  // leading run of free slots
       if (k == 0) {
         const unsigned long long te0 = clock64();
@@ -803,17 +852,20 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
         if (__any_sync(FULL, bad)) ok = false;
         continue;
       }
-      uint8_t* dst = ring_slot(smem, pipe, slot);
+      uint8_t* dst = LT ? smem + OFF_RING + (size_t)slot * LT_SLOT_BYTES : ring_slot(smem, pipe, slot);
       uint64_t* fb = full_bar(smem, pipe, slot);
       const int c = c0 + lane;
       if (lane < k) {
         mbar_arrive_expect_tx(fb, stage_bytes);
         bulk_g2s(dst, wbase + (int64_t)c * STAGE_A_BYTES, STAGE_A_BYTES, fb);
-        if (isD)
+        if (LT)  // the tile's B operand of this stage, one image
+          bulk_g2s(dst + STAGE_A_BYTES, (isD ? p.atl : p.xtl) + ((int64_t)u * nc + c) * LT_IMG_BYTES,
+                   bbytes, fb);
+        else if (isD)
           bulk_g2s(dst + STAGE_A_BYTES, p.aimg + ((int64_t)c * p.TK + pos0) * IMG_BYTES,
                    (uint32_t)nt * IMG_BYTES, fb);
       }
-      if (!isD) {
+      if (!LT && !isD) {
         for (int tl = 0; tl < nt; ++tl) {
           const int tk = __shfl_sync(FULL, tok, tl);
           if (lane < k)
@@ -833,10 +885,10 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
   }
   // let every issued copy land before the ring is reused or the CTA exits
   const uint32_t issued = rs.seq - seq_start;
-  const uint32_t n = issued < (uint32_t)NSLOT ? issued : (uint32_t)NSLOT;
+  const uint32_t n = issued < (uint32_t)NS ? issued : (uint32_t)NS;
   for (uint32_t s = rs.seq - n; s != rs.seq; ++s) {
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(full_bar(smem, pipe, (int)(s % NSLOT)), (s / NSLOT) & 1u)) {
+    while (!mbar_try_wait(full_bar(smem, pipe, (int)(s % NS)), (s / NS) & 1u)) {
       if (globaltimer_ns() - t0 > p.timeout_ns) break;
     }
   }
@@ -1018,6 +1070,172 @@ __device__ void stream_epilogue(const EngineParams& p, uint8_t* smem, const Stre
   }
 }
 
+// ---- phase C, large T*K: one pipeline over tiles -------------------------------------------
+// Tensor memory: LT_NACC accumulators of LT_ACC_COLS columns, then NSF
+// scale-factor buffers of LT_SF_COLS (A: 4 columns, B: 4 per 128 columns).
+__device__ __forceinline__ uint32_t lt_acc(int b) { return (uint32_t)b * LT_ACC_COLS; }
+__device__ __forceinline__ uint32_t lt_sf(int i) { return (uint32_t)(LT_NACC * LT_ACC_COLS + i * LT_SF_COLS); }
+
+// MMA issuer of the tile stream (one thread): per stage the weight scales and
+// the tile's 1-2 scale blocks go to tensor memory, then two MMAs (K = 64 each,
+// N = 8 per position of the tile) accumulate.
+__device__ void stream_mma_lt(const EngineParams& p, uint8_t* smem, uint32_t tmem, RoleState& rs) {
+  JobEntry* jq = job_queue(smem, 0);
+  const uint32_t ring0 = smem_u32(smem + OFF_RING);
+  const bool prof = p.prof != nullptr;
+  unsigned long long t_full = 0, t_issue = 0, t_acc = 0;
+  bool ok = true;
+  for (;;) {
+    JobEntry* en = jq + (rs.qk % JQ);
+    if (!wait_entry(p, en, rs.qk)) return;
+    const int job = *reinterpret_cast<volatile int32_t*>(&en->job);
+    if (job < 0) { ++rs.qk; break; }
+    const int s0 = en->s0, nc = en->nc, nt = en->nt, wj = en->wj;
+    ++rs.qk;
+    if (!ok) continue;
+    const int b = wj % LT_NACC;
+    const uint32_t use = (uint32_t)(wj / LT_NACC);
+    const unsigned long long ta0 = pclock(prof);
+    if (use > 0 &&
+        !wait_mbar(acce_bar(smem, 0, b), (use - 1) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, wj)) {
+      ok = false;
+      continue;
+    }
+    t_acc += pclock(prof) - ta0;
+    tc_fence_after();
+    const uint32_t tacc = tmem + lt_acc(b);
+    const int n = nt * NTERM, nblk = (n + 127) / 128;
+    const uint32_t idesc0 = mxf4_idesc(n, 0u), idesc1 = mxf4_idesc(n, 2u);
+    for (int c = 0; c < nc; ++c) {
+      const uint32_t s = (uint32_t)s0 + c;
+      const int slot = (int)(s % LT_NSLOT);
+      const unsigned long long tf0 = pclock(prof);
+      if (!wait_mbar(full_bar(smem, 0, slot), (s / LT_NSLOT) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, s)) {
+        ok = false;
+        break;
+      }
+      const unsigned long long tm0 = pclock(prof);
+      t_full += tm0 - tf0;
+      const uint32_t sa = ring0 + (uint32_t)slot * LT_SLOT_BYTES, sb = sa + STAGE_A_BYTES;
+      const uint32_t tsf = tmem + lt_sf((int)(rs.sfc++ % NSF));
+      tmem_cp_sf(tsf, smem_desc(sa + STAGE_CODE_BYTES, 0, 128));
+      for (int q = 0; q < nblk; ++q) tmem_cp_sf(tsf + 4 + 4 * q, smem_desc(sb + q * 512, 0, 128));
+      const uint32_t bc = sb + LT_SF_BYTES;
+      mma_mxf4(tacc, smem_desc(sa, 128, 256), smem_desc(bc, 128, IMG_CODE_BYTES), idesc0, tsf, tsf + 4,
+               c > 0 ? 1u : 0u);
+      mma_mxf4(tacc, smem_desc(sa + 4096, 128, 256), smem_desc(bc + 256, 128, IMG_CODE_BYTES), idesc1,
+               tsf | (2u << 30), (tsf + 4) | (2u << 30), 1u);
+      tc_commit(empty_bar(smem, 0, slot));
+      t_issue += pclock(prof) - tm0;
+    }
+    if (ok) tc_commit(accf_bar(smem, 0, b));
+  }
+  if (prof) {
+    atomicAdd(p.prof + PF_MMA_FULL, t_full);
+    atomicAdd(p.prof + PF_MMA_ISSUE, t_issue);
+    atomicAdd(p.prof + PF_MMA_ACC, t_acc);
+  }
+}
+
+// Epilogue of the tile stream (warps 4..7, warp q reading tensor-memory lanes
+// 32q..32q+31): as stream_epilogue, over up to LT_MAX positions; the SwiGLU
+// term images are written into the tile images of the down jobs.
+__device__ void stream_epilogue_lt(const EngineParams& p, uint8_t* smem, const StreamCtx& cx, uint32_t tmem,
+                                   RoleState& rs) {
+  const int lane = threadIdx.x & 31, q = (threadIdx.x >> 5) & 3;
+  JobEntry* jq = job_queue(smem, 0);
+  uint32_t* ready = p.sync + SY_READY;
+  const int nsd = p.I / KS;
+  const bool prof = p.prof != nullptr;
+  unsigned long long t_wait = 0, t_work = 0, n_jobs = 0;
+  const unsigned long long t_begin = pclock(prof);
+  bool ok = true;
+  float av[LT_MAX];
+  for (;;) {
+    JobEntry* en = jq + (rs.qk % JQ);
+    if (!wait_entry(p, en, rs.qk)) return;
+    const int job = *reinterpret_cast<volatile int32_t*>(&en->job);
+    if (job < 0) { ++rs.qk; break; }
+    const int wj = en->wj;
+    const int u = en->unit, rb = en->rb, isD = en->isD, pos0 = en->pos0, nt = en->nt;
+    ++rs.qk;
+    if (!ok) continue;
+    ++n_jobs;
+    const uint32_t gc = isD ? 0u : rs.gcount++;
+    const int b = wj % LT_NACC;
+    const unsigned long long tw0 = pclock(prof);
+    if (!wait_mbar(accf_bar(smem, 0, b), (uint32_t)(wj / LT_NACC) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, wj)) {
+      ok = false;
+      continue;
+    }
+    const unsigned long long tk0 = pclock(prof);
+    t_wait += tk0 - tw0;
+    tc_fence_after();
+    const uint32_t tacc = tmem + ((uint32_t)(32 * q) << 16) + lt_acc(b);
+    if (!isD) {
+      const int xb = (int)(gc & 1u);
+      float* xc = reinterpret_cast<float*>(smem + OFF_XCH) + xb * LT_MAX * 4;
+      for (int j = 0; j < nt; ++j) {
+        float v[NTERM];
+        tmem_ld8(tacc + j * NTERM, v);
+        float sum = v[NTERM - 1];
+#pragma unroll
+        for (int k = NTERM - 2; k >= 0; --k) sum += v[k];
+        const float other = __shfl_xor_sync(FULL, sum, 16);
+        const float g = lane < 16 ? sum : other, up = lane < 16 ? other : sum;
+        const float a = g / (1.0f + expf(-g)) * up;
+        av[j] = a;
+        float am = fabsf(a);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(FULL, am, o));
+        if (lane == 0) xc[j * 4 + q] = am;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xch_bar(smem, 0, xb));
+      if (!wait_mbar(xch_bar(smem, 0, xb), (gc >> 1) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, wj)) {
+        ok = false;
+        continue;
+      }
+      const int i0 = rb * GU_I_ROWS, sD = i0 / KS, kk = (i0 % KS) / 64, kc = q >> 1;
+      uint8_t* img = p.atl + ((int64_t)u * nsd + sD) * LT_IMG_BYTES;
+      for (int j = 0; j < nt; ++j) {
+        const int s0 = term0_exp(fmaxf(xc[j * 4 + q], xc[j * 4 + (q ^ 1)]));
+        const uint32_t word = term_word<16>(e2m1_terms(av[j], s0), lane);
+        if (lane < 16)
+          *reinterpret_cast<uint32_t*>(img + lt_code_offset(j) + kk * 256 + kc * 128 + (lane >> 1) * 16 +
+                                       (q & 1) * 8 + (lane & 1) * 4) = word;
+        if ((q & 1) == 0 && lane < NTERM) img[lt_sf_offset(j, lane, 2 * kk + kc)] = (uint8_t)(term_exp(s0, lane) + 127);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        fence_proxy_async_global();
+        __threadfence();
+        red_release_add_u32(ready + u, 1u);
+      }
+    } else {
+      const int h0 = rb * JOB_ROWS;
+      for (int j = 0; j < nt; ++j) {
+        float v[NTERM];
+        tmem_ld8(tacc + j * NTERM, v);
+        float sum = v[NTERM - 1];
+#pragma unroll
+        for (int k = NTERM - 2; k >= 0; --k) sum += v[k];
+        p.ypair[(int64_t)(pos0 + j) * p.H + h0 + 32 * q + lane] = sum * ld_tab(cx.wpos + pos0 + j, cx.global);
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(acce_bar(smem, 0, b));
+    t_work += pclock(prof) - tk0;
+  }
+  if (prof && lane == 0) {
+    atomicAdd(p.prof + PF_EPI_WAIT, t_wait);
+    atomicAdd(p.prof + PF_EPI_WORK, t_work);
+    atomicAdd(p.prof + PF_EPI_TOTAL, pclock(prof) - t_begin);
+    if (q == 0) atomicAdd(p.prof + PF_JOBS, n_jobs);
+  }
+}
+
 // ---- phase D: combine (+ RMSNorm) ------------------------------------------------------------
 __device__ __forceinline__ void store_bf16x4(__nv_bfloat16* dst, float4 v) {
   __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
@@ -1097,6 +1315,7 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
                            bool stamp) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool small = p.TK <= SMALL_PAIRS;
+  const bool tiles = use_tiles(p.TK, p.E);
   CtaTables& tb = tables(smem);
   for (int layer = 0; layer < p.L; ++layer) {
     const LayerPtrs& lp = p.layers[layer];
@@ -1120,22 +1339,37 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
       phase_permute_large(p, smem);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 3)) return;
       if (p.route_only) return;
+      if (tiles) {
+        phase_tile_gather(p);
+        if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 6)) return;
+      }
       cx = StreamCtx{p.units, p.dunits, p.tokpos, p.wpos, (int)ld_cg_u32(p.n_units), (int)ld_cg_u32(p.n_units + 1), true};
       inv = p.inv;
     }
     if (st) st[4] = globaltimer_ns();
     fence_proxy_async_smem();  // the ring held routing scratch written by generic stores
     __syncthreads();
-    if (warp < EPI_WARP0) {
-      const int pipe = warp >> 1;
-      if ((warp & 1) == 0) {
-        stream_producer(p, lp, smem, cx, pipe, rs);
+    if (!tiles) {  // two pipelines per CTA, units of <= NT_MAX positions
+      if (warp < EPI_WARP0) {
+        const int pipe = warp >> 1;
+        if ((warp & 1) == 0) {
+          stream_producer<false>(p, lp, smem, cx, pipe, rs);
+        } else {
+          if (lane == 0) stream_mma(p, smem, tmem, pipe, rs);
+          __syncwarp();
+        }
       } else {
-        if (lane == 0) stream_mma(p, smem, tmem, pipe, rs);
-        __syncwarp();
+        stream_epilogue(p, smem, cx, tmem, (warp - EPI_WARP0) / 4, rs);
       }
-    } else {
-      stream_epilogue(p, smem, cx, tmem, (warp - EPI_WARP0) / 4, rs);
+    } else {  // one pipeline per CTA over tiles of <= LT_MAX positions
+      if (warp == 0) {
+        stream_producer<true>(p, lp, smem, cx, 0, rs);
+      } else if (warp == 1) {
+        if (lane == 0) stream_mma_lt(p, smem, tmem, rs);
+        __syncwarp();
+      } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
+        stream_epilogue_lt(p, smem, cx, tmem, rs);
+      }
     }
     if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 4)) return;
     if (st) st[5] = globaltimer_ns();

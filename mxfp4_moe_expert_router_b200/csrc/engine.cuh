@@ -57,11 +57,45 @@ constexpr int NACC = 2;                                  // accumulator buffers 
 constexpr int ACC_COLS = NT_MAX * NTERM;                 // 32 columns per buffer
 constexpr int NSF = 4;                                   // scale-factor buffers per pipeline
 constexpr int SF_COLS = 8;                               // A (4 columns) + B (4 columns)
-constexpr int TMEM_COLS = 256;
+constexpr int TMEM_COLS = 512;                          // the whole tensor memory of the SM
 static_assert(NPIPE * (NACC * ACC_COLS + NSF * SF_COLS) <= TMEM_COLS, "tensor memory budget");
 // a batch's stages must occupy distinct slots whose previous use is already issued
 static_assert(PRODUCER_BATCH <= NSLOT && PRODUCER_BATCH < 32, "producer batch");
 constexpr int SMALL_PAIRS = 256;                         // T*K up to this: routing done per CTA
+
+// ---- large T*K: tile stream --------------------------------------------------------------
+// With many tokens per expert (T*K >= LT_MIN_PER_EXPERT * E) a unit ("tile")
+// holds up to LT_MAX consecutive positions of one expert's segment and one MMA
+// covers all of them (N = 8 per position, up to 192).  Per (tile, 128-K stage)
+// the B operand is one image: LT_SF_BLOCKS blocks of 512 bytes in the
+// scale-factor copy layout (the scale of column n = 8 tl + k sits in block
+// n / 128, row n % 32, bytes 4 ((n / 32) % 4) + block index), then LT_MAX x 512
+// bytes of E2M1 term codes (position tl at LT_SF_BYTES + tl * 512, the layout
+// of a single image's codes).  One bulk copy of LT_SF_BYTES + nt * 512 bytes
+// brings a tile's B operand for a stage.
+constexpr int LT_MAX = 24;
+constexpr int LT_MIN_PER_EXPERT = 8;                     // T*K / E from which tiles are used
+constexpr int LT_SF_BLOCKS = 2;                          // 32-row copies covering N <= 256
+constexpr int LT_SF_BYTES = LT_SF_BLOCKS * 512;
+constexpr int LT_CODE_BYTES = LT_MAX * IMG_CODE_BYTES;   // 12288
+constexpr int LT_IMG_BYTES = LT_SF_BYTES + LT_CODE_BYTES;  // 13312
+constexpr int LT_SLOT_BYTES = STAGE_A_BYTES + LT_IMG_BYTES;       // 22016
+constexpr int LT_NSLOT = 9;                              // one pipeline
+constexpr int LT_ACC_COLS = LT_MAX * NTERM;              // 192
+constexpr int LT_NACC = 2;
+constexpr int LT_SF_COLS = 4 + 4 * LT_SF_BLOCKS;         // 12
+static_assert(LT_NACC * LT_ACC_COLS + NSF * LT_SF_COLS <= TMEM_COLS, "tensor memory budget (tiles)");
+static_assert(LT_NSLOT <= NPIPE * NSLOT, "tile ring barriers");
+static_assert(8 * LT_MAX <= 128 * LT_SF_BLOCKS, "tile scale-factor blocks");
+// Byte offset in a tile image of the scale of position tl, term k, block kb.
+__host__ __device__ constexpr int lt_sf_offset(int tl, int k, int kb) {
+  return (tl / 16) * 512 + (8 * (tl % 4) + k) * 16 + 4 * ((tl % 16) / 4) + kb;
+}
+__host__ __device__ constexpr int lt_code_offset(int tl) { return LT_SF_BYTES + tl * IMG_CODE_BYTES; }
+// Whether a launch of T*K pairs over E experts streams tiles.
+__host__ __device__ inline bool use_tiles(int64_t TK, int E) {
+  return TK > SMALL_PAIRS && TK >= (int64_t)LT_MIN_PER_EXPERT * E;
+}
 constexpr int STAMPS_PER_LAYER = 7;  // x converted, logits (CTA 0), prepared, top-k, routed, streamed, combined
 
 // sync word layout (uint32)
@@ -77,6 +111,8 @@ enum : uint32_t {
 
 // Upper bounds of the unit tables for T*K pairs over E experts.
 __host__ __device__ inline int max_units(int E, int64_t TK) { return (int)((E < TK ? E : TK) + TK / NT_MAX + 1); }
+// Tiles of the large path (at most LT_MAX positions each).
+__host__ __device__ inline int max_tiles(int E, int64_t TK) { return (int)((E < TK ? E : TK) + TK / LT_MAX + 1); }
 __host__ __device__ inline int max_dunits(int E, int64_t TK) { return (int)((E < TK ? E : TK) + TK / ND_MAX + 1); }
 
 // Router split of H into HS parts of H / HS elements (a multiple of 8).
@@ -115,6 +151,8 @@ struct EngineParams {
   int32_t* dunits;            // [Dmax][4] down units (expert, pos0, nt <= ND_MAX, gate/up unit)
   int32_t* n_units;           // [2] gate/up units, down units
   uint8_t* aimg;              // [I/KS][TK][IMG_BYTES] E2M1 term images of the SwiGLU output
+  uint8_t* xtl;               // large T*K: [tiles][H/KS][LT_IMG_BYTES] x term images per tile
+  uint8_t* atl;               // large T*K: [tiles][I/KS][LT_IMG_BYTES] SwiGLU term images per tile
   float* ypair;               // [TK][H]
   uint32_t* sync;             // see SY_*
   uint64_t* stamps;           // null or [1 + MAX_LAYERS * STAMPS_PER_LAYER] %globaltimer ns (CTA 0)

@@ -25,6 +25,8 @@ struct moe_mxfp4 {
   double* logits = nullptr;
   uint8_t* xt = nullptr;
   uint8_t* aimg = nullptr;
+  uint8_t* xtl = nullptr;  // large T*k only
+  uint8_t* atl = nullptr;
   __nv_bfloat16* xnext = nullptr;
   int32_t *idx = nullptr, *counts = nullptr, *offsets = nullptr, *perm = nullptr, *inv = nullptr,
           *tokpos = nullptr, *units = nullptr, *dunits = nullptr, *n_units = nullptr;
@@ -88,6 +90,7 @@ EngineParams base_params(const moe_mxfp4* h, int T) {
   p.idx = h->idx; p.wts = h->wts; p.counts = h->counts; p.offsets = h->offsets;
   p.perm = h->perm; p.inv = h->inv; p.tokpos = h->tokpos; p.wpos = h->wpos;
   p.units = h->units; p.dunits = h->dunits; p.n_units = h->n_units; p.aimg = h->aimg;
+  p.xtl = h->xtl; p.atl = h->atl;
   p.ypair = h->ypair;
   p.sync = h->sync;
   p.stamps = h->stamps;
@@ -191,6 +194,10 @@ int32_t moe_mxfp4_create(const moe_config_t* cfg, const uint8_t* const* gate_cod
        dalloc(h, &h->stamps, (size_t)(1 + MAX_LAYERS * STAMPS_PER_LAYER) * 8) &&
        dalloc(h, &h->prof, (size_t)PROF_COUNTERS * 8) &&
        dalloc(h, &h->x_stage, (size_t)Tm * H * 2) && dalloc(h, &h->y_stage, (size_t)Tm * H * 2);
+  if (ok && use_tiles(TKm, E)) {  // tile images of the large-T*k stream
+    const size_t tiles = (size_t)max_tiles(E, TKm);
+    ok = dalloc(h, &h->xtl, tiles * (H / KS) * LT_IMG_BYTES) && dalloc(h, &h->atl, tiles * (I / KS) * LT_IMG_BYTES);
+  }
   if (!ok) { free_all(h); delete h; cudaGetLastError(); return MOE_ERR_OOM; }
 
   // term images: the scale rows' padding bytes 4..15 are read by the
