@@ -1311,11 +1311,11 @@ __device__ void phase_combine_rmsnorm(const EngineParams& p, const int32_t* inv,
 
 // All layers; returns early (every thread of the CTA together) when a grid
 // barrier reports an error, or after routing in route-only mode.
+template <bool TILES>
 __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, RoleState& rs,
                            bool stamp) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool small = p.TK <= SMALL_PAIRS;
-  const bool tiles = use_tiles(p.TK, p.E);
   CtaTables& tb = tables(smem);
   for (int layer = 0; layer < p.L; ++layer) {
     const LayerPtrs& lp = p.layers[layer];
@@ -1339,7 +1339,7 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
       phase_permute_large(p, smem);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 3)) return;
       if (p.route_only) return;
-      if (tiles) {
+      if constexpr (TILES) {
         phase_tile_gather(p);
         if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 6)) return;
       }
@@ -1349,7 +1349,7 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
     if (st) st[4] = globaltimer_ns();
     fence_proxy_async_smem();  // the ring held routing scratch written by generic stores
     __syncthreads();
-    if (!tiles) {  // two pipelines per CTA, units of <= NT_MAX positions
+    if constexpr (!TILES) {  // two pipelines per CTA, units of <= NT_MAX positions
       if (warp < EPI_WARP0) {
         const int pipe = warp >> 1;
         if ((warp & 1) == 0) {
@@ -1383,6 +1383,9 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
   }
 }
 
+// Two instances: the pipeline stream (TILES = false) and the tile stream; each
+// holds only its own stream code.
+template <bool TILES>
 __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1414,7 +1417,7 @@ __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p
   const bool stamp = p.stamps != nullptr && blockIdx.x == 0 && threadIdx.x == 0;
   if (stamp) p.stamps[0] = globaltimer_ns();
   RoleState rs;
-  run_layers(p, smem, tmem, rs, stamp);
+  run_layers<TILES>(p, smem, tmem, rs, stamp);
   if (use_tmem) {
     // free tensor memory only once every MMA this CTA issued has completed
     if (warp < EPI_WARP0 && (warp & 1) && lane == 0) {
@@ -1438,13 +1441,16 @@ __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p
 size_t engine_smem_bytes() { return SMEM_BYTES; }
 
 int engine_max_grid(int device, int* err) {
-  cudaError_t e = cudaFuncSetAttribute(engine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SMEM_BYTES);
-  if (e != cudaSuccess) { *err = (int)e; return 0; }
-  int per_sm = 0, sms = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, engine_kernel, THREADS, SMEM_BYTES);
-  if (e != cudaSuccess) { *err = (int)e; return 0; }
-  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+  int per_sm = ~0u >> 1, sms = 0;
+  for (const void* k : {(const void*)engine_kernel<false>, (const void*)engine_kernel<true>}) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) { *err = (int)e; return 0; }
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, THREADS, SMEM_BYTES);
+    if (e != cudaSuccess) { *err = (int)e; return 0; }
+    per_sm = n < per_sm ? n : per_sm;
+  }
+  cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
   if (e != cudaSuccess) { *err = (int)e; return 0; }
   *err = 0;
   return per_sm * sms;
@@ -1452,8 +1458,9 @@ int engine_max_grid(int device, int* err) {
 
 cudaError_t engine_launch(const EngineParams& p, int grid, cudaStream_t s) {
   void* args[] = {const_cast<EngineParams*>(&p)};
-  return cudaLaunchCooperativeKernel((const void*)engine_kernel, dim3(grid), dim3(THREADS), args,
-                                     SMEM_BYTES, s);
+  const void* k = use_tiles(p.TK, p.E) && !p.route_only ? (const void*)engine_kernel<true>
+                                                        : (const void*)engine_kernel<false>;
+  return cudaLaunchCooperativeKernel(k, dim3(grid), dim3(THREADS), args, SMEM_BYTES, s);
 }
 
 }  // namespace moe
