@@ -381,7 +381,7 @@ def main():
                          "traffic": traffic, "kernel": "engine_kernel"},
             "gpu_launches": args.steps,
             "phase_us_last_step": {k: round(v / 1e3, 2) for k, v in
-                                   zip(("convert_x", "router_logits", "grid_wait", "topk", "permute", "stream",
+                                   zip(("router_logits", "x_images", "route_wait", "topk_or_tables", "permute", "stream",
                                        "combine"), phases[:7])},
             "e2e": e2e,
             "cpu_baseline": cpu,

@@ -165,9 +165,11 @@ MOE_API int32_t moe_status(moe_mxfp4_t* h, void* stream);
 /*
  * moe_phase_ns -- tracing: synchronise `stream`, then write to the HOST array
  * ns_out up to max_n durations (ns, %globaltimer of CTA 0) of the last
- * moe_forward of the handle, seven per layer: CTA 0's activation conversion
- * and router logits, the wait for the rest of the grid, top-k, permutation +
- * unit tables, the MXFP4 weight stream, combine (+ RMSNorm).
+ * moe_forward of the handle, seven per layer, as seen by CTA 0: router
+ * logits; x term images (T*K <= 256: after arriving at the routing barrier);
+ * the wait for the routing; top-k (T*K <= 256: the copy of the routing
+ * tables); permutation + unit tables (+ tile gather); the MXFP4 weight
+ * stream; combine (+ RMSNorm).
  * Values of a launch that stopped early are unspecified.
  */
 MOE_API int32_t moe_phase_ns(moe_mxfp4_t* h, uint64_t* ns_out, int32_t max_n, void* stream);

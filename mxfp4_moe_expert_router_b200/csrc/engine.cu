@@ -246,26 +246,14 @@ __device__ __forceinline__ RouterWork router_work(const EngineParams& p) {
   return RouterWork{c, g, 0, 1};
 }
 
-// L2 prefetch of the router weight rows this CTA's dot products will read.
-__device__ void router_prefetch(const EngineParams& p, const LayerPtrs& lp) {
-  const RouterWork rw = router_work(p);
-  const int hpart = p.H / p.HS;
-#pragma unroll 1
-  for (int hs = rw.hs0; hs < p.HS; hs += rw.hstep) {
-    const int ne = (p.E - rw.e0 + rw.estep - 1) / rw.estep;
-#pragma unroll 1
-    for (int k = (int)threadIdx.x; k < ne; k += THREADS)
-      prefetch_l2_bulk(lp.router_w + (int64_t)(rw.e0 + k * rw.estep) * p.H + hs * hpart, (uint32_t)hpart * 4u);
-  }
-}
-
-// Sum over the warp of 16 values per lane, reduce-scatter order: afterwards
-// lane l holds the total of value l % 16 (16 double shuffles instead of 80).
-__device__ __forceinline__ double warp_sum16(double (&v)[RTC], int lane) {
-  static_assert(RTC == 16, "reduce-scatter written for 16 values");
+// Sum over the warp of P values per lane (P a power of two <= 32),
+// reduce-scatter order: afterwards lane l holds the total of value l % P
+// (P - 1 + 5 - log2 P double shuffles instead of 5 P).
+template <int P>
+__device__ __forceinline__ double warp_sum_rs(double (&v)[P], int lane) {
 #pragma unroll
-  for (int st = 0; st < 4; ++st) {
-    const int n = 8 >> st;  // values kept after this step
+  for (int st = 0; (1 << st) < P; ++st) {
+    const int n = P >> (st + 1);  // values kept after this step
     const bool hi = (lane >> st) & 1;
 #pragma unroll
     for (int k = 0; k < n; ++k) {
@@ -274,19 +262,67 @@ __device__ __forceinline__ double warp_sum16(double (&v)[RTC], int lane) {
       v[k] = keep + __shfl_xor_sync(FULL, send, 1 << st);
     }
   }
-  return v[0] + __shfl_xor_sync(FULL, v[0], 16);
+  double r = v[0];
+#pragma unroll
+  for (int o = P; o < 32; o <<= 1) r += __shfl_xor_sync(FULL, r, o);
+  return r;
 }
+
+// Router dot products of one token chunk of nt <= NT tokens: warp per expert
+// k of this CTA, lanes along this H part, fp64 accumulation (bf16 x as fp64
+// in xd[RTC][hpart]; rows nt..NT-1 are ignored), fp32 weights, then one
+// reduce-scatter over the lanes.
+// (Scalar arguments: a reference to the kernel's parameter block would move
+// that block to local memory for the whole kernel.)
+__host__ __device__ constexpr int pow2_at_least(int n) { return n <= 1 ? 1 : 2 * pow2_at_least((n + 1) / 2); }
+template <int NT>
+__device__ __forceinline__ void router_dots(const double* xd, const float* wsm, const float* router_w,
+                                         int nexp, int e0, int estep, int H, int hpart, int hs,
+                                         double* logits, int T, int t0, int nt, int E) {
+  constexpr int P = pow2_at_least(NT);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int k = warp; k < nexp; k += WARPS) {
+    const int e = e0 + k * estep;
+    const float* wr = wsm ? wsm + (size_t)k * hpart : router_w + (int64_t)e * H + hs * hpart;
+    double acc[P];
+#pragma unroll
+    for (int j = 0; j < P; ++j) acc[j] = 0.0;
+#pragma unroll 4
+    for (int h = lane; h < hpart; h += 32) {
+      const double w = (double)wr[h];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) acc[j] = fma(xd[j * hpart + h], w, acc[j]);
+    }
+    const double v = warp_sum_rs<P>(acc, lane);  // lane l (< nt <= NT) holds token t0 + l
+    if (lane < nt) logits[((int64_t)hs * T + t0 + lane) * E + e] = v;
+  }
+}
+
+// One token chunk: nt rounded up to 1, 2, 4, 8, 9, 12 or 16.
+__device__ __noinline__ void router_chunk(const double* xd, const float* wsm, const float* router_w,
+                                          int nexp, int e0, int estep, int H, int hpart, int hs,
+                                          double* logits, int T, int t0, int nt, int E) {
+#define MOE_ROUTER_DOTS(NT) router_dots<NT>(xd, wsm, router_w, nexp, e0, estep, H, hpart, hs, logits, T, t0, nt, E)
+  if (nt == 1) MOE_ROUTER_DOTS(1);
+  else if (nt == 2) MOE_ROUTER_DOTS(2);
+  else if (nt <= 4) MOE_ROUTER_DOTS(4);
+  else if (nt <= 8) MOE_ROUTER_DOTS(8);
+  else if (nt == 9) MOE_ROUTER_DOTS(9);
+  else if (nt <= 12) MOE_ROUTER_DOTS(12);
+  else MOE_ROUTER_DOTS(16);
+#undef MOE_ROUTER_DOTS
+}
+
 // x[t] (bf16) -> xt[stage][t]: per 32-element block one warp expands the values
 // into NTERM E2M1 terms (codes at the MMA's B-operand rows, scales at the
-// scale-factor rows of the image).
-__device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const __nv_bfloat16* x,
-                              int layer, uint8_t* smem, uint64_t* stamp) {
-  const int T = p.T, H = p.H, E = p.E;
+// scale-factor rows of the image).  Also the layer-input copy of the optional
+// per-layer output.
+__device__ void phase_images(const EngineParams& p, const __nv_bfloat16* x, int layer) {
+  const int T = p.T, H = p.H;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t gt = (int64_t)blockIdx.x * THREADS + threadIdx.x;
   const int64_t gs = (int64_t)gridDim.x * THREADS;
   const int64_t wg = (int64_t)blockIdx.x * WARPS + warp, ws = (int64_t)gridDim.x * WARPS;
-  router_prefetch(p, lp);
   const int nblk = H / 32;
   const int64_t ntask = p.route_only ? 0 : (int64_t)T * nblk;  // routing alone needs no images
   for (int64_t task = wg; task < ntask; task += ws) {
@@ -302,13 +338,20 @@ __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const 
     *reinterpret_cast<uint32_t*>(img + kk * 256 + kc * 128 + (lane >> 2) * 16 + (lane & 3) * 4) = word;
     if (lane < NTERM) img[IMG_CODE_BYTES + lane * 16 + b] = (uint8_t)(term_exp(s0, lane) + 127);
   }
-  if (stamp) stamp[0] = globaltimer_ns();
   if (p.layer_io) {
     const int64_t n8 = (int64_t)T * H / 8;
     const uint4* s8 = reinterpret_cast<const uint4*>(x);
     uint4* d8 = reinterpret_cast<uint4*>(p.layer_io + (int64_t)layer * T * H);
     for (int64_t i = gt; i < n8; i += gs) d8[i] = __ldcg(s8 + i);
   }
+}
+
+// Router partial logits (and the per-layer resets of the stream's counters).
+__device__ void phase_router(const EngineParams& p, const LayerPtrs& lp, const __nv_bfloat16* x,
+                             uint8_t* smem) {
+  const int T = p.T, H = p.H, E = p.E;
+  const int64_t gt = (int64_t)blockIdx.x * THREADS + threadIdx.x;
+  const int64_t gs = (int64_t)gridDim.x * THREADS;
   // per-layer resets of the stream's counters (used only after the next barrier)
   const int umax = max_units(E, p.TK);
   if (gt == 0) p.sync[SY_JOBS] = 0u;
@@ -327,52 +370,52 @@ __device__ void phase_prepare(const EngineParams& p, const LayerPtrs& lp, const 
   float* wsm = reinterpret_cast<float*>(xd + (size_t)RTC * hpart);
   const int nexp = rw.e0 < E ? (E - rw.e0 + rw.estep - 1) / rw.estep : 0;
   const bool wstaged = ((size_t)RTC * hpart * 8 + (size_t)nexp * hpart * 4) <= RING_BYTES;
+  const int hp8 = hpart / 8, hp4 = hpart / 4;  // 16-byte loads (H / HS is a multiple of 8)
   for (int hs = rw.hs0; hs < HS; hs += rw.hstep) {
-    if (wstaged) {
-      __syncthreads();  // the previous part's readers are done
-      const int hp4 = hpart / 4;
-      for (int i = threadIdx.x; i < nexp * hp4; i += THREADS) {
-        const int k = i / hp4, h4 = i - k * hp4;
-        reinterpret_cast<float4*>(wsm)[i] =
-            __ldg(reinterpret_cast<const float4*>(lp.router_w + (int64_t)(rw.e0 + k * rw.estep) * H + hs * hpart) + h4);
-      }
-    }
     for (int t0 = 0; t0 < T; t0 += RTC) {
       const int nt = min(RTC, T - t0);
       __syncthreads();  // the previous chunk's readers are done
-      const int hp8 = hpart / 8;  // 8 bf16 per 16-byte load (H / HS is a multiple of 8)
-#pragma unroll 4
-      for (int i = threadIdx.x; i < nt * hp8; i += THREADS) {
-        const int t = i / hp8, h8 = i - t * hp8;
-        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(x + (int64_t)(t0 + t) * H + hs * hpart) + h8);
-        double* d = xd + (size_t)t * hpart + h8 * 8;
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+      // stage the chunk's x slice as fp64 and, with a part's first chunk, the
+      // part's weight slices; a thread's loads are all in flight before its
+      // stores (one memory round trip for both)
+      const int nx = nt * hp8, nw = (t0 == 0 && wstaged) ? nexp * hp4 : 0;
+      constexpr int RB = 2;
+#pragma unroll 1
+      for (int i0 = threadIdx.x; i0 < nx + nw; i0 += RB * THREADS) {
+        uint4 v[RB];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          d[2 * q] = (double)__uint_as_float(u[q] << 16);
-          d[2 * q + 1] = (double)__uint_as_float(u[q] & 0xFFFF0000u);
+        for (int r = 0; r < RB; ++r) {
+          const int i = i0 + r * THREADS;
+          if (i < nx) {
+            const int t = i / hp8, h8 = i - t * hp8;
+            v[r] = __ldcg(reinterpret_cast<const uint4*>(x + (int64_t)(t0 + t) * H + hs * hpart) + h8);
+          } else if (i < nx + nw) {
+            const int k = (i - nx) / hp4, h4 = (i - nx) - k * hp4;
+            v[r] = __ldg(reinterpret_cast<const uint4*>(lp.router_w + (int64_t)(rw.e0 + k * rw.estep) * H + hs * hpart) + h4);
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < RB; ++r) {
+          const int i = i0 + r * THREADS;
+          if (i < nx) {
+            const int t = i / hp8, h8 = i - t * hp8;
+            double* d = xd + (size_t)t * hpart + h8 * 8;
+            const uint32_t u[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              d[2 * q] = (double)__uint_as_float(u[q] << 16);
+              d[2 * q + 1] = (double)__uint_as_float(u[q] & 0xFFFF0000u);
+            }
+          } else if (i < nx + nw) {
+            reinterpret_cast<uint4*>(wsm)[i - nx] = v[r];
+          }
         }
       }
       __syncthreads();
-      for (int k = warp; k < nexp; k += WARPS) {
-        const int e = rw.e0 + k * rw.estep;
-        const float* wr = wstaged ? wsm + (size_t)k * hpart : lp.router_w + (int64_t)e * H + hs * hpart;
-        double acc[RTC];
-#pragma unroll
-        for (int j = 0; j < RTC; ++j) acc[j] = 0.0;
-#pragma unroll 4
-        for (int h = lane; h < hpart; h += 32) {
-          const double w = (double)wr[h];
-#pragma unroll
-          for (int j = 0; j < RTC; ++j)
-            if (j < nt) acc[j] = fma(xd[j * hpart + h], w, acc[j]);
-        }
-        const double v = warp_sum16(acc, lane);  // lane l (< 16) holds token t0 + l
-        if (lane < nt) p.logits[((int64_t)hs * T + t0 + lane) * E + e] = v;
-      }
+      router_chunk(xd, wstaged ? wsm : nullptr, lp.router_w, nexp, rw.e0, rw.estep, H, hpart, hs, p.logits,
+                   T, t0, nt, E);
     }
   }
-  if (stamp) stamp[1] = globaltimer_ns();
 }
 
 // ---- phase B: top-k, weights, permutation ------------------------------------------------
@@ -385,67 +428,144 @@ __device__ __forceinline__ double key_value(uint64_t k) {
   return __longlong_as_double((long long)b);
 }
 
-// One warp: logits of token t (partials summed in order, plus bias), the K
-// largest (descending, ties to the lower expert), weights exp(l - lmax) / sum
-// over the K.  Lane r < K writes slot r.  The token's keys (order-preserving
-// 64-bit images of the fp64 logits) sit in the warp's shared-memory row; each
-// of the K rounds takes every lane's best key, then the warp-wide maximum
-// (the lower expert on equal keys), and removes the winner.  Kept out of line
-// and without unrolled sorting networks: the code runs once per layer and its
-// instruction fetch, not its arithmetic, sets its latency.
+// Key order: descending key, ascending expert on equal keys.
+__device__ __forceinline__ bool key_before(uint64_t ka, int ea, uint64_t kb, int eb) {
+  return ka > kb || (ka == kb && ea < eb);
+}
+__device__ __forceinline__ void key_exchange(uint64_t& ka, int& ea, uint64_t& kb, int& eb) {
+  if (key_before(kb, eb, ka, ea)) {
+    const uint64_t tk = ka; ka = kb; kb = tk;
+    const int te = ea; ea = eb; eb = te;
+  }
+}
+// The best of a lane's NK keys (a pairwise tournament; on equal keys the
+// lower index, which is the lower expert, wins).
+template <int NK>
+__device__ __forceinline__ void lane_best(const uint64_t (&key)[NK], uint64_t& best, int& bj) {
+  uint64_t k[NK];
+  int j[NK];
+#pragma unroll
+  for (int i = 0; i < NK; ++i) { k[i] = key[i]; j[i] = i; }
+#pragma unroll
+  for (int w = 1; w < NK; w <<= 1)
+#pragma unroll
+    for (int i = 0; i + w < NK; i += 2 * w)
+      if (k[i + w] > k[i]) { k[i] = k[i + w]; j[i] = j[i + w]; }
+  best = k[0];
+  bj = j[0];
+}
+
+// One warp: logits of token t (the H-part partials summed pairwise, plus
+// bias), the K largest (descending, ties to the lower expert), weights
+// exp(l - lmax) / sum over the K (fp32).  Lane r < K writes slot r and, when
+// `sel` is given, sets bit t of the winner's token mask sel[e * tw + t / 32].
+// Expert e = lane + 32 j is key j of its lane (an order-preserving 64-bit
+// image of the fp64 logit, in registers, NK >= E / 32 per lane).  Each of
+// the K rounds finds the warp-wide maximum of the lanes' best keys (the lower
+// expert on equal keys): one reduction of the keys' upper words, and only
+// when several lanes share that word, two more.  The winning lane then moves
+// to its next key: with four keys a lane keeps them sorted (five exchanges)
+// and shifts; with more it rescans them (a tournament).
 // (Scalar arguments: a reference to the kernel's parameter block would move
 // that block to local memory for the whole kernel.)
-__device__ __noinline__ void topk_row(const double* logits, int T, int E, int K, int HS,
-                                      const float* bias, int t, uint64_t* keys, int32_t* out_idx,
-                                      float* out_w) {
+template <int NK>
+__device__ __noinline__ void topk_nk(const double* logits, int T, int E, int K, int HS,
+                                     const float* bias, int t, int32_t* out_idx, float* out_w,
+                                     uint32_t* sel, int tw) {
   const int lane = threadIdx.x & 31;
-  // all of a lane's partial loads in flight at once (four experts x MAX_HSPLIT parts)
-#pragma unroll 1
-  for (int e0 = lane; e0 < E; e0 += 128) {
+  uint64_t key[NK];
+  // four experts per lane at a time, all their partial loads in flight at once
+#pragma unroll
+  for (int c = 0; c < NK / 4; ++c) {
     double part[4][MAX_HSPLIT];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int hs = 0; hs < MAX_HSPLIT; ++hs) {
-        const int e = e0 + 32 * i;
+        const int e = 32 * (4 * c + i) + lane;
         part[i][hs] = (hs < HS && e < E) ? __ldcg(logits + ((int64_t)hs * T + t) * E + e) : 0.0;
       }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int e = e0 + 32 * i;
-      double l = 0.0;
-#pragma unroll
-      for (int hs = 0; hs < MAX_HSPLIT; ++hs) l += part[i][hs];
-      if (e < E) keys[e] = order_key(bias ? l + (double)bias[e] : l);
+      const int e = 32 * (4 * c + i) + lane;
+      static_assert(MAX_HSPLIT == 8, "pairwise sum written for 8 parts");
+      const double l = ((part[i][0] + part[i][1]) + (part[i][2] + part[i][3])) +
+                       ((part[i][4] + part[i][5]) + (part[i][6] + part[i][7]));
+      key[4 * c + i] = e < E ? order_key(bias ? l + (double)bias[e] : l) : 0ull;
     }
   }
-  __syncwarp();
+  uint64_t best;
+  int be;  // expert of `best`
+  int ex[4];
+  if constexpr (NK == 4) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) ex[j] = 32 * j + lane;
+    key_exchange(key[0], ex[0], key[1], ex[1]);
+    key_exchange(key[2], ex[2], key[3], ex[3]);
+    key_exchange(key[0], ex[0], key[2], ex[2]);
+    key_exchange(key[1], ex[1], key[3], ex[3]);
+    key_exchange(key[1], ex[1], key[2], ex[2]);
+    best = key[0];
+    be = ex[0];
+  } else {
+    int bj;
+    lane_best<NK>(key, best, bj);
+    be = 32 * bj + lane;
+  }
   int my_e = -1;
   double my_l = 0.0, lmax = 0.0;
 #pragma unroll 1
   for (int r = 0; r < K; ++r) {
-    uint64_t best = 0ull;
-    int be = E;
-#pragma unroll 1
-    for (int e = lane; e < E; e += 32) {
-      const uint64_t k = keys[e];
-      if (k > best) { best = k; be = e; }  // ascending e: equal keys keep the lower expert
-    }
     const uint32_t hi = __reduce_max_sync(FULL, (uint32_t)(best >> 32));
-    const uint32_t lo = __reduce_max_sync(FULL, (uint32_t)(best >> 32) == hi ? (uint32_t)best : 0u);
-    const uint64_t top = ((uint64_t)hi << 32) | lo;
-    const int esel = (int)__reduce_min_sync(FULL, best == top ? (uint32_t)be : 0xFFFFFFFFu);
-    if (lane == (esel & 31)) keys[esel] = 0ull;
-    __syncwarp();
-    const double v = key_value(top);
+    const uint32_t tied = __ballot_sync(FULL, (uint32_t)(best >> 32) == hi);
+    uint32_t lo, esel;
+    if ((tied & (tied - 1u)) == 0u) {  // one lane holds the maximum
+      const int wl = __ffs(tied) - 1;
+      lo = __shfl_sync(FULL, (uint32_t)best, wl);
+      esel = (uint32_t)__shfl_sync(FULL, be, wl);
+    } else {
+      lo = __reduce_max_sync(FULL, (uint32_t)(best >> 32) == hi ? (uint32_t)best : 0u);
+      const uint64_t top = ((uint64_t)hi << 32) | lo;
+      esel = __reduce_min_sync(FULL, best == top ? (uint32_t)be : 0xFFFFFFFFu);
+    }
+    if ((uint32_t)be == esel) {  // the winner's lane moves to its next key
+      if constexpr (NK == 4) {
+        key[0] = key[1]; key[1] = key[2]; key[2] = key[3]; key[3] = 0ull;
+        ex[0] = ex[1]; ex[1] = ex[2]; ex[2] = ex[3]; ex[3] = 0x7FFFFFFF;
+        best = key[0];
+        be = ex[0];
+      } else {
+#pragma unroll
+        for (int j = 0; j < NK; ++j)
+          if (32 * j + lane == be) key[j] = 0ull;
+        int bj;
+        lane_best<NK>(key, best, bj);
+        be = 32 * bj + lane;
+      }
+    }
+    const double v = key_value(((uint64_t)hi << 32) | lo);
     if (r == 0) lmax = v;
-    if (lane == r) { my_e = esel; my_l = v; }
+    if (lane == r) { my_e = (int)esel; my_l = v; }
   }
-  const double ex = lane < K ? exp(my_l - lmax) : 0.0;
-  double sum = ex;
+  const float w = lane < K ? expf((float)(my_l - lmax)) : 0.f;
+  float sum = w;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(FULL, sum, o);
-  if (lane < K) { out_idx[lane] = my_e; out_w[lane] = (float)(ex / sum); }
+  if (lane < K) {
+    out_idx[lane] = my_e;
+    out_w[lane] = w / sum;
+    if (sel) atomicOr(sel + my_e * tw + (t >> 5), 1u << (t & 31));
+  }
+}
+
+// Top-k of token t with the smallest key list that holds E experts.
+__device__ __noinline__ void topk_row(const double* logits, int T, int E, int K, int HS,
+                                         const float* bias, int t, int32_t* out_idx, float* out_w,
+                                         uint32_t* sel, int tw) {
+  static_assert(MAX_EXPERTS == 512, "key lists of 4, 8 and 16 per lane");
+  if (E <= 128) topk_nk<4>(logits, T, E, K, HS, bias, t, out_idx, out_w, sel, tw);
+  else if (E <= 256) topk_nk<8>(logits, T, E, K, HS, bias, t, out_idx, out_w, sel, tw);
+  else topk_nk<16>(logits, T, E, K, HS, bias, t, out_idx, out_w, sel, tw);
 }
 
 // Exclusive scan of n <= 512 ints in shared memory by one warp (in place);
@@ -507,68 +627,109 @@ __device__ __noinline__ void build_units(const int32_t* counts, const int32_t* o
   }
 }
 
-// Small T*K: every CTA routes all tokens itself (no barrier); CTA 0 also writes
-// the maps to global memory.
-__device__ void phase_route_small(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem,
-                                  uint64_t* stamp) {
+// Small T*K: the routing of all tokens by one CTA, into its shared-memory
+// tables and the global maps at once.  Every expert keeps a mask of the
+// tokens that chose it (a token chooses an expert at most once), so its count
+// is the mask's population, and the stable position of pair (t, r) is the
+// expert's offset plus the number of earlier tokens in its mask.  Counts and
+// unit counts (ceil(count / NT_MAX)) are scanned together as one packed word.
+__device__ void phase_route_small(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem) {
   CtaTables& tb = tables(smem);
   const int T = p.T, E = p.E, K = p.K, TK = p.TK;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint64_t* keys = reinterpret_cast<uint64_t*>(ring_slot(smem, 0, 0)) + warp * MAX_EXPERTS;
-  for (int t = warp; t < T; t += WARPS) topk_row(p.logits, T, E, K, p.HS, lp.router_b, t, keys, tb.idx + t * K, tb.w + t * K);
-  __syncthreads();  // the key rows share the ring with the histogram below
-  if (stamp) *stamp = globaltimer_ns();
-  int32_t* hist = reinterpret_cast<int32_t*>(ring_slot(smem, 0, 0));  // [WARPS][E] scratch
-  for (int i = threadIdx.x; i < WARPS * E; i += THREADS) hist[i] = 0;
+  const int warp = threadIdx.x >> 5;
+  const int tw = (T + 31) >> 5;  // mask words per expert
+  uint32_t* sel = reinterpret_cast<uint32_t*>(ring_slot(smem, 0, 0));  // [E][tw], idle ring
+  int32_t* pk = reinterpret_cast<int32_t*>(sel + E * tw);             // [E + 1] packed counts
+  for (int i = threadIdx.x; i < E * tw; i += THREADS) sel[i] = 0u;
   __syncthreads();
-  const int pr = threadIdx.x;  // TK <= SMALL_PAIRS <= THREADS: one pair per thread
-  const bool valid = pr < TK;
-  const int e = valid ? tb.idx[pr] : -1 - lane;
-  const uint32_t peers = __match_any_sync(FULL, e);
-  const int rank_w = __popc(peers & ((1u << lane) - 1u));
-  if (valid && lane == __ffs(peers) - 1) hist[warp * E + e] = __popc(peers);
+  for (int t = warp; t < T; t += WARPS)
+    topk_row(p.logits, T, E, K, p.HS, lp.router_b, t, tb.idx + t * K, tb.w + t * K, sel, tw);
   __syncthreads();
+  // per expert x (one thread each): count and unit count, packed; scanned
+  // within each 32-expert chunk by its warp, then offset by the chunk totals
+  int32_t* ctot = pk + MAX_EXPERTS + 1;  // [MAX_EXPERTS / 32] chunk totals
+  const int lane = threadIdx.x & 31;
+  int32_t vx[MAX_EXPERTS / THREADS + 1];
+#pragma unroll
+  for (int r = 0; r * THREADS < MAX_EXPERTS; ++r) {
+    const int x = r * THREADS + threadIdx.x;
+    int c = 0;
+    if (x < E)
+      for (int w = 0; w < tw; ++w) c += __popc(sel[x * tw + w]);
+    const int32_t v = (((c + NT_MAX - 1) / NT_MAX) << 16) | c;  // c <= 256, units <= 320
+    int32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(FULL, incl, o);
+      if (lane >= o) incl += y;
+    }
+    vx[r] = v;
+    if (x < E) pk[x] = incl - v;
+    if (lane == 31 && x - 31 < E) ctot[x >> 5] = incl;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r * THREADS < MAX_EXPERTS; ++r) {
+    const int x = r * THREADS + threadIdx.x;
+    if (x < E) {
+      int32_t base = 0;
+      for (int q = 0; q < (x >> 5); ++q) base += ctot[q];
+      const int32_t ex = base + pk[x];
+      pk[x] = ex;
+      const int c = vx[r] & 0xFFFF, o = ex & 0xFFFF;
+      tb.counts[x] = c; p.counts[x] = c;
+      tb.offsets[x] = o; p.offsets[x] = o;
+      if (x == E - 1) {
+        const int32_t tot = ex + vx[r];
+        pk[E] = tot;
+        tb.offsets[E] = tot & 0xFFFF;
+        p.offsets[E] = tot & 0xFFFF;
+      }
+    }
+  }
+  __syncthreads();
+  for (int pr = threadIdx.x; pr < TK; pr += THREADS) {
+    const int e = tb.idx[pr], t = pr / K;
+    const uint32_t* m = sel + e * tw;
+    int before = __popc(m[t >> 5] & ((1u << (t & 31)) - 1u));
+    for (int w = 0; w < (t >> 5); ++w) before += __popc(m[w]);
+    const int pos = (pk[e] & 0xFFFF) + before;
+    const float wt = tb.w[pr];
+    tb.perm[pos] = pr; tb.inv[pr] = pos; tb.tokpos[pos] = t; tb.wpos[pos] = wt;
+    p.idx[pr] = e; p.wts[pr] = wt; p.perm[pos] = pr; p.inv[pr] = pos; p.tokpos[pos] = t; p.wpos[pos] = wt;
+  }
+  // gate/up units of <= NT_MAX consecutive positions of one expert's segment;
+  // the down units are the same ranges, each naming its gate/up unit
   for (int x = threadIdx.x; x < E; x += THREADS) {
-    int32_t c = 0;
-    for (int w = 0; w < WARPS; ++w) c += hist[w * E + x];
-    tb.counts[x] = c;
-    tb.offsets[x] = c;
+    const int c = pk[x + 1] - pk[x];  // packed difference: units << 16 | count
+    const int n = c & 0xFFFF, off = pk[x] & 0xFFFF, ub = pk[x] >> 16;
+    for (int s = 0; s * NT_MAX < n; ++s) {
+      const int4 gu = make_int4(x, off + s * NT_MAX, min(NT_MAX, n - s * NT_MAX), 0);
+      const int4 dn = make_int4(gu.x, gu.y, gu.z, ub + s);
+      reinterpret_cast<int4*>(tb.units)[ub + s] = gu;
+      reinterpret_cast<int4*>(tb.dunits)[ub + s] = dn;
+      reinterpret_cast<int4*>(p.units)[ub + s] = gu;
+      reinterpret_cast<int4*>(p.dunits)[ub + s] = dn;
+    }
   }
-  __syncthreads();
-  if (warp == 0) warp_exclusive_scan(tb.offsets, E, tb.offsets + E);
-  __syncthreads();
-  if (valid) {
-    int32_t before = 0;
-    for (int w = 0; w < warp; ++w) before += hist[w * E + e];
-    const int pos = tb.offsets[e] + before + rank_w;
-    tb.perm[pos] = pr;
-    tb.inv[pr] = pos;
-    tb.tokpos[pos] = pr / K;
-    tb.wpos[pos] = tb.w[pr];
+  if (threadIdx.x == 0) {
+    const int nu = pk[E] >> 16;
+    tb.n_units = nu; tb.n_dunits = nu;
+    p.n_units[0] = nu; p.n_units[1] = nu;
   }
-  __syncthreads();
-  build_units(tb.counts, tb.offsets, E, hist, tb.units, tb.dunits, &tb.n_units, &tb.n_dunits, NT_MAX);
-  __syncthreads();
-  // publish: the maps of the ABI and the stream's tables
-  for (int i = threadIdx.x; i < TK; i += THREADS) {
-    p.idx[i] = tb.idx[i]; p.wts[i] = tb.w[i]; p.perm[i] = tb.perm[i]; p.inv[i] = tb.inv[i];
-    p.tokpos[i] = tb.tokpos[i]; p.wpos[i] = tb.wpos[i];
-  }
-  for (int i = threadIdx.x; i < E; i += THREADS) p.counts[i] = tb.counts[i];
-  for (int i = threadIdx.x; i <= E; i += THREADS) p.offsets[i] = tb.offsets[i];
-  for (int i = threadIdx.x; i < tb.n_units * 4; i += THREADS) p.units[i] = tb.units[i];
-  for (int i = threadIdx.x; i < tb.n_dunits * 4; i += THREADS) p.dunits[i] = tb.dunits[i];
-  if (threadIdx.x == 0) { p.n_units[0] = tb.n_units; p.n_units[1] = tb.n_dunits; }
 }
 
 // Small T*K: the grid barrier after the router phase.  The CTA that arrives
 // last computes the routing once (top-k, permutation, unit tables) and
 // publishes it before releasing the barrier; every other CTA then copies the
 // stream's tables (a few KB) into shared memory.  One CTA reading all partial
-// logits is much faster than every CTA reading them at once.  Bounded like
-// grid_barrier; false on timeout or a recorded error.
-__device__ bool route_barrier(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem, uint32_t where,
-                              uint64_t* stamp) {
+// logits is much faster than every CTA reading them at once.  While the
+// routing runs, every CTA writes its share of the x term images and counts
+// itself in sync[SY_XDONE]; the stream's producers wait for the full count
+// before their first gate/up stage.  Bounded like grid_barrier; false on
+// timeout or a recorded error.
+__device__ bool route_barrier(const EngineParams& p, const LayerPtrs& lp, const __nv_bfloat16* x,
+                              int layer, uint8_t* smem, uint32_t where, uint64_t* stamp) {
   CtaTables& tb = tables(smem);
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -580,17 +741,32 @@ __device__ bool route_barrier(const EngineParams& p, const LayerPtrs& lp, uint8_
     tb.gen = (int32_t)gen;
   }
   __syncthreads();
-  int ok = 1;
-  if (tb.last) {
-    phase_route_small(p, lp, smem, stamp);
+  const bool last = tb.last != 0;
+  if (last) {
+    phase_route_small(p, lp, smem);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      // every CTA has arrived and touches the count again only after it sees
+      // the new generation: a plain store resets it, and the release orders
+      // it and all tables before that generation
+      __threadfence();
+      *reinterpret_cast<volatile uint32_t*>(p.sync + SY_BAR_COUNT) = 0u;
+      st_release_u32(p.sync + SY_BAR_GEN, (uint32_t)tb.gen + 1u);
+    }
+  }
+  if (!p.route_only) {
+    phase_images(p, x, layer);
     __syncthreads();
     if (threadIdx.x == 0) {
       __threadfence();
-      atomicExch(p.sync + SY_BAR_COUNT, 0u);
-      __threadfence();
-      st_release_u32(p.sync + SY_BAR_GEN, (uint32_t)tb.gen + 1u);
-      if (error_set(p.sync)) ok = 0;
+      atomicAdd(p.sync + SY_XDONE, 1u);
     }
+  }
+  if (stamp) stamp[0] = globaltimer_ns();
+  int ok = 1;
+  if (last) {
+    if (threadIdx.x == 0 && error_set(p.sync)) ok = 0;
+    if (stamp) stamp[1] = stamp[0];
     return __syncthreads_and(ok) != 0;
   }
   if (threadIdx.x == 0) {
@@ -608,7 +784,7 @@ __device__ bool route_barrier(const EngineParams& p, const LayerPtrs& lp, uint8_
     if (ok && error_set(p.sync)) ok = 0;
   }
   if (!__syncthreads_and(ok)) return false;
-  if (stamp) stamp[0] = globaltimer_ns();
+  if (stamp) stamp[1] = globaltimer_ns();
   if (p.route_only) return true;
   const int nu = ld_cg_u32(p.n_units), nd = ld_cg_u32(p.n_units + 1);
   const uint4* su = reinterpret_cast<const uint4*>(p.units);
@@ -626,12 +802,11 @@ __device__ bool route_barrier(const EngineParams& p, const LayerPtrs& lp, uint8_
 }
 
 // Large T*K, step 1: top-k of every token, distributed over all warps.
-__device__ void phase_topk_large(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem) {
+__device__ void phase_topk_large(const EngineParams& p, const LayerPtrs& lp) {
   const int warp = threadIdx.x >> 5;
   const int64_t wg = (int64_t)blockIdx.x * WARPS + warp, ws = (int64_t)gridDim.x * WARPS;
-  uint64_t* keys = reinterpret_cast<uint64_t*>(ring_slot(smem, 0, 0)) + warp * MAX_EXPERTS;
   for (int64_t t = wg; t < p.T; t += ws)
-    topk_row(p.logits, p.T, p.E, p.K, p.HS, lp.router_b, (int)t, keys, p.idx + t * p.K, p.wts + t * p.K);
+    topk_row(p.logits, p.T, p.E, p.K, p.HS, lp.router_b, (int)t, p.idx + t * p.K, p.wts + t * p.K, nullptr, 0);
 }
 
 // Large T*K, step 2: counts/offsets in every CTA (shared-memory histogram),
@@ -769,6 +944,12 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
   const int64_t n_gu = (int64_t)cx.n_units * gub, n_all = n_gu + (int64_t)cx.n_dunits * db;
   const int nc_gu = p.H / KS, nc_d = p.I / KS;
   const uint32_t need = (uint32_t)gub * 4u;  // readiness signals per gate/up unit: 4 warps per job
+  bool xwait = !LT && !cx.global;  // x term images written during the routing (small T*K)
+  // Units of at most NT_MAX positions read most expert weights once: the
+  // weight stages go to L2 as evict-first, so that the routing's working set
+  // (code, router weights, activations, tables) stays in L2 across launches.
+  // Tiles re-read each expert's weights once per tile and keep the default.
+  const uint64_t wpolicy = LT ? 0ull : l2_evict_first();
   const uint32_t seq_start = rs.seq;
   bool ok = true;
   unsigned long long t_empty = 0, t_ready = 0;
@@ -816,6 +997,26 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
       if (!ok) continue;  // publishes the end entry
       fence_proxy_async_global();  // the images were written by generic stores of other CTAs
     }
+    if (!isD && xwait) {  // every CTA's x images, before the first gate/up stage
+      xwait = false;
+      const unsigned long long tr0 = clock64();
+      if (lane == 0 && ld_acquire_u32(p.sync + SY_XDONE) < gridDim.x) {
+        const uint64_t t0 = globaltimer_ns();
+        uint32_t spins = 0;
+        while (ld_acquire_u32(p.sync + SY_XDONE) < gridDim.x) {
+          if ((++spins & 15u) == 0u) {
+            if (error_set(p.sync)) { ok = false; break; }
+            if (globaltimer_ns() - t0 > p.timeout_ns) { set_error(p.sync, DEV_TIMEOUT_IMAGES, (uint32_t)j); ok = false; break; }
+          }
+          __nanosleep(32);
+        }
+      }
+      ok = __shfl_sync(FULL, ok, 0);
+      __syncwarp();  // orders lane 0's acquire before every lane's copies
+      t_ready += clock64() - tr0;
+      if (!ok) continue;  // publishes the end entry
+      fence_proxy_async_global();  // the images were written by generic stores of other CTAs
+    }
     if (lane == 0) {
       JobEntry* en = jq + (rs.qk % JQ);
       en->job = (int32_t)j; en->s0 = (int32_t)rs.seq; en->nc = nc; en->unit = u; en->rb = rb;
@@ -857,7 +1058,8 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
       const int c = c0 + lane;
       if (lane < k) {
         mbar_arrive_expect_tx(fb, stage_bytes);
-        bulk_g2s(dst, wbase + (int64_t)c * STAGE_A_BYTES, STAGE_A_BYTES, fb);
+        if constexpr (LT) bulk_g2s(dst, wbase + (int64_t)c * STAGE_A_BYTES, STAGE_A_BYTES, fb);
+        else bulk_g2s_hint(dst, wbase + (int64_t)c * STAGE_A_BYTES, STAGE_A_BYTES, fb, wpolicy);
         if (LT)  // the tile's B operand of this stage, one image
           bulk_g2s(dst + STAGE_A_BYTES, (isD ? p.atl : p.xtl) + ((int64_t)u * nc + c) * LT_IMG_BYTES,
                    bbytes, fb);
@@ -1315,25 +1517,28 @@ template <bool TILES>
 __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, RoleState& rs,
                            bool stamp) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool small = p.TK <= SMALL_PAIRS;
+  const bool small = !TILES && p.TK <= SMALL_PAIRS;  // the tile stream runs only above SMALL_PAIRS
   CtaTables& tb = tables(smem);
   for (int layer = 0; layer < p.L; ++layer) {
     const LayerPtrs& lp = p.layers[layer];
     const __nv_bfloat16* x = layer == 0 ? p.x_in : p.xnext;
     uint64_t* st = stamp ? p.stamps + 1 + layer * STAMPS_PER_LAYER : nullptr;
-    phase_prepare(p, lp, x, layer, smem, st);
+    phase_router(p, lp, x, smem);
+    if (st) st[0] = globaltimer_ns();
     StreamCtx cx;
     const int32_t* inv;
     if (small) {
-      if (!route_barrier(p, lp, smem, 10 * layer + 1, st ? st + 2 : nullptr)) return;
+      if (!route_barrier(p, lp, x, layer, smem, 10 * layer + 1, st ? st + 1 : nullptr)) return;
       if (p.route_only) return;
       if (st) st[3] = globaltimer_ns();
       cx = StreamCtx{tb.units, tb.dunits, tb.tokpos, tb.wpos, tb.n_units, tb.n_dunits, false};
       inv = tb.inv;
     } else {
+      phase_images(p, x, layer);
+      if (st) st[1] = globaltimer_ns();
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 1)) return;
       if (st) st[2] = globaltimer_ns();
-      phase_topk_large(p, lp, smem);
+      phase_topk_large(p, lp);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 2)) return;
       if (st) st[3] = globaltimer_ns();
       phase_permute_large(p, smem);
@@ -1373,6 +1578,9 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
     }
     if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 4)) return;
     if (st) st[5] = globaltimer_ns();
+    // every producer has passed its image wait and every CTA has counted
+    // itself: the count restarts for the next layer or launch
+    if (blockIdx.x == 0 && threadIdx.x == 0) p.sync[SY_XDONE] = 0u;
     if (layer + 1 < p.L) {
       phase_combine_rmsnorm(p, inv, smem);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 5)) return;

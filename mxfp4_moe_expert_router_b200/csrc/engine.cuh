@@ -96,17 +96,18 @@ __host__ __device__ constexpr int lt_code_offset(int tl) { return LT_SF_BYTES + 
 __host__ __device__ inline bool use_tiles(int64_t TK, int E) {
   return TK > SMALL_PAIRS && TK >= (int64_t)LT_MIN_PER_EXPERT * E;
 }
-constexpr int STAMPS_PER_LAYER = 7;  // x converted, logits (CTA 0), prepared, top-k, routed, streamed, combined
+constexpr int STAMPS_PER_LAYER = 7;  // router, x images, routing wait, top-k / tables, permutation, stream, combine (CTA 0)
 
 // sync word layout (uint32)
 enum : int {
   SY_BAR_COUNT = 0, SY_BAR_GEN = 1, SY_JOBS = 2, SY_ERROR = 3, SY_ERRINFO = 4,
+  SY_XDONE = 5,  // CTAs whose x term images of this layer are written (small T*K)
   SY_READY = 8,  // ready[unit] from here
 };
 // device-side error codes (status word)
 enum : uint32_t {
   DEV_OK = 0, DEV_TIMEOUT_BARRIER = 1, DEV_TIMEOUT_PIPE = 2, DEV_TIMEOUT_READY = 3,
-  DEV_TIMEOUT_QUEUE = 4,
+  DEV_TIMEOUT_QUEUE = 4, DEV_TIMEOUT_IMAGES = 5,
 };
 
 // Upper bounds of the unit tables for T*K pairs over E experts.

@@ -78,6 +78,22 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src, uint32
       ::"r"(smem_u32(dst_smem)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 
+// The same copy with an L2 cache policy (from l2_evict_first()).
+__device__ __forceinline__ void bulk_g2s_hint(void* dst_smem, const void* src, uint32_t bytes,
+                                              uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+      ::"r"(smem_u32(dst_smem)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy) : "memory");
+}
+
+// L2 policy for data read once: its lines are the first to be replaced, so a
+// large stream does not push the small, reused working set out of L2.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t policy;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
+  return policy;
+}
+
 // Prefetch `bytes` of global memory into L2 (16-byte aligned address, size a
 // multiple of 16); no data is returned.
 __device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
