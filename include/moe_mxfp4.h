@@ -139,7 +139,10 @@ MOE_API int32_t moe_route(moe_mxfp4_t* h, int32_t layer, const void* x_bf16, int
  * NULL or a [num_layers+1][T][H] bf16 buffer that receives every layer's
  * input (slot l) and the final output (slot num_layers).  x and y may not
  * overlap.  T == 0 is a no-op.  Errors: MOE_ERR_INVALID_ARG, MOE_ERR_CUDA;
- * device-side timeouts are reported by the next moe_status.
+ * device-side timeouts are reported by the next moe_status.  The call only
+ * enqueues the launch (no synchronisation, no host reads of device memory),
+ * so it may be captured into a CUDA graph; calls on one handle must not run
+ * concurrently (they share its workspace).
  */
 MOE_API int32_t moe_forward(moe_mxfp4_t* h, const void* x_bf16, int32_t T, void* y_bf16,
                     void* layer_io_bf16, void* stream);
