@@ -133,12 +133,13 @@ __device__ bool grid_barrier(uint32_t* sync, uint64_t timeout_ns, uint32_t where
   __syncthreads();
   int ok = 1;
   if (threadIdx.x == 0) {
+    // the arrival releases this CTA's writes; the last arrival acquires them
+    // all, resets the count (every CTA touches it again only after it sees
+    // the new generation) and releases the new generation
     const uint32_t gen = ld_volatile_u32(sync + SY_BAR_GEN);
-    __threadfence();
-    const uint32_t prev = atomicAdd(sync + SY_BAR_COUNT, 1u);
+    const uint32_t prev = atom_add_acq_rel_u32(sync + SY_BAR_COUNT, 1u);
     if (prev == gridDim.x - 1) {
-      atomicExch(sync + SY_BAR_COUNT, 0u);
-      __threadfence();
+      *reinterpret_cast<volatile uint32_t*>(sync + SY_BAR_COUNT) = 0u;
       st_release_u32(sync + SY_BAR_GEN, gen + 1);
     } else {
       const uint64_t t0 = globaltimer_ns();
@@ -150,8 +151,8 @@ __device__ bool grid_barrier(uint32_t* sync, uint64_t timeout_ns, uint32_t where
         }
         __nanosleep(64);
       }
+      __threadfence();
     }
-    __threadfence();
     if (ok && error_set(sync)) ok = 0;
   }
   return __syncthreads_and(ok) != 0;
@@ -733,10 +734,10 @@ __device__ bool route_barrier(const EngineParams& p, const LayerPtrs& lp, const 
   CtaTables& tb = tables(smem);
   __syncthreads();
   if (threadIdx.x == 0) {
+    // the arrival releases this CTA's partial logits and, for the last CTA,
+    // acquires everyone else's
     const uint32_t gen = ld_volatile_u32(p.sync + SY_BAR_GEN);
-    __threadfence();
-    const uint32_t prev = atomicAdd(p.sync + SY_BAR_COUNT, 1u);
-    __threadfence();
+    const uint32_t prev = atom_add_acq_rel_u32(p.sync + SY_BAR_COUNT, 1u);
     tb.last = prev == gridDim.x - 1;
     tb.gen = (int32_t)gen;
   }
@@ -786,17 +787,32 @@ __device__ bool route_barrier(const EngineParams& p, const LayerPtrs& lp, const 
   if (!__syncthreads_and(ok)) return false;
   if (stamp) stamp[1] = globaltimer_ns();
   if (p.route_only) return true;
-  const int nu = ld_cg_u32(p.n_units), nd = ld_cg_u32(p.n_units + 1);
-  const uint4* su = reinterpret_cast<const uint4*>(p.units);
-  const uint4* sd = reinterpret_cast<const uint4*>(p.dunits);
-  for (int i = threadIdx.x; i < nu; i += THREADS) reinterpret_cast<uint4*>(tb.units)[i] = ld_cg_v4(su + i);
-  for (int i = threadIdx.x; i < nd; i += THREADS) reinterpret_cast<uint4*>(tb.dunits)[i] = ld_cg_v4(sd + i);
-  for (int i = threadIdx.x; i < p.TK; i += THREADS) {
-    tb.tokpos[i] = (int32_t)ld_cg_u32(p.tokpos + i);
-    tb.wpos[i] = __uint_as_float(ld_cg_u32(p.wpos + i));
-    tb.inv[i] = (int32_t)ld_cg_u32(p.inv + i);
+  // one round trip: every entry the tables can hold for this T*K is loaded
+  // at once, the counts alongside (entries past them are never read)
+  static_assert(THREADS >= SMALL_UNITS && THREADS >= SMALL_PAIRS, "one table entry per thread");
+  const int i = threadIdx.x;
+  const int ucap = min(max_units(p.E, p.TK), SMALL_UNITS);
+  uint4 gu = {}, dn = {};
+  uint32_t tp = 0, wp = 0, iv = 0;
+  if (i < ucap) {
+    gu = ld_cg_v4(reinterpret_cast<const uint4*>(p.units) + i);
+    dn = ld_cg_v4(reinterpret_cast<const uint4*>(p.dunits) + i);
   }
-  if (threadIdx.x == 0) { tb.n_units = nu; tb.n_dunits = nd; }
+  if (i < p.TK) {
+    tp = ld_cg_u32(p.tokpos + i);
+    wp = ld_cg_u32(p.wpos + i);
+    iv = ld_cg_u32(p.inv + i);
+  }
+  if (i == 0) { tb.n_units = (int32_t)ld_cg_u32(p.n_units); tb.n_dunits = (int32_t)ld_cg_u32(p.n_units + 1); }
+  if (i < ucap) {
+    reinterpret_cast<uint4*>(tb.units)[i] = gu;
+    reinterpret_cast<uint4*>(tb.dunits)[i] = dn;
+  }
+  if (i < p.TK) {
+    tb.tokpos[i] = (int32_t)tp;
+    tb.wpos[i] = __uint_as_float(wp);
+    tb.inv[i] = (int32_t)iv;
+  }
   __syncthreads();
   return true;
 }

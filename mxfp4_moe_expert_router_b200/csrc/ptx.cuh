@@ -113,6 +113,14 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ---- acquire / release on global words -----------------------------------------
+// Atomic add at gpu scope with acquire and release semantics: earlier memory
+// operations of this thread are visible before it, later ones are ordered
+// after it.  Returns the previous value.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_u32(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
