@@ -419,6 +419,142 @@ __device__ void phase_router(const EngineParams& p, const LayerPtrs& lp, const _
   }
 }
 
+// Router for large T (tile-stream launches), on the fp64 MMA path
+// (mma.sync m8n8k4 f64: 256 exact fp64 FMAs from two register operands).
+// Each CTA takes the same (H part, experts) share as phase_router.  Token
+// chunks of RTB = 16 (two 8-row tiles) are staged as fp32 (exact for bf16) in
+// two buffers, the next chunk's loads in flight while this one computes.
+// Experts go in groups of 16 (two 8-column tiles).  The 12 warps split the H
+// part; their partial tiles meet in shared memory and are summed in warp
+// order (deterministic), then stored.
+constexpr int RTB = 16, REB = 16, RXL = 6;  // RXL: 16-byte x loads per thread and chunk
+static_assert(RTB * (8192 / MAX_HSPLIT / 8) <= RXL * THREADS, "chunk loads per thread");
+__device__ __forceinline__ void dmma_m8n8k4(double (&c)[2], double a, double b) {
+  asm("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+      : "+d"(c[0]), "+d"(c[1]) : "d"(a), "d"(b));
+}
+// (Out of line, with scalar arguments: the tile stream's code generation then
+// does not depend on this phase, and the kernel's parameter block stays out of
+// local memory.)
+__device__ __noinline__ void phase_router_tiles(const __nv_bfloat16* x, const float* router_w,
+                                                double* logits, uint32_t* sync, int T, int H, int E,
+                                                int TK, int HS, uint8_t* smem) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t gt = (int64_t)blockIdx.x * THREADS + threadIdx.x;
+  const int64_t gs = (int64_t)gridDim.x * THREADS;
+  // per-layer resets of the stream's counters (used only after the next barrier)
+  const int umax = max_units(E, TK);
+  if (gt == 0) sync[SY_JOBS] = 0u;
+  for (int64_t u = gt; u < umax; u += gs) sync[SY_READY + u] = 0u;
+
+  RouterWork rw;
+  {
+    const int g = (int)gridDim.x, c = (int)blockIdx.x;
+    rw = g >= HS ? RouterWork{c % HS, HS, c / HS, (g - c % HS + HS - 1) / HS} : RouterWork{c, g, 0, 1};
+  }
+  const int hpart = H / HS, hp8 = hpart / 8, hp4 = hpart / 4;
+  const int xstride = hpart + 4;  // the 8 rows of a tile fall in 8 different bank groups
+  const int nexp = rw.e0 < E ? (E - rw.e0 + rw.estep - 1) / rw.estep : 0;
+  const int ng = (nexp + REB - 1) / REB;
+  // shared memory: red [WARPS][4 tiles][64] doubles, x [2][RTB][xstride], then
+  // (when they fit) the part's weight rows [ng * REB][xstride]
+  double* red = reinterpret_cast<double*>(ring_slot(smem, 0, 0));
+  float* xs = reinterpret_cast<float*>(red + WARPS * 4 * 64);
+  float* wsm = xs + 2 * RTB * xstride;
+  const bool wstaged =
+      (size_t)WARPS * 4 * 64 * 8 + ((size_t)2 * RTB + (size_t)ng * REB) * xstride * 4 <= RING_BYTES;
+  const int nchunk = (T + RTB - 1) / RTB;
+  const int g8 = lane >> 2, q4 = lane & 3;  // fragment row/column group, k within the step
+  for (int hs = rw.hs0; hs < HS; hs += rw.hstep) {
+    __syncthreads();  // the previous part's readers are done
+    if (wstaged)
+      for (int i = threadIdx.x; i < nexp * hp4; i += THREADS) {
+        const int k = i / hp4, h4 = i - k * hp4;
+        *reinterpret_cast<uint4*>(wsm + (size_t)k * xstride + 4 * h4) =
+            __ldg(reinterpret_cast<const uint4*>(router_w + (int64_t)(rw.e0 + k * rw.estep) * H + hs * hpart) + h4);
+      }
+    uint4 xr[RXL];
+    auto load_chunk = [&](int c) {
+      const int t0 = c * RTB, nt = min(RTB, T - t0);
+#pragma unroll
+      for (int r = 0; r < RXL; ++r) {
+        const int i = threadIdx.x + r * THREADS;
+        if (i < nt * hp8) {
+          const int t = i / hp8, h8 = i - t * hp8;
+          xr[r] = __ldcg(reinterpret_cast<const uint4*>(x + (int64_t)(t0 + t) * H + hs * hpart) + h8);
+        }
+      }
+    };
+    auto store_chunk = [&](int c) {
+      const int t0 = c * RTB, nt = min(RTB, T - t0);
+      float* b = xs + (c & 1) * RTB * xstride;
+#pragma unroll
+      for (int r = 0; r < RXL; ++r) {
+        const int i = threadIdx.x + r * THREADS;
+        if (i < nt * hp8) {
+          const int t = i / hp8, h8 = i - t * hp8;
+          const uint32_t u[4] = {xr[r].x, xr[r].y, xr[r].z, xr[r].w};
+          float4* d = reinterpret_cast<float4*>(b + (size_t)t * xstride + h8 * 8);
+          d[0] = make_float4(__uint_as_float(u[0] << 16), __uint_as_float(u[0] & 0xFFFF0000u),
+                             __uint_as_float(u[1] << 16), __uint_as_float(u[1] & 0xFFFF0000u));
+          d[1] = make_float4(__uint_as_float(u[2] << 16), __uint_as_float(u[2] & 0xFFFF0000u),
+                             __uint_as_float(u[3] << 16), __uint_as_float(u[3] & 0xFFFF0000u));
+        }
+      }
+    };
+    load_chunk(0);
+    store_chunk(0);
+    __syncthreads();
+#pragma unroll 1
+    for (int c = 0; c < nchunk; ++c) {
+      const int t0 = c * RTB, nt = min(RTB, T - t0);
+      const bool next = c + 1 < nchunk;
+      if (next) load_chunk(c + 1);
+      const float* xb = xs + (c & 1) * RTB * xstride;
+#pragma unroll 1
+      for (int g = 0; g < ng; ++g) {
+        // operand rows of this lane: tokens g8 and 8 + g8, experts g * 16 + g8 and + 8
+        const float* xa0 = xb + (size_t)g8 * xstride + q4;
+        const float* xa1 = xa0 + (size_t)8 * xstride;
+        const float* wb[2];
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+          const int k = g * REB + 8 * n + g8;
+          wb[n] = wstaged ? wsm + (size_t)k * xstride + q4
+                          : router_w + (int64_t)(rw.e0 + min(k, nexp - 1) * rw.estep) * H + hs * hpart + q4;
+        }
+        double acc[4][2] = {};
+#pragma unroll 2
+        for (int ks = warp; ks < hp4; ks += WARPS) {
+          const int h = 4 * ks;
+          const double a0 = (double)xa0[h], a1 = (double)xa1[h];
+          const double b0 = (double)wb[0][h], b1 = (double)wb[1][h];
+          dmma_m8n8k4(acc[0], a0, b0);
+          dmma_m8n8k4(acc[1], a0, b1);
+          dmma_m8n8k4(acc[2], a1, b0);
+          dmma_m8n8k4(acc[3], a1, b1);
+        }
+        // lane l holds tile elements (row l / 4, columns 2 (l % 4) and + 1): index 2 l (+ 1) row-major
+#pragma unroll
+        for (int tile = 0; tile < 4; ++tile)
+          *reinterpret_cast<double2*>(red + ((size_t)warp * 4 + tile) * 64 + 2 * lane) =
+              make_double2(acc[tile][0], acc[tile][1]);
+        __syncthreads();
+        for (int o = threadIdx.x; o < 4 * 64; o += THREADS) {
+          const int tile = o >> 6, r = o & 63;
+          double v = 0.0;
+          for (int w = 0; w < WARPS; ++w) v += red[((size_t)w * 4 + tile) * 64 + r];
+          const int tl = 8 * (tile >> 1) + (r >> 3), k = g * REB + 8 * (tile & 1) + (r & 7);
+          if (tl < nt && k < nexp) logits[((int64_t)hs * T + t0 + tl) * E + rw.e0 + k * rw.estep] = v;
+        }
+        __syncthreads();
+      }
+      if (next) store_chunk(c + 1);
+      __syncthreads();
+    }
+  }
+}
+
 // ---- phase B: top-k, weights, permutation ------------------------------------------------
 __device__ __forceinline__ uint64_t order_key(double v) {
   const uint64_t b = (uint64_t)__double_as_longlong(v);
@@ -1539,7 +1675,8 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
     const LayerPtrs& lp = p.layers[layer];
     const __nv_bfloat16* x = layer == 0 ? p.x_in : p.xnext;
     uint64_t* st = stamp ? p.stamps + 1 + layer * STAMPS_PER_LAYER : nullptr;
-    phase_router(p, lp, x, smem);
+    if constexpr (TILES) phase_router_tiles(x, lp.router_w, p.logits, p.sync, p.T, p.H, p.E, p.TK, p.HS, smem);
+    else phase_router(p, lp, x, smem);
     if (st) st[0] = globaltimer_ns();
     StreamCtx cx;
     const int32_t* inv;
