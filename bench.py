@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--batches", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--large-kind", choices=("f16", "mxf4"), default="mxf4",
+                    help="weight stream for many positions per expert: bf16 tiles or E2M1 term tiles")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of replaying them as one CUDA graph")
     ap.add_argument("--e2e-steps", type=int, default=None)
@@ -290,6 +292,7 @@ def main():
 
     layers = [build_layer(mx, w, l, seed=0) for l in range(w.layers)]
     m = mx.Moe(w.hidden, w.inter, w.experts, w.top_k, T, layers)
+    m.moe_set_large_kind(m.LARGE_F16 if args.large_kind == "f16" else m.LARGE_MXF4)
     xs = token_blocks(w, T, args.batches, rank)
     hits = []
     for x in xs:
@@ -406,6 +409,7 @@ def main():
                        "l2": "no flush: ~%.0f MB of expert weights streamed per step > 126 MB L2"
                              % (alg_bytes / 1e6),
                        "parallelism": f"replicas x{world} (independent verify blocks)",
+                       "large_kind": args.large_kind,
                        "launch": "stream launches" if graph is None else
                                  "the timed moe_forward calls replayed as one CUDA graph"},
             "layer_us": ms_step * 1e3 / w.layers,

@@ -191,6 +191,17 @@ MOE_API int32_t moe_phase_ns(moe_mxfp4_t* h, uint64_t* ns_out, int32_t max_n, vo
 MOE_API int32_t moe_stream_profile(moe_mxfp4_t* h, int32_t enable, uint64_t* out, int32_t max_n,
                                    void* stream);
 
+/*
+ * moe_set_large_kind -- the weight stream used when a call has many positions
+ * per expert (T*K > 256 and T*K >= 8*E): 1 = E2M1 term tiles on the block-
+ * scaled fp4 tensor-core MMA (x and the SwiGLU output expanded into eight
+ * E2M1 terms), 2 = bf16 tiles on the bf16 tensor-core MMA (MXFP4 weights
+ * dequantised to bf16 in shared memory, x exact, the SwiGLU output as two
+ * bf16 terms).  Default 1 (the faster of the two on B200 at every measured
+ * size).  Errors: MOE_ERR_INVALID_ARG.
+ */
+MOE_API int32_t moe_set_large_kind(moe_mxfp4_t* h, int32_t kind);
+
 /* moe_set_timeout_ns -- bound of every device-side wait (default 2 s; env MOE_TIMEOUT_NS). */
 MOE_API int32_t moe_set_timeout_ns(moe_mxfp4_t* h, uint64_t ns);
 

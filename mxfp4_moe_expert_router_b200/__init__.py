@@ -20,7 +20,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_OOM, MOE_ERR_CUD
 EXPORTS = ("mxfp4_quantize", "moe_mxfp4_create", "moe_route", "moe_forward", "moe_forward_host",
            "moe_status", "moe_set_timeout_ns", "moe_engine_grid", "moe_mxfp4_destroy",
            "moe_status_str", "moe_route_static", "moe_phase_ns",
-           "moe_stream_profile")
+           "moe_stream_profile", "moe_set_large_kind")
 
 
 class MoeConfig(ctypes.Structure):
@@ -53,6 +53,7 @@ def _load():
         "moe_forward_host": (i32, [vp, vp, i32, vp, vp]),
         "moe_status": (i32, [vp, vp]),
         "moe_set_timeout_ns": (i32, [vp, u64]),
+        "moe_set_large_kind": (i32, [vp, i32]),
         "moe_engine_grid": (i32, [vp]),
         "moe_mxfp4_destroy": (None, [vp]),
         "moe_status_str": (ctypes.c_char_p, [i32]),
@@ -196,6 +197,12 @@ class Moe:
 
     def moe_set_timeout_ns(self, ns: int):
         _check(lib.moe_set_timeout_ns(self.handle, int(ns)), "moe_set_timeout_ns")
+
+    LARGE_MXF4, LARGE_F16 = 1, 2
+
+    def moe_set_large_kind(self, kind: int):
+        """Weight stream for many positions per expert: LARGE_MXF4 (default) or LARGE_F16."""
+        _check(lib.moe_set_large_kind(self.handle, int(kind)), "moe_set_large_kind")
 
     @property
     def grid(self) -> int:

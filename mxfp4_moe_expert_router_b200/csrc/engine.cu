@@ -1040,6 +1040,114 @@ __device__ void phase_tile_gather(const EngineParams& p) {
   }
 }
 
+// ---- bf16 tile stream: permutation into balanced tiles, gather of x ------------------------
+// Unit tables of the bf16 tile stream: an expert's segment of c positions
+// becomes nb = ceil(c / FT_MAX) tiles of c / nb or c / nb + 1 consecutive
+// positions (the larger ones first); the down units are the same tiles, each
+// naming itself.  scratch: E ints.
+__device__ __noinline__ void build_ftiles(const int32_t* counts, const int32_t* offsets, int E, int32_t* scratch,
+                                          int32_t* units, int32_t* dunits, int32_t* n_units, int32_t* n_dunits) {
+  const int warp = threadIdx.x >> 5;
+  for (int x = threadIdx.x; x < E; x += THREADS) scratch[x] = (counts[x] + FT_MAX - 1) / FT_MAX;
+  __syncthreads();
+  if (warp == 0) warp_exclusive_scan(scratch, E, n_units);
+  __syncthreads();
+  if (threadIdx.x == 0) *n_dunits = *n_units;
+  for (int x = threadIdx.x; x < E; x += THREADS) {
+    const int c = counts[x];
+    const int nb = (c + FT_MAX - 1) / FT_MAX;
+    if (nb == 0) continue;
+    const int base = c / nb, rem = c % nb;
+    int pos = offsets[x];
+    for (int s = 0; s < nb; ++s) {
+      const int n = base + (s < rem ? 1 : 0);
+      const int u = scratch[x] + s;
+      int32_t* g = units + (int64_t)u * 4;
+      g[0] = x; g[1] = pos; g[2] = n; g[3] = 0;
+      int32_t* d = dunits + (int64_t)u * 4;
+      d[0] = x; d[1] = pos; d[2] = n; d[3] = u;
+      pos += n;
+    }
+  }
+}
+
+// Large T*K, bf16 tiles, step 2: as phase_permute_large, with balanced tiles.
+__device__ void phase_permute_f16(const EngineParams& p, uint8_t* smem) {
+  CtaTables& tb = tables(smem);
+  const int E = p.E, K = p.K, TK = p.TK;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < E; i += THREADS) tb.counts[i] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < TK; i += THREADS) atomicAdd(&tb.counts[__ldcg(p.idx + i)], 1);
+  __syncthreads();
+  for (int i = threadIdx.x; i < E; i += THREADS) tb.offsets[i] = tb.counts[i];
+  __syncthreads();
+  if (warp == 0) warp_exclusive_scan(tb.offsets, E, tb.offsets + E);
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    int32_t* scratch = reinterpret_cast<int32_t*>(ring_slot(smem, 0, 0));
+    build_ftiles(tb.counts, tb.offsets, E, scratch, p.units, p.dunits, &tb.n_units, &tb.n_dunits);
+    __syncthreads();
+    for (int i = threadIdx.x; i < E; i += THREADS) p.counts[i] = tb.counts[i];
+    for (int i = threadIdx.x; i <= E; i += THREADS) p.offsets[i] = tb.offsets[i];
+    if (threadIdx.x == 0) { p.n_units[0] = tb.n_units; p.n_units[1] = tb.n_dunits; }
+  }
+  const int64_t wg = (int64_t)blockIdx.x * WARPS + warp, ws = (int64_t)gridDim.x * WARPS;
+  for (int64_t x = wg; x < E; x += ws) {
+    int run = tb.offsets[x];
+    for (int base = 0; base < TK; base += 32) {
+      const int pr = base + lane;
+      const bool hit = pr < TK && __ldcg(p.idx + pr) == (int)x;
+      const uint32_t b = __ballot_sync(FULL, hit);
+      if (hit) {
+        const int pos = run + __popc(b & ((1u << lane) - 1u));
+        p.perm[pos] = pr; p.inv[pr] = pos; p.tokpos[pos] = pr / K; p.wpos[pos] = __ldcg(p.wts + pr);
+      }
+      run += __popc(b);
+    }
+  }
+}
+
+// Large T*K, bf16 tiles: the B block of every (tile, 64-K half-stage) of the
+// gate/up projection, gathered from the bf16 rows of x.  A warp moves one
+// (tile, half-stage): 8 lanes per position (16 bytes = 8 elements along K
+// each), four positions per step and eight steps of loads in flight.
+__device__ void phase_tile_gather_f16(const EngineParams& p, const __nv_bfloat16* x) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ns = p.H / FT_HK, nu = ld_cg_u32(p.n_units);
+  const int sub = lane >> 3, ch = lane & 7;  // position within a step of 4, chunk along K
+  const int64_t ntask = (int64_t)nu * ns;
+  for (int64_t us = (int64_t)blockIdx.x * WARPS + warp; us < ntask; us += (int64_t)gridDim.x * WARPS) {
+    const int u = (int)(us / ns), st = (int)(us % ns);
+    const int4 ur = __ldcg(reinterpret_cast<const int4*>(p.units) + u);
+    const int n = ur.z, rows = (n + 15) & ~15;
+    int tok[FT_MAX / 32];
+#pragma unroll
+    for (int i = 0; i < FT_MAX / 32; ++i) tok[i] = lane + 32 * i < n ? __ldcg(p.tokpos + ur.y + lane + 32 * i) : 0;
+    uint8_t* dst = p.xtf + us * FT_TERM_BYTES;
+    constexpr int STEPS = 8;
+    for (int tl0 = 0; tl0 < n; tl0 += 4 * STEPS) {
+      uint4 v[STEPS];
+#pragma unroll
+      for (int i = 0; i < STEPS; ++i) {
+        const int tl = tl0 + 4 * i + sub;
+        int t = 0;
+#pragma unroll
+        for (int q = 0; q < FT_MAX / 32; ++q) {
+          const int tq = __shfl_sync(FULL, tok[q], tl & 31);
+          if ((tl >> 5) == q) t = tq;
+        }
+        if (tl < n) v[i] = __ldcg(reinterpret_cast<const uint4*>(x + (int64_t)t * p.H + st * FT_HK) + ch);
+      }
+#pragma unroll
+      for (int i = 0; i < STEPS; ++i) {
+        const int tl = tl0 + 4 * i + sub;
+        if (tl < n) *reinterpret_cast<uint4*>(dst + ft_b_offset(tl, 8 * ch, rows)) = v[i];
+      }
+    }
+  }
+}
+
 // ---- phase C: the MXFP4 weight stream on tensor cores --------------------------------------
 struct StreamCtx {
   const int32_t* units;   // gate/up units
@@ -1609,6 +1717,425 @@ __device__ __forceinline__ float4 combine4(const EngineParams& p, const int32_t*
   return s;
 }
 
+// ---- bf16 tile stream roles ---------------------------------------------------------------
+// Three rings in the ring area: FT_RA raw weight half-stages, FT_NB B blocks,
+// FT_AB dequantised A blocks.  Barriers (pipe 0 / pipe 1 arrays):
+//   rawfull[i] = full(0, i)      producer's copies        rawempty[i] = empty(0, i)  converter warps
+//   bfull[i]   = full(1, i)      producer's copy          bempty[i]   = empty(1, i)  MMA commit
+//   afull[i]   = full(1, NB + i) converter warps          aempty[i]   = empty(1, NB + i)  MMA commit
+// and accf/acce(0, 0..1) between the MMA issuer and the epilogue warps.
+__device__ __forceinline__ uint8_t* ft_raw(uint8_t* smem, int i) { return smem + OFF_RING + (size_t)i * FT_RAW_BYTES; }
+__device__ __forceinline__ uint8_t* ft_b(uint8_t* smem, int i) {
+  return smem + OFF_RING + (size_t)FT_RA * FT_RAW_BYTES + (size_t)i * FT_TERM_BYTES;
+}
+__device__ __forceinline__ uint8_t* ft_a(uint8_t* smem, int i) {
+  return smem + OFF_RING + (size_t)FT_RA * FT_RAW_BYTES + (size_t)FT_NB * FT_TERM_BYTES + (size_t)i * FT_A_BYTES;
+}
+__device__ __forceinline__ uint64_t* rawfull_bar(uint8_t* smem, int i) { return full_bar(smem, 0, i); }
+__device__ __forceinline__ uint64_t* rawempty_bar(uint8_t* smem, int i) { return empty_bar(smem, 0, i); }
+__device__ __forceinline__ uint64_t* bfull_bar(uint8_t* smem, int i) { return full_bar(smem, 1, i); }
+__device__ __forceinline__ uint64_t* bempty_bar(uint8_t* smem, int i) { return empty_bar(smem, 1, i); }
+__device__ __forceinline__ uint64_t* afull_bar(uint8_t* smem, int i) { return full_bar(smem, 1, FT_NB + i); }
+__device__ __forceinline__ uint64_t* aempty_bar(uint8_t* smem, int i) { return empty_bar(smem, 1, FT_NB + i); }
+static_assert((size_t)FT_RA * FT_RAW_BYTES + (size_t)FT_NB * FT_TERM_BYTES + (size_t)FT_AB * FT_A_BYTES <= RING_BYTES,
+              "bf16 tile rings");
+static_assert(FT_RAW_BYTES % 128 == 0 && FT_TERM_BYTES % 128 == 0 && FT_A_BYTES % 128 == 0, "ring alignment");
+
+// kind::f16 instruction descriptor: bf16 A and B (K-major), fp32 D, M = 128.
+__device__ __forceinline__ uint32_t f16_idesc(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Bounded wait of lane 0 for a ring barrier's phase, shared with the warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const EngineParams& p, uint32_t info) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = wait_mbar(bar, parity, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, info);
+  return __shfl_sync(FULL, ok, 0) != 0;
+}
+
+// Producer warp of the bf16 tile stream: jobs -> queue entries (s0: first raw
+// half-stage sequence number, b0: first B block sequence number) -> copies.
+// Lane 0 issues; a down half-stage has two B blocks (the SwiGLU terms).
+__device__ void stream_producer_f16(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem,
+                                    const StreamCtx& cx, RoleState& rs) {
+  const int lane = threadIdx.x & 31;
+  JobEntry* jq = job_queue(smem, 0);
+  uint32_t* ready = p.sync + SY_READY;
+  const int gub = p.I / GU_I_ROWS, db = p.H / JOB_ROWS;
+  const int64_t n_gu = (int64_t)cx.n_units * gub, n_all = n_gu + (int64_t)cx.n_dunits * db;
+  const int nh_gu = p.H / FT_HK, nh_d = p.I / FT_HK;
+  const uint32_t need = (uint32_t)gub * 4u;
+  const uint32_t seq_start = rs.seq, b_start = rs.sfc;
+  bool ok = true;
+  unsigned long long t_empty = 0, t_ready = 0;
+  const unsigned long long t_begin = clock64();
+  fence_proxy_async_global();
+  const int64_t jbase = gridDim.x;
+  long long next = blockIdx.x;
+  for (;;) {
+    const int64_t j = __shfl_sync(FULL, next, 0);
+    if (j >= n_all || !ok) {
+      if (lane == 0) {
+        JobEntry* en = jq + (rs.qk % JQ);
+        en->job = -1; en->s0 = (int32_t)rs.seq; en->nc = 0; en->pad = (int32_t)rs.sfc;
+        __threadfence_block();
+        *reinterpret_cast<volatile int32_t*>(&en->flag) = rs.qk + 1;
+      }
+      ++rs.qk;
+      break;
+    }
+    if (lane == 0) next = jbase + atomicAdd(p.sync + SY_JOBS, 1u);
+    const bool isD = j >= n_gu;
+    const int64_t jj = isD ? j - n_gu : j;
+    const int per = isD ? db : gub;
+    const int u = (int)(jj / per), rb = (int)(jj % per);
+    const int4 ur = ld_tab(reinterpret_cast<const int4*>((isD ? cx.dunits : cx.units) + (int64_t)u * 4), cx.global);
+    const int e = ur.x, pos0 = ur.y, nt = ur.z;
+    const int nh = isD ? nh_d : nh_gu;
+    if (isD) {
+      const int gu = ur.w;
+      const unsigned long long tr0 = clock64();
+      if (ld_acquire_u32(ready + gu) < need) {
+        const uint64_t t0 = globaltimer_ns();
+        uint32_t spins = 0;
+        while (ld_acquire_u32(ready + gu) < need) {
+          if ((++spins & 15u) == 0u) {
+            if (error_set(p.sync)) { ok = false; break; }
+            if (globaltimer_ns() - t0 > p.timeout_ns) { set_error(p.sync, DEV_TIMEOUT_READY, gu); ok = false; break; }
+          }
+          __nanosleep(100);
+        }
+      }
+      t_ready += clock64() - tr0;
+      if (!ok) continue;
+      fence_proxy_async_global();  // the SwiGLU terms were written by generic stores of other CTAs
+    }
+    if (lane == 0) {
+      JobEntry* en = jq + (rs.qk % JQ);
+      en->job = (int32_t)j; en->s0 = (int32_t)rs.seq; en->nc = nh; en->unit = u; en->rb = rb;
+      en->isD = isD; en->e = e; en->pos0 = pos0; en->nt = nt; en->wj = rs.wj; en->pad = (int32_t)rs.sfc;
+      __threadfence_block();
+      *reinterpret_cast<volatile int32_t*>(&en->flag) = rs.qk + 1;
+    }
+    ++rs.qk;
+    ++rs.wj;
+    const uint8_t* wbase = isD ? lp.w_d + ((int64_t)e * db + rb) * (nh / 2) * STAGE_A_BYTES
+                               : lp.w_gu + ((int64_t)e * gub + rb) * (nh / 2) * STAGE_A_BYTES;
+    const int n16 = (nt + 15) & ~15;
+    const uint32_t bbytes = (uint32_t)n16 * FT_HK * 2u;
+    const int terms = isD ? 2 : 1;
+    for (int h = 0; h < nh && ok; ++h) {
+      // raw half-stage: codes of half h % 2 of stage h / 2, and that stage's scales
+      const uint32_t r = rs.seq;
+      const int ri = (int)(r % FT_RA);
+      const unsigned long long te0 = clock64();
+      if (r >= (uint32_t)FT_RA)
+        if (!warp_wait(rawempty_bar(smem, ri), ((r / FT_RA) + 1) & 1u, p, r)) { ok = false; break; }
+      if (lane == 0) {
+        uint64_t* fb = rawfull_bar(smem, ri);
+        const uint8_t* src = wbase + (int64_t)(h >> 1) * STAGE_A_BYTES;
+        mbar_arrive_expect_tx(fb, FT_RAW_BYTES);
+        bulk_g2s(ft_raw(smem, ri), src + (h & 1) * 4096, 4096, fb);
+        bulk_g2s(ft_raw(smem, ri) + 4096, src + STAGE_CODE_BYTES, 512, fb);
+      }
+      ++rs.seq;
+      for (int t = 0; t < terms; ++t) {
+        const uint32_t bq = rs.sfc;
+        const int bi = (int)(bq % FT_NB);
+        if (bq >= (uint32_t)FT_NB)
+          if (!warp_wait(bempty_bar(smem, bi), ((bq / FT_NB) + 1) & 1u, p, bq)) { ok = false; break; }
+        if (lane == 0) {
+          uint64_t* fb = bfull_bar(smem, bi);
+          const uint8_t* src = isD ? p.atf + (((int64_t)u * nh_d + h) * 2 + t) * FT_TERM_BYTES
+                                   : p.xtf + ((int64_t)u * nh_gu + h) * FT_TERM_BYTES;
+          mbar_arrive_expect_tx(fb, bbytes);
+          bulk_g2s(ft_b(smem, bi), src, bbytes, fb);
+        }
+        ++rs.sfc;
+      }
+      t_empty += clock64() - te0;
+    }
+  }
+  if (p.prof && lane == 0) {
+    atomicAdd(p.prof + PF_PROD_EMPTY, t_empty);
+    atomicAdd(p.prof + PF_PROD_READY, t_ready);
+    atomicAdd(p.prof + PF_PROD_TOTAL, clock64() - t_begin);
+    atomicAdd(p.prof + PF_STAGES, (unsigned long long)(rs.seq - seq_start));
+  }
+  // let every issued copy land before the rings are reused or the CTA exits
+  if (lane == 0) {
+    const uint32_t nr = min(rs.seq - seq_start, (uint32_t)FT_RA);
+    for (uint32_t r = rs.seq - nr; r != rs.seq; ++r) {
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(rawfull_bar(smem, (int)(r % FT_RA)), (r / FT_RA) & 1u))
+        if (globaltimer_ns() - t0 > p.timeout_ns) break;
+    }
+    const uint32_t nb = min(rs.sfc - b_start, (uint32_t)FT_NB);
+    for (uint32_t b = rs.sfc - nb; b != rs.sfc; ++b) {
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(bfull_bar(smem, (int)(b % FT_NB)), (b / FT_NB) & 1u))
+        if (globaltimer_ns() - t0 > p.timeout_ns) break;
+    }
+  }
+  __syncwarp();
+}
+
+// bf16 bits of the eight E2M1 magnitudes times 2^(sb - 127), as byte tables
+// for prmt: lo[0] (magnitudes 0..3) and lo[1] (4..7) hold the low bytes,
+// hi[0], hi[1] the high bytes.  Exact: every such product is a bf16 value
+// (normal for sb in [2, 252], where the exponent field is added directly).
+__device__ __forceinline__ void e2m1_bf16_tables(uint32_t sb, uint32_t (&lo)[2], uint32_t (&hi)[2]) {
+  uint32_t v[4];  // bf16 pairs (magnitude 2i in the low half, 2i + 1 in the high half)
+  if (sb >= 2u && sb <= 252u) {
+    const uint32_t d = (sb - 127u) << 7;  // added to each exponent field (two's complement)
+    const uint32_t dd = (d << 16) | (d & 0xFFFFu);
+    // magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 at 2^0: 0x0000 0x3F00 0x3F80 0x3FC0 0x4000 0x4040 0x4080 0x40C0
+    v[0] = (0x3F00u + d) << 16;
+    v[1] = __vadd2(0x3FC03F80u, dd);
+    v[2] = __vadd2(0x40404000u, dd);
+    v[3] = __vadd2(0x40C04080u, dd);
+  } else {
+    const float sc = sb == 0u ? __int_as_float(0x00400000) : sb == 255u ? __int_as_float(0x7FC00000)
+                                                                         : __int_as_float((int)(sb << 23));
+    const float mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(mag[2 * i] * sc));
+      const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(mag[2 * i + 1] * sc));
+      v[i] = a | (b << 16);
+    }
+  }
+  lo[0] = __byte_perm(v[0], v[1], 0x6420);
+  hi[0] = __byte_perm(v[0], v[1], 0x7531);
+  lo[1] = __byte_perm(v[2], v[3], 0x6420);
+  hi[1] = __byte_perm(v[2], v[3], 0x7531);
+}
+// Four E2M1 codes (16 bits, element i in bits 4i..4i+3) -> two bf16x2 words.
+__device__ __forceinline__ void e2m1x4_bf16(uint32_t c16, const uint32_t (&lo)[2], const uint32_t (&hi)[2],
+                                            uint32_t& w0, uint32_t& w1) {
+  const uint32_t sel = c16 & 0x7777u;
+  const uint32_t l4 = __byte_perm(lo[0], lo[1], sel), h4 = __byte_perm(hi[0], hi[1], sel);
+  w0 = __byte_perm(l4, h4, 0x5140) | ((c16 << 12) & 0x8000u) | ((c16 << 24) & 0x80000000u);
+  w1 = __byte_perm(l4, h4, 0x7362) | ((c16 << 4) & 0x8000u) | ((c16 << 16) & 0x80000000u);
+}
+
+// Converter warps: each raw weight half-stage (128 rows x 64 K of codes, the
+// stage's scales) becomes a bf16 A block in the kind::f16 K-major layout.  An
+// item is one row's 32-element block: 16 bytes of codes and its scale in, 64
+// bytes of bf16 out.
+__device__ void stream_convert_f16(const EngineParams& p, uint8_t* smem, int ci, RoleState& rs) {
+  const int lane = threadIdx.x & 31;
+  JobEntry* jq = job_queue(smem, 0);
+  bool ok = true;
+  for (;;) {
+    JobEntry* en = jq + (rs.qk % JQ);
+    if (!wait_entry(p, en, rs.qk)) return;
+    const int job = *reinterpret_cast<volatile int32_t*>(&en->job);
+    if (job < 0) { ++rs.qk; break; }
+    const int s0 = en->s0, nh = en->nc;
+    ++rs.qk;
+    if (!ok) continue;
+    for (int h = 0; h < nh; ++h) {
+      const uint32_t r = (uint32_t)s0 + h;
+      const int ri = (int)(r % FT_RA), ai = (int)(r % FT_AB);
+      if (!warp_wait(rawfull_bar(smem, ri), (r / FT_RA) & 1u, p, r) ||
+          (r >= (uint32_t)FT_AB && !warp_wait(aempty_bar(smem, ai), ((r / FT_AB) + 1) & 1u, p, r))) {
+        ok = false;
+        break;
+      }
+      const uint8_t* raw = ft_raw(smem, ri);
+      uint8_t* out = ft_a(smem, ai);
+      const int kb0 = 2 * (h & 1);  // scale blocks of this half
+      for (int it = ci * 32 + lane; it < 256; it += FT_CONV_WARPS * 32) {
+        const int m = it & 127, blk = it >> 7;
+        const uint4 cw = *reinterpret_cast<const uint4*>(raw + (m >> 3) * 256 + blk * 128 + (m & 7) * 16);
+        const uint32_t sb = raw[4096 + (m & 31) * 16 + (m >> 5) * 4 + kb0 + blk];
+        uint32_t lo[2], hi[2];
+        e2m1_bf16_tables(sb, lo, hi);
+        const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {  // elements 32 blk + 8 q .. + 7 of the half: chunk j = 4 blk + q
+          uint4 o;
+          e2m1x4_bf16(w[q] & 0xFFFFu, lo, hi, o.x, o.y);
+          e2m1x4_bf16(w[q] >> 16, lo, hi, o.z, o.w);
+          const int jc = 4 * blk + q;
+          *reinterpret_cast<uint4*>(out + (jc >> 1) * 4096 + (m >> 3) * 256 + (jc & 1) * 128 + (m & 7) * 16) = o;
+        }
+      }
+      fence_proxy_async_smem();  // the bf16 block is read by the tensor cores (async proxy)
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(afull_bar(smem, ai));
+        mbar_arrive(rawempty_bar(smem, ri));
+      }
+    }
+  }
+}
+
+// MMA issuer of the bf16 tile stream: per half-stage and B block 4 MMAs of
+// K = 16 (M = 128, N = n16) into the job's accumulator.
+__device__ void stream_mma_f16(const EngineParams& p, uint8_t* smem, uint32_t tmem, RoleState& rs) {
+  JobEntry* jq = job_queue(smem, 0);
+  const bool prof = p.prof != nullptr;
+  unsigned long long t_full = 0, t_issue = 0, t_acc = 0;
+  bool ok = true;
+  for (;;) {
+    JobEntry* en = jq + (rs.qk % JQ);
+    if (!wait_entry(p, en, rs.qk)) return;
+    const int job = *reinterpret_cast<volatile int32_t*>(&en->job);
+    if (job < 0) { ++rs.qk; break; }
+    const int s0 = en->s0, nh = en->nc, nt = en->nt, wj = en->wj, isD = en->isD, b0 = en->pad;
+    ++rs.qk;
+    if (!ok) continue;
+    const int b = wj & 1;
+    const uint32_t use = (uint32_t)(wj >> 1);
+    const unsigned long long ta0 = pclock(prof);
+    if (use > 0 && !wait_mbar(acce_bar(smem, 0, b), (use - 1) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, wj)) {
+      ok = false;
+      continue;
+    }
+    t_acc += pclock(prof) - ta0;
+    tc_fence_after();
+    const uint32_t tacc = tmem + (uint32_t)(b * FT_ACC_COLS);
+    const int n16 = (nt + 15) & ~15, terms = isD ? 2 : 1;
+    const uint32_t idesc = f16_idesc(n16);
+    for (int h = 0; h < nh && ok; ++h) {
+      const uint32_t r = (uint32_t)s0 + h;
+      const int ai = (int)(r % FT_AB);
+      const unsigned long long tf0 = pclock(prof);
+      if (!wait_mbar(afull_bar(smem, ai), (r / FT_AB) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, r)) {
+        ok = false;
+        break;
+      }
+      t_full += pclock(prof) - tf0;
+      const uint32_t sa = smem_u32(ft_a(smem, ai));
+      for (int t = 0; t < terms; ++t) {
+        const uint32_t bq = (uint32_t)b0 + h * terms + t;
+        const int bi = (int)(bq % FT_NB);
+        const unsigned long long tb0 = pclock(prof);
+        if (!wait_mbar(bfull_bar(smem, bi), (bq / FT_NB) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, bq)) {
+          ok = false;
+          break;
+        }
+        const unsigned long long tm0 = pclock(prof);
+        t_full += tm0 - tb0;
+        tc_fence_after();
+        const uint32_t sb = smem_u32(ft_b(smem, bi));
+#pragma unroll
+        for (int k16 = 0; k16 < FT_HK / 16; ++k16)
+          mma_bf16(tacc, smem_desc(sa + k16 * 4096, 128, 256), smem_desc(sb + k16 * n16 * 32, 128, 256), idesc,
+                   (h > 0 || t > 0 || k16 > 0) ? 1u : 0u);
+        tc_commit(bempty_bar(smem, bi));
+        t_issue += pclock(prof) - tm0;
+      }
+      if (!ok) break;
+      tc_commit(aempty_bar(smem, ai));
+    }
+    if (ok) tc_commit(accf_bar(smem, 0, b));
+  }
+  if (prof) {
+    atomicAdd(p.prof + PF_MMA_FULL, t_full);
+    atomicAdd(p.prof + PF_MMA_ISSUE, t_issue);
+    atomicAdd(p.prof + PF_MMA_ACC, t_acc);
+  }
+}
+
+// Epilogue warps of the bf16 tile stream (warp q reads accumulator rows
+// 32 q..32 q + 31).  Gate/up: SwiGLU of the gate and up rows (lanes l and
+// l + 16), written as two bf16 terms into the tile's down B blocks.  Down:
+// each position's column times its routing weight.
+__device__ void stream_epilogue_f16(const EngineParams& p, uint8_t* smem, const StreamCtx& cx, uint32_t tmem,
+                                    RoleState& rs) {
+  const int lane = threadIdx.x & 31, q = (threadIdx.x >> 5) & 3;
+  JobEntry* jq = job_queue(smem, 0);
+  uint32_t* ready = p.sync + SY_READY;
+  const int nhd = p.I / FT_HK;
+  const bool prof = p.prof != nullptr;
+  unsigned long long t_wait = 0, t_work = 0, n_jobs = 0;
+  const unsigned long long t_begin = pclock(prof);
+  bool ok = true;
+  for (;;) {
+    JobEntry* en = jq + (rs.qk % JQ);
+    if (!wait_entry(p, en, rs.qk)) return;
+    const int job = *reinterpret_cast<volatile int32_t*>(&en->job);
+    if (job < 0) { ++rs.qk; break; }
+    const int wj = en->wj;
+    const int u = en->unit, rb = en->rb, isD = en->isD, pos0 = en->pos0, nt = en->nt;
+    ++rs.qk;
+    if (!ok) continue;
+    ++n_jobs;
+    const int b = wj & 1;
+    const unsigned long long tw0 = pclock(prof);
+    if (!wait_mbar(accf_bar(smem, 0, b), (uint32_t)(wj >> 1) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, wj)) {
+      ok = false;
+      continue;
+    }
+    const unsigned long long tk0 = pclock(prof);
+    t_wait += tk0 - tw0;
+    tc_fence_after();
+    const uint32_t tacc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * FT_ACC_COLS);
+    const int n16 = (nt + 15) & ~15;
+    if (!isD) {
+      // rows 32 q + l: gate of I row i0 + 16 q + l for l < 16, up of the same row for l >= 16
+      const int i = rb * GU_I_ROWS + 16 * q + (lane & 15);
+      const int hD = i / FT_HK, k = i % FT_HK;
+      uint8_t* dst = p.atf + ((int64_t)u * nhd + hD) * 2 * FT_TERM_BYTES;
+      for (int j0 = 0; j0 < nt; j0 += 8) {
+        float v[8];
+        tmem_ld8(tacc + j0, v);
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const float other = __shfl_xor_sync(FULL, v[jj], 16);
+          const int j = j0 + jj;
+          if (lane < 16 && j < nt) {
+            const float g = v[jj], up = other;
+            const float a = g / (1.0f + expf(-g)) * up;
+            const __nv_bfloat16 h0 = __float2bfloat16_rn(a);
+            const __nv_bfloat16 h1 = __float2bfloat16_rn(a - __bfloat162float(h0));
+            *reinterpret_cast<__nv_bfloat16*>(dst + ft_b_offset(j, k, n16)) = h0;
+            *reinterpret_cast<__nv_bfloat16*>(dst + FT_TERM_BYTES + ft_b_offset(j, k, n16)) = h1;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        fence_proxy_async_global();
+        __threadfence();
+        red_release_add_u32(ready + u, 1u);
+      }
+    } else {
+      const int hrow = rb * JOB_ROWS + 32 * q + lane;
+      for (int j0 = 0; j0 < nt; j0 += 8) {
+        float v[8];
+        tmem_ld8(tacc + j0, v);
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int j = j0 + jj;
+          if (j < nt) p.ypair[(int64_t)(pos0 + j) * p.H + hrow] = v[jj] * ld_tab(cx.wpos + pos0 + j, cx.global);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(acce_bar(smem, 0, b));
+    t_work += pclock(prof) - tk0;
+  }
+  if (prof && lane == 0) {
+    atomicAdd(p.prof + PF_EPI_WAIT, t_wait);
+    atomicAdd(p.prof + PF_EPI_WORK, t_work);
+    atomicAdd(p.prof + PF_EPI_TOTAL, pclock(prof) - t_begin);
+    if (q == 0) atomicAdd(p.prof + PF_JOBS, n_jobs);
+  }
+}
+
 __device__ void phase_combine_out(const EngineParams& p, const int32_t* inv) {
   const int64_t gt = (int64_t)blockIdx.x * THREADS + threadIdx.x;
   const int64_t gs = (int64_t)gridDim.x * THREADS;
@@ -1665,17 +2192,19 @@ __device__ void phase_combine_rmsnorm(const EngineParams& p, const int32_t* inv,
 
 // All layers; returns early (every thread of the CTA together) when a grid
 // barrier reports an error, or after routing in route-only mode.
-template <bool TILES>
+// MODE 0: pipeline stream; MODE 1: E2M1 term tiles (kind::mxf4); MODE 2: bf16
+// tiles (kind::f16).  The tile modes run only above SMALL_PAIRS.
+template <int MODE>
 __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, RoleState& rs,
                            bool stamp) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool small = !TILES && p.TK <= SMALL_PAIRS;  // the tile stream runs only above SMALL_PAIRS
+  const bool small = MODE == 0 && p.TK <= SMALL_PAIRS;
   CtaTables& tb = tables(smem);
   for (int layer = 0; layer < p.L; ++layer) {
     const LayerPtrs& lp = p.layers[layer];
     const __nv_bfloat16* x = layer == 0 ? p.x_in : p.xnext;
     uint64_t* st = stamp ? p.stamps + 1 + layer * STAMPS_PER_LAYER : nullptr;
-    if constexpr (TILES) phase_router_tiles(x, lp.router_w, p.logits, p.sync, p.T, p.H, p.E, p.TK, p.HS, smem);
+    if constexpr (MODE != 0) phase_router_tiles(x, lp.router_w, p.logits, p.sync, p.T, p.H, p.E, p.TK, p.HS, smem);
     else phase_router(p, lp, x, smem);
     if (st) st[0] = globaltimer_ns();
     StreamCtx cx;
@@ -1687,18 +2216,22 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
       cx = StreamCtx{tb.units, tb.dunits, tb.tokpos, tb.wpos, tb.n_units, tb.n_dunits, false};
       inv = tb.inv;
     } else {
-      phase_images(p, x, layer);
+      if constexpr (MODE != 2) phase_images(p, x, layer);  // the bf16 tiles gather x itself
       if (st) st[1] = globaltimer_ns();
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 1)) return;
       if (st) st[2] = globaltimer_ns();
       phase_topk_large(p, lp);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 2)) return;
       if (st) st[3] = globaltimer_ns();
-      phase_permute_large(p, smem);
+      if constexpr (MODE == 2) phase_permute_f16(p, smem);
+      else phase_permute_large(p, smem);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 3)) return;
       if (p.route_only) return;
-      if constexpr (TILES) {
+      if constexpr (MODE == 1) {
         phase_tile_gather(p);
+        if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 6)) return;
+      } else if constexpr (MODE == 2) {
+        phase_tile_gather_f16(p, x);
         if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 6)) return;
       }
       cx = StreamCtx{p.units, p.dunits, p.tokpos, p.wpos, (int)ld_cg_u32(p.n_units), (int)ld_cg_u32(p.n_units + 1), true};
@@ -1707,7 +2240,7 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
     if (st) st[4] = globaltimer_ns();
     fence_proxy_async_smem();  // the ring held routing scratch written by generic stores
     __syncthreads();
-    if constexpr (!TILES) {  // two pipelines per CTA, units of <= NT_MAX positions
+    if constexpr (MODE == 0) {  // two pipelines per CTA, units of <= NT_MAX positions
       if (warp < EPI_WARP0) {
         const int pipe = warp >> 1;
         if ((warp & 1) == 0) {
@@ -1719,7 +2252,7 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
       } else {
         stream_epilogue(p, smem, cx, tmem, (warp - EPI_WARP0) / 4, rs);
       }
-    } else {  // one pipeline per CTA over tiles of <= LT_MAX positions
+    } else if constexpr (MODE == 1) {  // one pipeline per CTA over tiles of <= LT_MAX positions
       if (warp == 0) {
         stream_producer<true>(p, lp, smem, cx, 0, rs);
       } else if (warp == 1) {
@@ -1727,6 +2260,17 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
         __syncwarp();
       } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
         stream_epilogue_lt(p, smem, cx, tmem, rs);
+      }
+    } else {  // bf16 tiles: producer, MMA issuer, six converter warps, four epilogue warps
+      if (warp == 0) {
+        stream_producer_f16(p, lp, smem, cx, rs);
+      } else if (warp == 1) {
+        if (lane == 0) stream_mma_f16(p, smem, tmem, rs);
+        __syncwarp();
+      } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
+        stream_epilogue_f16(p, smem, cx, tmem, rs);
+      } else {
+        stream_convert_f16(p, smem, warp < EPI_WARP0 ? warp - 2 : warp - 6, rs);
       }
     }
     if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 4)) return;
@@ -1744,17 +2288,20 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
   }
 }
 
-// Two instances: the pipeline stream (TILES = false) and the tile stream; each
-// holds only its own stream code.
-template <bool TILES>
+// Three instances (MODE 0, 1, 2, see run_layers); each holds only its own
+// stream code.
+template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int pp = 0; pp < NPIPE; ++pp) {
       for (int i = 0; i < NSLOT; ++i) {
-        mbar_init(full_bar(smem, pp, i), 1);
-        mbar_init(empty_bar(smem, pp, i), 1);
+        // bf16 tiles: a raw slot is free once every converter warp has read
+        // it (rawempty_bar), an A block is full once every converter warp
+        // has written it (afull_bar)
+        mbar_init(full_bar(smem, pp, i), MODE == 2 && pp == 1 && i >= FT_NB ? FT_CONV_WARPS : 1);
+        mbar_init(empty_bar(smem, pp, i), MODE == 2 && pp == 0 ? FT_CONV_WARPS : 1);
       }
       for (int i = 0; i < NACC; ++i) {
         mbar_init(accf_bar(smem, pp, i), 1);
@@ -1778,7 +2325,7 @@ __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p
   const bool stamp = p.stamps != nullptr && blockIdx.x == 0 && threadIdx.x == 0;
   if (stamp) p.stamps[0] = globaltimer_ns();
   RoleState rs;
-  run_layers<TILES>(p, smem, tmem, rs, stamp);
+  run_layers<MODE>(p, smem, tmem, rs, stamp);
   if (use_tmem) {
     // free tensor memory only once every MMA this CTA issued has completed
     if (warp < EPI_WARP0 && (warp & 1) && lane == 0) {
@@ -1803,7 +2350,7 @@ size_t engine_smem_bytes() { return SMEM_BYTES; }
 
 int engine_max_grid(int device, int* err) {
   int per_sm = ~0u >> 1, sms = 0;
-  for (const void* k : {(const void*)engine_kernel<false>, (const void*)engine_kernel<true>}) {
+  for (const void* k : {(const void*)engine_kernel<0>, (const void*)engine_kernel<1>, (const void*)engine_kernel<2>}) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) { *err = (int)e; return 0; }
     int n = 0;
@@ -1819,8 +2366,9 @@ int engine_max_grid(int device, int* err) {
 
 cudaError_t engine_launch(const EngineParams& p, int grid, cudaStream_t s) {
   void* args[] = {const_cast<EngineParams*>(&p)};
-  const void* k = use_tiles(p.TK, p.E) && !p.route_only ? (const void*)engine_kernel<true>
-                                                        : (const void*)engine_kernel<false>;
+  const void* k = !use_tiles(p.TK, p.E) || p.route_only ? (const void*)engine_kernel<0>
+                  : p.large == LARGE_F16                  ? (const void*)engine_kernel<2>
+                                                          : (const void*)engine_kernel<1>;
   return cudaLaunchCooperativeKernel(k, dim3(grid), dim3(THREADS), args, SMEM_BYTES, s);
 }
 

@@ -92,6 +92,41 @@ __host__ __device__ constexpr int lt_sf_offset(int tl, int k, int kb) {
   return (tl / 16) * 512 + (8 * (tl % 4) + k) * 16 + 4 * ((tl % 16) / 4) + kb;
 }
 __host__ __device__ constexpr int lt_code_offset(int tl) { return LT_SF_BYTES + tl * IMG_CODE_BYTES; }
+// ---- large T*K: bf16 tile stream (kind::f16 on dequantised weights) ----------------------
+// The same tile jobs, with x in bf16 as the B operand (one term, exact) and
+// the MXFP4 weights dequantised to bf16 in shared memory by converter warps.
+// A tile holds up to FT_MAX positions (balanced split of an expert's
+// segment), padded to n16 (a multiple of 16) B rows, so one MMA has N = n16.
+// K runs in half-stages of 64: per half-stage the producer brings the half of
+// the packed weight stage (4096 bytes of codes + the stage's 512 scale bytes)
+// into the raw ring and the B block(s) into the B ring; a converter pass
+// turns the raw half into a bf16 A block; the MMA issuer runs 4 MMAs of
+// K = 16 per B block.  B blocks are K-major without swizzle: for K slice k16
+// [n16 / 8 row groups][2 core matrices along K][8 rows][16 bytes], slices
+// n16 * 32 bytes apart (ft_b_offset).  The down projection's B is the SwiGLU
+// output as two bf16 terms (leading term, then the remainder), two B blocks
+// per half-stage accumulated into the same accumulator.
+constexpr int FT_MAX = 128;
+constexpr int FT_HK = 64;                                 // K per half-stage
+constexpr int FT_TERM_BYTES = FT_MAX * FT_HK * 2;         // one B block at most: 16384
+constexpr int FT_RAW_BYTES = 4096 + 512;                  // codes of a half-stage + the stage's scales
+constexpr int FT_RA = 8;                                  // raw weight ring
+constexpr int FT_NB = 6;                                  // B ring
+constexpr int FT_AB = 3;                                  // dequantised A blocks
+constexpr int FT_A_BYTES = 128 * FT_HK * 2;               // 16384
+constexpr int FT_ACC_COLS = FT_MAX;                       // accumulator columns per job
+constexpr int FT_CONV_WARPS = 6;                          // warps 2, 3, 8..11
+static_assert(FT_RA <= NSLOT && FT_NB + FT_AB <= NSLOT, "bf16 tile barriers");
+static_assert(2 * FT_ACC_COLS <= TMEM_COLS, "tensor memory budget (bf16 tiles)");
+// Byte offset of element k (< FT_HK) of B row r in a block of `rows` rows.
+__host__ __device__ constexpr int ft_b_offset(int r, int k, int rows) {
+  return (k / 16) * rows * 32 + (r / 8) * 256 + ((k % 16) / 8) * 128 + (r % 8) * 16 + (k % 8) * 2;
+}
+// Tiles of the bf16 stream (at most FT_MAX positions each, balanced).
+__host__ __device__ inline int max_ftiles(int E, int64_t TK) { return (int)((E < TK ? E : TK) + TK / FT_MAX + 1); }
+// Large-T*K stream kind: 1 = E2M1 term tiles on kind::mxf4, 2 = bf16 tiles on kind::f16.
+enum : int { LARGE_MXF4 = 1, LARGE_F16 = 2 };
+
 // Whether a launch of T*K pairs over E experts streams tiles.
 __host__ __device__ inline bool use_tiles(int64_t TK, int E) {
   return TK > SMALL_PAIRS && TK >= (int64_t)LT_MIN_PER_EXPERT * E;
@@ -154,6 +189,9 @@ struct EngineParams {
   uint8_t* aimg;              // [I/KS][TK][IMG_BYTES] E2M1 term images of the SwiGLU output
   uint8_t* xtl;               // large T*K: [tiles][H/KS][LT_IMG_BYTES] x term images per tile
   uint8_t* atl;               // large T*K: [tiles][I/KS][LT_IMG_BYTES] SwiGLU term images per tile
+  uint8_t* xtf;               // bf16 tiles: [tiles][H/FT_HK][FT_TERM_BYTES] x per tile
+  uint8_t* atf;               // bf16 tiles: [tiles][I/FT_HK][2][FT_TERM_BYTES] SwiGLU output terms per tile
+  int large;                  // stream kind above SMALL_PAIRS with tiles: LARGE_MXF4 or LARGE_F16
   float* ypair;               // [TK][H]
   uint32_t* sync;             // see SY_*
   uint64_t* stamps;           // null or [1 + MAX_LAYERS * STAMPS_PER_LAYER] %globaltimer ns (CTA 0)

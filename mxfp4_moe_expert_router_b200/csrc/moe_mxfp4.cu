@@ -27,6 +27,9 @@ struct moe_mxfp4 {
   uint8_t* aimg = nullptr;
   uint8_t* xtl = nullptr;  // large T*k only
   uint8_t* atl = nullptr;
+  uint8_t* xtf = nullptr;  // large T*k only (bf16 tiles)
+  uint8_t* atf = nullptr;
+  int large = LARGE_MXF4;  // stream kind for large T*k
   __nv_bfloat16* xnext = nullptr;
   int32_t *idx = nullptr, *counts = nullptr, *offsets = nullptr, *perm = nullptr, *inv = nullptr,
           *tokpos = nullptr, *units = nullptr, *dunits = nullptr, *n_units = nullptr;
@@ -91,6 +94,7 @@ EngineParams base_params(const moe_mxfp4* h, int T) {
   p.perm = h->perm; p.inv = h->inv; p.tokpos = h->tokpos; p.wpos = h->wpos;
   p.units = h->units; p.dunits = h->dunits; p.n_units = h->n_units; p.aimg = h->aimg;
   p.xtl = h->xtl; p.atl = h->atl;
+  p.xtf = h->xtf; p.atf = h->atf; p.large = h->large;
   p.ypair = h->ypair;
   p.sync = h->sync;
   p.stamps = h->stamps;
@@ -197,6 +201,9 @@ int32_t moe_mxfp4_create(const moe_config_t* cfg, const uint8_t* const* gate_cod
   if (ok && use_tiles(TKm, E)) {  // tile images of the large-T*k stream
     const size_t tiles = (size_t)max_tiles(E, TKm);
     ok = dalloc(h, &h->xtl, tiles * (H / KS) * LT_IMG_BYTES) && dalloc(h, &h->atl, tiles * (I / KS) * LT_IMG_BYTES);
+    const size_t ftiles = (size_t)max_ftiles(E, TKm);
+    ok = ok && dalloc(h, &h->xtf, ftiles * (H / FT_HK) * FT_TERM_BYTES) &&
+         dalloc(h, &h->atf, ftiles * (I / FT_HK) * 2 * FT_TERM_BYTES);
   }
   if (!ok) { free_all(h); delete h; cudaGetLastError(); return MOE_ERR_OOM; }
 
@@ -257,6 +264,12 @@ int32_t moe_forward(moe_mxfp4_t* h, const void* x_bf16, int32_t T, void* y_bf16,
   p.layer_io = static_cast<__nv_bfloat16*>(layer_io_bf16);
   return engine_launch(p, h->grid, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK
                                                                                      : MOE_ERR_CUDA;
+}
+
+int32_t moe_set_large_kind(moe_mxfp4_t* h, int32_t kind) {
+  if (!h || (kind != LARGE_MXF4 && kind != LARGE_F16)) return MOE_ERR_INVALID_ARG;
+  h->large = kind;
+  return MOE_OK;
 }
 
 int32_t moe_status(moe_mxfp4_t* h, void* stream) {

@@ -105,6 +105,22 @@ def test_forward_matches_oracle(m, name):
     check_forward(y, x_values(xb), lw, w.top_k)
 
 
+@pytest.mark.parametrize("kind", ["mxf4", "f16"])
+@pytest.mark.parametrize("name,tokens", [("ragged_large", 80), ("ragged_large", 192)])
+def test_large_t_kinds_match_oracle(m, kind, name, tokens):
+    """Both weight streams for many positions per expert (E2M1 term tiles on the
+    fp4 MMA, bf16 tiles on the bf16 MMA): ragged tiles, T*K = 320 and 768."""
+    from tests.gpu_helpers import bf16_dev, check_forward, make_moe
+    H, I, E, k, _ = SHAPES[name]
+    w = synth.Workload(name, H, I, E, k, tokens, device_draw=False)
+    xb, lw, _ = quantized_layer_np(w, seed=23)
+    mo = make_moe(w, [lw])
+    mo.moe_set_large_kind(mo.LARGE_MXF4 if kind == "mxf4" else mo.LARGE_F16)
+    y = mo.moe_forward(bf16_dev(xb))
+    mo.moe_status()
+    check_forward(y, x_values(xb), lw, w.top_k)
+
+
 def test_forward_with_router_bias(m):
     from tests.gpu_helpers import bf16_dev, check_forward, make_moe
     w = _workload("ragged_large", zipf=1.2)
