@@ -158,6 +158,27 @@ MOE_API int32_t moe_forward_host(moe_mxfp4_t* h, const void* x_host, int32_t T, 
                          void* stream);
 
 /*
+ * moe_forward_host_async -- moe_forward with HOST input and output, without
+ * synchronising: the copy of x_host to one of two device staging slots (on
+ * an internal copy stream), the layers (on `stream`) and the copy of y back
+ * to y_host (on a second internal copy stream) are only enqueued, so a call's
+ * copies overlap the layers of its neighbours.  x_host must stay unchanged
+ * and y_host unread until the copies are done: moe_host_join, then a
+ * synchronisation of `stream` (or moe_status, which synchronises the copy
+ * streams too).  Pinned host memory gives the overlap; pageable memory works
+ * but serialises.  Errors: MOE_ERR_INVALID_ARG, MOE_ERR_CUDA; device-side
+ * timeouts are reported by the next moe_status.
+ */
+MOE_API int32_t moe_forward_host_async(moe_mxfp4_t* h, const void* x_host, int32_t T, void* y_host,
+                               void* stream);
+
+/*
+ * moe_host_join -- make `stream` wait (without blocking the host) for the
+ * output copies of every moe_forward_host_async call enqueued so far.
+ */
+MOE_API int32_t moe_host_join(moe_mxfp4_t* h, void* stream);
+
+/*
  * moe_status -- synchronise `stream`, then return and clear the device-side
  * status of the handle: MOE_OK, or MOE_ERR_TIMEOUT if a bounded wait inside
  * the engine expired (the handle's wait state is reset, so it stays usable).

@@ -20,7 +20,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_OOM, MOE_ERR_CUD
 EXPORTS = ("mxfp4_quantize", "moe_mxfp4_create", "moe_route", "moe_forward", "moe_forward_host",
            "moe_status", "moe_set_timeout_ns", "moe_engine_grid", "moe_mxfp4_destroy",
            "moe_status_str", "moe_route_static", "moe_phase_ns",
-           "moe_stream_profile", "moe_set_large_kind")
+           "moe_stream_profile", "moe_set_large_kind", "moe_forward_host_async", "moe_host_join")
 
 
 class MoeConfig(ctypes.Structure):
@@ -51,6 +51,8 @@ def _load():
         "moe_route": (i32, [vp, i32, vp, i32, vp, vp, vp, vp, vp, vp, vp]),
         "moe_forward": (i32, [vp, vp, i32, vp, vp, vp]),
         "moe_forward_host": (i32, [vp, vp, i32, vp, vp]),
+        "moe_forward_host_async": (i32, [vp, vp, i32, vp, vp]),
+        "moe_host_join": (i32, [vp, vp]),
         "moe_status": (i32, [vp, vp]),
         "moe_set_timeout_ns": (i32, [vp, u64]),
         "moe_set_large_kind": (i32, [vp, i32]),
@@ -171,6 +173,16 @@ class Moe:
         _check(lib.moe_forward_host(self.handle, _ptr(x_host), T, _ptr(y_host), _stream(stream)),
                "moe_forward_host")
         return y_host
+
+    def moe_forward_host_async(self, x_host, y_host, stream=None):
+        """Enqueue H2D of x_host, the layers, D2H into y_host (pinned); no synchronisation."""
+        _check(lib.moe_forward_host_async(self.handle, _ptr(x_host), x_host.shape[0], _ptr(y_host),
+                                          _stream(stream)), "moe_forward_host_async")
+        return y_host
+
+    def moe_host_join(self, stream=None):
+        """Make `stream` wait for every enqueued output copy of moe_forward_host_async."""
+        _check(lib.moe_host_join(self.handle, _stream(stream)), "moe_host_join")
 
     def moe_status(self, stream=None):
         _check(lib.moe_status(self.handle, _stream(stream)), "moe_status")

@@ -39,6 +39,11 @@ struct moe_mxfp4 {
   unsigned long long* prof = nullptr;
   bool profiling = false;
   __nv_bfloat16 *x_stage = nullptr, *y_stage = nullptr;
+  // moe_forward_host_async: two staging slots, copy streams and their events
+  __nv_bfloat16 *x_stage2[2] = {}, *y_stage2[2] = {};
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t ev_in[2] = {}, ev_k[2] = {}, ev_out[2] = {};
+  uint64_t host_seq = 0;
   std::vector<void*> allocs;
 };
 
@@ -56,8 +61,34 @@ bool dalloc(moe_mxfp4* h, T** out, size_t bytes) {
 }
 
 void free_all(moe_mxfp4* h) {
+  for (int i = 0; i < 2; ++i) {
+    if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+    if (h->ev_k[i]) cudaEventDestroy(h->ev_k[i]);
+    if (h->ev_out[i]) cudaEventDestroy(h->ev_out[i]);
+    h->ev_in[i] = h->ev_k[i] = h->ev_out[i] = nullptr;
+  }
+  if (h->h2d) cudaStreamDestroy(h->h2d);
+  if (h->d2h) cudaStreamDestroy(h->d2h);
+  h->h2d = h->d2h = nullptr;
   for (void* p : h->allocs) cudaFree(p);
   h->allocs.clear();
+}
+
+// Copy streams, events and the second staging slot of moe_forward_host_async,
+// created on first use.
+bool host_async_ready(moe_mxfp4* h) {
+  if (h->h2d) return true;
+  const size_t bytes = (size_t)h->cfg.max_tokens * h->cfg.hidden * 2;
+  h->x_stage2[0] = h->x_stage;
+  h->y_stage2[0] = h->y_stage;
+  if (!dalloc(h, &h->x_stage2[1], bytes) || !dalloc(h, &h->y_stage2[1], bytes)) return false;
+  for (int i = 0; i < 2; ++i)
+    if (cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h->ev_k[i], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming) != cudaSuccess)
+      return false;
+  return cudaStreamCreateWithFlags(&h->h2d, cudaStreamNonBlocking) == cudaSuccess &&
+         cudaStreamCreateWithFlags(&h->d2h, cudaStreamNonBlocking) == cudaSuccess;
 }
 
 size_t stage_bytes_gu(const moe_config_t& c) {
@@ -276,6 +307,8 @@ int32_t moe_status(moe_mxfp4_t* h, void* stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (h->h2d && (cudaStreamSynchronize(h->h2d) != cudaSuccess || cudaStreamSynchronize(h->d2h) != cudaSuccess))
+    return MOE_ERR_CUDA;
   uint32_t words[SY_READY] = {};
   if (cudaMemcpy(words, h->sync, sizeof(words), cudaMemcpyDeviceToHost) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -298,6 +331,43 @@ int32_t moe_forward_host(moe_mxfp4_t* h, const void* x_host, int32_t T, void* y_
   if (cudaMemcpyAsync(y_host, h->y_stage, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   return moe_status(h, stream);
+}
+
+int32_t moe_forward_host_async(moe_mxfp4_t* h, const void* x_host, int32_t T, void* y_host,
+                               void* stream) {
+  if (!h || T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x_host || !y_host) return MOE_ERR_INVALID_ARG;
+  if (!host_async_ready(h)) return MOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int k = (int)(h->host_seq & 1u);
+  const size_t bytes = (size_t)T * h->cfg.hidden * 2;
+  // slot k was last used two calls ago: its input is free once that call's
+  // layers ran, its output once that call's copy back finished
+  if (cudaStreamWaitEvent(h->h2d, h->ev_k[k], 0) != cudaSuccess ||
+      cudaMemcpyAsync(h->x_stage2[k], x_host, bytes, cudaMemcpyHostToDevice, h->h2d) != cudaSuccess ||
+      cudaEventRecord(h->ev_in[k], h->h2d) != cudaSuccess ||
+      cudaStreamWaitEvent(s, h->ev_in[k], 0) != cudaSuccess ||
+      cudaStreamWaitEvent(s, h->ev_out[k], 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int32_t st = moe_forward(h, h->x_stage2[k], T, h->y_stage2[k], nullptr, stream);
+  if (st != MOE_OK) return st;
+  if (cudaEventRecord(h->ev_k[k], s) != cudaSuccess ||
+      cudaStreamWaitEvent(h->d2h, h->ev_k[k], 0) != cudaSuccess ||
+      cudaMemcpyAsync(y_host, h->y_stage2[k], bytes, cudaMemcpyDeviceToHost, h->d2h) != cudaSuccess ||
+      cudaEventRecord(h->ev_out[k], h->d2h) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  ++h->host_seq;
+  return MOE_OK;
+}
+
+int32_t moe_host_join(moe_mxfp4_t* h, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (!h->h2d) return MOE_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int k = 0; k < 2; ++k)
+    if (cudaStreamWaitEvent(s, h->ev_out[k], 0) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
 }
 
 int32_t moe_phase_ns(moe_mxfp4_t* h, uint64_t* ns_out, int32_t max_n, void* stream) {
@@ -336,6 +406,10 @@ int32_t moe_engine_grid(const moe_mxfp4_t* h) { return h ? h->grid : 0; }
 
 void moe_mxfp4_destroy(moe_mxfp4_t* h) {
   if (!h) return;
+  if (h->h2d) {  // copies of moe_forward_host_async still in flight
+    cudaStreamSynchronize(h->h2d);
+    cudaStreamSynchronize(h->d2h);
+  }
   free_all(h);
   delete h;
 }

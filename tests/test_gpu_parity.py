@@ -251,3 +251,23 @@ def test_forward_captured_in_cuda_graph_matches_stream_launch(m):
     mo.moe_status()
     for y, r in zip(ys, ref):
         assert (bf16_host_bits(y) == r).all()
+
+
+def test_forward_host_async_matches_device(m):
+    """Pipelined host entry point: five calls over three token blocks (both
+    staging slots reused) give the device path's outputs bit for bit."""
+    import torch
+    from tests.gpu_helpers import bf16_dev, bf16_host_bits, make_moe
+    w = _workload("ragged_small")
+    lw = quantized_layer_np(w, seed=24)[1]
+    xbs = [quantized_layer_np(w, seed=25 + i)[0] for i in range(3)]
+    mo = make_moe(w, [lw])
+    ref = [bf16_host_bits(mo.moe_forward(bf16_dev(xb))) for xb in xbs]
+    xh = [torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory() for xb in xbs]
+    yh = [torch.empty((w.tokens, w.hidden), dtype=torch.bfloat16).pin_memory() for _ in range(5)]
+    for i in range(5):
+        mo.moe_forward_host_async(xh[i % 3], yh[i])
+    mo.moe_host_join()
+    mo.moe_status()
+    for i in range(5):
+        assert (bf16_host_bits(yh[i]) == ref[i % 3]).all(), i
