@@ -90,7 +90,7 @@ constexpr size_t OFF_DRAIN = OFF_XBAR + NPIPE * 2 * 8;              // [NPIPE]
 constexpr size_t OFF_TMEMBASE = OFF_DRAIN + NPIPE * 8;
 constexpr size_t OFF_JQ = align16(OFF_TMEMBASE + 8);                // [NPIPE][JQ]
 constexpr size_t OFF_XCH = align16(OFF_JQ + NPIPE * JQ * sizeof(JobEntry));  // [NPIPE][2][NT_MAX][4] floats
-constexpr size_t XCH_FLOATS = (NPIPE * 2 * NT_MAX > 2 * LT_MAX ? NPIPE * 2 * NT_MAX : 2 * LT_MAX) * 4;
+constexpr size_t XCH_FLOATS = (NPIPE * 2 * NT_MAX > 4 * LT_MAX ? NPIPE * 2 * NT_MAX : 4 * LT_MAX) * 4;
 constexpr size_t OFF_TABLES = align16(OFF_XCH + XCH_FLOATS * 4);
 constexpr size_t SMEM_BYTES = OFF_TABLES + sizeof(CtaTables);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -200,11 +200,12 @@ __device__ __forceinline__ float e2m1_value(uint32_t code) {
 // The NTERM E2M1 codes c_k of v = sum_k c_k 2^s_k (+ a residual below
 // 2^(s_0 - 21)); code k in bits 4k..4k+3.  Each step rounds the current
 // residual r to the nearest E2M1 multiple of 2^s_k and subtracts it exactly.
+template <int NT = NTERM>
 __device__ __forceinline__ uint32_t e2m1_terms(float v, int s0) {
   uint32_t w = 0;
   float r = v;
 #pragma unroll
-  for (int k = 0; k < NTERM; ++k) {
+  for (int k = 0; k < NT; ++k) {
     const int sk = term_exp(s0, k);
     const uint32_t c = f32x2_to_e2m1x2(0.f, r * pow2f(-sk)) & 0xFu;
     r = fmaf(-e2m1_value(c), pow2f(sk), r);
@@ -1000,41 +1001,47 @@ __device__ void phase_permute_large(const EngineParams& p, uint8_t* smem) {
 }
 
 // Large T*K: the x term images of every tile, gathered from the per-token
-// images (codes as they are, scale words into the tile's scale-factor blocks).
-// A warp moves GATHER_PER positions of one (tile, stage) per round, all loads
-// first.
-constexpr int GATHER_PER = 4;
+// images: the first LT_NTERM term rows of each position (row k of a token's
+// image becomes B row LT_NTERM * tl + k) and their scale words.  A warp moves
+// one (tile, stage): its 16-byte chunks (position, term, K chunk) and scale
+// words spread over the lanes, eight chunk loads of a lane in flight at once.
 __device__ void phase_tile_gather(const EngineParams& p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int ns = p.H / KS, nu = ld_cg_u32(p.n_units);
-  constexpr int NG = LT_MAX / GATHER_PER;
-  static_assert(LT_MAX % GATHER_PER == 0, "gather groups");
-  const int64_t ntask = (int64_t)nu * ns * NG;
-  for (int64_t task = (int64_t)blockIdx.x * WARPS + warp; task < ntask; task += (int64_t)gridDim.x * WARPS) {
-    const int g = (int)(task % NG);
-    const int64_t us = task / NG;  // tile * ns + stage
+  constexpr int CPP = LT_NTERM * 4;  // 16-byte chunks per position
+  const int64_t ntask = (int64_t)nu * ns;
+  for (int64_t us = (int64_t)blockIdx.x * WARPS + warp; us < ntask; us += (int64_t)gridDim.x * WARPS) {
     const int u = (int)(us / ns), st = (int)(us % ns);
     const int4 ur = __ldcg(reinterpret_cast<const int4*>(p.units) + u);
-    const int n = min(GATHER_PER, ur.z - g * GATHER_PER);
-    if (n <= 0) continue;
-    uint4 c[GATHER_PER];
-    uint32_t sfw[GATHER_PER];
+    const int n = ur.z;
+    static_assert(LT_MAX <= 64, "two token words per lane");
+    const int tok0 = lane < n ? __ldcg(p.tokpos + ur.y + lane) : 0;
+    const int tok1 = lane + 32 < n ? __ldcg(p.tokpos + ur.y + lane + 32) : 0;
+    const uint8_t* xs = p.xt + (int64_t)st * p.T * IMG_BYTES;
+    uint8_t* dst = p.xtl + us * LT_IMG_BYTES;
+    constexpr int B8 = 8;
+    for (int f0 = 0; f0 < n * CPP; f0 += 32 * B8) {
+      uint4 v[B8];
 #pragma unroll
-    for (int i = 0; i < GATHER_PER; ++i) {
-      if (i < n) {
-        const int tok = __ldcg(p.tokpos + ur.y + g * GATHER_PER + i);
-        const uint8_t* src = p.xt + ((int64_t)st * p.T + tok) * IMG_BYTES;
-        c[i] = __ldcg(reinterpret_cast<const uint4*>(src) + lane);
-        sfw[i] = __ldcg(reinterpret_cast<const uint32_t*>(src + IMG_CODE_BYTES + (lane & 7) * 16));
+      for (int i = 0; i < B8; ++i) {
+        const int f = f0 + 32 * i + lane, tl = f / CPP, r = f - tl * CPP, k = r >> 2, kch = r & 3;
+        const int ta = __shfl_sync(FULL, tok0, tl & 31), tb = __shfl_sync(FULL, tok1, tl & 31);
+        if (f < n * CPP)
+          v[i] = __ldcg(reinterpret_cast<const uint4*>(xs + (int64_t)(tl < 32 ? ta : tb) * IMG_BYTES + kch * 128 + k * 16));
+      }
+#pragma unroll
+      for (int i = 0; i < B8; ++i) {
+        const int f = f0 + 32 * i + lane, tl = f / CPP, r = f - tl * CPP, k = r >> 2, kch = r & 3;
+        if (f < n * CPP) *reinterpret_cast<uint4*>(dst + lt_row_offset(LT_NTERM * tl + k) + kch * 128) = v[i];
       }
     }
-    uint8_t* dst = p.xtl + us * LT_IMG_BYTES;
-#pragma unroll
-    for (int i = 0; i < GATHER_PER; ++i) {
-      if (i < n) {
-        const int tl = g * GATHER_PER + i;
-        reinterpret_cast<uint4*>(dst + lt_code_offset(tl))[lane] = c[i];
-        if (lane < NTERM) *reinterpret_cast<uint32_t*>(dst + lt_sf_offset(tl, lane, 0)) = sfw[i];
+    for (int f0 = 0; f0 < n * LT_NTERM; f0 += 32) {  // scale words: (position, term)
+      const int f = f0 + lane, tl = f / LT_NTERM, k = f - tl * LT_NTERM;
+      const int ta = __shfl_sync(FULL, tok0, tl & 31), tb = __shfl_sync(FULL, tok1, tl & 31);
+      if (f < n * LT_NTERM) {
+        const uint32_t w = __ldcg(reinterpret_cast<const uint32_t*>(xs + (int64_t)(tl < 32 ? ta : tb) * IMG_BYTES +
+                                                                   IMG_CODE_BYTES + k * 16));
+        *reinterpret_cast<uint32_t*>(dst + lt_sf_offset(f, 0)) = w;
       }
     }
   }
@@ -1203,7 +1210,7 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
   const int gub = p.I / GU_I_ROWS, db = p.H / JOB_ROWS;
   const int64_t n_gu = (int64_t)cx.n_units * gub, n_all = n_gu + (int64_t)cx.n_dunits * db;
   const int nc_gu = p.H / KS, nc_d = p.I / KS;
-  const uint32_t need = (uint32_t)gub * 4u;  // readiness signals per gate/up unit: 4 warps per job
+  const uint32_t need = (uint32_t)gub * (LT ? 8u : 4u);  // readiness signals per gate/up unit: epilogue warps per job
   bool xwait = !LT && !cx.global;  // x term images written during the routing (small T*K)
   // Units of at most NT_MAX positions read most expert weights once: the
   // weight stages go to L2 as evict-first, so that the routing's working set
@@ -1289,7 +1296,7 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
     const uint8_t* wbase = isD ? lp.w_d + ((int64_t)e * db + rb) * nc * STAGE_A_BYTES
                                : lp.w_gu + ((int64_t)e * gub + rb) * nc * STAGE_A_BYTES;
     const int tok = (!LT && !isD && lane < nt) ? ld_tab(cx.tokpos + pos0 + lane, cx.global) : 0;
-    const uint32_t bbytes = LT ? (uint32_t)(LT_SF_BYTES + nt * IMG_CODE_BYTES) : (uint32_t)nt * IMG_BYTES;
+    const uint32_t bbytes = LT ? (uint32_t)(LT_SF_BYTES + lt_cols(nt) * (IMG_CODE_BYTES / 8)) : (uint32_t)nt * IMG_BYTES;
     const uint32_t stage_bytes = STAGE_A_BYTES + bbytes;
     // Stages are issued in batches, one stage per lane: successive 1-D bulk
     // copies issued by one warp instruction each are serialised, while the
@@ -1566,7 +1573,7 @@ __device__ void stream_mma_lt(const EngineParams& p, uint8_t* smem, uint32_t tme
     t_acc += pclock(prof) - ta0;
     tc_fence_after();
     const uint32_t tacc = tmem + lt_acc(b);
-    const int n = nt * NTERM, nblk = (n + 127) / 128;
+    const int n = lt_cols(nt), nblk = (n + 127) / 128;
     const uint32_t idesc0 = mxf4_idesc(n, 0u), idesc1 = mxf4_idesc(n, 2u);
     for (int c = 0; c < nc; ++c) {
       const uint32_t s = (uint32_t)s0 + c;
@@ -1602,8 +1609,30 @@ __device__ void stream_mma_lt(const EngineParams& p, uint8_t* smem, uint32_t tme
 // Epilogue of the tile stream (warps 4..7, warp q reading tensor-memory lanes
 // 32q..32q+31): as stream_epilogue, over up to LT_MAX positions; the SwiGLU
 // term images are written into the tile images of the down jobs.
+// Sum of position j's LT_NTERM accumulator columns (this warp's 32 rows):
+// the eight columns from the aligned group holding the first, and the next
+// group when the terms cross into it; terms summed last to first.
+__device__ __forceinline__ float lt_position_sum(uint32_t tacc, int j) {
+  const int c0 = LT_NTERM * j, g0 = c0 & ~7;
+  float v[16];
+  tmem_ld8(tacc + g0, *reinterpret_cast<float(*)[8]>(v));
+  if (c0 + LT_NTERM > g0 + 8) tmem_ld8(tacc + g0 + 8, *reinterpret_cast<float(*)[8]>(v + 8));
+  float sum = 0.f;
+#pragma unroll
+  for (int k = LT_NTERM - 1; k >= 0; --k) {
+    float t = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i == c0 - g0 + k) t = v[i];
+    sum = k == LT_NTERM - 1 ? t : sum + t;
+  }
+  return sum;
+}
+// Eight epilogue warps in two sets (warps 4..7 and 8..11, each covering the
+// four accumulator lane quadrants); set `set` handles positions set, set + 2,
+// ..., with its own amax exchange buffers and barriers.
 __device__ void stream_epilogue_lt(const EngineParams& p, uint8_t* smem, const StreamCtx& cx, uint32_t tmem,
-                                   RoleState& rs) {
+                                   int set, RoleState& rs) {
   const int lane = threadIdx.x & 31, q = (threadIdx.x >> 5) & 3;
   JobEntry* jq = job_queue(smem, 0);
   uint32_t* ready = p.sync + SY_READY;
@@ -1636,13 +1665,9 @@ __device__ void stream_epilogue_lt(const EngineParams& p, uint8_t* smem, const S
     const uint32_t tacc = tmem + ((uint32_t)(32 * q) << 16) + lt_acc(b);
     if (!isD) {
       const int xb = (int)(gc & 1u);
-      float* xc = reinterpret_cast<float*>(smem + OFF_XCH) + xb * LT_MAX * 4;
-      for (int j = 0; j < nt; ++j) {
-        float v[NTERM];
-        tmem_ld8(tacc + j * NTERM, v);
-        float sum = v[NTERM - 1];
-#pragma unroll
-        for (int k = NTERM - 2; k >= 0; --k) sum += v[k];
+      float* xc = reinterpret_cast<float*>(smem + OFF_XCH) + (set * 2 + xb) * LT_MAX * 4;
+      for (int j = set; j < nt; j += 2) {
+        const float sum = lt_position_sum(tacc, j);
         const float other = __shfl_xor_sync(FULL, sum, 16);
         const float g = lane < 16 ? sum : other, up = lane < 16 ? other : sum;
         const float a = g / (1.0f + expf(-g)) * up;
@@ -1653,20 +1678,21 @@ __device__ void stream_epilogue_lt(const EngineParams& p, uint8_t* smem, const S
         if (lane == 0) xc[j * 4 + q] = am;
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(xch_bar(smem, 0, xb));
-      if (!wait_mbar(xch_bar(smem, 0, xb), (gc >> 1) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, wj)) {
+      if (lane == 0) mbar_arrive(xch_bar(smem, set, xb));
+      if (!wait_mbar(xch_bar(smem, set, xb), (gc >> 1) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, wj)) {
         ok = false;
         continue;
       }
       const int i0 = rb * GU_I_ROWS, sD = i0 / KS, kk = (i0 % KS) / 64, kc = q >> 1;
       uint8_t* img = p.atl + ((int64_t)u * nsd + sD) * LT_IMG_BYTES;
-      for (int j = 0; j < nt; ++j) {
+      for (int j = set; j < nt; j += 2) {
         const int s0 = term0_exp(fmaxf(xc[j * 4 + q], xc[j * 4 + (q ^ 1)]));
-        const uint32_t word = term_word<16>(e2m1_terms(av[j], s0), lane);
-        if (lane < 16)
-          *reinterpret_cast<uint32_t*>(img + lt_code_offset(j) + kk * 256 + kc * 128 + (lane >> 1) * 16 +
+        const uint32_t word = term_word<16>(e2m1_terms<LT_NTERM>(av[j], s0), lane);
+        if (lane < 2 * LT_NTERM)  // lane l: term l / 2, elements 8 (l % 2) .. + 7 of this warp's 16
+          *reinterpret_cast<uint32_t*>(img + lt_row_offset(LT_NTERM * j + (lane >> 1)) + kk * 256 + kc * 128 +
                                        (q & 1) * 8 + (lane & 1) * 4) = word;
-        if ((q & 1) == 0 && lane < NTERM) img[lt_sf_offset(j, lane, 2 * kk + kc)] = (uint8_t)(term_exp(s0, lane) + 127);
+        if ((q & 1) == 0 && lane < LT_NTERM)
+          img[lt_sf_offset(LT_NTERM * j + lane, 2 * kk + kc)] = (uint8_t)(term_exp(s0, lane) + 127);
       }
       __syncwarp();
       if (lane == 0) {
@@ -1676,12 +1702,8 @@ __device__ void stream_epilogue_lt(const EngineParams& p, uint8_t* smem, const S
       }
     } else {
       const int h0 = rb * JOB_ROWS;
-      for (int j = 0; j < nt; ++j) {
-        float v[NTERM];
-        tmem_ld8(tacc + j * NTERM, v);
-        float sum = v[NTERM - 1];
-#pragma unroll
-        for (int k = NTERM - 2; k >= 0; --k) sum += v[k];
+      for (int j = set; j < nt; j += 2) {
+        const float sum = lt_position_sum(tacc, j);
         p.ypair[(int64_t)(pos0 + j) * p.H + h0 + 32 * q + lane] = sum * ld_tab(cx.wpos + pos0 + j, cx.global);
       }
     }
@@ -2258,8 +2280,8 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
       } else if (warp == 1) {
         if (lane == 0) stream_mma_lt(p, smem, tmem, rs);
         __syncwarp();
-      } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
-        stream_epilogue_lt(p, smem, cx, tmem, rs);
+      } else if (warp >= EPI_WARP0) {
+        stream_epilogue_lt(p, smem, cx, tmem, warp >= EPI_WARP0 + 4 ? 1 : 0, rs);
       }
     } else {  // bf16 tiles: producer, MMA issuer, six converter warps, four epilogue warps
       if (warp == 0) {
@@ -2305,7 +2327,7 @@ __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p
       }
       for (int i = 0; i < NACC; ++i) {
         mbar_init(accf_bar(smem, pp, i), 1);
-        mbar_init(acce_bar(smem, pp, i), 4);
+        mbar_init(acce_bar(smem, pp, i), MODE == 1 && pp == 0 ? 8 : 4);  // tiles: eight epilogue warps
       }
       for (int i = 0; i < 2; ++i) mbar_init(xch_bar(smem, pp, i), 4);
       mbar_init(drain_bar(smem, pp), 1);

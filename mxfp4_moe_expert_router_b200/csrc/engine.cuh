@@ -66,32 +66,41 @@ constexpr int SMALL_PAIRS = 256;                         // T*K up to this: rout
 // ---- large T*K: tile stream --------------------------------------------------------------
 // With many tokens per expert (T*K >= LT_MIN_PER_EXPERT * E) a unit ("tile")
 // holds up to LT_MAX consecutive positions of one expert's segment and one MMA
-// covers all of them (N = 8 per position, up to 192).  Per (tile, 128-K stage)
-// the B operand is one image: LT_SF_BLOCKS blocks of 512 bytes in the
-// scale-factor copy layout (the scale of column n = 8 tl + k sits in block
-// n / 128, row n % 32, bytes 4 ((n / 32) % 4) + block index), then LT_MAX x 512
-// bytes of E2M1 term codes (position tl at LT_SF_BYTES + tl * 512, the layout
-// of a single image's codes).  One bulk copy of LT_SF_BYTES + nt * 512 bytes
-// brings a tile's B operand for a stage.
-constexpr int LT_MAX = 24;
+// covers all of them.  The tile stream carries LT_NTERM E2M1 terms of each
+// activation (the first LT_NTERM of the NTERM-term expansion; the residual is
+// below 2^-15 of the block maximum), so B row n = LT_NTERM * tl + k holds term
+// k of position tl, and N = lt_cols(nt) (rounded up to 8, at most 192).  Per
+// (tile, 128-K stage) the B operand is one image: LT_SF_BLOCKS blocks of 512
+// bytes in the scale-factor copy layout (the scale of row n sits in block
+// n / 128, row n % 32, bytes 4 ((n / 32) % 4) + block index: lt_sf_offset),
+// then the codes in 8-row groups of 512 bytes, row n at
+// lt_row_offset(n) + 256 kk + 128 kc for its four 16-byte chunks.  One bulk
+// copy of LT_SF_BYTES + lt_cols(nt) * 64 bytes brings a tile's B operand.
+constexpr int LT_NTERM = 5;
+constexpr int LT_MAX = 38;
 constexpr int LT_MIN_PER_EXPERT = 8;                     // T*K / E from which tiles are used
 constexpr int LT_SF_BLOCKS = 2;                          // 32-row copies covering N <= 256
 constexpr int LT_SF_BYTES = LT_SF_BLOCKS * 512;
-constexpr int LT_CODE_BYTES = LT_MAX * IMG_CODE_BYTES;   // 12288
+constexpr int LT_ACC_COLS = 192;                         // accumulator columns (B rows) at most
+constexpr int LT_CODE_BYTES = LT_ACC_COLS / 8 * IMG_CODE_BYTES;  // 12288
 constexpr int LT_IMG_BYTES = LT_SF_BYTES + LT_CODE_BYTES;  // 13312
 constexpr int LT_SLOT_BYTES = STAGE_A_BYTES + LT_IMG_BYTES;       // 22016
 constexpr int LT_NSLOT = 9;                              // one pipeline
-constexpr int LT_ACC_COLS = LT_MAX * NTERM;              // 192
 constexpr int LT_NACC = 2;
 constexpr int LT_SF_COLS = 4 + 4 * LT_SF_BLOCKS;         // 12
+static_assert(((LT_NTERM * LT_MAX + 7) & ~7) <= LT_ACC_COLS, "tile columns");
+static_assert(LT_NTERM <= NTERM, "tile terms are a prefix of the expansion");
 static_assert(LT_NACC * LT_ACC_COLS + NSF * LT_SF_COLS <= TMEM_COLS, "tensor memory budget (tiles)");
 static_assert(LT_NSLOT <= NPIPE * NSLOT, "tile ring barriers");
-static_assert(8 * LT_MAX <= 128 * LT_SF_BLOCKS, "tile scale-factor blocks");
-// Byte offset in a tile image of the scale of position tl, term k, block kb.
-__host__ __device__ constexpr int lt_sf_offset(int tl, int k, int kb) {
-  return (tl / 16) * 512 + (8 * (tl % 4) + k) * 16 + 4 * ((tl % 16) / 4) + kb;
+static_assert(LT_ACC_COLS <= 128 * LT_SF_BLOCKS, "tile scale-factor blocks");
+// B rows (= accumulator columns) of a tile of nt positions.
+__host__ __device__ constexpr int lt_cols(int nt) { return (LT_NTERM * nt + 7) & ~7; }
+// Byte offset in a tile image of B row n's first 16-byte chunk.
+__host__ __device__ constexpr int lt_row_offset(int n) { return LT_SF_BYTES + (n / 8) * IMG_CODE_BYTES + (n % 8) * 16; }
+// Byte offset in a tile image of the scale of B row n, 32-element block kb.
+__host__ __device__ constexpr int lt_sf_offset(int n, int kb) {
+  return (n / 128) * 512 + (n % 32) * 16 + 4 * ((n / 32) % 4) + kb;
 }
-__host__ __device__ constexpr int lt_code_offset(int tl) { return LT_SF_BYTES + tl * IMG_CODE_BYTES; }
 // ---- large T*K: bf16 tile stream (kind::f16 on dequantised weights) ----------------------
 // The same tile jobs, with x in bf16 as the B operand (one term, exact) and
 // the MXFP4 weights dequantised to bf16 in shared memory by converter warps.
