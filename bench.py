@@ -51,7 +51,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="decode_t9_h4096_e128", choices=sorted(synth.WORKLOADS))
-    ap.add_argument("--tokens", type=int, default=None, help="override T (sweep workload)")
+    ap.add_argument("--tokens", type=int, default=None, help="override T (default: the workload's own; 9 for the sweep)")
     ap.add_argument("--batches", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -277,8 +277,12 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     w = synth.WORKLOADS[args.workload]
-    T = args.tokens or (9 if args.workload.startswith("sweep") else w.tokens)
-    w = w.with_tokens(max(T, w.tokens)) if args.workload.startswith("sweep") else w
+    sweep = args.workload.startswith("sweep")
+    T = args.tokens or (9 if sweep else w.tokens)
+    if sweep:
+        w = w.with_tokens(max(T, w.tokens))
+    elif args.tokens:  # another token count on this workload's shapes
+        w = w.with_tokens(T)
 
     if args.impl == "reference":
         return run_reference(args, w, T, rank, world)
@@ -418,7 +422,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "mxfp4-w/fp32-acc",
             "data": "synthetic (seeded N(0,0.02) expert weights quantised to MXFP4, N(0,1) bf16 tokens)",
-            "config": {"workload": w.name if not args.workload.startswith("sweep") else f"{w.name}_t{T}",
+            "config": {"workload": w.name if not (sweep or args.tokens) else f"{w.name}_t{T}",
                        "hidden": w.hidden, "inter": w.inter, "experts": w.experts, "top_k": w.top_k,
                        "tokens_per_gpu": T, "layers": w.layers, "token_blocks": len(xs),
                        "mean_experts_hit": mean_hit,
