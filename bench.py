@@ -14,6 +14,10 @@ rotation), and the ~0.5 GB of expert weights one step streams exceeds the
 126 MB L2, so no L2 flush is inserted between steps.  The K timed calls are
 captured once into a CUDA graph and replayed (``--no-graph``: K stream
 launches); either way every step is a full engine launch on its own inputs.
+At verify-block sizes the line also carries ``ops_baseline``: the same calls as
+six launches per layer (``moe_forward_ops``: stream launches, a CUDA graph,
+and a CUDA graph of programmatic dependent launches) next to the engine's own
+launch, in µs per step.
 
 Under torchrun each rank runs the same layer on its own token blocks (independent
 verify steps: weak scaling, no collective on the data path); the timed region is
@@ -60,6 +64,8 @@ def parse_args():
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of replaying them as one CUDA graph")
     ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-ops-baseline", action="store_true",
+                    help="skip timing the operator-by-operator launches (moe_forward_ops)")
     return ap.parse_args()
 
 
@@ -101,6 +107,64 @@ def upload_graph(graph, stream):
     if rc != 0:
         raise RuntimeError(f"cuGraphUpload failed: {rc}")
     torch.cuda.synchronize()
+
+
+def time_calls(mx, stream, n: int, launch, use_graph: bool) -> float:
+    """Device time per call (us) of n calls launch(i, stream_handle): stream
+    launches, or the n calls captured into one CUDA graph and replayed."""
+    import torch
+    graph = None
+    if use_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            cap = mx._stream()
+            for i in range(n):
+                launch(i, cap)
+        upload_graph(graph, stream)
+    sp = mx._stream(stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    if graph is not None:
+        graph.replay()
+    else:
+        for i in range(n):
+            launch(i, sp)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    del graph
+    return e0.elapsed_time(e1) * 1e3 / n
+
+
+def ops_baseline(mx, m, stream, xptr, yptr, T: int, steps: int) -> dict:
+    """The same layer(s) as six launches per layer (moe_forward_ops) against the
+    single engine launch, each as stream launches and as a CUDA graph; the ops
+    also as a graph of programmatic dependent launches."""
+    def ops(flags):
+        def launch(i, sp):
+            st = mx.lib.moe_forward_ops(m.handle, xptr[i % len(xptr)], T, yptr, None, flags, sp)
+            if st != 0:
+                raise mx.MoeError(st, "moe_forward_ops")
+        return launch
+
+    def engine(i, sp):
+        st = mx.lib.moe_forward(m.handle, xptr[i % len(xptr)], T, yptr, None, sp)
+        if st != 0:
+            raise mx.MoeError(st, "moe_forward")
+
+    for i in range(3):
+        ops(mx.MOE_OPS_PDL)(i, mx._stream(stream))
+        ops(0)(i, mx._stream(stream))
+    m.moe_status()
+    res = {"engine_stream": time_calls(mx, stream, steps, engine, False),
+           "engine_graph": time_calls(mx, stream, steps, engine, True),
+           "ops_stream": time_calls(mx, stream, steps, ops(0), False),
+           "ops_graph": time_calls(mx, stream, steps, ops(0), True),
+           "ops_graph_pdl": time_calls(mx, stream, steps, ops(mx.MOE_OPS_PDL), True)}
+    m.moe_status()
+    return {"us_per_step": {k: round(v, 2) for k, v in res.items()},
+            "launches_per_step": {"engine": 1, "ops": 6 * m.cfg.num_layers}, "steps": steps,
+            "ops": "router partial logits; routing (1 CTA); x term images; gate/up + SwiGLU; down; combine"}
 
 
 def measured_peaks():
@@ -368,6 +432,11 @@ def main():
     achieved = alg_bytes / (ms_step * 1e-3) / 1e9
     traffic = profile_traffic()
 
+    # the pages' baseline execution model: one launch per operator
+    ops = None
+    if world == 1 and not args.no_ops_baseline and T * w.top_k <= 256:
+        ops = ops_baseline(mx, m, stream, xptr, yptr, T, max(1, min(args.steps, 500)))
+
     # end-to-end: the same metric through the public host-buffer entry point
     e2e = None
     if not args.no_e2e:
@@ -443,6 +512,7 @@ def main():
                                    zip(("router_logits", "x_images", "route_wait", "topk_or_tables", "permute", "stream",
                                        "combine"), phases[:7])},
             "e2e": e2e,
+            "ops_baseline": ops,
             "cpu_baseline": cpu,
             "clocks": clk,
         }

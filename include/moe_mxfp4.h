@@ -179,6 +179,29 @@ MOE_API int32_t moe_forward_host_async(moe_mxfp4_t* h, const void* x_host, int32
 MOE_API int32_t moe_host_join(moe_mxfp4_t* h, void* stream);
 
 /*
+ * moe_forward_ops -- the layers of moe_forward, operator by operator: per
+ * layer six launches on `stream` (router partial logits; routing by one CTA;
+ * x term images; gate/up + SwiGLU jobs; down jobs; combine, + RMSNorm between
+ * layers), each one CTA per SM except the routing (one CTA) and an RMSNorm
+ * combine (one CTA per token).  The results are bit-identical to moe_forward.
+ * It is the baseline the single persistent launch is measured against: the
+ * execution-model passages (TileRT blog "Breaking 1000 TPS", section on the
+ * execution model; HyperAI salon transcript "Speed is Intelligence", section
+ * on CUDA Graph and PDL) set a resident engine against operator-by-operator
+ * launches with CUDA graphs and programmatic dependent launch.
+ * flags: MOE_OPS_PDL launches every kernel as a programmatic dependent of its
+ * predecessor (it is scheduled while the predecessor drains, then waits for
+ * it before touching any data).  Arguments, layout and capture safety as for
+ * moe_forward.  Only T*K <= 256 (the verify-block sizes);
+ * larger calls return MOE_ERR_UNSUPPORTED_SHAPE.  Errors: MOE_ERR_INVALID_ARG,
+ * MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_CUDA; device-side timeouts are reported
+ * by the next moe_status.
+ */
+#define MOE_OPS_PDL 1
+MOE_API int32_t moe_forward_ops(moe_mxfp4_t* h, const void* x_bf16, int32_t T, void* y_bf16,
+                                void* layer_io_bf16, int32_t flags, void* stream);
+
+/*
  * moe_status -- synchronise `stream`, then return and clear the device-side
  * status of the handle: MOE_OK, or MOE_ERR_TIMEOUT if a bounded wait inside
  * the engine expired (the handle's wait state is reset, so it stays usable).
@@ -215,7 +238,7 @@ MOE_API int32_t moe_stream_profile(moe_mxfp4_t* h, int32_t enable, uint64_t* out
 /*
  * moe_set_large_kind -- the weight stream used when a call has many positions
  * per expert (T*K > 256 and T*K >= 8*E): 1 = E2M1 term tiles on the block-
- * scaled fp4 tensor-core MMA (x and the SwiGLU output expanded into eight
+ * scaled fp4 tensor-core MMA (x and the SwiGLU output expanded into five
  * E2M1 terms), 2 = bf16 tiles on the bf16 tensor-core MMA (MXFP4 weights
  * dequantised to bf16 in shared memory, x exact, the SwiGLU output as two
  * bf16 terms).  Default 1 (the faster of the two on B200 at every measured

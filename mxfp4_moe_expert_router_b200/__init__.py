@@ -20,7 +20,10 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_OOM, MOE_ERR_CUD
 EXPORTS = ("mxfp4_quantize", "moe_mxfp4_create", "moe_route", "moe_forward", "moe_forward_host",
            "moe_status", "moe_set_timeout_ns", "moe_engine_grid", "moe_mxfp4_destroy",
            "moe_status_str", "moe_route_static", "moe_phase_ns",
-           "moe_stream_profile", "moe_set_large_kind", "moe_forward_host_async", "moe_host_join")
+           "moe_stream_profile", "moe_set_large_kind", "moe_forward_host_async", "moe_host_join",
+           "moe_forward_ops")
+
+MOE_OPS_PDL = 1
 
 
 class MoeConfig(ctypes.Structure):
@@ -51,6 +54,7 @@ def _load():
         "moe_route": (i32, [vp, i32, vp, i32, vp, vp, vp, vp, vp, vp, vp]),
         "moe_forward": (i32, [vp, vp, i32, vp, vp, vp]),
         "moe_forward_host": (i32, [vp, vp, i32, vp, vp]),
+        "moe_forward_ops": (i32, [vp, vp, i32, vp, vp, i32, vp]),
         "moe_forward_host_async": (i32, [vp, vp, i32, vp, vp]),
         "moe_host_join": (i32, [vp, vp]),
         "moe_status": (i32, [vp, vp]),
@@ -165,6 +169,17 @@ class Moe:
                "moe_forward")
         return y
 
+    def moe_forward_ops(self, x, y=None, layer_io=None, pdl=True, stream=None):
+        """moe_forward as six launches per layer (one per operator); pdl: programmatic
+        dependent launches."""
+        import torch
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty((T, self.cfg.hidden), dtype=torch.bfloat16, device=x.device)
+        _check(lib.moe_forward_ops(self.handle, _ptr(x), T, _ptr(y), _ptr(layer_io),
+                                   MOE_OPS_PDL if pdl else 0, _stream(stream)), "moe_forward_ops")
+        return y
+
     def moe_forward_host(self, x_host, y_host=None, stream=None):
         import torch
         T = x_host.shape[0]
@@ -188,8 +203,9 @@ class Moe:
         _check(lib.moe_status(self.handle, _stream(stream)), "moe_status")
 
     def moe_phase_ns(self, stream=None):
-        """Durations (ns) of the last forward's phases, 7 per layer: x conversion and
-        router logits (CTA 0), grid wait, top-k, permute, stream, combine."""
+        """Durations (ns) of the last forward's phases as CTA 0 saw them, 7 per layer:
+        router logits, x term images, routing wait, top-k or table copy, permutation,
+        weight stream, combine."""
         n = self.cfg.num_layers * 7
         arr = (ctypes.c_uint64 * n)()
         _check(lib.moe_phase_ns(self.handle, arr, n, _stream(stream)), "moe_phase_ns")

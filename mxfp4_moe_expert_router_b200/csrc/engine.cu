@@ -1199,7 +1199,9 @@ __device__ bool wait_entry(const EngineParams& p, JobEntry* en, int32_t qk) {
 // term images are complete.  A stage is the job's weight stage plus one term
 // image per token (gate/up, from xt) or the unit's consecutive pair images
 // (down, from aimg).
-template <bool LT>
+// SPLIT (operator-by-operator launches only): 1 runs the gate/up jobs alone, 2
+// the down jobs alone (their gate/up units are then complete).
+template <bool LT, int SPLIT = 0>
 __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem,
                                 const StreamCtx& cx, int pipe, RoleState& rs) {
   constexpr int NS = LT ? LT_NSLOT : NSLOT;  // ring slots
@@ -1208,7 +1210,9 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
   JobEntry* jq = job_queue(smem, pipe);
   uint32_t* ready = p.sync + SY_READY;
   const int gub = p.I / GU_I_ROWS, db = p.H / JOB_ROWS;
-  const int64_t n_gu = (int64_t)cx.n_units * gub, n_all = n_gu + (int64_t)cx.n_dunits * db;
+  const int64_t n_gu = (int64_t)cx.n_units * gub;
+  const int64_t n_all = SPLIT == 1 ? n_gu : n_gu + (int64_t)cx.n_dunits * db;
+  const int64_t j0 = SPLIT == 2 ? n_gu : 0;  // first job of this launch
   const int nc_gu = p.H / KS, nc_d = p.I / KS;
   const uint32_t need = (uint32_t)gub * (LT ? 8u : 4u);  // readiness signals per gate/up unit: epilogue warps per job
   bool xwait = !LT && !cx.global;  // x term images written during the routing (small T*K)
@@ -1224,8 +1228,8 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
   fence_proxy_async_global();
   // the first job of every pipeline is static (no atomic round trip at the
   // start of the stream); later jobs come from the global counter
-  const int64_t jbase = (int64_t)NP * gridDim.x;
-  long long next = (int64_t)blockIdx.x + (int64_t)pipe * gridDim.x;
+  const int64_t jbase = j0 + (int64_t)NP * gridDim.x;
+  long long next = j0 + (int64_t)blockIdx.x + (int64_t)pipe * gridDim.x;
   for (;;) {
     const int64_t j = __shfl_sync(FULL, next, 0);
     if (j >= n_all || !ok) {
@@ -1238,7 +1242,7 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
       ++rs.qk;
       break;
     }
-    if (lane == 0) next = jbase + atomicAdd(p.sync + SY_JOBS, 1u);  // prefetch the following job
+    if (lane == 0) next = jbase + atomicAdd(p.sync + (SPLIT == 2 ? SY_JOBS2 : SY_JOBS), 1u);  // prefetch the following job
     const bool isD = j >= n_gu;
     const int64_t jj = isD ? j - n_gu : j;
     const int per = isD ? db : gub;
@@ -2310,8 +2314,56 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
   }
 }
 
-// Three instances (MODE 0, 1, 2, see run_layers); each holds only its own
-// stream code.
+// One operator of one layer per launch (MODE 3): the same phases as the
+// engine's small-T*K layer, with a kernel boundary instead of each grid-wide
+// wait.  The tables come from global memory; the down jobs start only after
+// every gate/up job has finished (their own launch).  Under programmatic
+// dependent launch a grid waits for its predecessor before it touches
+// anything, and lets its successor be scheduled right after that.
+template <int SPLIT>
+__device__ void op_stream(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem, uint32_t tmem,
+                          RoleState& rs) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const StreamCtx cx{p.units, p.dunits, p.tokpos, p.wpos, (int)ld_cg_u32(p.n_units),
+                     (int)ld_cg_u32(p.n_units + 1), true};
+  if (warp < EPI_WARP0) {
+    const int pipe = warp >> 1;
+    if ((warp & 1) == 0) {
+      stream_producer<false, SPLIT>(p, lp, smem, cx, pipe, rs);
+    } else {
+      if (lane == 0) stream_mma(p, smem, tmem, pipe, rs);
+      __syncwarp();
+    }
+  } else {
+    stream_epilogue(p, smem, cx, tmem, (warp - EPI_WARP0) / 4, rs);
+  }
+}
+
+__device__ void run_op(const EngineParams& p, uint8_t* smem, uint32_t tmem, RoleState& rs) {
+  const int layer = p.op_layer;
+  const LayerPtrs& lp = p.layers[layer];
+  const __nv_bfloat16* x = layer == 0 ? p.x_in : p.xnext;
+  grid_dependency_wait();
+  grid_launch_dependents();
+  switch (p.op) {
+    case OP_ROUTER: phase_router(p, lp, x, smem); break;
+    case OP_ROUTE:
+      if (threadIdx.x == 0) p.sync[SY_JOBS2] = 0u;
+      phase_route_small(p, lp, smem);
+      break;
+    case OP_IMAGES: phase_images(p, x, layer); break;
+    case OP_GATEUP: op_stream<1>(p, lp, smem, tmem, rs); break;
+    case OP_DOWN: op_stream<2>(p, lp, smem, tmem, rs); break;
+    case OP_COMBINE:
+      if (layer + 1 < p.L) phase_combine_rmsnorm(p, p.inv, smem);
+      else phase_combine_out(p, p.inv);
+      break;
+    default: break;
+  }
+}
+
+// Four instances: MODE 0, 1, 2 (see run_layers), each holding only its own
+// stream code, and MODE 3, one operator per launch (run_op).
 template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -2335,7 +2387,7 @@ __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p
     fence_mbar_init();
   }
   for (int i = threadIdx.x; i < NPIPE * JQ; i += THREADS) job_queue(smem, 0)[i].flag = 0;
-  const bool use_tmem = !p.route_only;
+  const bool use_tmem = !p.route_only && (MODE != 3 || p.op == OP_GATEUP || p.op == OP_DOWN);
   if (use_tmem && warp == 1) {
     tmem_alloc(tmem_base_word(smem), TMEM_COLS);
     tmem_relinquish();
@@ -2344,10 +2396,11 @@ __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = use_tmem ? *tmem_base_word(smem) : 0u;
-  const bool stamp = p.stamps != nullptr && blockIdx.x == 0 && threadIdx.x == 0;
+  const bool stamp = MODE != 3 && p.stamps != nullptr && blockIdx.x == 0 && threadIdx.x == 0;
   if (stamp) p.stamps[0] = globaltimer_ns();
   RoleState rs;
-  run_layers<MODE>(p, smem, tmem, rs, stamp);
+  if constexpr (MODE == 3) run_op(p, smem, tmem, rs);
+  else run_layers<MODE>(p, smem, tmem, rs, stamp);
   if (use_tmem) {
     // free tensor memory only once every MMA this CTA issued has completed
     if (warp < EPI_WARP0 && (warp & 1) && lane == 0) {
@@ -2372,7 +2425,8 @@ size_t engine_smem_bytes() { return SMEM_BYTES; }
 
 int engine_max_grid(int device, int* err) {
   int per_sm = ~0u >> 1, sms = 0;
-  for (const void* k : {(const void*)engine_kernel<0>, (const void*)engine_kernel<1>, (const void*)engine_kernel<2>}) {
+  for (const void* k : {(const void*)engine_kernel<0>, (const void*)engine_kernel<1>, (const void*)engine_kernel<2>,
+                        (const void*)engine_kernel<3>}) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) { *err = (int)e; return 0; }
     int n = 0;
@@ -2392,6 +2446,31 @@ cudaError_t engine_launch(const EngineParams& p, int grid, cudaStream_t s) {
                   : p.large == LARGE_F16                  ? (const void*)engine_kernel<2>
                                                           : (const void*)engine_kernel<1>;
   return cudaLaunchCooperativeKernel(k, dim3(grid), dim3(THREADS), args, SMEM_BYTES, s);
+}
+
+cudaError_t engine_launch_ops(const EngineParams& p0, int grid, bool pdl, cudaStream_t s) {
+  EngineParams p = p0;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = s;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  for (int l = 0; l < p0.L; ++l) {
+    for (int op = OP_ROUTER; op <= OP_COUNT; ++op) {
+      p.op = op;
+      p.op_layer = l;
+      // routing is one CTA's work; an RMSNorm combine takes one CTA per token
+      const int g = op == OP_ROUTE ? 1 : (op == OP_COMBINE && l + 1 < p0.L ? (p0.T < grid ? p0.T : grid) : grid);
+      cfg.gridDim = dim3(g);
+      const cudaError_t e = cudaLaunchKernelEx(&cfg, engine_kernel<3>, p);
+      if (e != cudaSuccess) return e;
+    }
+  }
+  return cudaSuccess;
 }
 
 }  // namespace moe

@@ -146,6 +146,7 @@ constexpr int STAMPS_PER_LAYER = 7;  // router, x images, routing wait, top-k / 
 enum : int {
   SY_BAR_COUNT = 0, SY_BAR_GEN = 1, SY_JOBS = 2, SY_ERROR = 3, SY_ERRINFO = 4,
   SY_XDONE = 5,  // CTAs whose x term images of this layer are written (small T*K)
+  SY_JOBS2 = 6,  // down-job counter of the operator-by-operator launches
   SY_READY = 8,  // ready[unit] from here
 };
 // device-side error codes (status word)
@@ -205,7 +206,14 @@ struct EngineParams {
   uint32_t* sync;             // see SY_*
   uint64_t* stamps;           // null or [1 + MAX_LAYERS * STAMPS_PER_LAYER] %globaltimer ns (CTA 0)
   unsigned long long* prof;   // null or [PROF_COUNTERS] summed SM-clock cycles (stream phase)
+  int op;                     // operator-by-operator launches: the OP_* this launch runs (0: whole engine)
+  int op_layer;               // ... and its layer
 };
+
+// The operators of one layer when every step is its own launch (small T*K):
+// router partial logits, routing (one CTA), x term images, gate/up jobs, down
+// jobs, combine.
+enum : int { OP_ROUTER = 1, OP_ROUTE, OP_IMAGES, OP_GATEUP, OP_DOWN, OP_COMBINE, OP_COUNT = OP_COMBINE };
 
 // stream-phase profile counters (SM-clock cycles summed over CTAs; the
 // epilogue ones also over its 8 warps)
@@ -217,6 +225,9 @@ enum : int {
 
 size_t engine_smem_bytes();
 cudaError_t engine_launch(const EngineParams& p, int grid, cudaStream_t s);
+// The same layer(s) as OP_COUNT launches per layer; pdl: each launch may start
+// while its predecessor drains (programmatic dependent launch).
+cudaError_t engine_launch_ops(const EngineParams& p, int grid, bool pdl, cudaStream_t s);
 int engine_max_grid(int device, int* err);
 
 cudaError_t quantize_launch(const void* w, int64_t rows, int64_t K, uint8_t* codes,

@@ -297,6 +297,28 @@ int32_t moe_forward(moe_mxfp4_t* h, const void* x_bf16, int32_t T, void* y_bf16,
                                                                                      : MOE_ERR_CUDA;
 }
 
+int32_t moe_forward_ops(moe_mxfp4_t* h, const void* x_bf16, int32_t T, void* y_bf16,
+                        void* layer_io_bf16, int32_t flags, void* stream) {
+  if (!h || T < 0 || T > h->cfg.max_tokens || (flags & ~MOE_OPS_PDL)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x_bf16 || !y_bf16 || !aligned16(x_bf16) || !aligned16(y_bf16) ||
+      (layer_io_bf16 && !aligned16(layer_io_bf16)))
+    return MOE_ERR_INVALID_ARG;
+  if ((int64_t)T * h->cfg.top_k > SMALL_PAIRS) return MOE_ERR_UNSUPPORTED_SHAPE;
+  const size_t bytes = (size_t)T * h->cfg.hidden * 2;
+  const char* xa = static_cast<const char*>(x_bf16);
+  const char* ya = static_cast<const char*>(y_bf16);
+  if (xa < ya + bytes && ya < xa + bytes) return MOE_ERR_INVALID_ARG;
+  EngineParams p = base_params(h, T);
+  p.stamps = nullptr;
+  p.x_in = static_cast<const __nv_bfloat16*>(x_bf16);
+  p.y_out = static_cast<__nv_bfloat16*>(y_bf16);
+  p.layer_io = static_cast<__nv_bfloat16*>(layer_io_bf16);
+  return engine_launch_ops(p, h->grid, (flags & MOE_OPS_PDL) != 0, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
 int32_t moe_set_large_kind(moe_mxfp4_t* h, int32_t kind) {
   if (!h || (kind != LARGE_MXF4 && kind != LARGE_F16)) return MOE_ERR_INVALID_ARG;
   h->large = kind;

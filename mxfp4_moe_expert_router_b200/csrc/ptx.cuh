@@ -112,6 +112,17 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---- programmatic dependent launch ----------------------------------------------
+// Wait until the grid this launch depends on has completed and its memory
+// operations are visible (returns at once for a launch without that dependency).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Allow the dependent launch to be scheduled before this grid completes.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- acquire / release on global words -----------------------------------------
 // Atomic add at gpu scope with acquire and release semantics: earlier memory
 // operations of this thread are visible before it, later ones are ordered
