@@ -21,7 +21,8 @@ EXPORTS = ("mxfp4_quantize", "moe_mxfp4_create", "moe_route", "moe_forward", "mo
            "moe_status", "moe_set_timeout_ns", "moe_engine_grid", "moe_mxfp4_destroy",
            "moe_status_str", "moe_route_static", "moe_phase_ns",
            "moe_stream_profile", "moe_set_large_kind", "moe_forward_host_async", "moe_host_join",
-           "moe_forward_ops")
+           "moe_forward_ops", "spec_verify_workspace_bytes", "spec_verify", "spec_verify_status",
+           "spec_exp")
 
 MOE_OPS_PDL = 1
 
@@ -66,6 +67,10 @@ def _load():
         "moe_stream_profile": (i32, [vp, i32, ctypes.POINTER(ctypes.c_uint64), i32, vp]),
         "moe_phase_ns": (i32, [vp, ctypes.POINTER(ctypes.c_uint64), i32, vp]),
         "moe_route_static": (i32, [vp, i32, i32, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, vp]),
+        "spec_verify_workspace_bytes": (i64, [i32, i32, i32]),
+        "spec_verify": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, i64, vp]),
+        "spec_verify_status": (i32, [vp, vp]),
+        "spec_exp": (i32, [vp, vp, i64, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -276,3 +281,47 @@ def moe_route_static(x, router_w, router_b, top_k, stream=None):
 def moe_mxfp4_create(hidden, inter, num_experts, top_k, max_tokens, layers, rms_eps=1e-6,
                      stream=None) -> Moe:
     return Moe(hidden, inter, num_experts, top_k, max_tokens, layers, rms_eps, stream)
+
+
+class SpecVerify:
+    """The speculative-verify acceptance step (``spec_verify`` in include/spec_verify.h)
+    for up to ``max_blocks`` verify blocks of ``gamma`` drafts over ``vocab`` tokens.
+    Owns the zero-filled device workspace."""
+
+    def __init__(self, max_blocks: int, gamma: int, vocab: int, device="cuda"):
+        import torch
+        self.max_blocks, self.gamma, self.vocab = max_blocks, gamma, vocab
+        nbytes = lib.spec_verify_workspace_bytes(max_blocks, gamma, vocab)
+        if nbytes < 0:
+            raise MoeError(MOE_ERR_INVALID_ARG, "spec_verify_workspace_bytes")
+        self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+    def __call__(self, target_logits, draft_logits, draft_tokens, r_accept, u_sample, n_out=None,
+                 tokens_out=None, stream=None):
+        """target_logits fp32 [B][G+1][V], draft_logits fp32 [B][G][V], draft_tokens
+        int32 [B][G], r_accept fp64 [B][G], u_sample fp64 [B] (CUDA) ->
+        (n_accepted int32 [B], tokens int32 [B][G+1])."""
+        import torch
+        B = target_logits.shape[0]
+        if B > self.max_blocks:
+            raise MoeError(MOE_ERR_INVALID_ARG, "spec_verify (more blocks than the workspace holds)")
+        dev = target_logits.device
+        if n_out is None:
+            n_out = torch.empty((B,), dtype=torch.int32, device=dev)
+        if tokens_out is None:
+            tokens_out = torch.empty((B, self.gamma + 1), dtype=torch.int32, device=dev)
+        _check(lib.spec_verify(_ptr(target_logits), _ptr(draft_logits), _ptr(draft_tokens), _ptr(r_accept),
+                               _ptr(u_sample), B, self.gamma, self.vocab, _ptr(n_out), _ptr(tokens_out),
+                               _ptr(self.workspace), self.workspace.numel(), _stream(stream)), "spec_verify")
+        return n_out, tokens_out
+
+    def status(self, stream=None):
+        _check(lib.spec_verify_status(_ptr(self.workspace), _stream(stream)), "spec_verify_status")
+
+
+def spec_exp(x, stream=None):
+    """The verify step's fp64 exp on a CUDA fp64 tensor (for accuracy tests)."""
+    import torch
+    y = torch.empty_like(x)
+    _check(lib.spec_exp(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "spec_exp")
+    return y

@@ -6,7 +6,7 @@
 
 nvcc cross-compiles without a GPU.  The library links the CUDA runtime
 statically and exports only the ``extern "C"`` entry points of
-``include/moe_mxfp4.h``.
+``include/moe_mxfp4.h`` and ``include/spec_verify.h``.
 """
 from __future__ import annotations
 
@@ -19,7 +19,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmoe_mxfp4.so")
-SOURCES = ["quantize.cu", "engine.cu", "moe_mxfp4.cu", "noalloc.cu"]
+SOURCES = ["quantize.cu", "engine.cu", "moe_mxfp4.cu", "noalloc.cu", "spec_verify.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -44,8 +44,9 @@ def up_to_date() -> bool:
     if not os.path.exists(LIB):
         return False
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(ROOT, "include", "moe_mxfp4.h"),
-                                                                os.path.abspath(__file__)]
+    inc = os.path.join(ROOT, "include")
+    deps = ([os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(inc, f) for f in os.listdir(inc)]
+            + [os.path.abspath(__file__)])
     return all(os.path.getmtime(d) <= t for d in deps if os.path.exists(d))
 
 

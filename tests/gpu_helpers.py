@@ -72,3 +72,30 @@ def check_forward(y_dev, x, lw, k, idx_gpu=None):
     ok, ratio = tolerance_ok(got, ref)
     assert ok, f"worst |err|/bound = {ratio:.3f}"
     return ratio
+
+
+def check_verify(inp, n_gpu, tok_gpu):
+    """spec_verify outputs against the oracle, block by block; returns the number of
+    unpinned blocks (a decision or draw within the oracle's rounding bound)."""
+    from oracle import spec
+    lt, ld, d, r, u = inp["lt"], inp["ld"], inp["d"], inp["r"], inp["u"]
+    B, G = d.shape
+    V = lt.shape[2]
+    loose = 0
+    for b in range(B):
+        res = spec.verify_block(lt[b], ld[b], d[b], r[b], float(u[b]))
+        n = int(n_gpu[b])
+        assert 0 <= n <= G
+        assert (tok_gpu[b, :n] == d[b, :n]).all() and (tok_gpu[b, n + 1:] == -1).all()
+        assert 0 <= tok_gpu[b, n] < V
+        if any(spec.decision_unpinned(rr, pp, qq, V) for rr, pp, qq in res["tested"]):
+            loose += 1
+            continue
+        assert n == res["n"], (b, n, res["n"])
+        unp, cands = spec.sample_unpinned(res["weights"], float(u[b]), V, res["kind"])
+        if unp:
+            loose += 1
+            assert int(tok_gpu[b, n]) in cands, (b, tok_gpu[b, n], cands)
+        else:
+            assert int(tok_gpu[b, n]) == res["tokens"][-1], (b, tok_gpu[b, n], res["tokens"][-1], res["kind"])
+    return loose

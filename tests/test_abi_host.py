@@ -1,7 +1,6 @@
 """Host-side checks of the C ABI that need no GPU.
 
-The library must load and export every function ``include/moe_mxfp4.h``
-declares; argument errors must be reported before any device work; a host
+The library must load and export every function ``include/*.h`` declares; argument errors must be reported before any device work; a host
 without a usable device must get MOE_ERR_DEVICE rather than a crash.
 """
 import ctypes
@@ -27,7 +26,7 @@ def _declared():
         if f.endswith(".h"):
             src = open(os.path.join(ROOT, "include", f)).read()
             src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-            names |= set(re.findall(r"^\s*(?:MOE_API\s+)?(?:int32_t|void|const char\*)\s+(\w+)\s*\(", src, re.M))
+            names |= set(re.findall(r"^\s*(?:MOE_API\s+)?(?:int32_t|int64_t|void|const char\*)\s+(\w+)\s*\(", src, re.M))
     return names
 
 
@@ -47,7 +46,7 @@ def test_exported_dynamic_symbols_are_only_the_abi(mx):
     import subprocess
     out = subprocess.run(["nm", "-D", "--defined-only", mx.LIB_PATH], capture_output=True, text=True).stdout
     exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
-    ours = {s for s in exported if s.startswith(("moe_", "mxfp4_"))}
+    ours = {s for s in exported if s.startswith(("moe_", "mxfp4_", "spec_"))}
     assert ours == _declared()
 
 
@@ -115,3 +114,34 @@ def test_null_handle_calls(mx):
     assert mx.lib.moe_set_timeout_ns(None, 5) == mx.MOE_ERR_INVALID_ARG
     assert mx.lib.moe_engine_grid(None) == 0
     mx.lib.moe_mxfp4_destroy(None)  # no-op
+    assert mx.lib.moe_forward_ops(None, p, 9, p, None, 0, None) == mx.MOE_ERR_INVALID_ARG
+
+
+def test_spec_verify_workspace_bounds(mx):
+    ws = mx.lib.spec_verify_workspace_bytes
+    assert ws(1, 8, 152064) > 0
+    assert ws(64, 8, 152064) > ws(1, 8, 152064)
+    assert ws(1, 0, 10) > 0
+    for bad in [(0, 8, 100), (1, -1, 100), (1, 17, 100), (1, 8, 0), (1, 8, (1 << 22) + 1)]:
+        assert ws(*bad) == -1, bad
+
+
+def test_spec_verify_argument_errors(mx):
+    f = mx.lib.spec_verify
+    p = ctypes.c_void_p(1 << 20)
+    n = mx.lib.spec_verify_workspace_bytes(2, 8, 1000)
+    assert f(p, p, p, p, p, 0, 8, 1000, p, p, p, n, None) == mx.MOE_OK  # no blocks: no-op
+    assert f(p, p, p, p, p, -1, 8, 1000, p, p, p, n, None) == mx.MOE_ERR_INVALID_ARG
+    assert f(p, p, p, p, p, 2, 8, 1000, p, p, p, n - 8, None) == mx.MOE_ERR_INVALID_ARG  # workspace too small
+    assert f(None, p, p, p, p, 2, 8, 1000, p, p, p, n, None) == mx.MOE_ERR_INVALID_ARG
+    assert f(p, None, p, p, p, 2, 8, 1000, p, p, p, n, None) == mx.MOE_ERR_INVALID_ARG
+    assert f(p, p, p, ctypes.c_void_p((1 << 20) + 4), p, 2, 8, 1000, p, p, p, n, None) == mx.MOE_ERR_INVALID_ARG
+    assert f(p, p, p, p, p, 2, 8, 1000, p, p, ctypes.c_void_p((1 << 20) + 8), n, None) == mx.MOE_ERR_INVALID_ARG
+    assert f(p, p, p, p, p, 2, 17, 1000, p, p, p, n, None) == mx.MOE_ERR_INVALID_ARG
+    assert mx.lib.spec_verify_status(None, None) == mx.MOE_ERR_INVALID_ARG
+    import torch
+    if not torch.cuda.is_available():  # valid arguments, no device
+        assert f(p, p, p, p, p, 2, 8, 1000, p, p, p, n, None) == mx.MOE_ERR_DEVICE
+        # G == 0 needs no draft arrays
+        n0 = mx.lib.spec_verify_workspace_bytes(2, 0, 1000)
+        assert f(p, None, None, None, p, 2, 0, 1000, p, p, p, n0, None) == mx.MOE_ERR_DEVICE
