@@ -72,10 +72,14 @@ def parse_args():
     return ap.parse_args()
 
 
+ENGINE_SOURCES = ("engine.cu", "engine.cuh", "ptx.cuh", "moe_mxfp4.cu")
+
+
 def source_digest() -> str:
+    """Digest of the sources engine_kernel is built from (and launched by)."""
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "mxfp4_moe_expert_router_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
+    for f in ENGINE_SOURCES:
+        with open(os.path.join(ROOT, "mxfp4_moe_expert_router_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
