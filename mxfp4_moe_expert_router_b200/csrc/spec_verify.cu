@@ -136,8 +136,8 @@ __device__ bool sv_grid_sync(uint32_t* hdr, uint32_t where) {
 // and 2^(j/32) comes correctly rounded from a 32-entry table in shared memory.
 // Error about 1 ulp.  Arguments here are l - max <= 0; below -708 (and for
 // -inf) it returns 0: such a term is under 2^-1021 of the row's largest, 1.
+// Branch-free, so that many calls schedule as straight-line code.
 __device__ __forceinline__ double sv_exp(double d, const double* tab) {
-  if (!(d > -708.0)) return 0.0;
   constexpr double INV_L = 0x1.71547652b82fep+5;         // 32 / ln2
   constexpr double L_HI = 0x1.62e42fefa39efp-1 / 32.0;   // ln2 / 32, leading part
   constexpr double L_LO = 0x1.abc9e3b39803fp-56 / 32.0;  // ln2 / 32 - L_HI
@@ -155,8 +155,11 @@ __device__ __forceinline__ double sv_exp(double d, const double* tab) {
   q *= r;  // exp(r) - 1
   const double T = tab[N & 31];
   const double e = fma(T, q, T);  // 2^(j/32) exp(r), in [0.98, 2.03)
-  // times 2^m, m = floor(N / 32): added to the exponent field (stays normal)
-  return __hiloint2double(__double2hiint(e) + ((N >> 5) << 20), __double2loint(e));
+  // times 2^m, m = floor(N / 32): added to the exponent field (stays normal
+  // above -708); below, and for -inf or NaN, the select gives 0 (no branch:
+  // the arithmetic above is then meaningless but harmless)
+  const double res = __hiloint2double(__double2hiint(e) + ((N >> 5) << 20), __double2loint(e));
+  return d > -708.0 ? res : 0.0;
 }
 
 __device__ __forceinline__ double warp_incl_scan(double v, int lane) {
