@@ -35,8 +35,7 @@ constexpr int SEG = 512;        // vocabulary entries per statistics segment
 constexpr int LPL = SEG / 32;   // ... per lane
 constexpr int SEGC = 256;       // vocabulary entries per weight segment
 constexpr int LPC = SEGC / 32;  // ... per lane
-constexpr int SB = 16;          // loads per lane batched together
-constexpr int SBR = 24;         // segment sums per lane batched together in the draw
+constexpr int SBR = 24;         // segment sums per lane loaded together in the draw
 constexpr uint64_t SV_TIMEOUT_NS = 2000000000ull;
 
 // workspace header (uint32 words), then %globaltimer stamps at byte 64
@@ -431,7 +430,7 @@ __device__ __forceinline__ int crossing_lane(double incl_plus_base, double t, do
 }
 
 // Sum of the segment weights W[s_lo, s_hi) in index order; loads in batches
-// of SB, all in flight together.
+// of SBR, all in flight together.
 __device__ __forceinline__ double range_sum(const double* W, int s_lo, int s_hi) {
   double c = 0.0;
   for (int s0 = s_lo; s0 < s_hi; s0 += SBR) {
