@@ -1,0 +1,44 @@
+"""bench.py's host logic on CPU: the roofline's byte count, the profile digest and the
+verify step's reference arm (the fp64 oracle on host cores)."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+import bench
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_algorithmic_bytes_closed_form():
+    w = synth.WORKLOADS["decode_t9_h4096_e128"]
+    # per hit expert: gate, up and down, each H*I elements at 4 bits + one scale byte per 32
+    per_expert = 3 * 4096 * 1536 * (0.5 + 1 / 32)
+    router = 128 * 4096 * 4          # fp32 router weights
+    xy = 2 * 9 * 4096 * 2            # bf16 x in, y out
+    assert bench.algorithmic_bytes(w, 9, 57) == pytest.approx(57 * per_expert + router + xy)
+    assert bench.algorithmic_bytes(w, 9, 0) == pytest.approx(router + xy)
+
+
+def test_committed_profile_matches_the_engine_sources():
+    """The decode profile's digest names the current engine sources, so the bench line
+    carries its DRAM traffic; any edit of those sources must come with a new capture."""
+    assert bench.profile_traffic() is not None
+    assert bench.profile_traffic() > bench.algorithmic_bytes(synth.WORKLOADS["decode_t9_h4096_e128"], 9, 50)
+
+
+def test_verify_reference_arm_prints_one_json_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "verify_tiny_v1000_g8", "--steps", "3", "--warmup", "1"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "blocks/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    assert d["config"]["workload"] == "verify_tiny_v1000_g8"
