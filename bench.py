@@ -613,7 +613,6 @@ def run_verify(args, w, rank, world):
     pass over them exceeds the L2 (no flush needed)."""
     import torch
     import torch.distributed as dist
-    from oracle import spec as ospec
     from synth.spec import verify_inputs
 
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -700,6 +699,7 @@ def run_verify(args, w, rank, world):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import spec as ospec  # the CPU-baseline leg only
         t0 = time.perf_counter()
         nb = 0
         while time.perf_counter() - t0 < 5.0 and nb < 64:
