@@ -67,16 +67,19 @@ def parse_args():
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of replaying them as one CUDA graph")
     ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--shard-i", action="store_true",
+                    help="I-sharded layer across the ranks (strong scaling): every rank streams its I-slice "
+                         "of the same token block; partials all-reduced (NCCL), then rounded to bf16")
     ap.add_argument("--no-ops-baseline", action="store_true",
                     help="skip timing the operator-by-operator launches (moe_forward_ops)")
     return ap.parse_args()
 
 
-ENGINE_SOURCES = ("engine.cu", "engine.cuh", "ptx.cuh", "moe_mxfp4.cu")
+ENGINE_SOURCES = ("engine.cu", "engine.cuh", "ptx.cuh")
 
 
 def source_digest() -> str:
-    """Digest of the sources engine_kernel is built from (and launched by)."""
+    """Digest of the sources engine_kernel's code is compiled from."""
     h = hashlib.sha256()
     for f in ENGINE_SOURCES:
         with open(os.path.join(ROOT, "mxfp4_moe_expert_router_b200", "csrc", f), "rb") as fh:
@@ -368,6 +371,8 @@ def main():
     import mxfp4_moe_expert_router_b200 as mx
 
     layers = [build_layer(mx, w, l, seed=0) for l in range(w.layers)]
+    if args.shard_i:
+        return run_shard_i(args, mx, w, T, layers, rank, world)
     m = mx.Moe(w.hidden, w.inter, w.experts, w.top_k, T, layers)
     m.moe_set_large_kind(m.LARGE_F16 if args.large_kind == "f16" else m.LARGE_MXF4)
     xs = token_blocks(w, T, args.batches, rank)
@@ -605,6 +610,79 @@ def run_reference(args, w, T, rank, world):
                                       f"by {len(hit)} hit experts"},
            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
+
+
+def run_shard_i(args, mx, w, T, layers, rank, world):
+    """The I-sharded layer: every rank holds rows [r*I/N, (r+1)*I/N) of each expert's
+    gate/up matrices and the same down columns, streams them for the same token
+    block (moe_forward_partial), the fp32 partials are summed across ranks (NCCL
+    all-reduce) and rounded to bf16 (moe_round_bf16).  Strong scaling: a step is one
+    token block, whatever N."""
+    import torch
+    import torch.distributed as dist
+    if w.layers != 1:
+        raise SystemExit("--shard-i: one layer per call")
+    shard = mx.shard_layer_i(layers[0], rank, world)
+    m = mx.Moe(w.hidden, w.inter // world, w.experts, w.top_k, T, [shard])
+    xs = token_blocks(w, T, args.batches, 0)  # the same token blocks on every rank
+    hits = []
+    for x in xs:
+        hits.append(int((m.moe_route(x, layer=0)["counts"] > 0).sum().item()))
+    part = torch.empty((T, w.hidden), dtype=torch.float32, device="cuda")
+    y = torch.empty((T, w.hidden), dtype=torch.bfloat16, device="cuda")
+
+    def step(i):
+        m.moe_forward_partial(xs[i % len(xs)], part)
+        if world > 1:
+            dist.all_reduce(part)
+        mx.round_bf16(part, y)
+
+    for i in range(args.warmup):
+        step(i)
+    m.moe_status()
+    stream = torch.cuda.current_stream()
+    clocks = ClockSampler(("GPU-" + str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid))
+                          if rank == 0 else None)
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    m.moe_status()
+    ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, "cuda")
+    us_step = ms * 1e3 / args.steps
+    mean_hit = float(np.mean([hits[i % len(hits)] for i in range(args.steps)]))
+    shard_w = synth.Workload(w.name, w.hidden, w.inter // world, w.experts, w.top_k, T)
+    alg = algorithmic_bytes(shard_w, T, mean_hit)
+    peak, peak_kind = measured_peaks()
+    achieved = alg / (us_step * 1e-6) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": T / (us_step * 1e-6), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": us_step / 1e3, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "mxfp4-w/fp32-acc",
+            "data": "synthetic (seeded N(0,0.02) expert weights quantised to MXFP4, N(0,1) bf16 tokens)",
+            "config": {"workload": w.name if not args.tokens else f"{w.name}_t{T}", "hidden": w.hidden,
+                       "inter": w.inter, "inter_per_rank": w.inter // world, "experts": w.experts,
+                       "top_k": w.top_k, "tokens": T, "parallelism": f"I-sharded x{world} (NCCL all-reduce)",
+                       "launch": "stream launches: moe_forward_partial, all-reduce, moe_round_bf16"},
+            "layer_us": us_step,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_source": peak_kind,
+                         "algorithmic_bytes_per_launch": alg, "traffic": None, "kernel": "engine_kernel",
+                         "per": "rank (its I-slice of the hit experts)"},
+            "gpu_launches": 3 * args.steps, "e2e": None, "cpu_baseline": None, "clocks": clk}), flush=True)
+    m.close()
+    if world > 1:
+        dist.destroy_process_group()
 
 
 def run_verify(args, w, rank, world):

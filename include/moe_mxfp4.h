@@ -148,6 +148,33 @@ MOE_API int32_t moe_forward(moe_mxfp4_t* h, const void* x_bf16, int32_t T, void*
                     void* layer_io_bf16, void* stream);
 
 /*
+ * moe_forward_partial -- one layer (a handle of num_layers == 1) with the
+ * output left as the fp32 sum over the k slots, in slot order, without the
+ * bf16 rounding: y_f32 [T][H] (device, 16-byte aligned).  It is one rank's
+ * share of an I-sharded layer. A handle built on rows [r*I/N, (r+1)*I/N) of
+ * every expert's gate and up matrices, and on the same columns of its down
+ * matrix (with their block scales), routes exactly as the unsharded layer.
+ * SwiGLU acts per intermediate row, so the N ranks' partials sum to the
+ * layer's output. moe_round_bf16 of that sum gives moe_forward's result, up to
+ * the fp32 summation order. With N = 1 it gives that result bit for bit. The
+ * sum over ranks is an all-reduce; the pages' deployment is one 8-GPU node
+ * (HyperAI salon transcript "Speed is Intelligence", GLM-5.1 case; bjdmk
+ * news, 8 GPUs per node). Arguments and capture safety as for moe_forward.
+ * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE (num_layers != 1),
+ * MOE_ERR_CUDA.
+ */
+MOE_API int32_t moe_forward_partial(moe_mxfp4_t* h, const void* x_bf16, int32_t T, float* y_f32,
+                                    void* stream);
+
+/*
+ * moe_round_bf16 -- out_bf16[i] = bf16(in_f32[i]) (round to nearest even) for
+ * n device values on `stream`; the last step of an I-sharded layer, after the
+ * partial outputs were summed.  Errors: MOE_ERR_INVALID_ARG (n < 0; null or
+ * misaligned pointers with n > 0), MOE_ERR_CUDA.
+ */
+MOE_API int32_t moe_round_bf16(const float* in_f32, void* out_bf16, int64_t n, void* stream);
+
+/*
  * moe_forward_host -- moe_forward with HOST input and output: copies
  * x_host [T][H] bf16 to the handle's device staging buffer, runs the layers,
  * copies y back to y_host [T][H] and synchronises `stream`.  Pinned host

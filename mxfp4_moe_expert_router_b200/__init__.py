@@ -22,7 +22,7 @@ EXPORTS = ("mxfp4_quantize", "moe_mxfp4_create", "moe_route", "moe_forward", "mo
            "moe_status_str", "moe_route_static", "moe_phase_ns",
            "moe_stream_profile", "moe_set_large_kind", "moe_forward_host_async", "moe_host_join",
            "moe_forward_ops", "spec_verify_workspace_bytes", "spec_verify", "spec_verify_status",
-           "spec_exp")
+           "spec_exp", "moe_forward_partial", "moe_round_bf16")
 
 MOE_OPS_PDL = 1
 
@@ -56,6 +56,8 @@ def _load():
         "moe_forward": (i32, [vp, vp, i32, vp, vp, vp]),
         "moe_forward_host": (i32, [vp, vp, i32, vp, vp]),
         "moe_forward_ops": (i32, [vp, vp, i32, vp, vp, i32, vp]),
+        "moe_forward_partial": (i32, [vp, vp, i32, vp, vp]),
+        "moe_round_bf16": (i32, [vp, vp, i64, vp]),
         "moe_forward_host_async": (i32, [vp, vp, i32, vp, vp]),
         "moe_host_join": (i32, [vp, vp]),
         "moe_status": (i32, [vp, vp]),
@@ -184,6 +186,17 @@ class Moe:
         _check(lib.moe_forward_ops(self.handle, _ptr(x), T, _ptr(y), _ptr(layer_io),
                                    MOE_OPS_PDL if pdl else 0, _stream(stream)), "moe_forward_ops")
         return y
+
+    def moe_forward_partial(self, x, y_f32=None, stream=None):
+        """One layer's fp32 output before the bf16 rounding: a rank's share of an
+        I-sharded layer (see ``shard_layer_i``)."""
+        import torch
+        T = x.shape[0]
+        if y_f32 is None:
+            y_f32 = torch.empty((T, self.cfg.hidden), dtype=torch.float32, device=x.device)
+        _check(lib.moe_forward_partial(self.handle, _ptr(x), T, _ptr(y_f32), _stream(stream)),
+               "moe_forward_partial")
+        return y_f32
 
     def moe_forward_host(self, x_host, y_host=None, stream=None):
         import torch
@@ -325,3 +338,27 @@ def spec_exp(x, stream=None):
     y = torch.empty_like(x)
     _check(lib.spec_exp(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "spec_exp")
     return y
+
+
+def round_bf16(y_f32, out=None, stream=None):
+    """bf16(y_f32), round to nearest even, on the device (``moe_round_bf16``)."""
+    import torch
+    if out is None:
+        out = torch.empty(y_f32.shape, dtype=torch.bfloat16, device=y_f32.device)
+    _check(lib.moe_round_bf16(_ptr(y_f32), _ptr(out), y_f32.numel(), _stream(stream)), "moe_round_bf16")
+    return out
+
+
+def shard_layer_i(layer: "LayerMX", rank: int, world: int) -> "LayerMX":
+    """Rank `rank` of `world`'s share of an I-sharded layer: rows [r*I/N, (r+1)*I/N)
+    of every expert's gate and up matrices, the same columns of its down matrix,
+    with their block scales; the router is replicated.  I/N must be a multiple of
+    128 (the engine's tiling)."""
+    E, I = layer.gate_codes.shape[0], layer.gate_codes.shape[1]
+    if world < 1 or not 0 <= rank < world or I % world or (I // world) % 128:
+        raise ValueError(f"cannot shard I = {I} over {world} ranks into multiples of 128")
+    i0, i1 = rank * I // world, (rank + 1) * I // world
+    rows = lambda t: t[:, i0:i1].contiguous()
+    return LayerMX(rows(layer.gate_codes), rows(layer.gate_scales), rows(layer.up_codes), rows(layer.up_scales),
+                   layer.down_codes[:, :, i0 // 2:i1 // 2].contiguous(),
+                   layer.down_scales[:, :, i0 // 32:i1 // 32].contiguous(), layer.router_w, layer.router_b)

@@ -19,7 +19,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmoe_mxfp4.so")
-SOURCES = ["quantize.cu", "engine.cu", "moe_mxfp4.cu", "noalloc.cu", "spec_verify.cu"]
+SOURCES = ["quantize.cu", "engine.cu", "moe_mxfp4.cu", "noalloc.cu", "spec_verify.cu", "partial.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -9,6 +9,7 @@
 #include <vector>
 
 #include "engine.cuh"
+#include "partial.cuh"
 
 using namespace moe;
 
@@ -315,6 +316,30 @@ int32_t moe_forward_ops(moe_mxfp4_t* h, const void* x_bf16, int32_t T, void* y_b
   p.y_out = static_cast<__nv_bfloat16*>(y_bf16);
   p.layer_io = static_cast<__nv_bfloat16*>(layer_io_bf16);
   return engine_launch_ops(p, h->grid, (flags & MOE_OPS_PDL) != 0, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+int32_t moe_forward_partial(moe_mxfp4_t* h, const void* x_bf16, int32_t T, float* y_f32, void* stream) {
+  if (!h || T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x_bf16 || !y_f32 || !aligned16(x_bf16) || !aligned16(y_f32)) return MOE_ERR_INVALID_ARG;
+  if (h->cfg.num_layers != 1) return MOE_ERR_UNSUPPORTED_SHAPE;
+  const int32_t st = moe_forward(h, x_bf16, T, h->y_stage, nullptr, stream);
+  if (st != MOE_OK) return st;
+  return combine_f32_launch(h->ypair, h->inv, T, h->cfg.top_k, h->cfg.hidden, y_f32,
+                            static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+int32_t moe_round_bf16(const float* in_f32, void* out_bf16, int64_t n, void* stream) {
+  if (n < 0 || (n > 0 && (!in_f32 || !out_bf16 || (reinterpret_cast<uintptr_t>(in_f32) & 3u) ||
+                          (reinterpret_cast<uintptr_t>(out_bf16) & 1u))))
+    return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  return round_bf16_launch(in_f32, static_cast<__nv_bfloat16*>(out_bf16), n, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }

@@ -45,3 +45,18 @@ def build_library():
     mod = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(mod)
     return mod.build()
+
+
+def shard_layer_np(lw, rank: int, world: int):
+    """Rank `rank` of `world`'s I-slice of an oracle layer (gate/up rows, down columns,
+    their block scales; the router replicated)."""
+    from oracle import moe as omoe
+    I = lw.gate_codes[0].shape[0]
+    i0, i1 = rank * I // world, (rank + 1) * I // world
+    rows = lambda a: [x[i0:i1].copy() for x in a]
+    return omoe.LayerWeights(
+        gate_codes=rows(lw.gate_codes), gate_scales=rows(lw.gate_scales),
+        up_codes=rows(lw.up_codes), up_scales=rows(lw.up_scales),
+        down_codes=[x[:, i0 // 2:i1 // 2].copy() for x in lw.down_codes],
+        down_scales=[x[:, i0 // 32:i1 // 32].copy() for x in lw.down_scales],
+        router_w=lw.router_w, router_b=lw.router_b)

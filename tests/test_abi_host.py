@@ -145,3 +145,12 @@ def test_spec_verify_argument_errors(mx):
         # G == 0 needs no draft arrays
         n0 = mx.lib.spec_verify_workspace_bytes(2, 0, 1000)
         assert f(p, None, None, None, p, 2, 0, 1000, p, p, p, n0, None) == mx.MOE_ERR_DEVICE
+
+
+def test_partial_and_round_argument_errors(mx):
+    p = ctypes.c_void_p(1 << 20)
+    assert mx.lib.moe_forward_partial(None, p, 9, p, None) == mx.MOE_ERR_INVALID_ARG
+    assert mx.lib.moe_round_bf16(p, p, -1, None) == mx.MOE_ERR_INVALID_ARG
+    assert mx.lib.moe_round_bf16(None, p, 4, None) == mx.MOE_ERR_INVALID_ARG
+    assert mx.lib.moe_round_bf16(ctypes.c_void_p((1 << 20) + 2), p, 4, None) == mx.MOE_ERR_INVALID_ARG
+    assert mx.lib.moe_round_bf16(None, None, 0, None) == mx.MOE_OK

@@ -244,3 +244,22 @@ def test_chain_rmsnorm_inputs():
     ms = (moe.rmsnorm(ys[0]) ** 2).mean(-1)
     assert np.allclose(ms, m / (m + moe.RMS_EPS), rtol=1e-14, atol=0)  # closed form with eps
     assert np.allclose((xs[1] ** 2).mean(-1), ms, rtol=2 ** -7, atol=0)  # after bf16 rounding
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_i_sharded_partials_sum_to_the_layer(world):
+    """SwiGLU acts per intermediate row, so splitting I across ranks (gate/up rows, down
+    columns) and summing the ranks' outputs gives the layer.  The routing depends only on
+    the router and is the same on every rank."""
+    from tests.helpers import quantized_layer_np, shard_layer_np, x_values
+    w = synth.Workload("shard", 256, 512, 8, 2, 9, device_draw=False)
+    xb, lw, _ = quantized_layer_np(w, seed=31)
+    x = x_values(xb)
+    full = moe.moe_layer(x, lw, w.top_k)
+    parts = [moe.moe_layer(x, shard_layer_np(lw, r, world), w.top_k) for r in range(world)]
+    for part in parts:
+        assert (part["idx"] == full["idx"]).all() and (part["perm"] == full["perm"]).all()
+    total = sum(part["y"] for part in parts)
+    assert np.allclose(total, full["y"], rtol=1e-12, atol=1e-12 * np.abs(full["y"]).max())
+    # a single rank is not the layer: every slice carries a share
+    assert not np.allclose(parts[0]["y"], full["y"], rtol=1e-3)
