@@ -65,3 +65,63 @@ def test_token_block_ids_bounds():
     assert bench.token_block_ids(3, 2) == [1192, 1193]
     with pytest.raises(ValueError):
         bench.token_block_ids(0, 65)
+
+
+def _shard_rank_main(rank, world, port, out):
+    """Rank r: the oracle's partial output over its I-slice, summed across ranks by an
+    all-reduce (gloo) -- the host composition of the I-sharded layer."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import synth
+    from oracle import moe
+    from tests.helpers import quantized_layer_np, shard_layer_np, x_values
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = synth.Workload("shard", 256, 256, 8, 2, 9, device_draw=False)
+        xb, lw, _ = quantized_layer_np(w, seed=61)
+        part = torch.from_numpy(moe.moe_layer(x_values(xb), shard_layer_np(lw, rank, world), w.top_k)["y"])
+        dist.all_reduce(part)
+        full = moe.moe_layer(x_values(xb), lw, w.top_k)["y"]
+        out.put((rank, float(np.abs(part.numpy() - full).max() / np.abs(full).max())))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_all_reduce_i_shards_to_the_layer():
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r for r, _ in res] == [0, 1]
+    assert all(err < 1e-12 for _, err in res), res
+
+
+def test_shard_layer_i_slices_like_the_oracle_side():
+    """The binding's I-slicer (torch, any device) against the oracle-side slicer."""
+    import numpy as np
+    import torch
+    import synth
+    from tests.helpers import build_library, quantized_layer_np, shard_layer_np
+    build_library()
+    import mxfp4_moe_expert_router_b200 as mx
+    w = synth.Workload("shard", 256, 512, 4, 2, 9, device_draw=False)
+    _, lw, _ = quantized_layer_np(w, seed=62)
+    st = lambda a: torch.from_numpy(np.stack(a))
+    layer = mx.LayerMX(st(lw.gate_codes), st(lw.gate_scales), st(lw.up_codes), st(lw.up_scales),
+                       st(lw.down_codes), st(lw.down_scales), torch.from_numpy(lw.router_w), None)
+    for world in (1, 2, 4):
+        for r in range(world):
+            a, b = mx.shard_layer_i(layer, r, world), shard_layer_np(lw, r, world)
+            for k in ("gate_codes", "gate_scales", "up_codes", "up_scales", "down_codes", "down_scales"):
+                assert (getattr(a, k).numpy() == np.stack(getattr(b, k))).all(), (world, r, k)
+    with pytest.raises(ValueError):
+        mx.shard_layer_i(layer, 0, 8)  # 512 / 8 = 64 rows
