@@ -160,8 +160,10 @@ MOE_API int32_t moe_forward(moe_mxfp4_t* h, const void* x_bf16, int32_t T, void*
  * sum over ranks is an all-reduce; the pages' deployment is one 8-GPU node
  * (HyperAI salon transcript "Speed is Intelligence", GLM-5.1 case; bjdmk
  * news, 8 GPUs per node). Arguments and capture safety as for moe_forward.
- * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE (num_layers != 1),
- * MOE_ERR_CUDA.
+ * The handle's bf16 staging output serves as scratch, and it is also slot 0
+ * of moe_forward_host_async. So order the call after any such copies still in
+ * flight (moe_host_join on `stream`). Errors: MOE_ERR_INVALID_ARG,
+ * MOE_ERR_UNSUPPORTED_SHAPE (num_layers != 1), MOE_ERR_CUDA.
  */
 MOE_API int32_t moe_forward_partial(moe_mxfp4_t* h, const void* x_bf16, int32_t T, float* y_f32,
                                     void* stream);
@@ -178,8 +180,10 @@ MOE_API int32_t moe_round_bf16(const float* in_f32, void* out_bf16, int64_t n, v
  * moe_forward_host -- moe_forward with HOST input and output: copies
  * x_host [T][H] bf16 to the handle's device staging buffer, runs the layers,
  * copies y back to y_host [T][H] and synchronises `stream`.  Pinned host
- * memory gives asynchronous copies; pageable memory works too.  Returns the
- * first error, device-side errors included.
+ * memory gives asynchronous copies; pageable memory works too.  Its staging
+ * buffers are slot 0 of moe_forward_host_async, whose copies and layers in
+ * flight it waits for first.  Returns the first error, device-side errors
+ * included.
  */
 MOE_API int32_t moe_forward_host(moe_mxfp4_t* h, const void* x_host, int32_t T, void* y_host,
                          void* stream);

@@ -112,6 +112,17 @@ int32_t validate_cfg(const moe_config_t* c) {
   return MOE_OK;
 }
 
+// x_stage / y_stage double as slot 0 of moe_forward_host_async.  Before another
+// call writes them, `s` waits for that slot's last copy in, layers and copy out
+// (events that were never recorded are complete).
+cudaError_t wait_async_slot0(const moe_mxfp4* h, cudaStream_t s) {
+  if (!h->h2d) return cudaSuccess;
+  cudaError_t e = cudaStreamWaitEvent(s, h->ev_in[0], 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, h->ev_k[0], 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, h->ev_out[0], 0);
+  return e;
+}
+
 EngineParams base_params(const moe_mxfp4* h, int T) {
   EngineParams p{};
   p.H = h->cfg.hidden; p.I = h->cfg.inter; p.E = h->cfg.num_experts; p.K = h->cfg.top_k;
@@ -371,7 +382,8 @@ int32_t moe_forward_host(moe_mxfp4_t* h, const void* x_host, int32_t T, void* y_
   if (!x_host || !y_host) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t bytes = (size_t)T * h->cfg.hidden * 2;
-  if (cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+  if (wait_async_slot0(h, s) != cudaSuccess ||
+      cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   int32_t st = moe_forward(h, h->x_stage, T, h->y_stage, nullptr, stream);
   if (st != MOE_OK) return st;
