@@ -68,8 +68,15 @@ def parse_args():
                     help="launch the timed steps one by one instead of replaying them as one CUDA graph")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--shard-i", action="store_true",
-                    help="I-sharded layer across the ranks (strong scaling): every rank streams its I-slice "
-                         "of the same token block; partials all-reduced (NCCL), then rounded to bf16")
+                    help="I-sharded layer across the ranks (the default with more than one rank): every rank "
+                         "streams its I-slice of the same token block; the partials are summed by the engine's "
+                         "fused all-reduce (peer loads) and rounded to bf16")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with more than one rank: independent replicas (each rank its own token blocks, no "
+                         "collective on the data path) instead of the I-sharded layer")
+    ap.add_argument("--nccl-allreduce", action="store_true",
+                    help="I-sharded layer: sum the partials with an NCCL all-reduce between launches instead of "
+                         "the fused all-reduce")
     ap.add_argument("--no-ops-baseline", action="store_true",
                     help="skip timing the operator-by-operator launches (moe_forward_ops)")
     return ap.parse_args()
@@ -146,6 +153,24 @@ def time_calls(mx, stream, n: int, launch, use_graph: bool) -> float:
     return e0.elapsed_time(e1) * 1e3 / n
 
 
+def per_call_times(m, mx, stream, step, n: int) -> dict:
+    """Device time of each of n stream-launched calls, an event pair around each:
+    median / p10 / p90 in us (the graph replay gives only the mean)."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    torch.cuda.synchronize()
+    for i, (a, b) in enumerate(ev):
+        a.record(stream)
+        step(i)
+        b.record(stream)
+    torch.cuda.synchronize()
+    m.moe_status()
+    us = sorted(a.elapsed_time(b) * 1e3 for a, b in ev)
+    q = lambda f: us[min(len(us) - 1, int(f * (len(us) - 1) + 0.5))]
+    return {"median_us": q(0.5), "p10_us": q(0.1), "p90_us": q(0.9), "n": n,
+            "launch": "stream launches, an event pair around each call"}
+
+
 def ops_baseline(mx, m, stream, xptr, yptr, T: int, steps: int) -> dict:
     """The same layer(s) as six launches per layer (moe_forward_ops) against the
     single engine launch, each as stream launches and as a CUDA graph; the ops
@@ -184,6 +209,64 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except (OSError, KeyError, ValueError):
         return 6650.0, "fallback"
+
+
+def measured_bf16_tflops():
+    """Dense bf16 tensor peak (burst: the engine is timed alone), measured, else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback"
+
+
+# Tensor-core kinds of the large-T weight stream: nominal dense rate relative to
+# bf16 (B200: fp4 9, fp8 4.5, bf16 2.25 PFLOP/s) and the MMA columns each
+# activation value occupies in the gate/up and down projections.
+LARGE_KINDS = {
+    "mxf4": {"mma": "tcgen05.mma kind::mxf4 (E2M1 x E2M1, E8M0 scales)", "ratio_to_bf16": 4.0,
+             "terms_gate_up": 5, "terms_down": 5},
+    "f16": {"mma": "tcgen05.mma kind::f16 (bf16 x bf16, weights dequantised)", "ratio_to_bf16": 1.0,
+            "terms_gate_up": 1, "terms_down": 2},
+}
+
+
+def layer_flops(w: synth.Workload, T: int) -> float:
+    """Algorithmic FLOP of one call: 6 T k H I (gate, up, down) + 2 T H E (router), per layer."""
+    return (6.0 * T * w.top_k * w.hidden * w.inter + 2.0 * T * w.hidden * w.experts) * w.layers
+
+
+def roofline(w: synth.Workload, T: int, alg_bytes: float, ms_step: float, large_kind: str, traffic) -> dict:
+    """HBM roofline of the weight stream, or the tensor roofline where the tile stream's
+    arithmetic intensity exceeds the ridge of its kind (the FP4 peak divided by the term
+    expansion of the activations, over the HBM peak)."""
+    peak, peak_kind = measured_peaks()
+    achieved = alg_bytes / (ms_step * 1e-3) / 1e9
+    hbm = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+           "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg_bytes, "traffic": traffic,
+           "kernel": "engine_kernel"}
+    TK = T * w.top_k
+    if not (TK > 256 and TK >= 8 * w.experts):
+        return hbm
+    k = LARGE_KINDS[large_kind]
+    bf16, bf16_kind = measured_bf16_tflops()
+    kind_peak = bf16 * k["ratio_to_bf16"]
+    flops = layer_flops(w, T)
+    terms = (2 * k["terms_gate_up"] + k["terms_down"]) / 3.0  # gate and up carry 2/3 of the FLOP
+    intensity = flops / alg_bytes
+    ridge = kind_peak / terms * 1e12 / (peak * 1e9)
+    if intensity <= ridge:
+        hbm["intensity_flop_per_byte"] = intensity
+        hbm["ridge_flop_per_byte"] = ridge
+        return hbm
+    tf = flops / (ms_step * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": tf, "peak": kind_peak, "unit": "TFLOP/s", "frac": tf / kind_peak,
+            "peak_source": f"{bf16_kind} bf16 {bf16:.1f} TFLOP/s x {k['ratio_to_bf16']:g} (nominal ratio of "
+                           f"{k['mma']} to bf16 on B200)",
+            "algorithmic_flop_per_launch": flops, "mma_columns_per_value": terms,
+            "frac_of_term_adjusted_peak": tf / (kind_peak / terms),
+            "intensity_flop_per_byte": intensity, "ridge_flop_per_byte": ridge,
+            "traffic": None, "kernel": "engine_kernel", "hbm": hbm}
 
 
 class ClockSampler:
@@ -289,46 +372,76 @@ def algorithmic_bytes(w: synth.Workload, T: int, hit: int) -> float:
 
 # ---- the CPU oracle as baseline / reference arm --------------------------------------------------
 
-def oracle_sample(w: synth.Workload, T: int, layer_dev, x_dev, budget_s: float):
-    """Time the oracle on a bounded sample of one layer; returns (layer seconds estimate, info).
+def cpu_model() -> str:
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
-    Untimed: regenerate the hit experts' bf16 weights (same device generator as
-    the GPU path), copy them to the host and quantise them with the oracle.
-    Timed: oracle routing of the whole block, then dequantisation + SwiGLU FFN +
-    weighting of as many hit experts (in expert order) as fit in ``budget_s``.
-    The layer time is extrapolated by the fraction of hit experts done.
-    """
+
+def oracle_prepare(w: synth.Workload, layer_dev, x_dev, n_experts: int):
+    """Untimed set-up of the oracle baseline: the block's fp64 inputs, its routing, and the
+    oracle's own MXFP4 codes of the first n hit experts (quantised from the same seeded bf16
+    weights as the GPU's)."""
     import torch
     from oracle import moe, mxfp4
     xb = x_dev.view(torch.int16).cpu().numpy().view(np.uint16)
     x = mxfp4.bf16_to_f64(xb)
     rw = layer_dev.router_w.cpu().numpy()
     rb = None if layer_dev.router_b is None else layer_dev.router_b.cpu().numpy()
-    t0 = time.perf_counter()
     idx, wts, _ = moe.route(x, rw, rb, w.top_k)
     counts, offsets, perm, inv = moe.permute(idx, w.experts)
-    t_route = time.perf_counter() - t0
     hit = [int(e) for e in np.nonzero(counts)[0]]
-    t_ffn, done = 0.0, 0
-    flat_w = wts.reshape(-1)
-    for e in hit:
-        q = {}
-        for kind in ("gate", "up", "down"):
-            bits = synth.expert_torch(w, 0, e, kind).view(torch.int16).cpu().numpy().view(np.uint16)
-            q[kind] = mxfp4.quantize(bits)
-        t1 = time.perf_counter()
-        seg = perm[offsets[e]:offsets[e + 1]]
-        wg = mxfp4.dequantize(*q["gate"])
-        wu = mxfp4.dequantize(*q["up"])
-        wd = mxfp4.dequantize(*q["down"])
-        _ = moe.expert_ffn(x[seg // w.top_k], wg, wu, wd) * flat_w[seg][:, None]
-        t_ffn += time.perf_counter() - t1
-        done += 1
-        if t_ffn + t_route >= budget_s or done >= 16:
-            break
-    layer_s = t_route + t_ffn * len(hit) / done
-    return layer_s, {"experts_timed": done, "experts_hit": len(hit), "route_s": t_route,
-                     "ffn_s_timed": t_ffn}
+    q = {}
+    dev = x_dev.device
+    for e in hit[:n_experts]:
+        q[e] = {kind: mxfp4.quantize(synth.expert_torch(w, 0, e, kind, device=dev)
+                                     .view(torch.int16).cpu().numpy().view(np.uint16))
+                for kind in ("gate", "up", "down")}
+    return {"x": x, "rw": rw, "rb": rb, "hit": hit, "q": q, "offsets": offsets, "perm": perm,
+            "flat_w": wts.reshape(-1)}
+
+
+def oracle_step(w: synth.Workload, prep, e: int):
+    """One timed sample of the oracle: the routing of the whole block, then one hit expert
+    (dequantise + SwiGLU FFN + routing weight).  Returns (route s, expert s)."""
+    from oracle import moe, mxfp4
+    t0 = time.perf_counter()
+    moe.permute(moe.route(prep["x"], prep["rw"], prep["rb"], w.top_k)[0], w.experts)
+    t1 = time.perf_counter()
+    q = prep["q"][e]
+    seg = prep["perm"][prep["offsets"][e]:prep["offsets"][e + 1]]
+    wg, wu, wd = (mxfp4.dequantize(*q[k]) for k in ("gate", "up", "down"))
+    _ = moe.expert_ffn(prep["x"][seg // w.top_k], wg, wu, wd) * prep["flat_w"][seg][:, None]
+    return t1 - t0, time.perf_counter() - t1
+
+
+def oracle_baseline(w: synth.Workload, T: int, layer_dev, x_dev, n_experts: int = 4, reps: int = 3):
+    """The oracle on this host's cores, BLAS on all threads and on one: per setting, `reps`
+    repetitions of (routing of the block + n hit experts), median taken; the layer time is
+    routing + (hit experts) x (median time of one expert)."""
+    from threadpoolctl import threadpool_limits
+    prep = oracle_prepare(w, layer_dev, x_dev, n_experts)
+    out = {}
+    for label, limit in (("all", None), ("one", 1)):
+        with threadpool_limits(limits=limit, user_api="blas"):
+            threads = blas_threads()
+            routes, experts = [], []
+            for _ in range(reps):
+                for i, e in enumerate(prep["q"]):
+                    r, x = oracle_step(w, prep, e)
+                    experts.append(x)
+                    if i == 0:
+                        routes.append(r)
+            t_route, t_exp = statistics.median(routes), statistics.median(experts)
+            out[label] = {"threads": threads, "route_s": t_route, "expert_s": t_exp,
+                          "layer_s": t_route + t_exp * len(prep["hit"])}
+    out["hit"] = len(prep["hit"])
+    out["experts_timed"] = len(prep["q"])
+    return out
 
 
 def blas_threads() -> int:
@@ -371,7 +484,7 @@ def main():
     import mxfp4_moe_expert_router_b200 as mx
 
     layers = [build_layer(mx, w, l, seed=0) for l in range(w.layers)]
-    if args.shard_i:
+    if args.shard_i or (world > 1 and not args.replicas and w.layers == 1):
         return run_shard_i(args, mx, w, T, layers, rank, world)
     m = mx.Moe(w.hidden, w.inter, w.experts, w.top_k, T, layers)
     m.moe_set_large_kind(m.LARGE_F16 if args.large_kind == "f16" else m.LARGE_MXF4)
@@ -433,6 +546,7 @@ def main():
     clk = clocks.stop()
     m.moe_status()
     phases = m.moe_phase_ns()  # the last timed step, CTA 0's view
+    per_call = per_call_times(m, mx, stream, step, min(args.steps, 200))
     ms_total = max_over_ranks(ev0.elapsed_time(ev1), dist if world > 1 else None, "cuda")
     ms_step = ms_total / args.steps
     tokens_per_s = job_tokens_per_s(world, T, args.steps, ms_total / 1e3)
@@ -444,7 +558,8 @@ def main():
                                    for x in xs[:2]]))
     peak, peak_kind = measured_peaks()
     achieved = alg_bytes / (ms_step * 1e-3) / 1e9
-    traffic = profile_traffic()
+    # the committed capture is of the decode workload's engine launch
+    traffic = profile_traffic() if (w.name == "decode_t9_h4096_e128" and T == w.tokens) else None
 
     # the pages' baseline execution model: one launch per operator
     ops = None
@@ -456,7 +571,7 @@ def main():
     if not args.no_e2e:
         xh = [x.cpu().pin_memory() for x in xs]
         yh = torch.empty((T, w.hidden), dtype=torch.bfloat16).pin_memory()
-        n_e2e = args.e2e_steps or max(1, min(args.steps, 500))
+        n_e2e = args.e2e_steps or 500
         for i in range(min(3, n_e2e)):
             m.moe_forward_host(xh[i % len(xh)], yh)
         if world > 1:
@@ -490,14 +605,20 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        layer_s, info = oracle_sample(w, T, layers[0], xs[0], budget_s=6.0)
-        cpu = {"value": T / layer_s if w.layers == 1 else T / (layer_s * w.layers),
-               "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"fp64 numpy oracle, layer 0, token block 0: routing of all {T} tokens + "
-                         f"{info['experts_timed']} of {info['experts_hit']} hit experts "
-                         f"(dequantise + SwiGLU FFN), extrapolated to all hit experts"
-                         + (f" and {w.layers} layers" if w.layers > 1 else ""),
-               "layer_s_estimate": layer_s}
+        ob = oracle_baseline(w, T, layers[0], xs[0])
+        layers_n = w.layers
+        cpu = {"value": T / (ob["all"]["layer_s"] * layers_n), "unit": "tokens/s",
+               "cores": ob["all"]["threads"], "kind": "oracle",
+               "sample": f"fp64 numpy oracle, layer 0, token block 0, median of 3: routing of all {T} tokens "
+                         f"+ each of {ob['experts_timed']} hit experts (dequantise + SwiGLU FFN); layer time = "
+                         f"routing + {ob['hit']} hit experts x median expert time"
+                         + (f", x {layers_n} layers" if layers_n > 1 else ""),
+               "cpu_model": cpu_model(), "cpu_count": os.cpu_count(),
+               "layer_s_estimate": ob["all"]["layer_s"] * layers_n,
+               "blas_one_thread": {"value": T / (ob["one"]["layer_s"] * layers_n), "unit": "tokens/s",
+                                   "threads": ob["one"]["threads"],
+                                   "layer_s_estimate": ob["one"]["layer_s"] * layers_n},
+               "timed_s": {k: {"route": ob[k]["route_s"], "expert": ob[k]["expert_s"]} for k in ("all", "one")}}
 
     if rank == 0:
         out = {
@@ -517,10 +638,8 @@ def main():
                                  "the timed moe_forward calls replayed as one CUDA graph"},
             "layer_us": ms_step * 1e3 / w.layers,
             "weight_stream_gbs": achieved,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "peak_source": peak_kind,
-                         "algorithmic_bytes_per_launch": alg_bytes,
-                         "traffic": traffic, "kernel": "engine_kernel"},
+            "roofline": roofline(w, T, alg_bytes, ms_step, args.large_kind, traffic),
+            "per_call": per_call,
             "gpu_launches": args.steps,
             "phase_us_last_step": {k: round(v / 1e3, 2) for k, v in
                                    zip(("router_logits", "x_images", "route_wait", "topk_or_tables", "permute", "stream",
@@ -549,93 +668,107 @@ def chain_hits(m, mx, w, T, x):
 
 
 def run_reference(args, w, T, rank, world):
-    """The fp64 CPU oracle on this host's cores, rank 0 only; each step a bounded sample."""
+    """The fp64 CPU oracle on this host's cores as the reference arm, rank 0 only.
+
+    Each timed step is a measured, bounded sample of the layer: the oracle's
+    routing of the whole token block, then one whole hit expert (dequantise +
+    SwiGLU FFN + routing weight), the experts taken in turn from the first few
+    hit ones.  ``ms_per_step`` is that step's measured time.  ``value`` is the
+    layer's tokens/s extrapolated from the medians (routing + hit experts x
+    one expert), reported with the extrapolation's inputs."""
     if rank != 0:
         return
     import torch
-    have_cuda = torch.cuda.is_available()
-    dev = "cuda" if have_cuda else "cpu"
-    from oracle import moe, mxfp4
-    # inputs: same recipe as the GPU arm (device draws when a GPU is present)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
     x = synth.draw_torch(1000, 0, "x", -1, (T, w.hidden), 1.0, device=dev)
-    xb = x.view(torch.int16).cpu().numpy().view(np.uint16)
-    xv = mxfp4.bf16_to_f64(xb)
     dense = synth.layer_inputs_torch(w, 0, 0, tokens=T, device=dev)
-    rw = dense["router_w"].cpu().numpy()
-    rb = None if dense["router_b"] is None else dense["router_b"].cpu().numpy()
-    idx, wts, _ = moe.route(xv, rw, rb, w.top_k)
-    counts, offsets, perm, inv = moe.permute(idx, w.experts)
-    hit = [int(e) for e in np.nonzero(counts)[0]]
-    # per-step sample: a slice of R rows of each projection of one hit expert
-    q = {}
-    e0 = hit[0]
-    for kind in ("gate", "up", "down"):
-        bits = synth.expert_torch(w, 0, e0, kind, device=dev).view(torch.int16).cpu().numpy().view(np.uint16)
-        q[kind] = mxfp4.quantize(bits)
-    seg = perm[offsets[e0]:offsets[e0 + 1]]
-    xr = xv[seg // w.top_k]
 
-    def expert_slice(frac):
-        ri, rh = max(1, int(w.inter * frac)), max(1, int(w.hidden * frac))
-        wg = mxfp4.dequantize(q["gate"][0][:ri], q["gate"][1][:ri])
-        wu = mxfp4.dequantize(q["up"][0][:ri], q["up"][1][:ri])
-        a = moe.silu(xr @ wg.T) * (xr @ wu.T)
-        full_a = np.zeros((xr.shape[0], w.inter))
-        full_a[:, :ri] = a
-        wd = mxfp4.dequantize(q["down"][0][:rh], q["down"][1][:rh])
-        return full_a @ wd.T
+    class _L:  # the two dense router tensors oracle_prepare reads
+        router_w, router_b = dense["router_w"], dense["router_b"]
 
-    t0 = time.perf_counter()
-    expert_slice(1.0)
-    t_expert = time.perf_counter() - t0
-    budget = 90.0
-    frac = min(1.0, max(1.0 / 64, budget / max(1, args.steps + args.warmup) / max(t_expert, 1e-6)))
-    for _ in range(args.warmup):
-        expert_slice(frac)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        expert_slice(frac)
-    el = time.perf_counter() - t0
-    layer_s = (el / args.steps) / frac * len(hit) * w.layers
+    prep = oracle_prepare(w, _L, x, n_experts=min(4, max(1, args.steps + args.warmup)))
+    experts = list(prep["q"])
+    for i in range(args.warmup):
+        oracle_step(w, prep, experts[i % len(experts)])
+    routes, times, steps_s = [], [], []
+    t_all = time.perf_counter()
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        r, e = oracle_step(w, prep, experts[i % len(experts)])
+        steps_s.append(time.perf_counter() - t0)
+        routes.append(r)
+        times.append(e)
+    wall = time.perf_counter() - t_all
+    hit = len(prep["hit"])
+    layer_s = (statistics.median(routes) + statistics.median(times) * hit) * w.layers
     value = T / layer_s
+    ms_step = wall * 1e3 / max(1, args.steps)
     out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": layer_s * 1e3, "higher_is_better": True,
+           "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "impl": "reference",
            "config": {"workload": w.name, "hidden": w.hidden, "inter": w.inter, "experts": w.experts,
                       "top_k": w.top_k, "tokens_per_gpu": T, "layers": w.layers},
+           "step": "measured: oracle routing of all %d tokens + one whole hit expert (of %d hit)" % (T, hit),
+           "value_basis": {"layer_s_extrapolated": layer_s, "route_s_median": statistics.median(routes),
+                           "expert_s_median": statistics.median(times), "hit_experts": hit,
+                           "layers": w.layers},
            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                            "sample": f"each step: dequantise + SwiGLU FFN of {frac:.3f} of the rows of one "
-                                      f"hit expert's projections; layer time extrapolated by rows and "
-                                      f"by {len(hit)} hit experts"},
+                            "cpu_model": cpu_model(), "cpu_count": os.cpu_count(),
+                            "sample": f"each step: the oracle's routing of the block + one of the first "
+                                      f"{len(experts)} hit experts in turn (measured); layer time = routing "
+                                      f"+ {hit} hit experts x the median expert time"},
            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
 
+def ishard_groups(inter: int, world: int):
+    """(group size g, groups): the largest g dividing `world` whose I-slices are multiples
+    of 128 (the engine's tiling); the world is then world / g groups of g ranks, each an
+    I-sharded layer on its own token blocks."""
+    for g in range(min(world, 8), 0, -1):
+        if world % g == 0 and inter % g == 0 and (inter // g) % 128 == 0:
+            return g, world // g
+    return 1, world
+
+
 def run_shard_i(args, mx, w, T, layers, rank, world):
-    """The I-sharded layer: every rank holds rows [r*I/N, (r+1)*I/N) of each expert's
-    gate/up matrices and the same down columns, streams them for the same token
-    block (moe_forward_partial), the fp32 partials are summed across ranks (NCCL
-    all-reduce) and rounded to bf16 (moe_round_bf16).  Strong scaling: a step is one
-    token block, whatever N."""
+    """The I-sharded layer: each rank of a group of g holds rows [r*I/g, (r+1)*I/g) of
+    every expert's gate/up matrices and the same down columns, and streams them for the
+    group's token block; the engine's last combine sums the g fp32 partials over NVLink
+    peer loads (moe_forward_ishard, one launch per step) and rounds to bf16.  With
+    --nccl-allreduce the partials are summed by an NCCL all-reduce between launches
+    (moe_forward_partial, all-reduce, moe_round_bf16).  Strong scaling within a group."""
     import torch
     import torch.distributed as dist
     if w.layers != 1:
         raise SystemExit("--shard-i: one layer per call")
-    shard = mx.shard_layer_i(layers[0], rank, world)
-    m = mx.Moe(w.hidden, w.inter // world, w.experts, w.top_k, T, [shard])
-    xs = token_blocks(w, T, args.batches, 0)  # the same token blocks on every rank
-    hits = []
-    for x in xs:
-        hits.append(int((m.moe_route(x, layer=0)["counts"] > 0).sum().item()))
+    g, groups = ishard_groups(w.inter, world)
+    my_group, grank = rank // g, rank % g
+    pgs = [dist.new_group(list(range(k * g, (k + 1) * g))) for k in range(groups)] if world > 1 else [None]
+    pg = pgs[my_group]
+    shard = mx.shard_layer_i(layers[0], grank, g)
+    m = mx.Moe(w.hidden, w.inter // g, w.experts, w.top_k, T, [shard])
+    xs = token_blocks(w, T, args.batches, my_group)  # the same token blocks within a group
+    hits = [int((m.moe_route(x, layer=0)["counts"] > 0).sum().item()) for x in xs]
     part = torch.empty((T, w.hidden), dtype=torch.float32, device="cuda")
     y = torch.empty((T, w.hidden), dtype=torch.bfloat16, device="cuda")
+    fused = not args.nccl_allreduce
+    opened = []
+    if fused:
+        if g > 1:
+            opened = mx.connect_ishard(m, pg)
+        else:
+            m.moe_ishard_attach(0, 1, [m.moe_ishard_region()[0]])
 
     def step(i):
-        m.moe_forward_partial(xs[i % len(xs)], part)
-        if world > 1:
-            dist.all_reduce(part)
-        mx.round_bf16(part, y)
+        if fused:
+            m.moe_forward_ishard(xs[i % len(xs)], y)
+        else:
+            m.moe_forward_partial(xs[i % len(xs)], part)
+            if g > 1:
+                dist.all_reduce(part, group=pg)
+            mx.round_bf16(part, y)
 
     for i in range(args.warmup):
         step(i)
@@ -660,26 +793,67 @@ def run_shard_i(args, mx, w, T, layers, rank, world):
     ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, "cuda")
     us_step = ms * 1e3 / args.steps
     mean_hit = float(np.mean([hits[i % len(hits)] for i in range(args.steps)]))
-    shard_w = synth.Workload(w.name, w.hidden, w.inter // world, w.experts, w.top_k, T)
+    shard_w = synth.Workload(w.name, w.hidden, w.inter // g, w.experts, w.top_k, T)
     alg = algorithmic_bytes(shard_w, T, mean_hit)
     peak, peak_kind = measured_peaks()
     achieved = alg / (us_step * 1e-6) / 1e9
+    # end to end: every step copies its token block from pinned host memory and its
+    # output back (the group's rank 0 would hand y on; every rank copies it here)
+    e2e = None
+    if not args.no_e2e:
+        xh = [x.cpu().pin_memory() for x in xs]
+        yh = torch.empty((T, w.hidden), dtype=torch.bfloat16).pin_memory()
+        xd = torch.empty_like(xs[0])
+        n_e2e = args.e2e_steps or max(args.steps, 100)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for i in range(n_e2e):
+            xd.copy_(xh[i % len(xh)], non_blocking=True)
+            if fused:
+                m.moe_forward_ishard(xd, y)
+            else:
+                m.moe_forward_partial(xd, part)
+                if g > 1:
+                    dist.all_reduce(part, group=pg)
+                mx.round_bf16(part, y)
+            yh.copy_(y, non_blocking=True)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        m.moe_status()
+        el = max_over_ranks(a0.elapsed_time(a1) / 1e3, dist if world > 1 else None, "cuda")
+        e2e = {"value": groups * T * n_e2e / el, "unit": "tokens/s", "steps": n_e2e,
+               "h2d_bytes_per_step": T * w.hidden * 2, "d2h_bytes_per_step": T * w.hidden * 2,
+               "api": "moe_forward_ishard on a device copy of pinned host tokens, output copied back"
+                      if fused else "moe_forward_partial + all-reduce + moe_round_bf16, host copies each step"}
+    if world > 1:
+        dist.barrier()
+    for b in opened:
+        mx.moe_ishard_ipc_close(b)
     if rank == 0:
+        how = ("one launch per step: moe_forward_ishard (engine + fused all-reduce over peer loads)" if fused else
+               "stream launches: moe_forward_partial, NCCL all-reduce, moe_round_bf16")
         print(json.dumps({
-            "metric": METRIC, "value": T / (us_step * 1e-6), "unit": "tokens/s", "n_gpus": world,
+            "metric": METRIC, "value": groups * T / (us_step * 1e-6), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": us_step / 1e3, "higher_is_better": True,
-            "scaling": "strong", "vs_baseline": None, "dtype": "mxfp4-w/fp32-acc",
+            "scaling": "strong" if groups == 1 else "weak", "vs_baseline": None, "dtype": "mxfp4-w/fp32-acc",
             "data": "synthetic (seeded N(0,0.02) expert weights quantised to MXFP4, N(0,1) bf16 tokens)",
             "config": {"workload": w.name if not args.tokens else f"{w.name}_t{T}", "hidden": w.hidden,
-                       "inter": w.inter, "inter_per_rank": w.inter // world, "experts": w.experts,
-                       "top_k": w.top_k, "tokens": T, "parallelism": f"I-sharded x{world} (NCCL all-reduce)",
-                       "launch": "stream launches: moe_forward_partial, all-reduce, moe_round_bf16"},
+                       "inter": w.inter, "inter_per_rank": w.inter // g, "experts": w.experts,
+                       "top_k": w.top_k, "tokens": T, "ishard_group": g, "groups": groups,
+                       "parallelism": f"I-sharded x{g}" + (f", {groups} groups on their own token blocks"
+                                                            if groups > 1 else ""),
+                       "allreduce": "fused (peer loads in the engine's last combine)" if fused else "NCCL",
+                       "launch": how},
             "layer_us": us_step,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_source": peak_kind,
                          "algorithmic_bytes_per_launch": alg, "traffic": None, "kernel": "engine_kernel",
                          "per": "rank (its I-slice of the hit experts)"},
-            "gpu_launches": 3 * args.steps, "e2e": None, "cpu_baseline": None, "clocks": clk}), flush=True)
+            "gpu_launches": (1 if fused else 3) * args.steps, "e2e": e2e, "cpu_baseline": None,
+            "clocks": clk}), flush=True)
     m.close()
     if world > 1:
         dist.destroy_process_group()

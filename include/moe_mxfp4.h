@@ -169,6 +169,50 @@ MOE_API int32_t moe_forward_partial(moe_mxfp4_t* h, const void* x_bf16, int32_t 
                                     void* stream);
 
 /*
+ * The I-sharded layer with a fused one-shot all-reduce.  The pages' deployment
+ * is one node of 8 GPUs (HyperAI salon transcript "Speed is Intelligence",
+ * GLM-5.1 case; bjdmk.com.cn news, section "1T模型，千token每秒"); splitting
+ * every expert's intermediate dimension over the GPUs gives each the same
+ * share of every hit expert's bytes whatever the routing skew, and leaves one
+ * exchange: the sum of the per-rank partial outputs.  Instead of a separate
+ * all-reduce launch, the engine's last combine does it: each rank writes its
+ * fp32 partial into its own region, publishes the call's epoch into every
+ * rank's region (system-scope release), waits until its own region holds the
+ * epoch from every rank (bounded; a timeout is MOE_ERR_TIMEOUT at moe_status),
+ * and sums the ranks' partials in rank order with plain loads of the peers'
+ * memory (NVLink), then rounds to bf16.  Every rank's y is bit-identical.
+ * No multicast copy is involved.
+ *
+ * Set-up, once per handle (a handle of num_layers == 1 built on the rank's
+ * I-slice, see moe_forward_partial):
+ *   moe_ishard_region      the handle's region: MAX_RANKS epoch words, then two
+ *                          slots of [max_tokens][hidden] fp32 (allocated and
+ *                          zeroed on the first call; synchronises the device).
+ *   moe_ishard_ipc_handle  its 64-byte CUDA IPC handle, to send to the peers.
+ *   moe_ishard_ipc_open    map a peer's region (from its handle) on the current
+ *                          device; moe_ishard_ipc_close unmaps it.
+ *   moe_ishard_attach      rank, world (1..8) and every rank's region as the
+ *                          current device addresses it (regions[rank] must be
+ *                          this handle's own); restarts the epochs and clears
+ *                          this region's epoch words (synchronises the device),
+ *                          so every rank must attach before any rank calls
+ *                          (a barrier over the ranks), also after a timeout.
+ * Then moe_forward_ishard(h, x, T, y) on every rank, the same calls in the same
+ * order (each call is one epoch).  x must be the same on every rank.  Errors:
+ * MOE_ERR_INVALID_ARG (null or misaligned pointers, rank/world out of range,
+ * not attached), MOE_ERR_UNSUPPORTED_SHAPE (num_layers != 1), MOE_ERR_OOM,
+ * MOE_ERR_CUDA.
+ */
+#define MOE_IPC_HANDLE_BYTES 64
+MOE_API int32_t moe_ishard_region(moe_mxfp4_t* h, void** base_out, uint64_t* bytes_out);
+MOE_API int32_t moe_ishard_ipc_handle(moe_mxfp4_t* h, void* handle_out);
+MOE_API int32_t moe_ishard_ipc_open(const void* handle, void** base_out);
+MOE_API int32_t moe_ishard_ipc_close(void* base);
+MOE_API int32_t moe_ishard_attach(moe_mxfp4_t* h, int32_t rank, int32_t world, void* const* regions);
+MOE_API int32_t moe_forward_ishard(moe_mxfp4_t* h, const void* x_bf16, int32_t T, void* y_bf16,
+                                   void* stream);
+
+/*
  * moe_round_bf16 -- out_bf16[i] = bf16(in_f32[i]) (round to nearest even) for
  * n device values on `stream`; the last step of an I-sharded layer, after the
  * partial outputs were summed.  Errors: MOE_ERR_INVALID_ARG (n < 0; null or
@@ -301,12 +345,14 @@ MOE_API void moe_mxfp4_destroy(moe_mxfp4_t* h);
  * kernel's shared-memory limit); make that first call before any stream
  * capture.  All calls share the array: calls whose kernels overlap on the GPU
  * race and give wrong outputs, so serialise them.  The call clears the words
- * that must start at zero itself.  Sizes whose working memory exceeds the
- * array (roughly T*(8*num_experts + 4*hidden) bytes) return
+ * that must start at zero itself.  The working memory of a call is
+ * 64*T*num_experts + 36*min(num_experts, T*top_k) + 17*T*top_k bytes plus
+ * under 2 KB of alignment (fp64 partial logits, unit tables, barrier words):
+ * T up to about 1000 at num_experts = 128, top_k = 8.  Larger sizes return
  * MOE_ERR_UNSUPPORTED_SHAPE; hidden must be a multiple of 128 (at most 8192),
  * num_experts <= 512, top_k <= min(num_experts, 32).  T == 0 is a no-op.
- * There is no status query: a device-side wait that times out leaves the
- * outputs undefined.
+ * A device-side wait that runs out (bound: 2 s, or env MOE_TIMEOUT_NS) leaves
+ * the outputs undefined; moe_route_static_status reports it.
  */
 #define MOE_ROUTE_STATIC_SCRATCH_BYTES (8u << 20)
 MOE_API int32_t moe_route_static(const void* x_bf16, int32_t T, int32_t hidden,
@@ -314,6 +360,16 @@ MOE_API int32_t moe_route_static(const void* x_bf16, int32_t T, int32_t hidden,
                                  int32_t num_experts, int32_t top_k, int32_t* topk_idx,
                                  float* topk_w, int32_t* counts, int32_t* offsets, int32_t* perm,
                                  int32_t* inv_perm, void* stream);
+
+/*
+ * moe_route_static_status -- synchronise `stream`, then return and clear the
+ * device-side status of the moe_route_static calls made on the current device:
+ * MOE_OK, or MOE_ERR_TIMEOUT if a bounded wait of the last such call ran out
+ * (its outputs are then undefined).  It allocates nothing either.  MOE_OK when
+ * no call was made on this device; MOE_ERR_CUDA if the synchronisation or the
+ * read of the status word fails.
+ */
+MOE_API int32_t moe_route_static_status(void* stream);
 
 /* moe_status_str -- static English text for a status code. */
 MOE_API const char* moe_status_str(int32_t status);

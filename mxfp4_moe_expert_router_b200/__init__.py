@@ -19,12 +19,16 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_OOM, MOE_ERR_CUD
 
 EXPORTS = ("mxfp4_quantize", "moe_mxfp4_create", "moe_route", "moe_forward", "moe_forward_host",
            "moe_status", "moe_set_timeout_ns", "moe_engine_grid", "moe_mxfp4_destroy",
-           "moe_status_str", "moe_route_static", "moe_phase_ns",
+           "moe_status_str", "moe_route_static", "moe_route_static_status", "moe_phase_ns",
            "moe_stream_profile", "moe_set_large_kind", "moe_forward_host_async", "moe_host_join",
            "moe_forward_ops", "spec_verify_workspace_bytes", "spec_verify", "spec_verify_status",
-           "spec_exp", "moe_forward_partial", "moe_round_bf16")
+           "spec_exp", "moe_forward_partial", "moe_round_bf16", "moe_ishard_region", "moe_ishard_ipc_handle",
+           "moe_ishard_ipc_open", "moe_ishard_ipc_close", "moe_ishard_attach", "moe_forward_ishard")
 
 MOE_OPS_PDL = 1
+MOE_ROUTE_STATIC_SCRATCH_BYTES = 8 << 20  # the header's static working memory of moe_route_static
+MOE_IPC_HANDLE_BYTES = 64
+AR_MAX_RANKS, AR_FLAG_BYTES = 8, 256  # layout of an I-shard region: epoch words, then two fp32 slots
 
 
 class MoeConfig(ctypes.Structure):
@@ -58,6 +62,12 @@ def _load():
         "moe_forward_ops": (i32, [vp, vp, i32, vp, vp, i32, vp]),
         "moe_forward_partial": (i32, [vp, vp, i32, vp, vp]),
         "moe_round_bf16": (i32, [vp, vp, i64, vp]),
+        "moe_ishard_region": (i32, [vp, ctypes.POINTER(vp), ctypes.POINTER(u64)]),
+        "moe_ishard_ipc_handle": (i32, [vp, vp]),
+        "moe_ishard_ipc_open": (i32, [vp, ctypes.POINTER(vp)]),
+        "moe_ishard_ipc_close": (i32, [vp]),
+        "moe_ishard_attach": (i32, [vp, i32, i32, pp]),
+        "moe_forward_ishard": (i32, [vp, vp, i32, vp, vp]),
         "moe_forward_host_async": (i32, [vp, vp, i32, vp, vp]),
         "moe_host_join": (i32, [vp, vp]),
         "moe_status": (i32, [vp, vp]),
@@ -69,6 +79,7 @@ def _load():
         "moe_stream_profile": (i32, [vp, i32, ctypes.POINTER(ctypes.c_uint64), i32, vp]),
         "moe_phase_ns": (i32, [vp, ctypes.POINTER(ctypes.c_uint64), i32, vp]),
         "moe_route_static": (i32, [vp, i32, i32, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_route_static_status": (i32, [vp]),
         "spec_verify_workspace_bytes": (i64, [i32, i32, i32]),
         "spec_verify": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, i64, vp]),
         "spec_verify_status": (i32, [vp, vp]),
@@ -198,6 +209,32 @@ class Moe:
                "moe_forward_partial")
         return y_f32
 
+    # -- I-sharded layer with the fused all-reduce ----------------------------------------------
+    def moe_ishard_region(self):
+        """(device address, bytes) of this handle's all-reduce region (allocated on first use)."""
+        base, n = ctypes.c_void_p(0), ctypes.c_uint64(0)
+        _check(lib.moe_ishard_region(self.handle, ctypes.byref(base), ctypes.byref(n)), "moe_ishard_region")
+        return int(base.value), int(n.value)
+
+    def moe_ishard_ipc_handle(self) -> bytes:
+        buf = ctypes.create_string_buffer(MOE_IPC_HANDLE_BYTES)
+        _check(lib.moe_ishard_ipc_handle(self.handle, buf), "moe_ishard_ipc_handle")
+        return buf.raw
+
+    def moe_ishard_attach(self, rank: int, world: int, regions):
+        """Every rank's region (device addresses as this GPU sees them; own at `rank`)."""
+        arr = (ctypes.c_void_p * world)(*[int(r) for r in regions])
+        _check(lib.moe_ishard_attach(self.handle, rank, world, ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))),
+               "moe_ishard_attach")
+
+    def moe_forward_ishard(self, x, y=None, stream=None):
+        import torch
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty((T, self.cfg.hidden), dtype=torch.bfloat16, device=x.device)
+        _check(lib.moe_forward_ishard(self.handle, _ptr(x), T, _ptr(y), _stream(stream)), "moe_forward_ishard")
+        return y
+
     def moe_forward_host(self, x_host, y_host=None, stream=None):
         import torch
         T = x_host.shape[0]
@@ -289,6 +326,71 @@ def moe_route_static(x, router_w, router_b, top_k, stream=None):
                                                          "perm", "inv_perm")], _stream(stream)),
            "moe_route_static")
     return out
+
+
+def moe_route_static_status(stream=None) -> int:
+    """Synchronise the stream; MOE_OK, or MOE_ERR_TIMEOUT (then cleared) if the last
+    ``moe_route_static`` call on the current device ran out of its wait bound."""
+    return int(lib.moe_route_static_status(_stream(stream)))
+
+
+def moe_ishard_ipc_open(handle: bytes) -> int:
+    """Map a peer's all-reduce region (its 64-byte IPC handle) on the current device."""
+    base = ctypes.c_void_p(0)
+    _check(lib.moe_ishard_ipc_open(ctypes.create_string_buffer(bytes(handle), MOE_IPC_HANDLE_BYTES),
+                                   ctypes.byref(base)), "moe_ishard_ipc_open")
+    return int(base.value)
+
+
+def moe_ishard_ipc_close(base: int):
+    _check(lib.moe_ishard_ipc_close(ctypes.c_void_p(base)), "moe_ishard_ipc_close")
+
+
+class _DeviceSpan:
+    """A raw device address range seen through __cuda_array_interface__ (no copy)."""
+
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr, "data": (int(ptr), False),
+                                         "version": 2, "strides": None}
+
+
+def region_views(base: int, max_tokens: int, hidden: int):
+    """Torch views of an I-shard region: (epoch words as int32 [8], partial slots fp32 [2][T][H])."""
+    import torch
+    flags = torch.as_tensor(_DeviceSpan(base, (AR_MAX_RANKS,), "<i4"), device="cuda")
+    parts = torch.as_tensor(_DeviceSpan(base + AR_FLAG_BYTES, (2, max_tokens, hidden), "<f4"), device="cuda")
+    return flags, parts
+
+
+def exchange_ipc_handles(handle: bytes, group=None) -> list:
+    """All ranks' IPC handles, in rank order (torch.distributed all-gather of the bytes)."""
+    import torch.distributed as dist
+    out = [None] * dist.get_world_size(group)
+    dist.all_gather_object(out, bytes(handle), group=group)
+    return [bytes(h) for h in out]
+
+
+def connect_ishard(m: "Moe", group=None, opener=None):
+    """Attach handle `m` (this rank's I-slice) to every rank's region: export this
+    rank's region, gather all handles, map the peers' regions (``opener``: the
+    mapping call, moe_ishard_ipc_open by default).  Returns the mapped peer
+    addresses (to close with moe_ishard_ipc_close when done)."""
+    import torch.distributed as dist
+    opener = opener or moe_ishard_ipc_open
+    rank, world = dist.get_rank(group), dist.get_world_size(group)
+    own, _ = m.moe_ishard_region()
+    handles = exchange_ipc_handles(m.moe_ishard_ipc_handle(), group)
+    regions, opened = [], []
+    for r, h in enumerate(handles):
+        if r == rank:
+            regions.append(own)
+        else:
+            b = opener(h)
+            opened.append(b)
+            regions.append(b)
+    m.moe_ishard_attach(rank, world, regions)
+    dist.barrier(group)  # every rank's epoch words are cleared before any rank publishes
+    return opened
 
 
 def moe_mxfp4_create(hidden, inter, num_experts, top_k, max_tokens, layers, rms_eps=1e-6,

@@ -49,6 +49,12 @@ namespace moe {
 namespace {
 
 constexpr uint32_t FULL = 0xFFFFFFFFu;
+// Bound of the drains before a CTA reuses or releases memory that bulk copies
+// or MMAs it already issued still target (the ring, tensor memory).  Issued
+// work completes on its own within microseconds, so this bound is fixed and
+// independent of the caller's wait bound: a short p.timeout_ns stops new work
+// early but never frees shared or tensor memory under work in flight.
+constexpr uint64_t DRAIN_NS = 2000000000ull;
 constexpr int SMALL_UNITS = 256 + SMALL_PAIRS / NT_MAX;
 constexpr int SMALL_DUNITS = 256 + SMALL_PAIRS / ND_MAX;
 
@@ -1362,7 +1368,7 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
   for (uint32_t s = rs.seq - n; s != rs.seq; ++s) {
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(full_bar(smem, pipe, (int)(s % NS)), (s / NS) & 1u)) {
-      if (globaltimer_ns() - t0 > p.timeout_ns) break;
+      if (globaltimer_ns() - t0 > DRAIN_NS) break;
     }
   }
 }
@@ -1902,13 +1908,13 @@ __device__ void stream_producer_f16(const EngineParams& p, const LayerPtrs& lp, 
     for (uint32_t r = rs.seq - nr; r != rs.seq; ++r) {
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(rawfull_bar(smem, (int)(r % FT_RA)), (r / FT_RA) & 1u))
-        if (globaltimer_ns() - t0 > p.timeout_ns) break;
+        if (globaltimer_ns() - t0 > DRAIN_NS) break;
     }
     const uint32_t nb = min(rs.sfc - b_start, (uint32_t)FT_NB);
     for (uint32_t b = rs.sfc - nb; b != rs.sfc; ++b) {
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(bfull_bar(smem, (int)(b % FT_NB)), (b / FT_NB) & 1u))
-        if (globaltimer_ns() - t0 > p.timeout_ns) break;
+        if (globaltimer_ns() - t0 > DRAIN_NS) break;
     }
   }
   __syncwarp();
@@ -2175,44 +2181,177 @@ __device__ void phase_combine_out(const EngineParams& p, const int32_t* inv) {
   }
 }
 
-// Per token (one CTA each): y = bf16(combine); x_next = bf16(y / sqrt(mean(y^2) + eps)).
-__device__ void phase_combine_rmsnorm(const EngineParams& p, const int32_t* inv, uint8_t* smem) {
-  CtaTables& tb = tables(smem);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int MAXV = (8192 / 4 + THREADS - 1) / THREADS;
-  for (int t = blockIdx.x; t < p.T; t += gridDim.x) {
-    float4 yv[MAXV];
-    float ss = 0.f;
-#pragma unroll
-    for (int i = 0; i < MAXV; ++i) {
-      const int h = (threadIdx.x + i * THREADS) * 4;
-      if (h < p.H) {
-        float4 s = combine4(p, inv, t, h);
-        s.x = __bfloat162float(__float2bfloat16_rn(s.x));
-        s.y = __bfloat162float(__float2bfloat16_rn(s.y));
-        s.z = __bfloat162float(__float2bfloat16_rn(s.z));
-        s.w = __bfloat162float(__float2bfloat16_rn(s.w));
-        yv[i] = s;
-        ss += s.x * s.x + s.y * s.y + s.z * s.z + s.w * s.w;
+// I-sharded layer, last step: the fused one-shot all-reduce (see AllReduce in
+// engine.cuh).  This rank's fp32 partial (the slot-order combine) goes to slot
+// epoch % 2 of its own region; after a grid barrier CTA 0 publishes the epoch
+// to every rank (system-scope release); every CTA waits, bounded, until every
+// rank's epoch is in its own region (system-scope acquire), then sums its
+// share of [T][H] over the ranks in rank order -- the same operations on
+// every rank, so every rank's y is bit-identical -- and rounds to bf16.
+// Returns false (every thread of the CTA) on a timeout or a recorded error.
+__device__ bool phase_allreduce_out(const EngineParams& p, const int32_t* inv, int layer) {
+  const int64_t gt = (int64_t)blockIdx.x * THREADS + threadIdx.x;
+  const int64_t gs = (int64_t)gridDim.x * THREADS;
+  const int H4 = p.H / 4, world = p.ar.world, rank = p.ar.rank;
+  const uint32_t epoch = p.ar.epoch;
+  const int64_t slot = (int64_t)(epoch & 1u) * p.ar.slot_floats;
+  float* mine = reinterpret_cast<float*>(p.ar.region[rank] + AR_FLAG_BYTES) + slot;
+  for (int64_t g = gt; g < (int64_t)p.T * H4; g += gs) {
+    const int t = (int)(g / H4), h = (int)(g % H4) * 4;
+    *reinterpret_cast<float4*>(mine + (int64_t)t * p.H + h) = combine4(p, inv, t, h);
+  }
+  if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 8)) return false;
+  if (blockIdx.x == 0 && (int)threadIdx.x < world) {
+    // the barrier acquired every CTA's partial; make it visible system-wide
+    // before the epoch
+    __threadfence_system();
+    st_release_sys_u32(reinterpret_cast<uint32_t*>(p.ar.region[threadIdx.x]) + rank, epoch);
+  }
+  int ok = 1;
+  if (threadIdx.x == 0) {
+    const uint32_t* flags = reinterpret_cast<const uint32_t*>(p.ar.region[rank]);
+    const uint64_t t0 = globaltimer_ns();
+    for (int r = 0; r < world && ok; ++r) {
+      uint32_t spins = 0;
+      while (ld_acquire_sys_u32(flags + r) < epoch) {
+        if ((++spins & 15u) == 0u) {
+          if (error_set(p.sync)) { ok = 0; break; }
+          if (globaltimer_ns() - t0 > p.timeout_ns) { set_error(p.sync, DEV_TIMEOUT_PEER, (uint32_t)r); ok = 0; break; }
+        }
+        __nanosleep(64);
       }
     }
+  }
+  if (!__syncthreads_and(ok)) return false;
+  __nv_bfloat16* dump = p.layer_io ? p.layer_io + (int64_t)p.L * p.T * p.H : nullptr;
+  for (int64_t g = gt; g < (int64_t)p.T * H4; g += gs) {
+    const int t = (int)(g / H4), h = (int)(g % H4) * 4;
+    const int64_t off = slot + (int64_t)t * p.H + h;
+    float4 s = ld_volatile_f4(reinterpret_cast<const float*>(p.ar.region[0] + AR_FLAG_BYTES) + off);
+    for (int r = 1; r < world; ++r) {
+      const float4 v = ld_volatile_f4(reinterpret_cast<const float*>(p.ar.region[r] + AR_FLAG_BYTES) + off);
+      s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    }
+    store_bf16x4(p.y_out + (int64_t)t * p.H + h, s);
+    if (dump) store_bf16x4(dump + (int64_t)t * p.H + h, s);
+  }
+  return true;
+}
+
+// RMSNorm between chained layers: y = bf16(combine); x_next = bf16(y * r),
+// r = 1 / sqrt(mean(y^2) + eps).  A token's H values are cut into RMS_CHUNKS
+// chunks.  The sum of squares of a chunk is reduced in a fixed order (each
+// thread one float4, then the warp, then the warps in order), and a token's
+// sum is its chunk sums added in chunk order, so the result does not depend
+// on how chunks are spread over CTAs.  The engine spreads the T * RMS_CHUNKS
+// chunks over the whole grid (partial sums, a grid barrier, then the scaling
+// of each chunk); the operator-by-operator launch runs all chunks of a token
+// in one CTA.  Both give the same bits.
+constexpr int RMS_CHUNKS = 16;
+static_assert(8192 / RMS_CHUNKS / 4 <= THREADS, "one float4 of a chunk per thread");
+
+// The bf16-rounded combine of this thread's float4 of chunk c of token t (zero
+// past the chunk), and its sum of squares.
+__device__ __forceinline__ float4 rms_chunk_values(const EngineParams& p, const int32_t* inv, int t, int c,
+                                                   bool& mine) {
+  const int cl4 = p.H / RMS_CHUNKS / 4;
+  mine = (int)threadIdx.x < cl4;
+  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (mine) {
+    s = combine4(p, inv, t, c * (p.H / RMS_CHUNKS) + 4 * (int)threadIdx.x);
+    s.x = __bfloat162float(__float2bfloat16_rn(s.x));
+    s.y = __bfloat162float(__float2bfloat16_rn(s.y));
+    s.z = __bfloat162float(__float2bfloat16_rn(s.z));
+    s.w = __bfloat162float(__float2bfloat16_rn(s.w));
+  }
+  return s;
+}
+
+// Sum of squares of chunk c of token t, fixed reduction order; every thread
+// of the CTA gets the result.  Also returns this thread's values.
+__device__ float rms_chunk_ss(const EngineParams& p, const int32_t* inv, int t, int c, float* red,
+                              float4& v, bool& mine) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = rms_chunk_values(p, inv, t, c, mine);
+  float ss = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(FULL, ss, o);
-    if (lane == 0) tb.red[warp] = ss;
-    __syncthreads();
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(FULL, ss, o);
+  __syncthreads();  // red is free
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < WARPS; ++w) tot += red[w];
+  return tot;
+}
+
+__device__ __forceinline__ void rms_chunk_store(const EngineParams& p, int t, int c, float4 v, bool mine, float r) {
+  if (mine)
+    store_bf16x4(p.xnext + (int64_t)t * p.H + c * (p.H / RMS_CHUNKS) + 4 * (int)threadIdx.x,
+                 make_float4(v.x * r, v.y * r, v.z * r, v.w * r));
+}
+
+__device__ __forceinline__ float rms_scale(const EngineParams& p, float tot) {
+  return 1.0f / sqrtf(tot / (float)p.H + p.rms_eps);
+}
+
+// Engine, step 1 of 2: the chunk sums of squares of every (token, chunk) task,
+// spread over the grid, into part[t * RMS_CHUNKS + c].
+__device__ void phase_rms_partials(const EngineParams& p, const int32_t* inv, float* part, uint8_t* smem) {
+  CtaTables& tb = tables(smem);
+  for (int task = blockIdx.x; task < p.T * RMS_CHUNKS; task += gridDim.x) {
+    float4 v;
+    bool mine;
+    const float ss = rms_chunk_ss(p, inv, task / RMS_CHUNKS, task % RMS_CHUNKS, tb.red, v, mine);
+    if (threadIdx.x == 0) part[task] = ss;
+  }
+}
+
+// Engine, step 2 of 2 (after a grid barrier): each token's sum from its chunk
+// sums in chunk order, then the scaled bf16 values of every task's chunk.
+__device__ void phase_rms_apply(const EngineParams& p, const int32_t* inv, const float* part) {
+  for (int task = blockIdx.x; task < p.T * RMS_CHUNKS; task += gridDim.x) {
+    const int t = task / RMS_CHUNKS, c = task % RMS_CHUNKS;
     float tot = 0.f;
 #pragma unroll
-    for (int w = 0; w < WARPS; ++w) tot += tb.red[w];
-    const float r = 1.0f / sqrtf(tot / (float)p.H + p.rms_eps);
-#pragma unroll
-    for (int i = 0; i < MAXV; ++i) {
-      const int h = (threadIdx.x + i * THREADS) * 4;
-      if (h < p.H) {
-        const float4 s = yv[i];
-        store_bf16x4(p.xnext + (int64_t)t * p.H + h, make_float4(s.x * r, s.y * r, s.z * r, s.w * r));
-      }
+    for (int q = 0; q < RMS_CHUNKS; ++q) tot += __ldcg(part + t * RMS_CHUNKS + q);
+    bool mine;
+    const float4 v = rms_chunk_values(p, inv, t, c, mine);
+    rms_chunk_store(p, t, c, v, mine, rms_scale(p, tot));
+  }
+}
+
+// Operator-by-operator launch: every chunk of a token in one CTA (tokens over
+// the CTAs), the same arithmetic in the same order as the two engine steps.
+__device__ void phase_combine_rmsnorm(const EngineParams& p, const int32_t* inv, uint8_t* smem) {
+  CtaTables& tb = tables(smem);
+  for (int t = blockIdx.x; t < p.T; t += gridDim.x) {
+    float tot = 0.f;
+    for (int c = 0; c < RMS_CHUNKS; ++c) {
+      float4 v;
+      bool mine;
+      tot += rms_chunk_ss(p, inv, t, c, tb.red, v, mine);
+    }
+    const float r = rms_scale(p, tot);
+    for (int c = 0; c < RMS_CHUNKS; ++c) {
+      bool mine;
+      const float4 v = rms_chunk_values(p, inv, t, c, mine);
+      rms_chunk_store(p, t, c, v, mine, r);
     }
     __syncthreads();
+  }
+}
+
+// L2 prefetch of this CTA's 1/gridDim share of `bytes` (a multiple of 16) at
+// `base` (16-byte aligned), in bulk prefetches of at most 16 KB.
+__device__ void prefetch_share(const void* base, size_t bytes) {
+  const size_t share = ((bytes + gridDim.x - 1) / gridDim.x + 15) & ~size_t(15);
+  const size_t b0 = (size_t)blockIdx.x * share;
+  if (b0 >= bytes) return;
+  const size_t b1 = b0 + share < bytes ? b0 + share : bytes;
+  for (size_t o = b0; o < b1; o += 16384) {
+    const size_t n = b1 - o < 16384 ? b1 - o : 16384;
+    prefetch_l2_bulk(static_cast<const uint8_t*>(base) + o, (uint32_t)n);
   }
 }
 
@@ -2264,6 +2403,11 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
       inv = p.inv;
     }
     if (st) st[4] = globaltimer_ns();
+    // the next layer's router weights go to L2 while this layer streams (its
+    // expert weights are evict-first, so they stay): every CTA prefetches its
+    // share, a few tens of KB, without waiting for it
+    if (layer + 1 < p.L && threadIdx.x == 32 * (WARPS - 1))
+      prefetch_share(p.layers[layer + 1].router_w, (size_t)p.E * p.H * 4);
     fence_proxy_async_smem();  // the ring held routing scratch written by generic stores
     __syncthreads();
     if constexpr (MODE == 0) {  // two pipelines per CTA, units of <= NT_MAX positions
@@ -2305,8 +2449,15 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
     // itself: the count restarts for the next layer or launch
     if (blockIdx.x == 0 && threadIdx.x == 0) p.sync[SY_XDONE] = 0u;
     if (layer + 1 < p.L) {
-      phase_combine_rmsnorm(p, inv, smem);
+      // the partial logits are not read again in this layer: they hold the
+      // chunk sums of squares until the next layer's router overwrites them
+      float* part = reinterpret_cast<float*>(p.logits);
+      phase_rms_partials(p, inv, part, smem);
+      if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 7)) return;
+      phase_rms_apply(p, inv, part);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 5)) return;
+    } else if (p.ar.world > 0) {
+      if (!phase_allreduce_out(p, inv, layer)) return;
     } else {
       phase_combine_out(p, inv);
     }
@@ -2408,7 +2559,7 @@ __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p
       tc_commit(db);
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(db, 0u)) {
-        if (globaltimer_ns() - t0 > p.timeout_ns) { set_error(p.sync, DEV_TIMEOUT_PIPE, 0xFFFFu); break; }
+        if (globaltimer_ns() - t0 > DRAIN_NS) { set_error(p.sync, DEV_TIMEOUT_PIPE, 0xFFFFu); break; }
       }
     }
     __syncwarp();

@@ -152,7 +152,7 @@ enum : int {
 // device-side error codes (status word)
 enum : uint32_t {
   DEV_OK = 0, DEV_TIMEOUT_BARRIER = 1, DEV_TIMEOUT_PIPE = 2, DEV_TIMEOUT_READY = 3,
-  DEV_TIMEOUT_QUEUE = 4, DEV_TIMEOUT_IMAGES = 5,
+  DEV_TIMEOUT_QUEUE = 4, DEV_TIMEOUT_IMAGES = 5, DEV_TIMEOUT_PEER = 6,
 };
 
 // Upper bounds of the unit tables for T*K pairs over E experts.
@@ -170,6 +170,29 @@ struct LayerPtrs {
   const float* router_w;  // [E][H]
   const float* router_b;  // [E] or null
 };
+
+// ---- I-sharded layer with the fused one-shot all-reduce --------------------------------
+// Every rank owns one region in its own memory: MAX_RANKS epoch words (the
+// flag rank r last published into this region, at word r), padded to
+// AR_FLAG_BYTES, then two slots of [max_tokens][H] fp32 partial outputs.
+// A call of epoch e (1, 2, ... on every rank alike) writes this rank's
+// partial into slot e % 2 of its own region, publishes e into word `rank` of
+// every rank's region, waits until its own region holds e (or more) from
+// every rank, then sums the ranks' slot e % 2 in rank order (peer loads) and
+// rounds to bf16.  Two slots suffice: a rank can write slot e % 2 again only
+// at epoch e + 2, after every rank has published epoch e + 1, which each does
+// only after it finished reading epoch e.
+constexpr int MAX_RANKS = 8;
+constexpr int AR_FLAG_BYTES = 256;
+struct AllReduce {
+  int rank, world;            // world == 0: not an I-sharded call
+  uint32_t epoch;
+  int64_t slot_floats;        // floats per partial slot (max_tokens * H)
+  uint8_t* region[MAX_RANKS]; // every rank's region, as this GPU addresses it (own: local)
+};
+__host__ __device__ inline size_t ar_region_bytes(int64_t max_tokens, int H) {
+  return AR_FLAG_BYTES + 2 * (size_t)max_tokens * H * 4;
+}
 
 struct EngineParams {
   int H, I, E, K, T, TK, L;  // hidden, inter, experts, top_k, tokens, T*K, layers to run
@@ -206,6 +229,7 @@ struct EngineParams {
   uint32_t* sync;             // see SY_*
   uint64_t* stamps;           // null or [1 + MAX_LAYERS * STAMPS_PER_LAYER] %globaltimer ns (CTA 0)
   unsigned long long* prof;   // null or [PROF_COUNTERS] summed SM-clock cycles (stream phase)
+  AllReduce ar;               // I-sharded layer: the fused all-reduce of the last combine
   int op;                     // operator-by-operator launches: the OP_* this launch runs (0: whole engine)
   int op_layer;               // ... and its layer
 };

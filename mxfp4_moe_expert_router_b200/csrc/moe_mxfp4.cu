@@ -45,6 +45,14 @@ struct moe_mxfp4 {
   cudaStream_t h2d = nullptr, d2h = nullptr;
   cudaEvent_t ev_in[2] = {}, ev_k[2] = {}, ev_out[2] = {};
   uint64_t host_seq = 0;
+  // I-sharded layer with the fused all-reduce: this handle's region (own
+  // allocation, so that it can be exported by CUDA IPC), every rank's region
+  // as this GPU addresses it, and the epoch of the last call
+  uint8_t* ar_region = nullptr;
+  size_t ar_bytes = 0;
+  int ar_rank = -1, ar_world = 0;
+  uint32_t ar_epoch = 0;
+  uint8_t* ar_regions[MAX_RANKS] = {};
   std::vector<void*> allocs;
 };
 
@@ -342,6 +350,100 @@ int32_t moe_forward_partial(moe_mxfp4_t* h, const void* x_bf16, int32_t T, float
                             static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
+}
+
+int32_t moe_ishard_region(moe_mxfp4_t* h, void** base_out, uint64_t* bytes_out) {
+  if (!h || !base_out || !bytes_out) return MOE_ERR_INVALID_ARG;
+  if (h->cfg.num_layers != 1) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!h->ar_region) {
+    const size_t bytes = ar_region_bytes(h->cfg.max_tokens, h->cfg.hidden);
+    void* p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) { cudaGetLastError(); return MOE_ERR_OOM; }
+    if (cudaMemset(p, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+      cudaFree(p);
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    h->allocs.push_back(p);
+    h->ar_region = static_cast<uint8_t*>(p);
+    h->ar_bytes = bytes;
+  }
+  *base_out = h->ar_region;
+  *bytes_out = h->ar_bytes;
+  return MOE_OK;
+}
+
+int32_t moe_ishard_ipc_handle(moe_mxfp4_t* h, void* handle_out) {
+  if (!h || !handle_out) return MOE_ERR_INVALID_ARG;
+  void* base = nullptr;
+  uint64_t bytes = 0;
+  const int32_t st = moe_ishard_region(h, &base, &bytes);
+  if (st != MOE_OK) return st;
+  cudaIpcMemHandle_t ipc;
+  static_assert(sizeof(ipc) == MOE_IPC_HANDLE_BYTES, "IPC handle size");
+  if (cudaIpcGetMemHandle(&ipc, base) != cudaSuccess) { cudaGetLastError(); return MOE_ERR_CUDA; }
+  std::memcpy(handle_out, &ipc, sizeof(ipc));
+  return MOE_OK;
+}
+
+int32_t moe_ishard_ipc_open(const void* handle, void** base_out) {
+  if (!handle || !base_out) return MOE_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t ipc;
+  std::memcpy(&ipc, handle, sizeof(ipc));
+  void* p = nullptr;
+  if (cudaIpcOpenMemHandle(&p, ipc, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+    cudaGetLastError();
+    *base_out = nullptr;
+    return MOE_ERR_CUDA;
+  }
+  *base_out = p;
+  return MOE_OK;
+}
+
+int32_t moe_ishard_ipc_close(void* base) {
+  if (!base) return MOE_ERR_INVALID_ARG;
+  if (cudaIpcCloseMemHandle(base) != cudaSuccess) { cudaGetLastError(); return MOE_ERR_CUDA; }
+  return MOE_OK;
+}
+
+int32_t moe_ishard_attach(moe_mxfp4_t* h, int32_t rank, int32_t world, void* const* regions) {
+  if (!h || !regions || world < 1 || world > MAX_RANKS || rank < 0 || rank >= world) return MOE_ERR_INVALID_ARG;
+  if (h->cfg.num_layers != 1) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!h->ar_region || regions[rank] != h->ar_region) return MOE_ERR_INVALID_ARG;
+  for (int r = 0; r < world; ++r)
+    if (!regions[r] || !aligned16(regions[r])) return MOE_ERR_INVALID_ARG;
+  // epochs restart at 1: clear the epoch words the peers publish into
+  if (cudaMemset(h->ar_region, 0, AR_FLAG_BYTES) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  for (int r = 0; r < MAX_RANKS; ++r) h->ar_regions[r] = r < world ? static_cast<uint8_t*>(regions[r]) : nullptr;
+  h->ar_rank = rank;
+  h->ar_world = world;
+  h->ar_epoch = 0;
+  return MOE_OK;
+}
+
+int32_t moe_forward_ishard(moe_mxfp4_t* h, const void* x_bf16, int32_t T, void* y_bf16, void* stream) {
+  if (!h || T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (h->ar_world < 1) return MOE_ERR_INVALID_ARG;  // not attached
+  if (T == 0) return MOE_OK;
+  if (!x_bf16 || !y_bf16 || !aligned16(x_bf16) || !aligned16(y_bf16)) return MOE_ERR_INVALID_ARG;
+  const size_t bytes = (size_t)T * h->cfg.hidden * 2;
+  const char* xa = static_cast<const char*>(x_bf16);
+  const char* ya = static_cast<const char*>(y_bf16);
+  if (xa < ya + bytes && ya < xa + bytes) return MOE_ERR_INVALID_ARG;
+  EngineParams p = base_params(h, T);
+  p.x_in = static_cast<const __nv_bfloat16*>(x_bf16);
+  p.y_out = static_cast<__nv_bfloat16*>(y_bf16);
+  p.ar.rank = h->ar_rank;
+  p.ar.world = h->ar_world;
+  p.ar.epoch = h->ar_epoch + 1;
+  p.ar.slot_floats = (int64_t)h->cfg.max_tokens * h->cfg.hidden;
+  for (int r = 0; r < MAX_RANKS; ++r) p.ar.region[r] = h->ar_regions[r];
+  if (engine_launch(p, h->grid, static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  h->ar_epoch = p.ar.epoch;
+  return MOE_OK;
 }
 
 int32_t moe_round_bf16(const float* in_f32, void* out_bf16, int64_t n, void* stream) {

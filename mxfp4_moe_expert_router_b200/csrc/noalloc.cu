@@ -140,3 +140,35 @@ extern "C" MOE_API int32_t moe_route_static(const void* x_bf16, int32_t T, int32
   if (cudaMemsetAsync(p.sync, 0, SY_READY * sizeof(uint32_t), cs) != cudaSuccess) return MOE_ERR_CUDA;
   return engine_launch(p, grid, cs) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
+
+// The status word of the routing kernel sits at the start of the array (the
+// sync region is at offset 0 for every size), so its address does not depend
+// on the sizes of the last call.
+extern "C" MOE_API int32_t moe_route_static_status(void* stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return MOE_ERR_DEVICE; }
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_DEVICE;
+  void* base = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    base = g_scratch_ptr[dev];
+  }
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(cs) != cudaSuccess) { cudaGetLastError(); return MOE_ERR_CUDA; }
+  if (!base) return MOE_OK;  // no call on this device yet
+  uint32_t* sync = static_cast<uint32_t*>(base);
+  uint32_t words[2] = {};
+  static_assert(SY_ERRINFO == SY_ERROR + 1, "status and info words are adjacent");
+  if (cudaMemcpyAsync(words, sync + SY_ERROR, sizeof(words), cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
+      cudaStreamSynchronize(cs) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  if (words[0] == DEV_OK) return MOE_OK;
+  if (cudaMemsetAsync(sync, 0, SY_READY * sizeof(uint32_t), cs) != cudaSuccess ||
+      cudaStreamSynchronize(cs) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return MOE_ERR_TIMEOUT;
+}

@@ -154,3 +154,19 @@ def test_partial_and_round_argument_errors(mx):
     assert mx.lib.moe_round_bf16(None, p, 4, None) == mx.MOE_ERR_INVALID_ARG
     assert mx.lib.moe_round_bf16(ctypes.c_void_p((1 << 20) + 2), p, 4, None) == mx.MOE_ERR_INVALID_ARG
     assert mx.lib.moe_round_bf16(None, None, 0, None) == mx.MOE_OK
+
+
+def test_route_static_size_formula_on_the_host(mx):
+    """The header's working-memory formula of moe_route_static: the first T beyond it is
+    refused before any device work (so this runs without a GPU)."""
+    p = ctypes.c_void_p(1 << 20)
+    limit = mx.MOE_ROUTE_STATIC_SCRATCH_BYTES
+    for H, E, k in [(256, 16, 4), (4096, 128, 8), (7168, 256, 8)]:
+        T = 1
+        while 64 * T * E + 36 * min(E, T * k) + 17 * T * k <= limit:
+            T += 1
+        assert mx.lib.moe_route_static(p, T, H, p, None, E, k, p, p, p, p, p, p, None) == \
+            mx.MOE_ERR_UNSUPPORTED_SHAPE, (H, E, k, T)
+    import torch
+    if not torch.cuda.is_available():  # no device: the status query has nothing to report
+        assert mx.lib.moe_route_static_status(None) in (mx.MOE_OK, mx.MOE_ERR_DEVICE, mx.MOE_ERR_CUDA)

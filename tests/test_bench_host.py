@@ -59,3 +59,33 @@ def test_moe_reference_arm_prints_the_contract_line():
     assert d["metric"] == bench.METRIC and d["config"]["workload"] == "tiny_h256_e8"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_roofline_bound_follows_the_intensity():
+    """Tensor roofline where the tile stream's intensity exceeds its kind's ridge (the sweep at
+    T = 4608), HBM below it (T = 576) and on the verify-block path."""
+    w = synth.WORKLOADS["sweep_h7168_e256"]
+    by = lambda T: bench.algorithmic_bytes(w, T, 256)
+    r = bench.roofline(w.with_tokens(4608), 4608, by(4608), 13.0, "mxf4", None)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    flops = 6.0 * 4608 * 8 * 7168 * 2048 + 2.0 * 4608 * 7168 * 256
+    assert r["algorithmic_flop_per_launch"] == pytest.approx(flops)
+    assert r["achieved"] == pytest.approx(flops / 13.0e-3 / 1e12)
+    bf16, _ = bench.measured_bf16_tflops()
+    assert r["peak"] == pytest.approx(4.0 * bf16)
+    assert bench.roofline(w.with_tokens(576), 576, by(576), 2.3, "mxf4", None)["bound"] == "hbm"
+    d = synth.WORKLOADS["decode_t9_h4096_e128"]
+    r = bench.roofline(d, 9, bench.algorithmic_bytes(d, 9, 57), 0.11, "mxf4", 1.0)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["traffic"] == 1.0
+
+
+def test_ishard_groups_keep_slices_on_the_engine_tiling():
+    assert bench.ishard_groups(1536, 1) == (1, 1)
+    assert bench.ishard_groups(1536, 2) == (2, 1)
+    assert bench.ishard_groups(1536, 4) == (4, 1)
+    assert bench.ishard_groups(1536, 8) == (4, 2)   # 1536 / 8 = 192 is not a multiple of 128
+    assert bench.ishard_groups(2048, 8) == (8, 1)
+    for inter in (1536, 2048):
+        for world in (1, 2, 3, 4, 6, 8):
+            g, groups = bench.ishard_groups(inter, world)
+            assert g * groups == world and (inter // g) % 128 == 0 and inter % g == 0

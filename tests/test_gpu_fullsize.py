@@ -1,13 +1,19 @@
-"""Parity at the full workload sizes, on sampled tokens.
+"""Parity at the full workload sizes.
 
-The GPU runs whole layers at the bench and parity sizes.
-- The oracle recomputes a few sampled tokens one by one.
-- It quantises the same seeded bf16 expert weights itself (nothing it uses comes
-  from the CUDA path), and checks that the GPU's codes and scales for those
-  experts are bit-identical.
-- It routes the sampled tokens in fp64 and evaluates their SwiGLU experts.
-- It compares each token's y row within the tolerance (the rms term over the
-  sampled rows).
+The GPU runs whole layers at the bench and parity sizes, then:
+- the routing of EVERY token is compared with the oracle's fp64 routing
+  (indices bit-exact except near ties, which are counted and must stay rare;
+  counts, offsets, perm and inv bit-exact; weights within 1e-5);
+- the output rows of sampled tokens are recomputed by the oracle one by one.
+  The oracle quantises the same seeded bf16 expert weights itself (nothing it
+  uses comes from the CUDA path), checks that the GPU's codes and scales of
+  those experts are bit-identical, and evaluates the sampled tokens' SwiGLU
+  experts expert by expert (a few experts in memory at a time).  Each row is
+  compared within the tolerance, the rms term over the sampled rows.
+Sampling: every token of the verify-block workloads (T = 9, every layer of
+the chain teacher-forced), and 16 tokens spread over the block for T >= 72,
+which puts sampled pairs in interior tiles and in both epilogue sets of the
+tile stream (checked).
 
 The oracle's quantiser runs in a spawn process pool.
 """
@@ -22,6 +28,8 @@ from oracle import moe, mxfp4
 from tests.helpers import tolerance_ok, x_values
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+LT_MAX = 38  # positions per tile of the tile stream (engine.cuh)
 
 
 def _quantize_bits(bits):
@@ -52,116 +60,155 @@ def _bits(t):
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-class ExpertCache:
-    """Oracle MXFP4 weights of one layer, quantised on demand and checked against the GPU's."""
+def sample_tokens(T: int, n: int = 16) -> list:
+    """Every token up to n, else n tokens spread evenly over [0, T) (first and last included)."""
+    if T <= n:
+        return list(range(T))
+    return sorted({int(v) for v in np.linspace(0, T - 1, n)})
 
-    def __init__(self, w, layer, gpu_layer, pool):
-        self.w, self.layer, self.g, self.pool, self.dense = w, layer, gpu_layer, pool, {}
 
-    def need(self, experts):
-        todo = [e for e in experts if e not in self.dense]
-        jobs = [(e, kind) for e in todo for kind in ("gate", "up", "down")]
-        bits = [_bits(synth.expert_torch(self.w, self.layer, e, kind, seed=0)) for e, kind in jobs]
-        res = self.pool.map(_quantize_bits, bits)
-        gpu = {"gate": (self.g.gate_codes, self.g.gate_scales), "up": (self.g.up_codes, self.g.up_scales),
-               "down": (self.g.down_codes, self.g.down_scales)}
+def oracle_rows(pool, w, layer, gpu_layer, xv, tokens, idx, wts, chunk=8):
+    """fp64 layer output rows of the sampled tokens (their routing idx/wts given).
+
+    Expert by expert, `chunk` experts at a time: the oracle quantises the
+    seeded bf16 weights, checks the GPU's codes and scales bit for bit,
+    dequantises, and adds each routed pair's weighted SwiGLU output; the k
+    contributions of a row are summed in slot order."""
+    users = {}
+    for j in range(len(tokens)):
+        for slot, e in enumerate(idx[j]):
+            users.setdefault(int(e), []).append((j, slot))
+    contrib = np.zeros((len(tokens), w.top_k, w.hidden))
+    gpu = {"gate": (gpu_layer.gate_codes, gpu_layer.gate_scales), "up": (gpu_layer.up_codes, gpu_layer.up_scales),
+           "down": (gpu_layer.down_codes, gpu_layer.down_scales)}
+    experts = sorted(users)
+    for c0 in range(0, len(experts), chunk):
+        part = experts[c0:c0 + chunk]
+        jobs = [(e, kind) for e in part for kind in ("gate", "up", "down")]
+        bits = [_bits(synth.expert_torch(w, layer, e, kind, seed=0)) for e, kind in jobs]
+        res = pool.map(_quantize_bits, bits)
         mats = {}
         for (e, kind), (c, s) in zip(jobs, res):
             gc, gs = gpu[kind]
             assert (gc[e].cpu().numpy() == c).all(), f"codes of expert {e} {kind}"
             assert (gs[e].cpu().numpy() == s).all(), f"scales of expert {e} {kind}"
             mats[(e, kind)] = mxfp4.dequantize(c, s)
-        for e in todo:
-            self.dense[e] = (mats[(e, "gate")], mats[(e, "up")], mats[(e, "down")])
+        for e in part:
+            rows = users[e]
+            xr = np.stack([xv[tokens[j]] for j, _ in rows])
+            out = moe.expert_ffn(xr, mats[(e, "gate")], mats[(e, "up")], mats[(e, "down")])
+            for (j, slot), o in zip(rows, out):
+                contrib[j, slot] = wts[j][slot] * o
+        del mats
+    y = np.zeros((len(tokens), w.hidden))
+    for slot in range(w.top_k):  # slot order
+        y += contrib[:, slot]
+    return y
 
-    def token_y(self, x_row, idx_row, w_row):
-        y = np.zeros(self.w.hidden)
-        for e, wt in zip(idx_row, w_row):  # slot order
-            wg, wu, wd = self.dense[int(e)]
-            y += wt * moe.expert_ffn(x_row[None, :], wg, wu, wd)[0]
-        return y
 
-
-def _route_and_check(x, router_w, router_b, k, gpu_idx, tokens):
-    idx, w, lg = moe.route(x[tokens], router_w, router_b, k)
-    bound = moe.logit_error_bound(x[tokens], router_w, router_b)
+def _route_all(route, xv, rw, rb, k, T):
+    """Every token's routing against the oracle; returns (oracle idx, oracle-side weights of
+    the GPU's selection, unpinned count).  Near ties are counted and evaluated at the GPU's
+    own selection; everything else is bit-exact."""
+    idx, w, lg = moe.route(xv, rw, rb, k)
+    bound = moe.logit_error_bound(xv, rw, rb)
     loose = set(moe.unpinned_tokens(lg, bound, k).tolist())
-    for j, t in enumerate(tokens):
-        if j not in loose:
-            assert gpu_idx[t].tolist() == idx[j].tolist(), (t, gpu_idx[t], idx[j])
-        else:  # near tie: evaluate the layer at the GPU's own selection
-            p = moe.softmax(lg[j])
-            ps = p[gpu_idx[t]]
-            idx[j], w[j] = gpu_idx[t], ps / ps.sum()
-    return idx, w
+    g_idx = route["topk_idx"].cpu().numpy()
+    for t in range(T):
+        if t not in loose:
+            assert g_idx[t].tolist() == idx[t].tolist(), (t, g_idx[t], idx[t])
+    counts, offsets, perm, inv = moe.permute(g_idx, rw.shape[0])
+    assert (route["counts"].cpu().numpy() == counts).all()
+    assert (route["offsets"].cpu().numpy() == offsets).all()
+    assert (route["perm"].cpu().numpy() == perm).all()
+    assert (route["inv_perm"].cpu().numpy() == inv).all()
+    p = moe.softmax(lg)
+    ps = np.take_along_axis(p, g_idx.astype(np.int64), axis=-1)
+    ws = ps / ps.sum(-1, keepdims=True)
+    assert np.abs(route["topk_w"].cpu().numpy() - ws).max() <= 1e-5
+    # rare: a near tie needs a logit gap below ~1e-13 relative
+    assert len(loose) <= max(1, T // 500), f"{len(loose)} unpinned tokens of {T}"
+    return g_idx, ws, len(loose)
 
 
-def _run(mx, pool, w, T, tokens, layer_io=False):
+def _tile_coverage(route, tokens, k, E):
+    """(tile index within the expert's segment, epilogue set) of every sampled pair."""
+    inv = route["inv_perm"].cpu().numpy()
+    offsets = route["offsets"].cpu().numpy()
+    idx = route["topk_idx"].cpu().numpy()
+    cov = set()
+    for t in tokens:
+        for slot in range(k):
+            e = int(idx[t, slot])
+            p = int(inv[t * k + slot]) - int(offsets[e])
+            cov.add((p // LT_MAX, (p % LT_MAX) % 2))
+    return cov
+
+
+def _run(mx, w, T, layer_io=False):
     import torch
     import bench
     layers = [bench.build_layer(mx, w, l, seed=0) for l in range(w.layers)]
     m = mx.Moe(w.hidden, w.inter, w.experts, w.top_k, T, layers)
     x = synth.draw_torch(1000, 0, "x", -1, (T, w.hidden), 1.0)
-    route = m.moe_route(x, layer=0)
     io = torch.empty((w.layers + 1, T, w.hidden), dtype=torch.bfloat16, device="cuda") if layer_io else None
     y = m.moe_forward(x, layer_io=io)
     m.moe_status()
     dense = [synth.layer_inputs_torch(w, l, 0, tokens=T) for l in range(w.layers)]
-    return m, layers, x, route, y, io, dense
+    return m, layers, x, y, io, dense
 
 
-def _check_layer(pool, w, layer, gpu_layer, dense_l, x_bits, gpu_idx, got_rows, tokens, normalise):
-    xv = mxfp4.bf16_to_f64(x_bits)
+def _check_layer(m, pool, w, layer, gpu_layer, dense_l, x_dev, out_dev, tokens, normalise):
+    """Route every token of x_dev on the GPU and in the oracle, then the sampled rows of out_dev."""
+    import torch
+    T = x_dev.shape[0]
+    route = m.moe_route(x_dev.contiguous(), layer=layer)
+    m.moe_status()
+    xv = mxfp4.bf16_to_f64(_bits(x_dev))
     rw = dense_l["router_w"].cpu().numpy().astype(np.float64)
     rb = None if dense_l["router_b"] is None else dense_l["router_b"].cpu().numpy().astype(np.float64)
-    idx, wts = _route_and_check(xv, rw, rb, w.top_k, gpu_idx, tokens)
-    cache = ExpertCache(w, layer, gpu_layer, pool)
-    cache.need(sorted({int(e) for row in idx for e in row}))
-    ref = np.stack([cache.token_y(xv[t], idx[j], wts[j]) for j, t in enumerate(tokens)])
+    g_idx, ws, loose = _route_all(route, xv, rw, rb, w.top_k, T)
+    ref = oracle_rows(pool, w, layer, gpu_layer, xv, tokens, g_idx[tokens], ws[tokens])
     if normalise:
         ref = moe.round_bf16(moe.rmsnorm(ref))
-    ok, ratio = tolerance_ok(got_rows, ref)
+    got = x_values(out_dev[tokens].contiguous().view(torch.int16).cpu().numpy().view(np.uint16))
+    ok, ratio = tolerance_ok(got, ref)
     assert ok, f"layer {layer}: worst |err|/bound = {ratio:.3f}"
-    return ratio
+    return route, ratio, loose
 
 
-def _gpu_rows(t, tokens):
-    import torch
-    return x_values(t[tokens].contiguous().view(torch.int16).cpu().numpy().view(np.uint16))
-
-
-@pytest.mark.parametrize("name,tokens", [("decode_t9_h4096_e128", [0, 8]),
-                                         ("batched_t144_h6144_e256", [5, 143])])
-def test_single_layer_full_size(mx, pool, name, tokens):
+@pytest.mark.parametrize("name", ["decode_t9_h4096_e128", "batched_t144_h6144_e256"])
+def test_single_layer_full_size(mx, pool, name):
     w = synth.WORKLOADS[name]
-    m, layers, x, route, y, _, dense = _run(mx, pool, w, w.tokens, tokens)
-    gpu_idx = route["topk_idx"].cpu().numpy()
-    _check_layer(pool, w, 0, layers[0], dense[0], _bits(x), gpu_idx, _gpu_rows(y, tokens), tokens, False)
+    m, layers, x, y, _, dense = _run(mx, w, w.tokens)
+    tokens = sample_tokens(w.tokens)
+    _check_layer(m, pool, w, 0, layers[0], dense[0], x, y, tokens, False)
     m.close()
 
 
 def test_chain_full_size_teacher_forced(mx, pool):
-    """8-layer chain (Zipf-biased router): layers 0 and 7 on the GPU's own bf16 inputs."""
+    """8-layer chain (Zipf-biased router): every layer, every token, on the GPU's own bf16 inputs."""
     w = synth.WORKLOADS["chain8_t9_h6144_e256_zipf"]
-    tokens = [3]
-    m, layers, x, route, y, io, dense = _run(mx, pool, w, w.tokens, tokens, layer_io=True)
-    for l in (0, w.layers - 1):
-        xl = io[l]
-        r = m.moe_route(xl.contiguous(), layer=l)
-        gpu_idx = r["topk_idx"].cpu().numpy()
+    m, layers, x, y, io, dense = _run(mx, w, w.tokens, layer_io=True)
+    assert (io[w.layers] == y).all()
+    tokens = sample_tokens(w.tokens)
+    for l in range(w.layers):
         last = l == w.layers - 1
-        out = io[l + 1]
-        _check_layer(pool, w, l, layers[l], dense[l], _bits(xl), gpu_idx, _gpu_rows(out, tokens), tokens,
-                     normalise=not last)
+        _check_layer(m, pool, w, l, layers[l], dense[l], io[l], io[l + 1], tokens, normalise=not last)
     m.close()
 
 
-@pytest.mark.parametrize("T", [1, 72, 4608])
+@pytest.mark.parametrize("T", [1, 9, 72, 576, 4608])
 def test_sweep_full_size(mx, pool, T):
-    """H = 7168, E = 256: T = 1 (decode), 72 and 4608 (the large-T routing path)."""
+    """H = 7168, E = 256 over the token sweep: decode (1, 9), the pipeline stream with
+    grid-wide routing (72), the tile stream (576, 4608)."""
     w = synth.WORKLOADS["sweep_h7168_e256"].with_tokens(T)
-    tokens = [0] if T == 1 else [1, T - 1]
-    m, layers, x, route, y, _, dense = _run(mx, pool, w, T, tokens)
-    gpu_idx = route["topk_idx"].cpu().numpy()
-    _check_layer(pool, w, 0, layers[0], dense[0], _bits(x), gpu_idx, _gpu_rows(y, tokens), tokens, False)
+    m, layers, x, y, _, dense = _run(mx, w, T)
+    tokens = sample_tokens(T)
+    route, _, _ = _check_layer(m, pool, w, 0, layers[0], dense[0], x, y, tokens, False)
+    if T * w.top_k >= 8 * w.experts:  # tile stream: both epilogue sets, interior tiles at 4608
+        cov = _tile_coverage(route, tokens, w.top_k, w.experts)
+        assert {s for _, s in cov} == {0, 1}, cov
+        if T >= 4608:
+            assert max(t for t, _ in cov) >= 2, cov
     m.close()

@@ -125,3 +125,60 @@ def test_shard_layer_i_slices_like_the_oracle_side():
                 assert (getattr(a, k).numpy() == np.stack(getattr(b, k))).all(), (world, r, k)
     with pytest.raises(ValueError):
         mx.shard_layer_i(layer, 0, 8)  # 512 / 8 = 64 rows
+
+
+class _FakeHandle:
+    """Stands in for a Moe handle: a region address per rank, a recognisable IPC handle."""
+
+    def __init__(self, rank):
+        self.rank, self.attached = rank, None
+
+    def moe_ishard_region(self):
+        return 0x1000 * (self.rank + 1), 4096
+
+    def moe_ishard_ipc_handle(self):
+        return bytes([self.rank + 1]) * 64
+
+    def moe_ishard_attach(self, rank, world, regions):
+        self.attached = (rank, world, list(regions))
+
+
+def _ipc_rank_main(rank, world, port, out):
+    import torch.distributed as dist
+    from tests.helpers import build_library
+    build_library()
+    import mxfp4_moe_expert_router_b200 as mx
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        got = mx.exchange_ipc_handles(bytes([rank + 1]) * 64)
+        fake = _FakeHandle(rank)
+        # a peer's region as this rank maps it: tagged with the handle it came from
+        opened = mx.connect_ishard(fake, opener=lambda h: 0x100000 + h[0])
+        out.put((rank, [g[0] for g in got], fake.attached, opened))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ishard_handle_exchange_and_attach_order_under_gloo():
+    """connect_ishard over 3 gloo ranks: every rank gets all IPC handles in rank order,
+    maps each peer's, and attaches its own region at its rank and the mapped peers elsewhere."""
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    world = 3
+    procs = [ctx.Process(target=_ipc_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, tags, attached, opened in res:
+        assert tags == [1, 2, 3]
+        r, w, regions = attached
+        assert (r, w) == (rank, world)
+        expect = [0x1000 * (rank + 1) if s == rank else 0x100000 + s + 1 for s in range(world)]
+        assert regions == expect
+        assert opened == [0x100000 + s + 1 for s in range(world) if s != rank]
