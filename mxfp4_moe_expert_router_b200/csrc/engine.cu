@@ -103,7 +103,6 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert((size_t)WARPS * MAX_EXPERTS * 8 <= RING_BYTES, "routing scratch in ring");
 static_assert((size_t)16 * (8192 / MAX_HSPLIT) * 8 <= RING_BYTES, "router x slice in ring");
 static_assert((size_t)LT_NSLOT * LT_SLOT_BYTES <= RING_BYTES && LT_SLOT_BYTES % 16 == 0, "tile ring");
-static_assert(PRODUCER_BATCH <= LT_NSLOT, "producer batch (tiles)");
 static_assert(SLOT_BYTES % 16 == 0 && STAGE_A_BYTES % 16 == 0 && IMG_BYTES % 16 == 0, "bulk-copy alignment");
 // tensor memory: pipeline p's accumulators, then its scale-factor buffers
 __host__ __device__ constexpr uint32_t tm_acc(int pipe, int b) { return (uint32_t)(pipe * NACC + b) * ACC_COLS; }
@@ -126,6 +125,22 @@ __device__ __forceinline__ float* xch_buf(uint8_t* smem, int pipe, int i) {
   return reinterpret_cast<float*>(smem + OFF_XCH) + (pipe * 2 + i) * NT_MAX * 4;
 }
 __device__ __forceinline__ CtaTables& tables(uint8_t* smem) { return *reinterpret_cast<CtaTables*>(smem + OFF_TABLES); }
+
+// Stream modes: 0 = pipeline stream (units of <= NT_MAX positions, two
+// pipelines per CTA), 1 = tiles (<= LT_MAX positions, one row block per job),
+// 4 = tile pairs (<= LTA_MAX positions, LTA_R row blocks per job sharing each
+// B stage).  The tile modes run one pipeline per CTA.
+template <int TM> struct TileCfg;
+template <> struct TileCfg<1> {
+  static constexpr int R = 1, ACCW = LT_ACC_COLS, NACCV = LT_NACC, NS = LT_NSLOT,
+                       SLOTB = LT_SLOT_BYTES;
+};
+template <> struct TileCfg<4> {
+  static constexpr int R = LTA_R, ACCW = LTA_ACC_COLS, NACCV = LTA_NACC, NS = LTA_NSLOT,
+                       SLOTB = LTA_SLOT_BYTES;
+};
+static_assert((size_t)LTA_NSLOT * LTA_SLOT_BYTES <= RING_BYTES && LTA_SLOT_BYTES % 16 == 0, "tile pair ring");
+static_assert(PRODUCER_BATCH <= LT_NSLOT, "producer batch (tiles)");
 
 __device__ __forceinline__ void set_error(uint32_t* sync, uint32_t code, uint32_t info) {
   if (atomicCAS(sync + SY_ERROR, 0u, code) == 0u) atomicExch(sync + SY_ERRINFO, info);
@@ -969,8 +984,9 @@ __device__ void phase_topk_large(const EngineParams& p, const LayerPtrs& lp) {
 }
 
 // Large T*K, step 2: counts/offsets in every CTA (shared-memory histogram),
-// unit table by CTA 0, stable positions by one warp per expert (ballot scan).
-__device__ void phase_permute_large(const EngineParams& p, uint8_t* smem) {
+// unit table by CTA 0 (units of at most `us` positions), stable positions by
+// one warp per expert (ballot scan).
+__device__ void phase_permute_large(const EngineParams& p, uint8_t* smem, int us) {
   CtaTables& tb = tables(smem);
   const int E = p.E, K = p.K, TK = p.TK;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -984,8 +1000,7 @@ __device__ void phase_permute_large(const EngineParams& p, uint8_t* smem) {
   __syncthreads();
   if (blockIdx.x == 0) {
     int32_t* scratch = reinterpret_cast<int32_t*>(ring_slot(smem, 0, 0));
-    build_units(tb.counts, tb.offsets, E, scratch, p.units, p.dunits, &tb.n_units, &tb.n_dunits,
-                use_tiles(TK, E) ? LT_MAX : NT_MAX);
+    build_units(tb.counts, tb.offsets, E, scratch, p.units, p.dunits, &tb.n_units, &tb.n_dunits, us);
     for (int i = threadIdx.x; i < E; i += THREADS) p.counts[i] = tb.counts[i];
     for (int i = threadIdx.x; i <= E; i += THREADS) p.offsets[i] = tb.offsets[i];
     if (threadIdx.x == 0) { p.n_units[0] = tb.n_units; p.n_units[1] = tb.n_dunits; }
@@ -1207,20 +1222,25 @@ __device__ bool wait_entry(const EngineParams& p, JobEntry* en, int32_t qk) {
 // (down, from aimg).
 // SPLIT (operator-by-operator launches only): 1 runs the gate/up jobs alone, 2
 // the down jobs alone (their gate/up units are then complete).
-template <bool LT, int SPLIT = 0>
+template <int TM, int SPLIT = 0>
 __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem,
                                 const StreamCtx& cx, int pipe, RoleState& rs) {
-  constexpr int NS = LT ? LT_NSLOT : NSLOT;  // ring slots
+  constexpr bool LT = TM != 0;
+  constexpr int NS = TM == 1 ? LT_NSLOT : TM == 4 ? LTA_NSLOT : NSLOT;  // ring slots
+  constexpr int SLOTB = TM == 1 ? LT_SLOT_BYTES : TM == 4 ? LTA_SLOT_BYTES : SLOT_BYTES;
+  constexpr int R = TM == 4 ? LTA_R : 1;      // row blocks per job
   constexpr int NP = LT ? 1 : NPIPE;         // pipelines per CTA
+  constexpr int PB = PRODUCER_BATCH < NS ? PRODUCER_BATCH : NS;
   const int lane = threadIdx.x & 31;
   JobEntry* jq = job_queue(smem, pipe);
   uint32_t* ready = p.sync + SY_READY;
   const int gub = p.I / GU_I_ROWS, db = p.H / JOB_ROWS;
-  const int64_t n_gu = (int64_t)cx.n_units * gub;
-  const int64_t n_all = SPLIT == 1 ? n_gu : n_gu + (int64_t)cx.n_dunits * db;
+  const int gpu_ = gub / R, dpu = db / R;    // jobs per unit
+  const int64_t n_gu = (int64_t)cx.n_units * gpu_;
+  const int64_t n_all = SPLIT == 1 ? n_gu : n_gu + (int64_t)cx.n_dunits * dpu;
   const int64_t j0 = SPLIT == 2 ? n_gu : 0;  // first job of this launch
   const int nc_gu = p.H / KS, nc_d = p.I / KS;
-  const uint32_t need = (uint32_t)gub * (LT ? 8u : 4u);  // readiness signals per gate/up unit: epilogue warps per job
+  const uint32_t need = (uint32_t)gpu_ * (LT ? 8u : 4u);  // readiness signals per gate/up unit: epilogue warps per job
   bool xwait = !LT && !cx.global;  // x term images written during the routing (small T*K)
   // Units of at most NT_MAX positions read most expert weights once: the
   // weight stages go to L2 as evict-first, so that the routing's working set
@@ -1251,8 +1271,8 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
     if (lane == 0) next = jbase + atomicAdd(p.sync + (SPLIT == 2 ? SY_JOBS2 : SY_JOBS), 1u);  // prefetch the following job
     const bool isD = j >= n_gu;
     const int64_t jj = isD ? j - n_gu : j;
-    const int per = isD ? db : gub;
-    const int u = (int)(jj / per), rb = (int)(jj % per);
+    const int per = isD ? dpu : gpu_;
+    const int u = (int)(jj / per), rb = (int)(jj % per) * R;  // first row block of the job
     const int4 ur = ld_tab(reinterpret_cast<const int4*>((isD ? cx.dunits : cx.units) + (int64_t)u * 4), cx.global);
     const int e = ur.x, pos0 = ur.y, nt = ur.z;
     const int nc = isD ? nc_d : nc_gu;
@@ -1307,7 +1327,8 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
                                : lp.w_gu + ((int64_t)e * gub + rb) * nc * STAGE_A_BYTES;
     const int tok = (!LT && !isD && lane < nt) ? ld_tab(cx.tokpos + pos0 + lane, cx.global) : 0;
     const uint32_t bbytes = LT ? (uint32_t)(LT_SF_BYTES + lt_cols(nt) * (IMG_CODE_BYTES / 8)) : (uint32_t)nt * IMG_BYTES;
-    const uint32_t stage_bytes = STAGE_A_BYTES + bbytes;
+    const uint32_t stage_bytes = R * STAGE_A_BYTES + bbytes;
+    const int64_t rstep = (int64_t)nc * STAGE_A_BYTES;  // between the stages of consecutive row blocks
     // Stages are issued in batches, one stage per lane: successive 1-D bulk
     // copies issued by one warp instruction each are serialised, while the
     // copies of one instruction proceed in parallel.  A batch is the run of
@@ -1316,7 +1337,7 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
     // whenever the producer falls behind.
     int c0 = 0;
     while (c0 < nc && ok) {
-      const int nb = min(PRODUCER_BATCH, nc - c0);
+      const int nb = min(PB, nc - c0);
       const uint32_t s = rs.seq + lane;
       const int slot = (int)(s % NS);
       const uint32_t par = ((s / NS) + 1) & 1u;  // completion of the slot's previous use
@@ -1330,15 +1351,20 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
         if (__any_sync(FULL, bad)) ok = false;
         continue;
       }
-      uint8_t* dst = LT ? smem + OFF_RING + (size_t)slot * LT_SLOT_BYTES : ring_slot(smem, pipe, slot);
+      uint8_t* dst = LT ? smem + OFF_RING + (size_t)slot * SLOTB : ring_slot(smem, pipe, slot);
       uint64_t* fb = full_bar(smem, pipe, slot);
       const int c = c0 + lane;
       if (lane < k) {
         mbar_arrive_expect_tx(fb, stage_bytes);
-        if constexpr (LT) bulk_g2s(dst, wbase + (int64_t)c * STAGE_A_BYTES, STAGE_A_BYTES, fb);
-        else bulk_g2s_hint(dst, wbase + (int64_t)c * STAGE_A_BYTES, STAGE_A_BYTES, fb, wpolicy);
+        if constexpr (LT) {
+#pragma unroll
+          for (int r = 0; r < R; ++r)
+            bulk_g2s(dst + r * STAGE_A_BYTES, wbase + r * rstep + (int64_t)c * STAGE_A_BYTES, STAGE_A_BYTES, fb);
+        } else {
+          bulk_g2s_hint(dst, wbase + (int64_t)c * STAGE_A_BYTES, STAGE_A_BYTES, fb, wpolicy);
+        }
         if (LT)  // the tile's B operand of this stage, one image
-          bulk_g2s(dst + STAGE_A_BYTES, (isD ? p.atl : p.xtl) + ((int64_t)u * nc + c) * LT_IMG_BYTES,
+          bulk_g2s(dst + R * STAGE_A_BYTES, (isD ? p.atl : p.xtl) + ((int64_t)u * nc + c) * LT_IMG_BYTES,
                    bbytes, fb);
         else if (isD)
           bulk_g2s(dst + STAGE_A_BYTES, p.aimg + ((int64_t)c * p.TK + pos0) * IMG_BYTES,
@@ -1550,15 +1576,29 @@ __device__ void stream_epilogue(const EngineParams& p, uint8_t* smem, const Stre
 }
 
 // ---- phase C, large T*K: one pipeline over tiles -------------------------------------------
-// Tensor memory: LT_NACC accumulators of LT_ACC_COLS columns, then NSF
-// scale-factor buffers of LT_SF_COLS (A: 4 columns, B: 4 per 128 columns).
-__device__ __forceinline__ uint32_t lt_acc(int b) { return (uint32_t)b * LT_ACC_COLS; }
-__device__ __forceinline__ uint32_t lt_sf(int i) { return (uint32_t)(LT_NACC * LT_ACC_COLS + i * LT_SF_COLS); }
+// Tensor memory: NACCV accumulator sets of R accumulators of ACCW columns
+// (accumulator r of set b at (b R + r) ACCW), then NSF scale-factor buffers
+// of 4 R + 4 columns (A: 4 per row block, then B: 4 per 128 B rows).
+template <int TM>
+__device__ __forceinline__ uint32_t lt_acc(int b, int r) {
+  return (uint32_t)(b * TileCfg<TM>::R + r) * TileCfg<TM>::ACCW;
+}
+template <int TM>
+__device__ __forceinline__ uint32_t lt_sf(int i) {
+  using C = TileCfg<TM>;
+  return (uint32_t)(C::NACCV * C::R * C::ACCW + i * (4 * C::R + 4 * LT_SF_BLOCKS));
+}
+static_assert(LT_NACC * LT_ACC_COLS + NSF * (4 + 4 * LT_SF_BLOCKS) <= TMEM_COLS, "tensor memory (tiles)");
+static_assert(LTA_NACC * LTA_R * LTA_ACC_COLS + NSF * (4 * LTA_R + 4 * LT_SF_BLOCKS) <= TMEM_COLS,
+              "tensor memory (tile pairs)");
 
-// MMA issuer of the tile stream (one thread): per stage the weight scales and
-// the tile's 1-2 scale blocks go to tensor memory, then two MMAs (K = 64 each,
-// N = 8 per position of the tile) accumulate.
+// MMA issuer of the tile stream (one thread): per stage the weight scales of
+// the job's R row blocks and the tile's 1-2 scale blocks go to tensor memory,
+// then per row block two MMAs (K = 64 each, N = 8 per position of the tile)
+// accumulate into that row block's accumulator.
+template <int TM>
 __device__ void stream_mma_lt(const EngineParams& p, uint8_t* smem, uint32_t tmem, RoleState& rs) {
+  using C = TileCfg<TM>;
   JobEntry* jq = job_queue(smem, 0);
   const uint32_t ring0 = smem_u32(smem + OFF_RING);
   const bool prof = p.prof != nullptr;
@@ -1572,8 +1612,8 @@ __device__ void stream_mma_lt(const EngineParams& p, uint8_t* smem, uint32_t tme
     const int s0 = en->s0, nc = en->nc, nt = en->nt, wj = en->wj;
     ++rs.qk;
     if (!ok) continue;
-    const int b = wj % LT_NACC;
-    const uint32_t use = (uint32_t)(wj / LT_NACC);
+    const int b = wj % C::NACCV;
+    const uint32_t use = (uint32_t)(wj / C::NACCV);
     const unsigned long long ta0 = pclock(prof);
     if (use > 0 &&
         !wait_mbar(acce_bar(smem, 0, b), (use - 1) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, wj)) {
@@ -1582,28 +1622,34 @@ __device__ void stream_mma_lt(const EngineParams& p, uint8_t* smem, uint32_t tme
     }
     t_acc += pclock(prof) - ta0;
     tc_fence_after();
-    const uint32_t tacc = tmem + lt_acc(b);
     const int n = lt_cols(nt), nblk = (n + 127) / 128;
     const uint32_t idesc0 = mxf4_idesc(n, 0u), idesc1 = mxf4_idesc(n, 2u);
     for (int c = 0; c < nc; ++c) {
       const uint32_t s = (uint32_t)s0 + c;
-      const int slot = (int)(s % LT_NSLOT);
+      const int slot = (int)(s % C::NS);
       const unsigned long long tf0 = pclock(prof);
-      if (!wait_mbar(full_bar(smem, 0, slot), (s / LT_NSLOT) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, s)) {
+      if (!wait_mbar(full_bar(smem, 0, slot), (s / C::NS) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, s)) {
         ok = false;
         break;
       }
       const unsigned long long tm0 = pclock(prof);
       t_full += tm0 - tf0;
-      const uint32_t sa = ring0 + (uint32_t)slot * LT_SLOT_BYTES, sb = sa + STAGE_A_BYTES;
-      const uint32_t tsf = tmem + lt_sf((int)(rs.sfc++ % NSF));
-      tmem_cp_sf(tsf, smem_desc(sa + STAGE_CODE_BYTES, 0, 128));
-      for (int q = 0; q < nblk; ++q) tmem_cp_sf(tsf + 4 + 4 * q, smem_desc(sb + q * 512, 0, 128));
+      const uint32_t sa = ring0 + (uint32_t)slot * C::SLOTB, sb = sa + C::R * STAGE_A_BYTES;
+      const uint32_t tsf = tmem + lt_sf<TM>((int)(rs.sfc++ % NSF));
+      const uint32_t tsb = tsf + 4 * C::R;  // B scale columns
+#pragma unroll
+      for (int r = 0; r < C::R; ++r)
+        tmem_cp_sf(tsf + 4 * r, smem_desc(sa + r * STAGE_A_BYTES + STAGE_CODE_BYTES, 0, 128));
+      for (int q = 0; q < nblk; ++q) tmem_cp_sf(tsb + 4 * q, smem_desc(sb + q * 512, 0, 128));
       const uint32_t bc = sb + LT_SF_BYTES;
-      mma_mxf4(tacc, smem_desc(sa, 128, 256), smem_desc(bc, 128, IMG_CODE_BYTES), idesc0, tsf, tsf + 4,
-               c > 0 ? 1u : 0u);
-      mma_mxf4(tacc, smem_desc(sa + 4096, 128, 256), smem_desc(bc + 256, 128, IMG_CODE_BYTES), idesc1,
-               tsf | (2u << 30), (tsf + 4) | (2u << 30), 1u);
+#pragma unroll
+      for (int r = 0; r < C::R; ++r) {
+        const uint32_t tacc = tmem + lt_acc<TM>(b, r), ar = sa + r * STAGE_A_BYTES, tsa = tsf + 4 * r;
+        mma_mxf4(tacc, smem_desc(ar, 128, 256), smem_desc(bc, 128, IMG_CODE_BYTES), idesc0, tsa, tsb,
+                 c > 0 ? 1u : 0u);
+        mma_mxf4(tacc, smem_desc(ar + 4096, 128, 256), smem_desc(bc + 256, 128, IMG_CODE_BYTES), idesc1,
+                 tsa | (2u << 30), tsb | (2u << 30), 1u);
+      }
       tc_commit(empty_bar(smem, 0, slot));
       t_issue += pclock(prof) - tm0;
     }
@@ -1639,10 +1685,16 @@ __device__ __forceinline__ float lt_position_sum(uint32_t tacc, int j) {
   return sum;
 }
 // Eight epilogue warps in two sets (warps 4..7 and 8..11, each covering the
-// four accumulator lane quadrants); set `set` handles positions set, set + 2,
-// ..., with its own amax exchange buffers and barriers.
+// four accumulator lane quadrants), each with its own amax exchange buffers
+// and barriers.  Tiles (one row block per job): set `set` handles positions
+// set, set + 2, ...  Tile pairs: set `set` handles every position of row
+// block rb + set (its own accumulator).
+template <int TM>
 __device__ void stream_epilogue_lt(const EngineParams& p, uint8_t* smem, const StreamCtx& cx, uint32_t tmem,
                                    int set, RoleState& rs) {
+  using C = TileCfg<TM>;
+  static_assert(C::R == 1 || C::R == 2, "one row block per epilogue set");
+  const int J0 = C::R == 1 ? set : 0, JS = C::R == 1 ? 2 : 1, rs_ = C::R == 1 ? 0 : set;
   const int lane = threadIdx.x & 31, q = (threadIdx.x >> 5) & 3;
   JobEntry* jq = job_queue(smem, 0);
   uint32_t* ready = p.sync + SY_READY;
@@ -1663,20 +1715,21 @@ __device__ void stream_epilogue_lt(const EngineParams& p, uint8_t* smem, const S
     if (!ok) continue;
     ++n_jobs;
     const uint32_t gc = isD ? 0u : rs.gcount++;
-    const int b = wj % LT_NACC;
+    const int b = wj % C::NACCV;
     const unsigned long long tw0 = pclock(prof);
-    if (!wait_mbar(accf_bar(smem, 0, b), (uint32_t)(wj / LT_NACC) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, wj)) {
+    if (!wait_mbar(accf_bar(smem, 0, b), (uint32_t)(wj / C::NACCV) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, wj)) {
       ok = false;
       continue;
     }
     const unsigned long long tk0 = pclock(prof);
     t_wait += tk0 - tw0;
     tc_fence_after();
-    const uint32_t tacc = tmem + ((uint32_t)(32 * q) << 16) + lt_acc(b);
+    const uint32_t tacc = tmem + ((uint32_t)(32 * q) << 16) + lt_acc<TM>(b, rs_);
+    const int rbe = rb + rs_;  // this set's row block
     if (!isD) {
       const int xb = (int)(gc & 1u);
       float* xc = reinterpret_cast<float*>(smem + OFF_XCH) + (set * 2 + xb) * LT_MAX * 4;
-      for (int j = set; j < nt; j += 2) {
+      for (int j = J0; j < nt; j += JS) {
         const float sum = lt_position_sum(tacc, j);
         const float other = __shfl_xor_sync(FULL, sum, 16);
         const float g = lane < 16 ? sum : other, up = lane < 16 ? other : sum;
@@ -1693,9 +1746,9 @@ __device__ void stream_epilogue_lt(const EngineParams& p, uint8_t* smem, const S
         ok = false;
         continue;
       }
-      const int i0 = rb * GU_I_ROWS, sD = i0 / KS, kk = (i0 % KS) / 64, kc = q >> 1;
+      const int i0 = rbe * GU_I_ROWS, sD = i0 / KS, kk = (i0 % KS) / 64, kc = q >> 1;
       uint8_t* img = p.atl + ((int64_t)u * nsd + sD) * LT_IMG_BYTES;
-      for (int j = set; j < nt; j += 2) {
+      for (int j = J0; j < nt; j += JS) {
         const int s0 = term0_exp(fmaxf(xc[j * 4 + q], xc[j * 4 + (q ^ 1)]));
         const uint32_t word = term_word<16>(e2m1_terms<LT_NTERM>(av[j], s0), lane);
         if (lane < 2 * LT_NTERM)  // lane l: term l / 2, elements 8 (l % 2) .. + 7 of this warp's 16
@@ -1711,8 +1764,8 @@ __device__ void stream_epilogue_lt(const EngineParams& p, uint8_t* smem, const S
         red_release_add_u32(ready + u, 1u);
       }
     } else {
-      const int h0 = rb * JOB_ROWS;
-      for (int j = set; j < nt; j += 2) {
+      const int h0 = rbe * JOB_ROWS;
+      for (int j = J0; j < nt; j += JS) {
         const float sum = lt_position_sum(tacc, j);
         p.ypair[(int64_t)(pos0 + j) * p.H + h0 + 32 * q + lane] = sum * ld_tab(cx.wpos + pos0 + j, cx.global);
       }
@@ -2247,18 +2300,29 @@ __device__ bool phase_allreduce_out(const EngineParams& p, const int32_t* inv, i
 // chunks over the whole grid (partial sums, a grid barrier, then the scaling
 // of each chunk); the operator-by-operator launch runs all chunks of a token
 // in one CTA.  Both give the same bits.
-constexpr int RMS_CHUNKS = 16;
+constexpr int RMS_CHUNKS = 8;
 static_assert(8192 / RMS_CHUNKS / 4 <= THREADS, "one float4 of a chunk per thread");
 
 // The bf16-rounded combine of this thread's float4 of chunk c of token t (zero
-// past the chunk), and its sum of squares.
-__device__ __forceinline__ float4 rms_chunk_values(const EngineParams& p, const int32_t* inv, int t, int c,
-                                                   bool& mine) {
-  const int cl4 = p.H / RMS_CHUNKS / 4;
+// past the chunk): the k slot loads are issued before the adds, which stay in
+// slot order.  (Scalar arguments: out-of-line callers must not take the
+// kernel's parameter block by reference.)
+__device__ __forceinline__ float4 rms_chunk_values(const float* ypair, const int32_t* inv, int K, int H, int t,
+                                                   int c, bool& mine) {
+  const int cl4 = H / RMS_CHUNKS / 4;
   mine = (int)threadIdx.x < cl4;
   float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
   if (mine) {
-    s = combine4(p, inv, t, c * (p.H / RMS_CHUNKS) + 4 * (int)threadIdx.x);
+    const int h = c * (H / RMS_CHUNKS) + 4 * (int)threadIdx.x;
+    for (int s0 = 0; s0 < K; s0 += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (s0 + i < K) v[i] = __ldcg(reinterpret_cast<const float4*>(ypair + (int64_t)inv[t * K + s0 + i] * H + h));
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (s0 + i < K) { s.x += v[i].x; s.y += v[i].y; s.z += v[i].z; s.w += v[i].w; }
+    }
     s.x = __bfloat162float(__float2bfloat16_rn(s.x));
     s.y = __bfloat162float(__float2bfloat16_rn(s.y));
     s.z = __bfloat162float(__float2bfloat16_rn(s.z));
@@ -2267,12 +2331,10 @@ __device__ __forceinline__ float4 rms_chunk_values(const EngineParams& p, const 
   return s;
 }
 
-// Sum of squares of chunk c of token t, fixed reduction order; every thread
-// of the CTA gets the result.  Also returns this thread's values.
-__device__ float rms_chunk_ss(const EngineParams& p, const int32_t* inv, int t, int c, float* red,
-                              float4& v, bool& mine) {
+// Sum of squares of the values v (this thread's part of one chunk), fixed
+// reduction order; every thread of the CTA gets the result.
+__device__ float rms_chunk_ss(float4 v, float* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  v = rms_chunk_values(p, inv, t, c, mine);
   float ss = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(FULL, ss, o);
@@ -2285,58 +2347,62 @@ __device__ float rms_chunk_ss(const EngineParams& p, const int32_t* inv, int t, 
   return tot;
 }
 
-__device__ __forceinline__ void rms_chunk_store(const EngineParams& p, int t, int c, float4 v, bool mine, float r) {
+// x_next chunk = bf16(v * 1 / sqrt(tot / H + eps)).
+__device__ __forceinline__ void rms_chunk_store(__nv_bfloat16* xnext, int H, float eps, int t, int c, float4 v,
+                                                bool mine, float tot) {
+  const float r = 1.0f / sqrtf(tot / (float)H + eps);
   if (mine)
-    store_bf16x4(p.xnext + (int64_t)t * p.H + c * (p.H / RMS_CHUNKS) + 4 * (int)threadIdx.x,
+    store_bf16x4(xnext + (int64_t)t * H + c * (H / RMS_CHUNKS) + 4 * (int)threadIdx.x,
                  make_float4(v.x * r, v.y * r, v.z * r, v.w * r));
 }
 
-__device__ __forceinline__ float rms_scale(const EngineParams& p, float tot) {
-  return 1.0f / sqrtf(tot / (float)p.H + p.rms_eps);
-}
-
-// Engine, step 1 of 2: the chunk sums of squares of every (token, chunk) task,
-// spread over the grid, into part[t * RMS_CHUNKS + c].
-__device__ void phase_rms_partials(const EngineParams& p, const int32_t* inv, float* part, uint8_t* smem) {
-  CtaTables& tb = tables(smem);
-  for (int task = blockIdx.x; task < p.T * RMS_CHUNKS; task += gridDim.x) {
-    float4 v;
+// Engine: the chunk sums of squares of every (token, chunk) task, spread over
+// the grid, into part[t * RMS_CHUNKS + c]; a grid barrier; then each token's
+// sum from its chunk sums in chunk order and the scaled bf16 values of every
+// task's chunk.  A CTA's first task keeps its values in registers across the
+// barrier; further tasks (more than one per CTA) recompute them.  Returns
+// false on a barrier timeout or a recorded error.
+__device__ bool phase_rms(const float* ypair, const int32_t* inv, int K, int H, int T, float eps,
+                                       __nv_bfloat16* xnext, float* part, float* red, uint32_t* sync,
+                                       uint64_t timeout_ns, uint32_t where) {
+  const int ntask = T * RMS_CHUNKS;
+  float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f);
+  bool mine0 = false;
+  for (int task = blockIdx.x; task < ntask; task += gridDim.x) {
     bool mine;
-    const float ss = rms_chunk_ss(p, inv, task / RMS_CHUNKS, task % RMS_CHUNKS, tb.red, v, mine);
+    const float4 v = rms_chunk_values(ypair, inv, K, H, task / RMS_CHUNKS, task % RMS_CHUNKS, mine);
+    const float ss = rms_chunk_ss(v, red);
     if (threadIdx.x == 0) part[task] = ss;
+    if (task == (int)blockIdx.x) { v0 = v; mine0 = mine; }
   }
-}
-
-// Engine, step 2 of 2 (after a grid barrier): each token's sum from its chunk
-// sums in chunk order, then the scaled bf16 values of every task's chunk.
-__device__ void phase_rms_apply(const EngineParams& p, const int32_t* inv, const float* part) {
-  for (int task = blockIdx.x; task < p.T * RMS_CHUNKS; task += gridDim.x) {
+  if (!grid_barrier(sync, timeout_ns, where)) return false;
+  for (int task = blockIdx.x; task < ntask; task += gridDim.x) {
     const int t = task / RMS_CHUNKS, c = task % RMS_CHUNKS;
     float tot = 0.f;
 #pragma unroll
     for (int q = 0; q < RMS_CHUNKS; ++q) tot += __ldcg(part + t * RMS_CHUNKS + q);
-    bool mine;
-    const float4 v = rms_chunk_values(p, inv, t, c, mine);
-    rms_chunk_store(p, t, c, v, mine, rms_scale(p, tot));
+    bool mine = mine0;
+    float4 v = v0;
+    if (task != (int)blockIdx.x) v = rms_chunk_values(ypair, inv, K, H, t, c, mine);
+    rms_chunk_store(xnext, H, eps, t, c, v, mine, tot);
   }
+  return true;
 }
 
 // Operator-by-operator launch: every chunk of a token in one CTA (tokens over
-// the CTAs), the same arithmetic in the same order as the two engine steps.
+// the CTAs), the same arithmetic in the same order as phase_rms.
 __device__ void phase_combine_rmsnorm(const EngineParams& p, const int32_t* inv, uint8_t* smem) {
   CtaTables& tb = tables(smem);
   for (int t = blockIdx.x; t < p.T; t += gridDim.x) {
     float tot = 0.f;
     for (int c = 0; c < RMS_CHUNKS; ++c) {
-      float4 v;
       bool mine;
-      tot += rms_chunk_ss(p, inv, t, c, tb.red, v, mine);
+      tot += rms_chunk_ss(rms_chunk_values(p.ypair, inv, p.K, p.H, t, c, mine), tb.red);
     }
-    const float r = rms_scale(p, tot);
     for (int c = 0; c < RMS_CHUNKS; ++c) {
       bool mine;
-      const float4 v = rms_chunk_values(p, inv, t, c, mine);
-      rms_chunk_store(p, t, c, v, mine, r);
+      const float4 v = rms_chunk_values(p.ypair, inv, p.K, p.H, t, c, mine);
+      rms_chunk_store(p.xnext, p.H, p.rms_eps, t, c, v, mine, tot);
     }
     __syncthreads();
   }
@@ -2357,19 +2423,22 @@ __device__ void prefetch_share(const void* base, size_t bytes) {
 
 // All layers; returns early (every thread of the CTA together) when a grid
 // barrier reports an error, or after routing in route-only mode.
-// MODE 0: pipeline stream; MODE 1: E2M1 term tiles (kind::mxf4); MODE 2: bf16
-// tiles (kind::f16).  The tile modes run only above SMALL_PAIRS.
+// MODE 0: pipeline stream, one layer, plain combine (the decode kernel); MODE 5:
+// pipeline stream with chained layers (RMSNorm) or the fused all-reduce; MODE 1:
+// E2M1 term tiles (kind::mxf4); MODE 4: E2M1 term tile pairs (two row blocks per
+// job); MODE 2: bf16 tiles (kind::f16).  The tile modes run only above SMALL_PAIRS.
 template <int MODE>
 __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, RoleState& rs,
                            bool stamp) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool small = MODE == 0 && p.TK <= SMALL_PAIRS;
+  constexpr bool PIPE = MODE == 0 || MODE == 5;  // pipeline stream (units of <= NT_MAX positions)
+  const bool small = PIPE && p.TK <= SMALL_PAIRS;
   CtaTables& tb = tables(smem);
   for (int layer = 0; layer < p.L; ++layer) {
     const LayerPtrs& lp = p.layers[layer];
     const __nv_bfloat16* x = layer == 0 ? p.x_in : p.xnext;
     uint64_t* st = stamp ? p.stamps + 1 + layer * STAMPS_PER_LAYER : nullptr;
-    if constexpr (MODE != 0) phase_router_tiles(x, lp.router_w, p.logits, p.sync, p.T, p.H, p.E, p.TK, p.HS, smem);
+    if constexpr (!PIPE) phase_router_tiles(x, lp.router_w, p.logits, p.sync, p.T, p.H, p.E, p.TK, p.HS, smem);
     else phase_router(p, lp, x, smem);
     if (st) st[0] = globaltimer_ns();
     StreamCtx cx;
@@ -2389,10 +2458,10 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 2)) return;
       if (st) st[3] = globaltimer_ns();
       if constexpr (MODE == 2) phase_permute_f16(p, smem);
-      else phase_permute_large(p, smem);
+      else phase_permute_large(p, smem, MODE == 4 ? LTA_MAX : MODE == 1 ? LT_MAX : NT_MAX);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 3)) return;
       if (p.route_only) return;
-      if constexpr (MODE == 1) {
+      if constexpr (MODE == 1 || MODE == 4) {
         phase_tile_gather(p);
         if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 6)) return;
       } else if constexpr (MODE == 2) {
@@ -2410,11 +2479,11 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
       prefetch_share(p.layers[layer + 1].router_w, (size_t)p.E * p.H * 4);
     fence_proxy_async_smem();  // the ring held routing scratch written by generic stores
     __syncthreads();
-    if constexpr (MODE == 0) {  // two pipelines per CTA, units of <= NT_MAX positions
+    if constexpr (PIPE) {  // two pipelines per CTA, units of <= NT_MAX positions
       if (warp < EPI_WARP0) {
         const int pipe = warp >> 1;
         if ((warp & 1) == 0) {
-          stream_producer<false>(p, lp, smem, cx, pipe, rs);
+          stream_producer<0>(p, lp, smem, cx, pipe, rs);
         } else {
           if (lane == 0) stream_mma(p, smem, tmem, pipe, rs);
           __syncwarp();
@@ -2422,14 +2491,14 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
       } else {
         stream_epilogue(p, smem, cx, tmem, (warp - EPI_WARP0) / 4, rs);
       }
-    } else if constexpr (MODE == 1) {  // one pipeline per CTA over tiles of <= LT_MAX positions
+    } else if constexpr (MODE == 1 || MODE == 4) {  // one pipeline per CTA over tiles (pairs)
       if (warp == 0) {
-        stream_producer<true>(p, lp, smem, cx, 0, rs);
+        stream_producer<MODE>(p, lp, smem, cx, 0, rs);
       } else if (warp == 1) {
-        if (lane == 0) stream_mma_lt(p, smem, tmem, rs);
+        if (lane == 0) stream_mma_lt<MODE>(p, smem, tmem, rs);
         __syncwarp();
       } else if (warp >= EPI_WARP0) {
-        stream_epilogue_lt(p, smem, cx, tmem, warp >= EPI_WARP0 + 4 ? 1 : 0, rs);
+        stream_epilogue_lt<MODE>(p, smem, cx, tmem, warp >= EPI_WARP0 + 4 ? 1 : 0, rs);
       }
     } else {  // bf16 tiles: producer, MMA issuer, six converter warps, four epilogue warps
       if (warp == 0) {
@@ -2448,15 +2517,16 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
     // every producer has passed its image wait and every CTA has counted
     // itself: the count restarts for the next layer or launch
     if (blockIdx.x == 0 && threadIdx.x == 0) p.sync[SY_XDONE] = 0u;
-    if (layer + 1 < p.L) {
+    // MODE 0 runs single layers without the all-reduce (launch rule), so the
+    // decode kernel carries neither the RMSNorm nor the all-reduce code
+    if (MODE != 0 && layer + 1 < p.L) {
       // the partial logits are not read again in this layer: they hold the
       // chunk sums of squares until the next layer's router overwrites them
-      float* part = reinterpret_cast<float*>(p.logits);
-      phase_rms_partials(p, inv, part, smem);
-      if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 7)) return;
-      phase_rms_apply(p, inv, part);
+      if (!phase_rms(p.ypair, inv, p.K, p.H, p.T, p.rms_eps, p.xnext, reinterpret_cast<float*>(p.logits),
+                     tb.red, p.sync, p.timeout_ns, 10 * layer + 7))
+        return;
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 5)) return;
-    } else if (p.ar.world > 0) {
+    } else if (MODE != 0 && p.ar.world > 0) {
       if (!phase_allreduce_out(p, inv, layer)) return;
     } else {
       phase_combine_out(p, inv);
@@ -2480,7 +2550,7 @@ __device__ void op_stream(const EngineParams& p, const LayerPtrs& lp, uint8_t* s
   if (warp < EPI_WARP0) {
     const int pipe = warp >> 1;
     if ((warp & 1) == 0) {
-      stream_producer<false, SPLIT>(p, lp, smem, cx, pipe, rs);
+      stream_producer<0, SPLIT>(p, lp, smem, cx, pipe, rs);
     } else {
       if (lane == 0) stream_mma(p, smem, tmem, pipe, rs);
       __syncwarp();
@@ -2513,8 +2583,8 @@ __device__ void run_op(const EngineParams& p, uint8_t* smem, uint32_t tmem, Role
   }
 }
 
-// Four instances: MODE 0, 1, 2 (see run_layers), each holding only its own
-// stream code, and MODE 3, one operator per launch (run_op).
+// Six instances: MODE 0, 1, 2, 4, 5 (see run_layers), each holding only its
+// own stream code, and MODE 3, one operator per launch (run_op).
 template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -2530,7 +2600,7 @@ __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p
       }
       for (int i = 0; i < NACC; ++i) {
         mbar_init(accf_bar(smem, pp, i), 1);
-        mbar_init(acce_bar(smem, pp, i), MODE == 1 && pp == 0 ? 8 : 4);  // tiles: eight epilogue warps
+        mbar_init(acce_bar(smem, pp, i), (MODE == 1 || MODE == 4) && pp == 0 ? 8 : 4);  // tiles: eight epilogue warps
       }
       for (int i = 0; i < 2; ++i) mbar_init(xch_bar(smem, pp, i), 4);
       mbar_init(drain_bar(smem, pp), 1);
@@ -2577,7 +2647,7 @@ size_t engine_smem_bytes() { return SMEM_BYTES; }
 int engine_max_grid(int device, int* err) {
   int per_sm = ~0u >> 1, sms = 0;
   for (const void* k : {(const void*)engine_kernel<0>, (const void*)engine_kernel<1>, (const void*)engine_kernel<2>,
-                        (const void*)engine_kernel<3>}) {
+                        (const void*)engine_kernel<3>, (const void*)engine_kernel<4>, (const void*)engine_kernel<5>}) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) { *err = (int)e; return 0; }
     int n = 0;
@@ -2593,8 +2663,11 @@ int engine_max_grid(int device, int* err) {
 
 cudaError_t engine_launch(const EngineParams& p, int grid, cudaStream_t s) {
   void* args[] = {const_cast<EngineParams*>(&p)};
-  const void* k = !use_tiles(p.TK, p.E) || p.route_only ? (const void*)engine_kernel<0>
+  const bool plain = p.L == 1 && p.ar.world == 0;  // MODE 0's launch rule
+  const void* k = !use_tiles(p.TK, p.E) || p.route_only ? (plain || p.route_only ? (const void*)engine_kernel<0>
+                                                                                : (const void*)engine_kernel<5>)
                   : p.large == LARGE_F16                  ? (const void*)engine_kernel<2>
+                  : use_tile_pairs(p.TK, p.E, p.H)         ? (const void*)engine_kernel<4>
                                                           : (const void*)engine_kernel<1>;
   return cudaLaunchCooperativeKernel(k, dim3(grid), dim3(THREADS), args, SMEM_BYTES, s);
 }

@@ -93,6 +93,25 @@ static_assert(LT_NTERM <= NTERM, "tile terms are a prefix of the expansion");
 static_assert(LT_NACC * LT_ACC_COLS + NSF * LT_SF_COLS <= TMEM_COLS, "tensor memory budget (tiles)");
 static_assert(LT_NSLOT <= NPIPE * NSLOT, "tile ring barriers");
 static_assert(LT_ACC_COLS <= 128 * LT_SF_BLOCKS, "tile scale-factor blocks");
+// Tile pairs: with few positions per expert (T*K <= LTA_PER_EXPERT * E) a
+// tile holds at most LTA_MAX positions (N <= 96) and a job covers LTA_R = 2
+// consecutive row blocks that share every B stage: per stage the producer
+// brings the two 8704-byte weight stages and one B image, and the MMA issuer
+// accumulates into one tensor-memory accumulator per row block.  More of the
+// bytes in flight are then weights (the B image is read once per two row
+// blocks), which is what the stream is short of at these sizes.  Needs H % 256
+// == 0 (down jobs of 2 x 128 rows of H).
+constexpr int LTA_MAX = 22;
+constexpr int LTA_R = 2;
+constexpr int LTA_NACC = 2;                              // accumulator sets (of LTA_R accumulators)
+constexpr int LTA_PER_EXPERT = 24;
+constexpr int LTA_ACC_COLS = 112;                        // accumulator columns per row block at most
+constexpr int LTA_B_BYTES = LT_SF_BYTES + LTA_ACC_COLS / 8 * IMG_CODE_BYTES;  // 8192
+constexpr int LTA_SLOT_BYTES = LTA_R * STAGE_A_BYTES + LTA_B_BYTES;           // 25600
+constexpr int LTA_NSLOT = 7;
+static_assert(((LT_NTERM * LTA_MAX + 7) & ~7) <= LTA_ACC_COLS && LTA_ACC_COLS <= 128, "tile pair columns");
+static_assert(LTA_NACC * LTA_R * LTA_ACC_COLS + NSF * (4 * LTA_R + 4) <= TMEM_COLS, "tensor memory budget (tile pairs)");
+static_assert(LTA_NSLOT <= NPIPE * NSLOT, "tile pair ring barriers");
 // B rows (= accumulator columns) of a tile of nt positions.
 __host__ __device__ constexpr int lt_cols(int nt) { return (LT_NTERM * nt + 7) & ~7; }
 // Byte offset in a tile image of B row n's first 16-byte chunk.
@@ -140,6 +159,10 @@ enum : int { LARGE_MXF4 = 1, LARGE_F16 = 2 };
 __host__ __device__ inline bool use_tiles(int64_t TK, int E) {
   return TK > SMALL_PAIRS && TK >= (int64_t)LT_MIN_PER_EXPERT * E;
 }
+// Whether its tiles are streamed as tile pairs (two row blocks per job).
+__host__ __device__ inline bool use_tile_pairs(int64_t TK, int E, int H) {
+  return use_tiles(TK, E) && H % (LTA_R * JOB_ROWS) == 0 && TK <= (int64_t)LTA_PER_EXPERT * E;
+}
 constexpr int STAMPS_PER_LAYER = 7;  // router, x images, routing wait, top-k / tables, permutation, stream, combine (CTA 0)
 
 // sync word layout (uint32)
@@ -157,8 +180,8 @@ enum : uint32_t {
 
 // Upper bounds of the unit tables for T*K pairs over E experts.
 __host__ __device__ inline int max_units(int E, int64_t TK) { return (int)((E < TK ? E : TK) + TK / NT_MAX + 1); }
-// Tiles of the large path (at most LT_MAX positions each).
-__host__ __device__ inline int max_tiles(int E, int64_t TK) { return (int)((E < TK ? E : TK) + TK / LT_MAX + 1); }
+// Tiles of the large path (at most LT_MAX, or LTA_MAX for tile pairs, positions each).
+__host__ __device__ inline int max_tiles(int E, int64_t TK) { return (int)((E < TK ? E : TK) + TK / LTA_MAX + 1); }
 __host__ __device__ inline int max_dunits(int E, int64_t TK) { return (int)((E < TK ? E : TK) + TK / ND_MAX + 1); }
 
 // Router split of H into HS parts of H / HS elements (a multiple of 8).
