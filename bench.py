@@ -62,8 +62,9 @@ def parse_args():
     ap.add_argument("--batches", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--large-kind", choices=("f16", "mxf4"), default="mxf4",
-                    help="weight stream for many positions per expert: bf16 tiles or E2M1 term tiles")
+    ap.add_argument("--large-kind", choices=("f16", "mxf4", "mxf8"), default="mxf4",
+                    help="weight stream for many positions per expert: bf16 tiles, E2M1 term tiles or "
+                         "E4M3 term tiles")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of replaying them as one CUDA graph")
     ap.add_argument("--e2e-steps", type=int, default=None)
@@ -228,6 +229,8 @@ LARGE_KINDS = {
              "terms_gate_up": 5, "terms_down": 5},
     "f16": {"mma": "tcgen05.mma kind::f16 (bf16 x bf16, weights dequantised)", "ratio_to_bf16": 1.0,
             "terms_gate_up": 1, "terms_down": 2},
+    "mxf8": {"mma": "tcgen05.mma kind::mxf8f6f4 (E2M1 x E4M3, E8M0 scales)", "ratio_to_bf16": 2.0,
+             "terms_gate_up": 2, "terms_down": 3},
 }
 
 
@@ -487,7 +490,7 @@ def main():
     if args.shard_i or (world > 1 and not args.replicas and w.layers == 1):
         return run_shard_i(args, mx, w, T, layers, rank, world)
     m = mx.Moe(w.hidden, w.inter, w.experts, w.top_k, T, layers)
-    m.moe_set_large_kind(m.LARGE_F16 if args.large_kind == "f16" else m.LARGE_MXF4)
+    m.moe_set_large_kind({"f16": m.LARGE_F16, "mxf4": m.LARGE_MXF4, "mxf8": m.LARGE_MXF8}[args.large_kind])
     xs = token_blocks(w, T, args.batches, rank)
     hits = []
     for x in xs:

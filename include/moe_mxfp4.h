@@ -314,10 +314,17 @@ MOE_API int32_t moe_stream_profile(moe_mxfp4_t* h, int32_t enable, uint64_t* out
  * moe_set_large_kind -- the weight stream used when a call has many positions
  * per expert (T*K > 256 and T*K >= 8*E): 1 = E2M1 term tiles on the block-
  * scaled fp4 tensor-core MMA (x and the SwiGLU output expanded into five
- * E2M1 terms), 2 = bf16 tiles on the bf16 tensor-core MMA (MXFP4 weights
- * dequantised to bf16 in shared memory, x exact, the SwiGLU output as two
- * bf16 terms).  Default 1 (the faster of the two on B200 at every measured
- * size).  Errors: MOE_ERR_INVALID_ARG.
+ * E2M1 terms; with at most 24 positions per expert and hidden % 256 == 0,
+ * jobs of two row blocks share each activation stage), 2 = bf16 tiles on the
+ * bf16 tensor-core MMA (MXFP4 weights dequantised to bf16 in shared memory, x
+ * exact, the SwiGLU output as two bf16 terms), 3 = E4M3 term tiles on the
+ * block-scaled kind that takes E2M1 weights and E4M3 activations (the MXFP4
+ * weight codes rewritten in shared memory into that kind's 16-byte-chunk
+ * form; x as two E4M3 terms, the SwiGLU output as three).  Default 1.  The
+ * kinds are the ablation of the MXFP4 tensor-core paths (bjdmk.com.cn news,
+ * section "极致协同，通向千速之路", on MXFP4 for the experts; TileRT blog
+ * "Breaking 1000 TPS", section "第一次跃迁：Execution Model Revolution", on
+ * the tensor cores under the tile pipeline).  Errors: MOE_ERR_INVALID_ARG.
  */
 MOE_API int32_t moe_set_large_kind(moe_mxfp4_t* h, int32_t kind);
 

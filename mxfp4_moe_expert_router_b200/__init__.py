@@ -281,10 +281,10 @@ class Moe:
     def moe_set_timeout_ns(self, ns: int):
         _check(lib.moe_set_timeout_ns(self.handle, int(ns)), "moe_set_timeout_ns")
 
-    LARGE_MXF4, LARGE_F16 = 1, 2
+    LARGE_MXF4, LARGE_F16, LARGE_MXF8 = 1, 2, 3
 
     def moe_set_large_kind(self, kind: int):
-        """Weight stream for many positions per expert: LARGE_MXF4 (default) or LARGE_F16."""
+        """Weight stream for many positions per expert: LARGE_MXF4 (default), LARGE_F16 or LARGE_MXF8."""
         _check(lib.moe_set_large_kind(self.handle, int(kind)), "moe_set_large_kind")
 
     @property

@@ -96,7 +96,8 @@ constexpr size_t OFF_DRAIN = OFF_XBAR + NPIPE * 2 * 8;              // [NPIPE]
 constexpr size_t OFF_TMEMBASE = OFF_DRAIN + NPIPE * 8;
 constexpr size_t OFF_JQ = align16(OFF_TMEMBASE + 8);                // [NPIPE][JQ]
 constexpr size_t OFF_XCH = align16(OFF_JQ + NPIPE * JQ * sizeof(JobEntry));  // [NPIPE][2][NT_MAX][4] floats
-constexpr size_t XCH_FLOATS = (NPIPE * 2 * NT_MAX > 4 * LT_MAX ? NPIPE * 2 * NT_MAX : 4 * LT_MAX) * 4;
+constexpr size_t XCH_FLOATS = (NPIPE * 2 * NT_MAX > 4 * ET_MAX ? NPIPE * 2 * NT_MAX : 4 * ET_MAX) * 4;
+static_assert(ET_MAX >= LT_MAX, "amax exchange sized by the largest tile");
 constexpr size_t OFF_TABLES = align16(OFF_XCH + XCH_FLOATS * 4);
 constexpr size_t SMEM_BYTES = OFF_TABLES + sizeof(CtaTables);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -369,7 +370,62 @@ __device__ void phase_images(const EngineParams& p, const __nv_bfloat16* x, int 
   }
 }
 
+// ---- E4M3 term expansion (kind::mxf8f6f4 tiles) -------------------------------------------
+// Exponent of term 0 for a block with amax A: the least s with A <= 448 * 2^s
+// (A = m 2^E, m in [1, 2): s = E - 8 if m <= 1.75, else E - 7), kept in
+// [-118, 127] so that every term exponent s - ET_STEP k (k < 3) has an E8M0
+// byte in [1, 254].
+__device__ __forceinline__ int et_term0_exp(float amax) {
+  const uint32_t u = __float_as_uint(amax);
+  const int E = (int)((u >> 23) & 0xFF) - 127;
+  if (E < -126) return -118;  // zero or subnormal amax
+  const int s = (u & 0x7FFFFFu) <= 0x600000u ? E - 8 : E - 7;
+  return min(max(s, -118), 127);
+}
+// Term k's E4M3 code of v (residual after the previous terms in r, updated).
+__device__ __forceinline__ uint32_t et_term(float& r, int s0, int k) {
+  const int sk = s0 - ET_STEP * k;
+  const uint32_t c = f32_to_e4m3(r * pow2f(-sk));
+  r = fmaf(-e4m3_to_f32(c), pow2f(sk), r);
+  return c;
+}
+
+// x[t] (bf16) -> xe[stage][t]: per 32-element block one warp expands the
+// values into ET_XTERMS E4M3 terms (lane = element); term k's codes at
+// k * 128 + 32 b + lane, its scale byte at 256 + 4 k + b (b = the block in
+// the stage).  Also the layer-input copy of the optional per-layer output.
+__device__ void phase_images_e4m3(const EngineParams& p, const __nv_bfloat16* x, int layer) {
+  const int T = p.T, H = p.H;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t gt = (int64_t)blockIdx.x * THREADS + threadIdx.x;
+  const int64_t gs = (int64_t)gridDim.x * THREADS;
+  const int64_t wg = (int64_t)blockIdx.x * WARPS + warp, ws = (int64_t)gridDim.x * WARPS;
+  const int nblk = H / 32;
+  for (int64_t task = wg; task < (int64_t)T * nblk; task += ws) {
+    const int t = (int)(task / nblk), gb = (int)(task % nblk);
+    float r = __bfloat162float(__ldcg(x + (int64_t)t * H + gb * 32 + lane));
+    float am = fabsf(r);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(FULL, am, o));
+    const int s0 = et_term0_exp(am), b = gb % KB;
+    uint8_t* img = p.xe + ((int64_t)(gb / KB) * T + t) * ET_XIMG;
+#pragma unroll
+    for (int k = 0; k < ET_XTERMS; ++k) img[k * 128 + b * 32 + lane] = (uint8_t)et_term(r, s0, k);
+    if (lane < ET_XTERMS) img[256 + 4 * lane + b] = (uint8_t)(s0 - ET_STEP * lane + 127);
+  }
+  if (p.layer_io) {
+    const int64_t n8 = (int64_t)T * H / 8;
+    const uint4* s8 = reinterpret_cast<const uint4*>(x);
+    uint4* d8 = reinterpret_cast<uint4*>(p.layer_io + (int64_t)layer * T * H);
+    for (int64_t i = gt; i < n8; i += gs) d8[i] = __ldcg(s8 + i);
+  }
+}
+
 // Router partial logits (and the per-layer resets of the stream's counters).
+// RB: 16-byte loads in flight per thread while staging (the chained-layer
+// instance stages a few thousand per CTA in one or two round trips; the
+// single-layer decode instance keeps its register budget with 2).
+template <int RB = 2>
 __device__ void phase_router(const EngineParams& p, const LayerPtrs& lp, const __nv_bfloat16* x,
                              uint8_t* smem) {
   const int T = p.T, H = p.H, E = p.E;
@@ -402,7 +458,6 @@ __device__ void phase_router(const EngineParams& p, const LayerPtrs& lp, const _
       // part's weight slices; a thread's loads are all in flight before its
       // stores (one memory round trip for both)
       const int nx = nt * hp8, nw = (t0 == 0 && wstaged) ? nexp * hp4 : 0;
-      constexpr int RB = 2;
 #pragma unroll 1
       for (int i0 = threadIdx.x; i0 < nx + nw; i0 += RB * THREADS) {
         uint4 v[RB];
@@ -1068,6 +1123,52 @@ __device__ void phase_tile_gather(const EngineParams& p) {
   }
 }
 
+// Large T*K, E4M3 tiles: the x image of every (tile, stage), gathered from the
+// per-token images: term k of position tl is B row n = ET_XTERMS tl + k (its
+// 128 codes as eight 16-byte chunks at et_code_offset(n, 16 c, N)), its scale
+// word at lt_sf_offset(n, 0).  A warp moves one (tile, stage).
+__device__ void phase_tile_gather_e4m3(const EngineParams& p) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ns = p.H / KS, nu = ld_cg_u32(p.n_units);
+  constexpr int CPP = ET_XTERMS * 8;  // 16-byte chunks per position
+  const int64_t ntask = (int64_t)nu * ns;
+  for (int64_t us = (int64_t)blockIdx.x * WARPS + warp; us < ntask; us += (int64_t)gridDim.x * WARPS) {
+    const int u = (int)(us / ns), st = (int)(us % ns);
+    const int4 ur = __ldcg(reinterpret_cast<const int4*>(p.units) + u);
+    const int n = ur.z, N = et_cols(n, ET_XTERMS);
+    static_assert(ET_MAX <= 64, "two token words per lane");
+    const int tok0 = lane < n ? __ldcg(p.tokpos + ur.y + lane) : 0;
+    const int tok1 = lane + 32 < n ? __ldcg(p.tokpos + ur.y + lane + 32) : 0;
+    const uint8_t* xs = p.xe + (int64_t)st * p.T * ET_XIMG;
+    uint8_t* dst = p.xte + us * ET_XB_BYTES;
+    constexpr int B8 = 8;
+    for (int f0 = 0; f0 < n * CPP; f0 += 32 * B8) {
+      uint4 v[B8];
+#pragma unroll
+      for (int i = 0; i < B8; ++i) {
+        const int f = f0 + 32 * i + lane, tl = f / CPP, r = f - tl * CPP, k = r >> 3, c = r & 7;
+        const int ta = __shfl_sync(FULL, tok0, tl & 31), tb = __shfl_sync(FULL, tok1, tl & 31);
+        if (f < n * CPP)
+          v[i] = __ldcg(reinterpret_cast<const uint4*>(xs + (int64_t)(tl < 32 ? ta : tb) * ET_XIMG + k * 128 + c * 16));
+      }
+#pragma unroll
+      for (int i = 0; i < B8; ++i) {
+        const int f = f0 + 32 * i + lane, tl = f / CPP, r = f - tl * CPP, k = r >> 3, c = r & 7;
+        if (f < n * CPP) *reinterpret_cast<uint4*>(dst + et_code_offset(ET_XTERMS * tl + k, 16 * c, N)) = v[i];
+      }
+    }
+    for (int f0 = 0; f0 < n * ET_XTERMS; f0 += 32) {  // scale words: (position, term)
+      const int f = f0 + lane, tl = f / ET_XTERMS, k = f - tl * ET_XTERMS;
+      const int ta = __shfl_sync(FULL, tok0, tl & 31), tb = __shfl_sync(FULL, tok1, tl & 31);
+      if (f < n * ET_XTERMS) {
+        const uint32_t w =
+            __ldcg(reinterpret_cast<const uint32_t*>(xs + (int64_t)(tl < 32 ? ta : tb) * ET_XIMG + 256 + 4 * k));
+        *reinterpret_cast<uint32_t*>(dst + lt_sf_offset(f, 0)) = w;
+      }
+    }
+  }
+}
+
 // ---- bf16 tile stream: permutation into balanced tiles, gather of x ------------------------
 // Unit tables of the bf16 tile stream: an expert's segment of c positions
 // becomes nb = ceil(c / FT_MAX) tiles of c / nb or c / nb + 1 consecutive
@@ -1226,8 +1327,8 @@ template <int TM, int SPLIT = 0>
 __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem,
                                 const StreamCtx& cx, int pipe, RoleState& rs) {
   constexpr bool LT = TM != 0;
-  constexpr int NS = TM == 1 ? LT_NSLOT : TM == 4 ? LTA_NSLOT : NSLOT;  // ring slots
-  constexpr int SLOTB = TM == 1 ? LT_SLOT_BYTES : TM == 4 ? LTA_SLOT_BYTES : SLOT_BYTES;
+  constexpr int NS = TM == 1 ? LT_NSLOT : TM == 4 ? LTA_NSLOT : TM == 6 ? ET_NSLOT : NSLOT;  // ring slots
+  constexpr int SLOTB = TM == 1 ? LT_SLOT_BYTES : TM == 4 ? LTA_SLOT_BYTES : TM == 6 ? ET_SLOT_BYTES : SLOT_BYTES;
   constexpr int R = TM == 4 ? LTA_R : 1;      // row blocks per job
   constexpr int NP = LT ? 1 : NPIPE;         // pipelines per CTA
   constexpr int PB = PRODUCER_BATCH < NS ? PRODUCER_BATCH : NS;
@@ -1326,7 +1427,9 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
     const uint8_t* wbase = isD ? lp.w_d + ((int64_t)e * db + rb) * nc * STAGE_A_BYTES
                                : lp.w_gu + ((int64_t)e * gub + rb) * nc * STAGE_A_BYTES;
     const int tok = (!LT && !isD && lane < nt) ? ld_tab(cx.tokpos + pos0 + lane, cx.global) : 0;
-    const uint32_t bbytes = LT ? (uint32_t)(LT_SF_BYTES + lt_cols(nt) * (IMG_CODE_BYTES / 8)) : (uint32_t)nt * IMG_BYTES;
+    const uint32_t bbytes = TM == 6 ? (uint32_t)et_img_bytes(et_cols(nt, isD ? ET_ATERMS : ET_XTERMS))
+                            : LT    ? (uint32_t)(LT_SF_BYTES + lt_cols(nt) * (IMG_CODE_BYTES / 8))
+                                    : (uint32_t)nt * IMG_BYTES;
     const uint32_t stage_bytes = R * STAGE_A_BYTES + bbytes;
     const int64_t rstep = (int64_t)nc * STAGE_A_BYTES;  // between the stages of consecutive row blocks
     // Stages are issued in batches, one stage per lane: successive 1-D bulk
@@ -1364,7 +1467,9 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
           bulk_g2s_hint(dst, wbase + (int64_t)c * STAGE_A_BYTES, STAGE_A_BYTES, fb, wpolicy);
         }
         if (LT)  // the tile's B operand of this stage, one image
-          bulk_g2s(dst + R * STAGE_A_BYTES, (isD ? p.atl : p.xtl) + ((int64_t)u * nc + c) * LT_IMG_BYTES,
+          bulk_g2s(dst + R * STAGE_A_BYTES,
+                   TM == 6 ? (isD ? p.ate + ((int64_t)u * nc + c) * ET_AB_BYTES : p.xte + ((int64_t)u * nc + c) * ET_XB_BYTES)
+                           : (isD ? p.atl : p.xtl) + ((int64_t)u * nc + c) * LT_IMG_BYTES,
                    bbytes, fb);
         else if (isD)
           bulk_g2s(dst + STAGE_A_BYTES, p.aimg + ((int64_t)c * p.TK + pos0) * IMG_BYTES,
@@ -1767,6 +1872,245 @@ __device__ void stream_epilogue_lt(const EngineParams& p, uint8_t* smem, const S
       const int h0 = rbe * JOB_ROWS;
       for (int j = J0; j < nt; j += JS) {
         const float sum = lt_position_sum(tacc, j);
+        p.ypair[(int64_t)(pos0 + j) * p.H + h0 + 32 * q + lane] = sum * ld_tab(cx.wpos + pos0 + j, cx.global);
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(acce_bar(smem, 0, b));
+    t_work += pclock(prof) - tk0;
+  }
+  if (prof && lane == 0) {
+    atomicAdd(p.prof + PF_EPI_WAIT, t_wait);
+    atomicAdd(p.prof + PF_EPI_WORK, t_work);
+    atomicAdd(p.prof + PF_EPI_TOTAL, pclock(prof) - t_begin);
+    if (q == 0) atomicAdd(p.prof + PF_JOBS, n_jobs);
+  }
+}
+
+// ---- phase C, large T*K, E4M3 tiles on kind::mxf8f6f4 -----------------------------------------
+// Ring slot (ET_SLOT_BYTES): the packed weight stage (STAGE_A_BYTES, from the
+// producer), the tile's B image (from the producer), and the weight codes in
+// the kind's 16-byte-chunk form (ET_U_BYTES, from the converter warps; the
+// MMA still takes the weight scales from the packed stage).  Barriers: full
+// (0, slot) = the producer's copies, full (1, slot) = the converted codes (two
+// converter warps), empty (0, slot) = the MMAs done with the whole slot.
+// Tensor memory: 2 accumulators of ET_ACC_COLS, then NSF scale buffers of 12
+// columns (A: 4, B: 4 per 128 rows).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const EngineParams& p, uint32_t info);
+__device__ __forceinline__ uint32_t et_acc(int b) { return (uint32_t)b * ET_ACC_COLS; }
+__device__ __forceinline__ uint32_t et_sf(int i) { return (uint32_t)(2 * ET_ACC_COLS + i * (4 + 4 * LT_SF_BLOCKS)); }
+__device__ __forceinline__ uint8_t* et_slot(uint8_t* smem, int slot) { return smem + OFF_RING + (size_t)slot * ET_SLOT_BYTES; }
+constexpr int ET_U_OFF = STAGE_A_BYTES + ET_AB_BYTES;
+static_assert(ET_U_OFF % 128 == 0 && (size_t)ET_NSLOT * ET_SLOT_BYTES <= RING_BYTES, "E4M3 ring layout");
+
+// Converter warps (2 and 3): each packed 16-byte chunk (32 E2M1 codes of one
+// weight row: row m, K half kk, 32-element chunk c of the packed stage) becomes
+// the two 16-element chunks of K slice 2 kk + c in the kind's form: 8 packed
+// bytes, then 8 zero bytes.
+__device__ void stream_convert_e(const EngineParams& p, uint8_t* smem, int wl, RoleState& rs) {
+  const int lane = threadIdx.x & 31, tid = 32 * wl + lane;
+  JobEntry* jq = job_queue(smem, 0);
+  bool ok = true;
+  for (;;) {
+    JobEntry* en = jq + (rs.qk % JQ);
+    if (!wait_entry(p, en, rs.qk)) return;
+    const int job = *reinterpret_cast<volatile int32_t*>(&en->job);
+    if (job < 0) { ++rs.qk; break; }
+    const int s0 = en->s0, nc = en->nc;
+    ++rs.qk;
+    if (!ok) continue;
+    for (int c = 0; c < nc; ++c) {
+      const uint32_t s = (uint32_t)s0 + c;
+      const int slot = (int)(s % ET_NSLOT);
+      if (!warp_wait(full_bar(smem, 0, slot), (s / ET_NSLOT) & 1u, p, s)) { ok = false; break; }
+      const uint8_t* raw = et_slot(smem, slot);
+      uint8_t* u = et_slot(smem, slot) + ET_U_OFF;
+#pragma unroll 4
+      for (int i = tid; i < 128 * 4; i += 64) {
+        const int m = i >> 2, q = i & 3, kk = q >> 1, kc = q & 1;
+        const uint4 w = *reinterpret_cast<const uint4*>(raw + kk * 4096 + (m >> 3) * 256 + kc * 128 + (m & 7) * 16);
+        uint8_t* d = u + q * 4096 + (m >> 3) * 256 + (m & 7) * 16;
+        *reinterpret_cast<uint4*>(d) = make_uint4(w.x, w.y, 0u, 0u);
+        *reinterpret_cast<uint4*>(d + 128) = make_uint4(w.z, w.w, 0u, 0u);
+      }
+      fence_proxy_async_smem();  // read by the tensor cores (async proxy)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(full_bar(smem, 1, slot));
+    }
+  }
+}
+
+// MMA issuer of the E4M3 tiles (one thread): per stage the weight scales and
+// the tile's 1-2 scale blocks go to tensor memory, then four MMAs (K = 32
+// each, scale byte i of the stage's block column) accumulate.
+__device__ void stream_mma_e(const EngineParams& p, uint8_t* smem, uint32_t tmem, RoleState& rs) {
+  JobEntry* jq = job_queue(smem, 0);
+  const bool prof = p.prof != nullptr;
+  unsigned long long t_full = 0, t_issue = 0, t_acc = 0;
+  bool ok = true;
+  for (;;) {
+    JobEntry* en = jq + (rs.qk % JQ);
+    if (!wait_entry(p, en, rs.qk)) return;
+    const int job = *reinterpret_cast<volatile int32_t*>(&en->job);
+    if (job < 0) { ++rs.qk; break; }
+    const int s0 = en->s0, nc = en->nc, nt = en->nt, wj = en->wj, isD = en->isD;
+    ++rs.qk;
+    if (!ok) continue;
+    const int b = wj & 1;
+    const uint32_t use = (uint32_t)(wj >> 1);
+    const unsigned long long ta0 = pclock(prof);
+    if (use > 0 &&
+        !wait_mbar(acce_bar(smem, 0, b), (use - 1) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, wj)) {
+      ok = false;
+      continue;
+    }
+    t_acc += pclock(prof) - ta0;
+    tc_fence_after();
+    const uint32_t tacc = tmem + et_acc(b);
+    const int n = et_cols(nt, isD ? ET_ATERMS : ET_XTERMS), nblk = (n + 127) / 128;
+    for (int c = 0; c < nc; ++c) {
+      const uint32_t s = (uint32_t)s0 + c;
+      const int slot = (int)(s % ET_NSLOT);
+      const unsigned long long tf0 = pclock(prof);
+      if (!wait_mbar(full_bar(smem, 0, slot), (s / ET_NSLOT) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, s) ||
+          !wait_mbar(full_bar(smem, 1, slot), (s / ET_NSLOT) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, s)) {
+        ok = false;
+        break;
+      }
+      const unsigned long long tm0 = pclock(prof);
+      t_full += tm0 - tf0;
+      tc_fence_after();
+      const uint32_t sa = smem_u32(et_slot(smem, slot)), sb = sa + STAGE_A_BYTES, su = sa + ET_U_OFF;
+      const uint32_t tsf = tmem + et_sf((int)(rs.sfc++ % NSF)), tsb = tsf + 4;
+      tmem_cp_sf(tsf, smem_desc(sa + STAGE_CODE_BYTES, 0, 128));
+      for (int q = 0; q < nblk; ++q) tmem_cp_sf(tsb + 4 * q, smem_desc(sb + q * 512, 0, 128));
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        mma_mxf8(tacc, smem_desc(su + i * 4096, 128, 256), smem_desc(sb + LT_SF_BYTES + i * n * 32, 128, 256),
+                 mxf8_idesc(n, (uint32_t)i), tsf | ((uint32_t)i << 30), tsb | ((uint32_t)i << 30),
+                 (c > 0 || i > 0) ? 1u : 0u);
+      tc_commit(empty_bar(smem, 0, slot));
+      t_issue += pclock(prof) - tm0;
+    }
+    if (ok) tc_commit(accf_bar(smem, 0, b));
+  }
+  if (prof) {
+    atomicAdd(p.prof + PF_MMA_FULL, t_full);
+    atomicAdd(p.prof + PF_MMA_ISSUE, t_issue);
+    atomicAdd(p.prof + PF_MMA_ACC, t_acc);
+  }
+}
+
+// Sum of position j's NT accumulator columns (this warp's 32 rows), the
+// eight-column group holding the first and the next one when the terms cross
+// into it; terms summed last to first.
+template <int NT>
+__device__ __forceinline__ float et_position_sum(uint32_t tacc, int j) {
+  const int c0 = NT * j, g0 = c0 & ~7;
+  float v[16];
+  tmem_ld8(tacc + g0, *reinterpret_cast<float(*)[8]>(v));
+  if (c0 + NT > g0 + 8) tmem_ld8(tacc + g0 + 8, *reinterpret_cast<float(*)[8]>(v + 8));
+  float sum = 0.f;
+#pragma unroll
+  for (int k = NT - 1; k >= 0; --k) {
+    float t = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i == c0 - g0 + k) t = v[i];
+    sum = k == NT - 1 ? t : sum + t;
+  }
+  return sum;
+}
+
+// Epilogue of the E4M3 tiles: eight warps in two sets (positions set, set + 2,
+// ...), warp q reading accumulator rows 32 q .. 32 q + 31.  Gate/up: SwiGLU
+// of the gate and up rows (lanes l, l + 16), the block amax shared with warp
+// q ^ 1, ET_ATERMS E4M3 terms of the output written into the tile's down
+// image (row n = 3 j + k, this warp's 16 elements at 16 (q % 2) of block
+// 2 kk + q / 2); down: the position's column sum times the routing weight.
+__device__ void stream_epilogue_e(const EngineParams& p, uint8_t* smem, const StreamCtx& cx, uint32_t tmem,
+                                  int set, RoleState& rs) {
+  const int lane = threadIdx.x & 31, q = (threadIdx.x >> 5) & 3;
+  JobEntry* jq = job_queue(smem, 0);
+  uint32_t* ready = p.sync + SY_READY;
+  const int nsd = p.I / KS;
+  const bool prof = p.prof != nullptr;
+  unsigned long long t_wait = 0, t_work = 0, n_jobs = 0;
+  const unsigned long long t_begin = pclock(prof);
+  bool ok = true;
+  float av[ET_MAX];
+  for (;;) {
+    JobEntry* en = jq + (rs.qk % JQ);
+    if (!wait_entry(p, en, rs.qk)) return;
+    const int job = *reinterpret_cast<volatile int32_t*>(&en->job);
+    if (job < 0) { ++rs.qk; break; }
+    const int wj = en->wj;
+    const int u = en->unit, rb = en->rb, isD = en->isD, pos0 = en->pos0, nt = en->nt;
+    ++rs.qk;
+    if (!ok) continue;
+    ++n_jobs;
+    const uint32_t gc = isD ? 0u : rs.gcount++;
+    const int b = wj & 1;
+    const unsigned long long tw0 = pclock(prof);
+    if (!wait_mbar(accf_bar(smem, 0, b), (uint32_t)(wj >> 1) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, wj)) {
+      ok = false;
+      continue;
+    }
+    const unsigned long long tk0 = pclock(prof);
+    t_wait += tk0 - tw0;
+    tc_fence_after();
+    const uint32_t tacc = tmem + ((uint32_t)(32 * q) << 16) + et_acc(b);
+    if (!isD) {
+      const int xb = (int)(gc & 1u);
+      float* xc = reinterpret_cast<float*>(smem + OFF_XCH) + (set * 2 + xb) * ET_MAX * 4;
+      for (int j = set; j < nt; j += 2) {
+        const float sum = et_position_sum<ET_XTERMS>(tacc, j);
+        const float other = __shfl_xor_sync(FULL, sum, 16);
+        const float g = lane < 16 ? sum : other, up = lane < 16 ? other : sum;
+        const float a = g / (1.0f + expf(-g)) * up;
+        av[j] = a;
+        float am = fabsf(a);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(FULL, am, o));
+        if (lane == 0) xc[j * 4 + q] = am;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xch_bar(smem, set, xb));
+      if (!wait_mbar(xch_bar(smem, set, xb), (gc >> 1) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, wj)) {
+        ok = false;
+        continue;
+      }
+      const int i0 = rb * GU_I_ROWS, sD = i0 / KS, blk = 2 * ((i0 % KS) / 64) + (q >> 1);
+      const int N = et_cols(nt, ET_ATERMS);
+      uint8_t* img = p.ate + ((int64_t)u * nsd + sD) * ET_AB_BYTES;
+      const int e0 = 32 * blk + 16 * (q & 1);  // this warp's first element of the stage
+      for (int j = set; j < nt; j += 2) {
+        const int s0 = et_term0_exp(fmaxf(xc[j * 4 + q], xc[j * 4 + (q ^ 1)]));
+        float r = av[j];
+#pragma unroll
+        for (int k = 0; k < ET_ATERMS; ++k) {
+          const uint32_t c = et_term(r, s0, k);
+          // lanes 4 w .. 4 w + 3 (w < 4) pack their bytes into one word: elements e0 + 4 w .. + 3
+          const uint32_t c1 = __shfl_down_sync(FULL, c, 1), c2 = __shfl_down_sync(FULL, c, 2),
+                         c3 = __shfl_down_sync(FULL, c, 3);
+          if (lane < 16 && (lane & 3) == 0)
+            *reinterpret_cast<uint32_t*>(img + et_code_offset(ET_ATERMS * j + k, e0 + lane, N)) =
+                c | (c1 << 8) | (c2 << 16) | (c3 << 24);
+        }
+        if ((q & 1) == 0 && lane < ET_ATERMS)
+          img[lt_sf_offset(ET_ATERMS * j + lane, blk)] = (uint8_t)(s0 - ET_STEP * lane + 127);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        fence_proxy_async_global();
+        __threadfence();
+        red_release_add_u32(ready + u, 1u);
+      }
+    } else {
+      const int h0 = rb * JOB_ROWS;
+      for (int j = set; j < nt; j += 2) {
+        const float sum = et_position_sum<ET_ATERMS>(tacc, j);
         p.ypair[(int64_t)(pos0 + j) * p.H + h0 + 32 * q + lane] = sum * ld_tab(cx.wpos + pos0 + j, cx.global);
       }
     }
@@ -2426,7 +2770,8 @@ __device__ void prefetch_share(const void* base, size_t bytes) {
 // MODE 0: pipeline stream, one layer, plain combine (the decode kernel); MODE 5:
 // pipeline stream with chained layers (RMSNorm) or the fused all-reduce; MODE 1:
 // E2M1 term tiles (kind::mxf4); MODE 4: E2M1 term tile pairs (two row blocks per
-// job); MODE 2: bf16 tiles (kind::f16).  The tile modes run only above SMALL_PAIRS.
+// job); MODE 6: E4M3 term tiles (kind::mxf8f6f4); MODE 2: bf16 tiles
+// (kind::f16).  The tile modes run only above SMALL_PAIRS.
 template <int MODE>
 __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, RoleState& rs,
                            bool stamp) {
@@ -2439,7 +2784,7 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
     const __nv_bfloat16* x = layer == 0 ? p.x_in : p.xnext;
     uint64_t* st = stamp ? p.stamps + 1 + layer * STAMPS_PER_LAYER : nullptr;
     if constexpr (!PIPE) phase_router_tiles(x, lp.router_w, p.logits, p.sync, p.T, p.H, p.E, p.TK, p.HS, smem);
-    else phase_router(p, lp, x, smem);
+    else phase_router<MODE == 5 ? 10 : 2>(p, lp, x, smem);
     if (st) st[0] = globaltimer_ns();
     StreamCtx cx;
     const int32_t* inv;
@@ -2450,7 +2795,8 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
       cx = StreamCtx{tb.units, tb.dunits, tb.tokpos, tb.wpos, tb.n_units, tb.n_dunits, false};
       inv = tb.inv;
     } else {
-      if constexpr (MODE != 2) phase_images(p, x, layer);  // the bf16 tiles gather x itself
+      if constexpr (MODE == 6) phase_images_e4m3(p, x, layer);
+      else if constexpr (MODE != 2) phase_images(p, x, layer);  // the bf16 tiles gather x itself
       if (st) st[1] = globaltimer_ns();
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 1)) return;
       if (st) st[2] = globaltimer_ns();
@@ -2458,11 +2804,14 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 2)) return;
       if (st) st[3] = globaltimer_ns();
       if constexpr (MODE == 2) phase_permute_f16(p, smem);
-      else phase_permute_large(p, smem, MODE == 4 ? LTA_MAX : MODE == 1 ? LT_MAX : NT_MAX);
+      else phase_permute_large(p, smem, MODE == 6 ? ET_MAX : MODE == 4 ? LTA_MAX : MODE == 1 ? LT_MAX : NT_MAX);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 3)) return;
       if (p.route_only) return;
       if constexpr (MODE == 1 || MODE == 4) {
         phase_tile_gather(p);
+        if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 6)) return;
+      } else if constexpr (MODE == 6) {
+        phase_tile_gather_e4m3(p);
         if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 6)) return;
       } else if constexpr (MODE == 2) {
         phase_tile_gather_f16(p, x);
@@ -2499,6 +2848,17 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
         __syncwarp();
       } else if (warp >= EPI_WARP0) {
         stream_epilogue_lt<MODE>(p, smem, cx, tmem, warp >= EPI_WARP0 + 4 ? 1 : 0, rs);
+      }
+    } else if constexpr (MODE == 6) {  // E4M3 tiles: producer, MMA issuer, two converter warps, eight epilogue warps
+      if (warp == 0) {
+        stream_producer<6>(p, lp, smem, cx, 0, rs);
+      } else if (warp == 1) {
+        if (lane == 0) stream_mma_e(p, smem, tmem, rs);
+        __syncwarp();
+      } else if (warp < EPI_WARP0) {
+        stream_convert_e(p, smem, warp - 2, rs);
+      } else {
+        stream_epilogue_e(p, smem, cx, tmem, warp >= EPI_WARP0 + 4 ? 1 : 0, rs);
       }
     } else {  // bf16 tiles: producer, MMA issuer, six converter warps, four epilogue warps
       if (warp == 0) {
@@ -2583,8 +2943,8 @@ __device__ void run_op(const EngineParams& p, uint8_t* smem, uint32_t tmem, Role
   }
 }
 
-// Six instances: MODE 0, 1, 2, 4, 5 (see run_layers), each holding only its
-// own stream code, and MODE 3, one operator per launch (run_op).
+// Seven instances: MODE 0, 1, 2, 4, 5, 6 (see run_layers), each holding only
+// its own stream code, and MODE 3, one operator per launch (run_op).
 template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -2595,12 +2955,14 @@ __global__ void __launch_bounds__(THREADS, 1) engine_kernel(const EngineParams p
         // bf16 tiles: a raw slot is free once every converter warp has read
         // it (rawempty_bar), an A block is full once every converter warp
         // has written it (afull_bar)
-        mbar_init(full_bar(smem, pp, i), MODE == 2 && pp == 1 && i >= FT_NB ? FT_CONV_WARPS : 1);
+        // E4M3 tiles: pipe 1's full barriers announce the converted weight codes (two warps)
+        mbar_init(full_bar(smem, pp, i), MODE == 2 && pp == 1 && i >= FT_NB ? FT_CONV_WARPS
+                                         : MODE == 6 && pp == 1 ? 2 : 1);
         mbar_init(empty_bar(smem, pp, i), MODE == 2 && pp == 0 ? FT_CONV_WARPS : 1);
       }
       for (int i = 0; i < NACC; ++i) {
         mbar_init(accf_bar(smem, pp, i), 1);
-        mbar_init(acce_bar(smem, pp, i), (MODE == 1 || MODE == 4) && pp == 0 ? 8 : 4);  // tiles: eight epilogue warps
+        mbar_init(acce_bar(smem, pp, i), (MODE == 1 || MODE == 4 || MODE == 6) && pp == 0 ? 8 : 4);  // tiles: eight epilogue warps
       }
       for (int i = 0; i < 2; ++i) mbar_init(xch_bar(smem, pp, i), 4);
       mbar_init(drain_bar(smem, pp), 1);
@@ -2647,7 +3009,8 @@ size_t engine_smem_bytes() { return SMEM_BYTES; }
 int engine_max_grid(int device, int* err) {
   int per_sm = ~0u >> 1, sms = 0;
   for (const void* k : {(const void*)engine_kernel<0>, (const void*)engine_kernel<1>, (const void*)engine_kernel<2>,
-                        (const void*)engine_kernel<3>, (const void*)engine_kernel<4>, (const void*)engine_kernel<5>}) {
+                        (const void*)engine_kernel<3>, (const void*)engine_kernel<4>, (const void*)engine_kernel<5>,
+                        (const void*)engine_kernel<6>}) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) { *err = (int)e; return 0; }
     int n = 0;
@@ -2667,6 +3030,7 @@ cudaError_t engine_launch(const EngineParams& p, int grid, cudaStream_t s) {
   const void* k = !use_tiles(p.TK, p.E) || p.route_only ? (plain || p.route_only ? (const void*)engine_kernel<0>
                                                                                 : (const void*)engine_kernel<5>)
                   : p.large == LARGE_F16                  ? (const void*)engine_kernel<2>
+                  : p.large == LARGE_MXF8                 ? (const void*)engine_kernel<6>
                   : use_tile_pairs(p.TK, p.E, p.H)         ? (const void*)engine_kernel<4>
                                                           : (const void*)engine_kernel<1>;
   return cudaLaunchCooperativeKernel(k, dim3(grid), dim3(THREADS), args, SMEM_BYTES, s);

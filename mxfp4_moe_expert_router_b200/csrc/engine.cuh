@@ -153,7 +153,50 @@ __host__ __device__ constexpr int ft_b_offset(int r, int k, int rows) {
 // Tiles of the bf16 stream (at most FT_MAX positions each, balanced).
 __host__ __device__ inline int max_ftiles(int E, int64_t TK) { return (int)((E < TK ? E : TK) + TK / FT_MAX + 1); }
 // Large-T*K stream kind: 1 = E2M1 term tiles on kind::mxf4, 2 = bf16 tiles on kind::f16.
-enum : int { LARGE_MXF4 = 1, LARGE_F16 = 2 };
+// ---- large T*K: E4M3 term tiles on kind::mxf8f6f4 ---------------------------------------
+// The block-scaled kind that takes E2M1 weights and E4M3 activations.  Each
+// activation value is an exact-to-fp32-rounding sum of block-scaled E4M3
+// terms with fixed exponent steps: s_0 = the least s with amax <= 448 * 2^s
+// for the 32-element block, s_k = s_0 - 4 k, each term rounding the remaining
+// residual to nearest.  x takes ET_XTERMS = 2 terms (bf16 has 8 significant
+// bits: exact except for about 6e-5 of the values, worst residual 3e-7 of the
+// block max), the SwiGLU output ET_ATERMS = 3 (residual below 6e-5 of the
+// block max).  A tile holds at most ET_MAX positions; its B rows are
+// n = terms * tl + k, N rounded up to 16.
+// The weights stay packed MXFP4 in HBM and in the ring; two converter warps
+// rewrite each stage's codes into the kind's shared-memory form for 4-bit
+// data, 16 elements per 16-byte chunk: 8 packed bytes (element 2j in the low
+// nibble of byte j), then 8 zero bytes.  8-bit operands are K-major 8-row x
+// 16-byte core matrices; an MMA covers K = 32 (one scale block, selected by
+// the scale-factor byte index).
+// Per-token x images: [H/KS][T][ET_XIMG] bytes: term k's 128 codes at k * 128,
+// its 4 block scales at 256 + 4 k.  Tile images (B operand of one stage):
+// the scale-factor block (LT_SF_BYTES, lt_sf_offset layout), then the codes of
+// K slice i (32 elements) at LT_SF_BYTES + i * N * 32 as [N/8][2][8][16].
+constexpr int ET_XTERMS = 2, ET_ATERMS = 3;
+constexpr int ET_STEP = 4;                               // exponent step between terms
+constexpr int ET_MAX = 64;
+constexpr int ET_XIMG = 272;                             // per-token x image bytes per stage
+constexpr int ET_ACC_COLS = 192;                         // 3 terms x 64 positions
+constexpr int ET_XB_BYTES = LT_SF_BYTES + 4 * 128 * 32;  // gate/up B image at most (N <= 128)
+constexpr int ET_AB_BYTES = LT_SF_BYTES + 4 * ET_ACC_COLS * 32;  // down B image at most (N <= 192)
+constexpr int ET_U_BYTES = 128 * KS;                     // a stage's codes in the 16-byte-chunk form
+constexpr int ET_SLOT_BYTES = STAGE_A_BYTES + ET_AB_BYTES + ET_U_BYTES;  // raw stage, B image, converted A
+constexpr int ET_NSLOT = 4;
+static_assert(ET_ATERMS * ET_MAX <= ET_ACC_COLS && ET_XTERMS * ET_MAX <= 128, "E4M3 tile columns");
+static_assert(2 * ET_ACC_COLS + NSF * (4 + 4 * LT_SF_BLOCKS) <= TMEM_COLS, "tensor memory (E4M3 tiles)");
+static_assert(ET_SLOT_BYTES % 128 == 0 && ET_NSLOT <= NPIPE * NSLOT, "E4M3 tile ring");
+// B rows of a tile of nt positions with `terms` terms per position (a multiple of 16).
+__host__ __device__ constexpr int et_cols(int nt, int terms) { return (terms * nt + 15) & ~15; }
+// Byte offset in an E4M3 tile image of element e (0..127 of the stage) of B row n, N rows.
+__host__ __device__ constexpr int et_code_offset(int n, int e, int N) {
+  return LT_SF_BYTES + (e / 32) * N * 32 + (n / 8) * 256 + ((e % 32) / 16) * 128 + (n % 8) * 16 + (e % 16);
+}
+__host__ __device__ constexpr int et_img_bytes(int N) { return LT_SF_BYTES + 4 * N * 32; }
+// Tiles of the E4M3 stream (at most ET_MAX positions each).
+__host__ __device__ inline int max_etiles(int E, int64_t TK) { return (int)((E < TK ? E : TK) + TK / ET_MAX + 1); }
+
+enum : int { LARGE_MXF4 = 1, LARGE_F16 = 2, LARGE_MXF8 = 3 };
 
 // Whether a launch of T*K pairs over E experts streams tiles.
 __host__ __device__ inline bool use_tiles(int64_t TK, int E) {
@@ -247,7 +290,10 @@ struct EngineParams {
   uint8_t* atl;               // large T*K: [tiles][I/KS][LT_IMG_BYTES] SwiGLU term images per tile
   uint8_t* xtf;               // bf16 tiles: [tiles][H/FT_HK][FT_TERM_BYTES] x per tile
   uint8_t* atf;               // bf16 tiles: [tiles][I/FT_HK][2][FT_TERM_BYTES] SwiGLU output terms per tile
-  int large;                  // stream kind above SMALL_PAIRS with tiles: LARGE_MXF4 or LARGE_F16
+  uint8_t* xe;                // E4M3 tiles: [H/KS][T][ET_XIMG] per-token x term images
+  uint8_t* xte;               // E4M3 tiles: [tiles][H/KS][ET_XB_BYTES] x tile images
+  uint8_t* ate;               // E4M3 tiles: [tiles][I/KS][ET_AB_BYTES] SwiGLU output tile images
+  int large;                  // stream kind above SMALL_PAIRS with tiles: LARGE_MXF4, LARGE_F16 or LARGE_MXF8
   float* ypair;               // [TK][H]
   uint32_t* sync;             // see SY_*
   uint64_t* stamps;           // null or [1 + MAX_LAYERS * STAMPS_PER_LAYER] %globaltimer ns (CTA 0)

@@ -28,6 +28,7 @@ struct moe_mxfp4 {
   uint8_t* aimg = nullptr;
   uint8_t* xtl = nullptr;  // large T*k only
   uint8_t* atl = nullptr;
+  uint8_t *xe = nullptr, *xte = nullptr, *ate = nullptr;  // large T*k only (E4M3 tiles)
   uint8_t* xtf = nullptr;  // large T*k only (bf16 tiles)
   uint8_t* atf = nullptr;
   int large = LARGE_MXF4;  // stream kind for large T*k
@@ -146,6 +147,7 @@ EngineParams base_params(const moe_mxfp4* h, int T) {
   p.units = h->units; p.dunits = h->dunits; p.n_units = h->n_units; p.aimg = h->aimg;
   p.xtl = h->xtl; p.atl = h->atl;
   p.xtf = h->xtf; p.atf = h->atf; p.large = h->large;
+  p.xe = h->xe; p.xte = h->xte; p.ate = h->ate;
   p.ypair = h->ypair;
   p.sync = h->sync;
   p.stamps = h->stamps;
@@ -255,6 +257,9 @@ int32_t moe_mxfp4_create(const moe_config_t* cfg, const uint8_t* const* gate_cod
     const size_t ftiles = (size_t)max_ftiles(E, TKm);
     ok = ok && dalloc(h, &h->xtf, ftiles * (H / FT_HK) * FT_TERM_BYTES) &&
          dalloc(h, &h->atf, ftiles * (I / FT_HK) * 2 * FT_TERM_BYTES);
+    const size_t etiles = (size_t)max_etiles(E, TKm);
+    ok = ok && dalloc(h, &h->xe, (size_t)(H / KS) * Tm * ET_XIMG) &&
+         dalloc(h, &h->xte, etiles * (H / KS) * ET_XB_BYTES) && dalloc(h, &h->ate, etiles * (I / KS) * ET_AB_BYTES);
   }
   if (!ok) { free_all(h); delete h; cudaGetLastError(); return MOE_ERR_OOM; }
 
@@ -458,7 +463,7 @@ int32_t moe_round_bf16(const float* in_f32, void* out_bf16, int64_t n, void* str
 }
 
 int32_t moe_set_large_kind(moe_mxfp4_t* h, int32_t kind) {
-  if (!h || (kind != LARGE_MXF4 && kind != LARGE_F16)) return MOE_ERR_INVALID_ARG;
+  if (!h || (kind != LARGE_MXF4 && kind != LARGE_F16 && kind != LARGE_MXF8)) return MOE_ERR_INVALID_ARG;
   h->large = kind;
   return MOE_OK;
 }

@@ -8,6 +8,7 @@
 #pragma once
 #include <stdint.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace moe {
 
@@ -197,6 +198,21 @@ __device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float hi, float lo) {
   return r;
 }
 
+// ---- E4M3 ------------------------------------------------------------------------
+// fp32 -> E4M3 code (low byte), round to nearest even, saturating to +-448.
+__device__ __forceinline__ uint32_t f32_to_e4m3(float v) {
+  uint32_t r;
+  asm("{\n .reg .b16 h;\n cvt.rn.satfinite.e4m3x2.f32 h, %1, %2;\n cvt.u32.u16 %0, h;\n}\n"
+      : "=r"(r) : "f"(0.f), "f"(v));
+  return r & 0xFFu;
+}
+// E4M3 code (low byte) -> its value, exact (every E4M3 value is an f16 value).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+  uint32_t r;
+  asm("{\n .reg .b16 h;\n cvt.u16.u32 h, %1;\n cvt.rn.f16x2.e4m3x2 %0, h;\n}\n" : "=r"(r) : "r"(code & 0xFFu));
+  return __half2float(__ushort_as_half((unsigned short)(r & 0xFFFFu)));
+}
+
 // Named barrier among `count` threads (id 1..15; 0 is __syncthreads).
 __device__ __forceinline__ void named_barrier(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -258,6 +274,25 @@ __device__ __forceinline__ void mma_mxf4(uint32_t tmem_d, uint64_t adesc, uint64
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n}\n"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
+// Instruction descriptor of kind::mxf8f6f4 with E2M1 A and E4M3 B (E8M0
+// scales per 32 elements), M = 128, K-major A and B, N columns; sf = the
+// scale-factor byte (0..3, one 32-element block) used by this MMA.
+__device__ __forceinline__ uint32_t mxf8_idesc(int n, uint32_t sf) {
+  return (sf << 4) | (5u << 7) | (0u << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) |
+         ((uint32_t)(128 >> 4) << 24) | (sf << 29);
+}
+
+// D[128 x N] (+)= (A * 2^SFA) (B * 2^SFB)^T over K = 32, fp32 accumulate in
+// tensor memory; issued by one thread.
+__device__ __forceinline__ void mma_mxf8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n}\n"
       ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
       : "memory");
 }

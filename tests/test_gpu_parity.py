@@ -108,20 +108,22 @@ def test_forward_matches_oracle(m, name):
     check_forward(y, x_values(xb), lw, w.top_k)
 
 
-@pytest.mark.parametrize("kind", ["mxf4", "f16"])
+@pytest.mark.parametrize("kind", ["mxf4", "f16", "mxf8"])
 @pytest.mark.parametrize("name,tokens", [("ragged_large", 80), ("ragged_large", 192), ("pairs", 80),
-                                         ("pairs", 96), ("pairs", 101)])
+                                         ("pairs", 96), ("pairs", 101), ("pairs", 300)])
 def test_large_t_kinds_match_oracle(m, kind, name, tokens):
-    """Both weight streams for many positions per expert (E2M1 term tiles on the
-    fp4 MMA, bf16 tiles on the bf16 MMA): ragged tiles, T*K = 320 and 768 with one
-    row block per job, T*K = 320 and 384 as tile pairs (segments split into tiles
-    of at most 22), T*K = 404 back on single row blocks."""
+    """The three weight streams for many positions per expert (E2M1 term tiles on
+    the fp4 MMA, bf16 tiles on the bf16 MMA, E4M3 term tiles on the fp8/fp6/fp4
+    MMA): ragged tiles, T*K = 320 and 768 with one row block per job, T*K = 320
+    and 384 as tile pairs (segments split into tiles of at most 22), T*K = 404
+    back on single row blocks, T*K = 1200 (75 positions per expert: several
+    tiles of every kind per expert)."""
     from tests.gpu_helpers import bf16_dev, check_forward, make_moe
     H, I, E, k, _ = SHAPES[name]
     w = synth.Workload(name, H, I, E, k, tokens, device_draw=False)
     xb, lw, _ = quantized_layer_np(w, seed=23)
     mo = make_moe(w, [lw])
-    mo.moe_set_large_kind(mo.LARGE_MXF4 if kind == "mxf4" else mo.LARGE_F16)
+    mo.moe_set_large_kind({"mxf4": mo.LARGE_MXF4, "f16": mo.LARGE_F16, "mxf8": mo.LARGE_MXF8}[kind])
     y = mo.moe_forward(bf16_dev(xb))
     mo.moe_status()
     check_forward(y, x_values(xb), lw, w.top_k)
