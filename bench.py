@@ -458,6 +458,9 @@ def blas_threads() -> int:
 
 # ---- main ------------------------------------------------------------------------------------------
 
+PHASES = ("router_logits", "x_images", "route_wait", "topk_or_tables", "permute", "stream", "combine")
+
+
 def main():
     args = parse_args()
     import torch
@@ -645,8 +648,9 @@ def main():
             "per_call": per_call,
             "gpu_launches": args.steps,
             "phase_us_last_step": {k: round(v / 1e3, 2) for k, v in
-                                   zip(("router_logits", "x_images", "route_wait", "topk_or_tables", "permute", "stream",
-                                       "combine"), phases[:7])},
+                                   zip(PHASES, phases[:7])},
+            "phase_us_mean_over_layers": None if w.layers == 1 else
+                {k: round(float(np.mean(phases[i::7][:w.layers])) / 1e3, 2) for i, k in enumerate(PHASES)},
             "e2e": e2e,
             "ops_baseline": ops,
             "cpu_baseline": cpu,

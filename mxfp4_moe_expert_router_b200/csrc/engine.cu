@@ -338,9 +338,11 @@ __device__ __noinline__ void router_chunk(const double* xd, const float* wsm, co
 }
 
 // x[t] (bf16) -> xt[stage][t]: per 32-element block one warp expands the values
-// into NTERM E2M1 terms (codes at the MMA's B-operand rows, scales at the
-// scale-factor rows of the image).  Also the layer-input copy of the optional
-// per-layer output.
+// into E2M1 terms (codes at the MMA's B-operand rows, scales at the
+// scale-factor rows of the image): all NTERM, or the first NT (the tile
+// streams read only LT_NTERM; term rows past NT get zero codes).  Also the
+// layer-input copy of the optional per-layer output.
+template <int NT = NTERM>
 __device__ void phase_images(const EngineParams& p, const __nv_bfloat16* x, int layer) {
   const int T = p.T, H = p.H;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -356,7 +358,7 @@ __device__ void phase_images(const EngineParams& p, const __nv_bfloat16* x, int 
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(FULL, am, o));
     const int s0 = term0_exp(am);
-    const uint32_t word = term_word<32>(e2m1_terms(v, s0), lane);
+    const uint32_t word = term_word<32>(e2m1_terms<NT>(v, s0), lane);
     const int b = gb % KB, kk = b >> 1, kc = b & 1;
     uint8_t* img = p.xt + ((int64_t)(gb / KB) * T + t) * IMG_BYTES;
     *reinterpret_cast<uint32_t*>(img + kk * 256 + kc * 128 + (lane >> 2) * 16 + (lane & 3) * 4) = word;
@@ -2777,13 +2779,17 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
                            bool stamp) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr bool PIPE = MODE == 0 || MODE == 5;  // pipeline stream (units of <= NT_MAX positions)
-  const bool small = PIPE && p.TK <= SMALL_PAIRS;
+  // MODE 0 is launched only for T*K <= SMALL_PAIRS: its routing is always per CTA
+  const bool small = PIPE && (MODE == 0 || p.TK <= SMALL_PAIRS);
   CtaTables& tb = tables(smem);
   for (int layer = 0; layer < p.L; ++layer) {
     const LayerPtrs& lp = p.layers[layer];
     const __nv_bfloat16* x = layer == 0 ? p.x_in : p.xnext;
     uint64_t* st = stamp ? p.stamps + 1 + layer * STAMPS_PER_LAYER : nullptr;
+    // the fp64 MMA router wherever the routing is grid-wide (T*K > SMALL_PAIRS):
+    // from a few dozen tokens its 8-token tiles are full enough to pay
     if constexpr (!PIPE) phase_router_tiles(x, lp.router_w, p.logits, p.sync, p.T, p.H, p.E, p.TK, p.HS, smem);
+    else if (MODE == 5 && !small) phase_router_tiles(x, lp.router_w, p.logits, p.sync, p.T, p.H, p.E, p.TK, p.HS, smem);
     else phase_router<MODE == 5 ? 10 : 2>(p, lp, x, smem);
     if (st) st[0] = globaltimer_ns();
     StreamCtx cx;
@@ -2796,6 +2802,7 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
       inv = tb.inv;
     } else {
       if constexpr (MODE == 6) phase_images_e4m3(p, x, layer);
+      else if constexpr (MODE == 1 || MODE == 4) phase_images<LT_NTERM>(p, x, layer);
       else if constexpr (MODE != 2) phase_images(p, x, layer);  // the bf16 tiles gather x itself
       if (st) st[1] = globaltimer_ns();
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 1)) return;
@@ -3026,9 +3033,11 @@ int engine_max_grid(int device, int* err) {
 
 cudaError_t engine_launch(const EngineParams& p, int grid, cudaStream_t s) {
   void* args[] = {const_cast<EngineParams*>(&p)};
-  const bool plain = p.L == 1 && p.ar.world == 0;  // MODE 0's launch rule
-  const void* k = !use_tiles(p.TK, p.E) || p.route_only ? (plain || p.route_only ? (const void*)engine_kernel<0>
-                                                                                : (const void*)engine_kernel<5>)
+  // MODE 0's launch rule: routing per CTA (T*K <= SMALL_PAIRS), one layer, no
+  // all-reduce (or routing only); every other pipeline launch takes MODE 5
+  const bool plain = p.TK <= SMALL_PAIRS && ((p.L == 1 && p.ar.world == 0) || p.route_only);
+  const void* k = !use_tiles(p.TK, p.E) || p.route_only ? (plain ? (const void*)engine_kernel<0>
+                                                                 : (const void*)engine_kernel<5>)
                   : p.large == LARGE_F16                  ? (const void*)engine_kernel<2>
                   : p.large == LARGE_MXF8                 ? (const void*)engine_kernel<6>
                   : use_tile_pairs(p.TK, p.E, p.H)         ? (const void*)engine_kernel<4>
