@@ -96,7 +96,7 @@ constexpr size_t OFF_DRAIN = OFF_XBAR + NPIPE * 2 * 8;              // [NPIPE]
 constexpr size_t OFF_TMEMBASE = OFF_DRAIN + NPIPE * 8;
 constexpr size_t OFF_JQ = align16(OFF_TMEMBASE + 8);                // [NPIPE][JQ]
 constexpr size_t OFF_XCH = align16(OFF_JQ + NPIPE * JQ * sizeof(JobEntry));  // [NPIPE][2][NT_MAX][4] floats
-constexpr size_t XCH_FLOATS = (NPIPE * 2 * NT_MAX > 4 * ET_MAX ? NPIPE * 2 * NT_MAX : 4 * ET_MAX) * 4;
+constexpr size_t XCH_FLOATS = (NPIPE * 2 * NT_BIG > 4 * ET_MAX ? NPIPE * 2 * NT_BIG : 4 * ET_MAX) * 4;
 static_assert(ET_MAX >= LT_MAX, "amax exchange sized by the largest tile");
 constexpr size_t OFF_TABLES = align16(OFF_XCH + XCH_FLOATS * 4);
 constexpr size_t SMEM_BYTES = OFF_TABLES + sizeof(CtaTables);
@@ -114,6 +114,26 @@ __host__ __device__ constexpr uint32_t tm_sf(int pipe, int i) {
 __device__ __forceinline__ uint8_t* ring_slot(uint8_t* smem, int pipe, int s) {
   return smem + OFF_RING + ((size_t)pipe * NSLOT + s) * SLOT_BYTES;
 }
+// The pipeline stream for units of at most U positions (NT_MAX, or NT_BIG
+// for big units): ring slots and tensor-memory accumulators.
+template <int U> struct PipeCfg;
+template <> struct PipeCfg<NT_MAX> {
+  static constexpr int NS = NSLOT, SLOTB = SLOT_BYTES, ACCW = ACC_COLS;
+};
+template <> struct PipeCfg<NT_BIG> {
+  static constexpr int NS = NSLOT_BIG, SLOTB = SLOT_BYTES_BIG, ACCW = ACC_COLS_BIG;
+};
+static_assert((size_t)NPIPE * NSLOT_BIG * SLOT_BYTES_BIG <= RING_BYTES && SLOT_BYTES_BIG % 16 == 0, "big-unit ring");
+template <int U>
+__device__ __forceinline__ uint32_t pipe_ring(uint8_t* smem, int pipe) {
+  return smem_u32(smem + OFF_RING + (size_t)pipe * PipeCfg<U>::NS * PipeCfg<U>::SLOTB);
+}
+template <int U>
+__device__ __forceinline__ uint32_t pipe_acc(int pipe, int b) { return (uint32_t)(pipe * NACC + b) * PipeCfg<U>::ACCW; }
+template <int U>
+__device__ __forceinline__ uint32_t pipe_sf(int pipe, int i) {
+  return (uint32_t)(NPIPE * NACC * PipeCfg<U>::ACCW + (pipe * NSF + i) * SF_COLS);
+}
 __device__ __forceinline__ uint64_t* full_bar(uint8_t* smem, int pipe, int s) { return reinterpret_cast<uint64_t*>(smem + OFF_FULL) + pipe * NSLOT + s; }
 __device__ __forceinline__ uint64_t* empty_bar(uint8_t* smem, int pipe, int s) { return reinterpret_cast<uint64_t*>(smem + OFF_EMPTY) + pipe * NSLOT + s; }
 __device__ __forceinline__ uint64_t* accf_bar(uint8_t* smem, int pipe, int b) { return reinterpret_cast<uint64_t*>(smem + OFF_ACCF) + pipe * NACC + b; }
@@ -122,8 +142,8 @@ __device__ __forceinline__ uint64_t* xch_bar(uint8_t* smem, int pipe, int i) { r
 __device__ __forceinline__ uint64_t* drain_bar(uint8_t* smem, int pipe) { return reinterpret_cast<uint64_t*>(smem + OFF_DRAIN) + pipe; }
 __device__ __forceinline__ uint32_t* tmem_base_word(uint8_t* smem) { return reinterpret_cast<uint32_t*>(smem + OFF_TMEMBASE); }
 __device__ __forceinline__ JobEntry* job_queue(uint8_t* smem, int pipe) { return reinterpret_cast<JobEntry*>(smem + OFF_JQ) + pipe * JQ; }
-__device__ __forceinline__ float* xch_buf(uint8_t* smem, int pipe, int i) {
-  return reinterpret_cast<float*>(smem + OFF_XCH) + (pipe * 2 + i) * NT_MAX * 4;
+__device__ __forceinline__ float* xch_buf(uint8_t* smem, int pipe, int i, int u = NT_MAX) {
+  return reinterpret_cast<float*>(smem + OFF_XCH) + (pipe * 2 + i) * u * 4;
 }
 __device__ __forceinline__ CtaTables& tables(uint8_t* smem) { return *reinterpret_cast<CtaTables*>(smem + OFF_TABLES); }
 
@@ -1078,6 +1098,47 @@ __device__ void phase_permute_large(const EngineParams& p, uint8_t* smem, int us
   }
 }
 
+// Big units: the x image of every (stage, permuted position), copied from
+// its token's image, so that a unit's B operand is one contiguous run of
+// positions (one bulk copy per stage).  In the scale row r of position j < 4
+// of a unit, bytes 4..7 take the scale bytes of row r of position j + 4 when
+// the unit has it (B row 32 + 8 j + r's scales, for tensor-memory column 5).
+// A warp moves one (unit, stage): 40 16-byte chunks per position (32 of
+// codes, then the 8 scale rows), eight chunks per lane in flight.
+__device__ void phase_pos_gather(const EngineParams& p) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int CPP = IMG_BYTES / 16, CCODE = IMG_CODE_BYTES / 16;
+  const int ns = p.H / KS, nu = ld_cg_u32(p.n_units);
+  const int64_t ntask = (int64_t)nu * ns;
+  for (int64_t us = (int64_t)blockIdx.x * WARPS + warp; us < ntask; us += (int64_t)gridDim.x * WARPS) {
+    const int u = (int)(us / ns), st = (int)(us % ns);
+    const int4 ur = __ldcg(reinterpret_cast<const int4*>(p.units) + u);
+    const int pos0 = ur.y, n = ur.z;  // n <= NT_BIG
+    const int tok = lane < n ? __ldcg(p.tokpos + pos0 + lane) : 0;
+    const uint8_t* xs = p.xt + (int64_t)st * p.T * IMG_BYTES;
+    uint4* dst = reinterpret_cast<uint4*>(p.xp + ((int64_t)st * p.TK + pos0) * IMG_BYTES);
+    constexpr int B8 = 8;
+    for (int f0 = 0; f0 < n * CPP; f0 += 32 * B8) {
+      uint4 v[B8];
+#pragma unroll
+      for (int i = 0; i < B8; ++i) {
+        const int f = f0 + 32 * i + lane, j = f / CPP, ch = f - j * CPP;
+        const int tj = __shfl_sync(FULL, tok, j & 7), tp = __shfl_sync(FULL, tok, (j + NT_MAX) & 7);
+        if (f < n * CPP) {
+          v[i] = __ldcg(reinterpret_cast<const uint4*>(xs + (int64_t)tj * IMG_BYTES) + ch);
+          if (ch >= CCODE && j < NT_MAX && j + NT_MAX < n)  // the partner's scale bytes of this row
+            v[i].y = __ldcg(reinterpret_cast<const uint32_t*>(xs + (int64_t)tp * IMG_BYTES + 16 * ch));
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < B8; ++i) {
+        const int f = f0 + 32 * i + lane;
+        if (f < n * CPP) dst[f] = v[i];
+      }
+    }
+  }
+}
+
 // Large T*K: the x term images of every tile, gathered from the per-token
 // images: the first LT_NTERM term rows of each position (row k of a token's
 // image becomes B row LT_NTERM * tl + k) and their scale words.  A warp moves
@@ -1328,9 +1389,13 @@ __device__ bool wait_entry(const EngineParams& p, JobEntry* en, int32_t qk) {
 template <int TM, int SPLIT = 0>
 __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint8_t* smem,
                                 const StreamCtx& cx, int pipe, RoleState& rs) {
-  constexpr bool LT = TM != 0;
-  constexpr int NS = TM == 1 ? LT_NSLOT : TM == 4 ? LTA_NSLOT : TM == 6 ? ET_NSLOT : NSLOT;  // ring slots
-  constexpr int SLOTB = TM == 1 ? LT_SLOT_BYTES : TM == 4 ? LTA_SLOT_BYTES : TM == 6 ? ET_SLOT_BYTES : SLOT_BYTES;
+  constexpr bool LT = TM == 1 || TM == 4 || TM == 6;  // tile modes (TM 0, 7: the pipeline stream)
+  constexpr int NS = TM == 1 ? LT_NSLOT : TM == 4 ? LTA_NSLOT : TM == 6 ? ET_NSLOT : TM == 7 ? NSLOT_BIG : NSLOT;
+  constexpr int SLOTB = TM == 1   ? LT_SLOT_BYTES
+                        : TM == 4 ? LTA_SLOT_BYTES
+                        : TM == 6 ? ET_SLOT_BYTES
+                        : TM == 7 ? SLOT_BYTES_BIG
+                                  : SLOT_BYTES;
   constexpr int R = TM == 4 ? LTA_R : 1;      // row blocks per job
   constexpr int NP = LT ? 1 : NPIPE;         // pipelines per CTA
   constexpr int PB = PRODUCER_BATCH < NS ? PRODUCER_BATCH : NS;
@@ -1428,7 +1493,7 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
     ++rs.wj;
     const uint8_t* wbase = isD ? lp.w_d + ((int64_t)e * db + rb) * nc * STAGE_A_BYTES
                                : lp.w_gu + ((int64_t)e * gub + rb) * nc * STAGE_A_BYTES;
-    const int tok = (!LT && !isD && lane < nt) ? ld_tab(cx.tokpos + pos0 + lane, cx.global) : 0;
+    const int tok = (!LT && TM != 7 && !isD && lane < nt) ? ld_tab(cx.tokpos + pos0 + lane, cx.global) : 0;
     const uint32_t bbytes = TM == 6 ? (uint32_t)et_img_bytes(et_cols(nt, isD ? ET_ATERMS : ET_XTERMS))
                             : LT    ? (uint32_t)(LT_SF_BYTES + lt_cols(nt) * (IMG_CODE_BYTES / 8))
                                     : (uint32_t)nt * IMG_BYTES;
@@ -1456,7 +1521,7 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
         if (__any_sync(FULL, bad)) ok = false;
         continue;
       }
-      uint8_t* dst = LT ? smem + OFF_RING + (size_t)slot * SLOTB : ring_slot(smem, pipe, slot);
+      uint8_t* dst = smem + OFF_RING + ((size_t)(LT ? 0 : pipe) * NS + slot) * SLOTB;
       uint64_t* fb = full_bar(smem, pipe, slot);
       const int c = c0 + lane;
       if (lane < k) {
@@ -1477,7 +1542,10 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
           bulk_g2s(dst + STAGE_A_BYTES, p.aimg + ((int64_t)c * p.TK + pos0) * IMG_BYTES,
                    (uint32_t)nt * IMG_BYTES, fb);
       }
-      if (!LT && !isD) {
+      if (TM == 7 && !isD) {  // big units: the unit's gathered positions, one copy
+        if (lane < k)
+          bulk_g2s(dst + STAGE_A_BYTES, p.xp + ((int64_t)c * p.TK + pos0) * IMG_BYTES, (uint32_t)nt * IMG_BYTES, fb);
+      } else if (!LT && !isD) {
         for (int tl = 0; tl < nt; ++tl) {
           const int tk = __shfl_sync(FULL, tok, tl);
           if (lane < k)
@@ -1510,9 +1578,11 @@ __device__ void stream_producer(const EngineParams& p, const LayerPtrs& lp, uint
 // go to tensor memory and two block-scaled MMAs (K = 64 each, N = 8 columns
 // per token or pair) accumulate into the job's tensor-memory buffer; the slot
 // is released by a commit when they complete.
+template <int U = NT_MAX>
 __device__ void stream_mma(const EngineParams& p, uint8_t* smem, uint32_t tmem, int pipe, RoleState& rs) {
+  using C = PipeCfg<U>;
   JobEntry* jq = job_queue(smem, pipe);
-  const uint32_t ring0 = smem_u32(ring_slot(smem, pipe, 0));
+  const uint32_t ring0 = pipe_ring<U>(smem, pipe);
   const bool prof = p.prof != nullptr;
   unsigned long long t_full = 0, t_issue = 0, t_acc = 0;
   bool ok = true;
@@ -1534,20 +1604,20 @@ __device__ void stream_mma(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
     }
     t_acc += pclock(prof) - ta0;
     tc_fence_after();
-    const uint32_t tacc = tmem + tm_acc(pipe, b);
+    const uint32_t tacc = tmem + pipe_acc<U>(pipe, b);
     const uint32_t idesc0 = mxf4_idesc(nt * NTERM, 0u), idesc1 = mxf4_idesc(nt * NTERM, 2u);
     for (int c = 0; c < nc; ++c) {
       const uint32_t s = (uint32_t)s0 + c;
-      const int slot = (int)(s % NSLOT);
+      const int slot = (int)(s % C::NS);
       const unsigned long long tf0 = pclock(prof);
-      if (!wait_mbar(full_bar(smem, pipe, slot), (s / NSLOT) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, s)) {
+      if (!wait_mbar(full_bar(smem, pipe, slot), (s / C::NS) & 1u, p.sync, p.timeout_ns, DEV_TIMEOUT_PIPE, s)) {
         ok = false;
         break;
       }
       const unsigned long long tm0 = pclock(prof);
       t_full += tm0 - tf0;
-      const uint32_t sa = ring0 + (uint32_t)slot * SLOT_BYTES, sb = sa + STAGE_A_BYTES;
-      const uint32_t tsf = tmem + tm_sf(pipe, (int)(rs.sfc++ % NSF));
+      const uint32_t sa = ring0 + (uint32_t)slot * C::SLOTB, sb = sa + STAGE_A_BYTES;
+      const uint32_t tsf = tmem + pipe_sf<U>(pipe, (int)(rs.sfc++ % NSF));
       tmem_cp_sf(tsf, smem_desc(sa + STAGE_CODE_BYTES, 0, 128));
       tmem_cp_sf(tsf + 4, smem_desc(sb + IMG_CODE_BYTES, 0, IMG_BYTES));
       mma_mxf4(tacc, smem_desc(sa, 128, 256), smem_desc(sb, 128, IMG_BYTES), idesc0, tsf, tsf + 4,
@@ -1574,6 +1644,7 @@ __device__ void stream_mma(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
 //     q ^ 1 through shared memory) goes to aimg and the unit's readiness
 //     counter is incremented once per warp.
 //   down: row h0 + 32 q + l of every pair, times the routing weight -> ypair.
+template <int U = NT_MAX>
 __device__ void stream_epilogue(const EngineParams& p, uint8_t* smem, const StreamCtx& cx,
                                 uint32_t tmem, int pipe, RoleState& rs) {
   const int lane = threadIdx.x & 31, q = (threadIdx.x >> 5) & 3;
@@ -1603,15 +1674,15 @@ __device__ void stream_epilogue(const EngineParams& p, uint8_t* smem, const Stre
     const unsigned long long tk0 = pclock(prof);
     t_wait += tk0 - tw0;
     tc_fence_after();
-    const uint32_t tacc = tmem + ((uint32_t)(32 * q) << 16) + tm_acc(pipe, b);
+    const uint32_t tacc = tmem + ((uint32_t)(32 * q) << 16) + pipe_acc<U>(pipe, b);
     if (!isD) {
-      float av[NT_MAX];
+      float av[U];
       // block amax of warps q and q ^ 1 meet in shared memory; the exchange
       // buffer alternates so that a warp one job ahead cannot overwrite it
       const int xb = (int)(gc & 1u);
-      float* xc = xch_buf(smem, pipe, xb);
+      float* xc = xch_buf(smem, pipe, xb, U);
 #pragma unroll
-      for (int j = 0; j < NT_MAX; ++j) {
+      for (int j = 0; j < U; ++j) {
         av[j] = 0.f;
         if (j < nt) {
           float v[NTERM];
@@ -1637,7 +1708,7 @@ __device__ void stream_epilogue(const EngineParams& p, uint8_t* smem, const Stre
       }
       const int i0 = rb * GU_I_ROWS, sD = i0 / KS, kk = (i0 % KS) / 64, kc = q >> 1;
 #pragma unroll
-      for (int j = 0; j < NT_MAX; ++j) {
+      for (int j = 0; j < U; ++j) {
         if (j < nt) {
           const int s0 = term0_exp(fmaxf(xc[j * 4 + q], xc[j * 4 + (q ^ 1)]));
           const uint32_t word = term_word<16>(e2m1_terms(av[j], s0), lane);
@@ -1645,8 +1716,12 @@ __device__ void stream_epilogue(const EngineParams& p, uint8_t* smem, const Stre
           if (lane < 16)
             *reinterpret_cast<uint32_t*>(img + kk * 256 + kc * 128 + (lane >> 1) * 16 + (q & 1) * 8 +
                                          (lane & 1) * 4) = word;
-          if ((q & 1) == 0 && lane < NTERM)
-            img[IMG_CODE_BYTES + lane * 16 + 2 * kk + kc] = (uint8_t)(term_exp(s0, lane) + 127);
+          if ((q & 1) == 0 && lane < NTERM) {
+            const uint8_t e8 = (uint8_t)(term_exp(s0, lane) + 127);
+            img[IMG_CODE_BYTES + lane * 16 + 2 * kk + kc] = e8;
+            // big units: positions 4..7 also at bytes 4..7 of position j - 4's scale rows
+            if (U == NT_BIG && j >= NT_MAX) img[IMG_CODE_BYTES + lane * 16 + 4 + 2 * kk + kc - NT_MAX * IMG_BYTES] = e8;
+          }
         }
       }
       __syncwarp();
@@ -1658,7 +1733,7 @@ __device__ void stream_epilogue(const EngineParams& p, uint8_t* smem, const Stre
     } else {
       const int h0 = rb * JOB_ROWS;
 #pragma unroll
-      for (int j = 0; j < ND_MAX; ++j) {
+      for (int j = 0; j < (U > ND_MAX ? U : ND_MAX); ++j) {
         if (j < nt) {
           float v[NTERM];
           tmem_ld8(tacc + j * NTERM, v);
@@ -2778,9 +2853,9 @@ template <int MODE>
 __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, RoleState& rs,
                            bool stamp) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr bool PIPE = MODE == 0 || MODE == 5;  // pipeline stream (units of <= NT_MAX positions)
+  constexpr bool PIPE = MODE == 0 || MODE == 5 || MODE == 7;  // pipeline stream (MODE 7: big units)
   // MODE 0 is launched only for T*K <= SMALL_PAIRS: its routing is always per CTA
-  const bool small = PIPE && (MODE == 0 || p.TK <= SMALL_PAIRS);
+  const bool small = PIPE && MODE != 7 && (MODE == 0 || p.TK <= SMALL_PAIRS);
   CtaTables& tb = tables(smem);
   for (int layer = 0; layer < p.L; ++layer) {
     const LayerPtrs& lp = p.layers[layer];
@@ -2789,7 +2864,7 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
     // the fp64 MMA router wherever the routing is grid-wide (T*K > SMALL_PAIRS):
     // from a few dozen tokens its 8-token tiles are full enough to pay
     if constexpr (!PIPE) phase_router_tiles(x, lp.router_w, p.logits, p.sync, p.T, p.H, p.E, p.TK, p.HS, smem);
-    else if (MODE == 5 && !small) phase_router_tiles(x, lp.router_w, p.logits, p.sync, p.T, p.H, p.E, p.TK, p.HS, smem);
+    else if (MODE != 0 && !small) phase_router_tiles(x, lp.router_w, p.logits, p.sync, p.T, p.H, p.E, p.TK, p.HS, smem);
     else phase_router<MODE == 5 ? 10 : 2>(p, lp, x, smem);
     if (st) st[0] = globaltimer_ns();
     StreamCtx cx;
@@ -2811,11 +2886,14 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 2)) return;
       if (st) st[3] = globaltimer_ns();
       if constexpr (MODE == 2) phase_permute_f16(p, smem);
-      else phase_permute_large(p, smem, MODE == 6 ? ET_MAX : MODE == 4 ? LTA_MAX : MODE == 1 ? LT_MAX : NT_MAX);
+      else phase_permute_large(p, smem, MODE == 6 ? ET_MAX : MODE == 4 ? LTA_MAX : MODE == 1 ? LT_MAX : MODE == 7 ? NT_BIG : NT_MAX);
       if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 3)) return;
       if (p.route_only) return;
       if constexpr (MODE == 1 || MODE == 4) {
         phase_tile_gather(p);
+        if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 6)) return;
+      } else if constexpr (MODE == 7) {
+        phase_pos_gather(p);
         if (!grid_barrier(p.sync, p.timeout_ns, 10 * layer + 6)) return;
       } else if constexpr (MODE == 6) {
         phase_tile_gather_e4m3(p);
@@ -2835,17 +2913,18 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
       prefetch_share(p.layers[layer + 1].router_w, (size_t)p.E * p.H * 4);
     fence_proxy_async_smem();  // the ring held routing scratch written by generic stores
     __syncthreads();
-    if constexpr (PIPE) {  // two pipelines per CTA, units of <= NT_MAX positions
+    if constexpr (PIPE) {  // two pipelines per CTA, units of <= NT_MAX (MODE 7: NT_BIG) positions
+      constexpr int U = MODE == 7 ? NT_BIG : NT_MAX;
       if (warp < EPI_WARP0) {
         const int pipe = warp >> 1;
         if ((warp & 1) == 0) {
-          stream_producer<0>(p, lp, smem, cx, pipe, rs);
+          stream_producer<MODE == 7 ? 7 : 0>(p, lp, smem, cx, pipe, rs);
         } else {
-          if (lane == 0) stream_mma(p, smem, tmem, pipe, rs);
+          if (lane == 0) stream_mma<U>(p, smem, tmem, pipe, rs);
           __syncwarp();
         }
       } else {
-        stream_epilogue(p, smem, cx, tmem, (warp - EPI_WARP0) / 4, rs);
+        stream_epilogue<U>(p, smem, cx, tmem, (warp - EPI_WARP0) / 4, rs);
       }
     } else if constexpr (MODE == 1 || MODE == 4) {  // one pipeline per CTA over tiles (pairs)
       if (warp == 0) {
@@ -3017,7 +3096,7 @@ int engine_max_grid(int device, int* err) {
   int per_sm = ~0u >> 1, sms = 0;
   for (const void* k : {(const void*)engine_kernel<0>, (const void*)engine_kernel<1>, (const void*)engine_kernel<2>,
                         (const void*)engine_kernel<3>, (const void*)engine_kernel<4>, (const void*)engine_kernel<5>,
-                        (const void*)engine_kernel<6>}) {
+                        (const void*)engine_kernel<6>, (const void*)engine_kernel<7>}) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) { *err = (int)e; return 0; }
     int n = 0;
@@ -3034,10 +3113,14 @@ int engine_max_grid(int device, int* err) {
 cudaError_t engine_launch(const EngineParams& p, int grid, cudaStream_t s) {
   void* args[] = {const_cast<EngineParams*>(&p)};
   // MODE 0's launch rule: routing per CTA (T*K <= SMALL_PAIRS), one layer, no
-  // all-reduce (or routing only); every other pipeline launch takes MODE 5
+  // all-reduce (or routing only); big units (MODE 7) for grid-wide routing
+  // with at least BIG_MIN_PER_EXPERT positions per expert; every other
+  // pipeline launch takes MODE 5
   const bool plain = p.TK <= SMALL_PAIRS && ((p.L == 1 && p.ar.world == 0) || p.route_only);
-  const void* k = !use_tiles(p.TK, p.E) || p.route_only ? (plain ? (const void*)engine_kernel<0>
-                                                                 : (const void*)engine_kernel<5>)
+  const void* pipe_k = plain                                         ? (const void*)engine_kernel<0>
+                       : !p.route_only && use_big_units(p.TK, p.E) ? (const void*)engine_kernel<7>
+                                                                     : (const void*)engine_kernel<5>;
+  const void* k = !use_tiles(p.TK, p.E) || p.route_only ? pipe_k
                   : p.large == LARGE_F16                  ? (const void*)engine_kernel<2>
                   : p.large == LARGE_MXF8                 ? (const void*)engine_kernel<6>
                   : use_tile_pairs(p.TK, p.E, p.H)         ? (const void*)engine_kernel<4>

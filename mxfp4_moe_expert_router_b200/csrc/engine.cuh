@@ -62,6 +62,22 @@ static_assert(NPIPE * (NACC * ACC_COLS + NSF * SF_COLS) <= TMEM_COLS, "tensor me
 // a batch's stages must occupy distinct slots whose previous use is already issued
 static_assert(PRODUCER_BATCH <= NSLOT && PRODUCER_BATCH < 32, "producer batch");
 constexpr int SMALL_PAIRS = 256;                         // T*K up to this: routing done per CTA
+// Big units (grid-wide routing without tiles, at least BIG_MIN_PER_EXPERT
+// positions per expert on average): units of up to NT_BIG positions, so that
+// an expert hit by 5..8 positions streams its weights once.  The B operand is
+// a unit's run of per-position x images (one bulk copy per stage) in which
+// positions 4..7 also have their scale bytes at bytes 4..7 of the scale rows
+// of positions 0..3: one 32-row scale-factor copy then fills the B scale
+// columns 4 (B rows 0..31) and 5 (rows 32..63), and the stage takes the same
+// two MMAs (N = 8 nt <= 64) as a unit of NT_MAX.
+constexpr int NT_BIG = 8;
+constexpr int BIG_MIN_PER_EXPERT = 4;
+constexpr int SLOT_BYTES_BIG = STAGE_A_BYTES + NT_BIG * IMG_BYTES;  // 13824
+constexpr int NSLOT_BIG = 7;                             // per pipeline
+constexpr int ACC_COLS_BIG = NT_BIG * NTERM;             // 64 columns per buffer
+static_assert(NPIPE * (NACC * ACC_COLS_BIG + NSF * SF_COLS) <= TMEM_COLS, "tensor memory budget (big units)");
+static_assert(NSLOT_BIG <= NSLOT, "big-unit ring barriers");
+static_assert(NT_BIG == 2 * NT_MAX, "positions 4..7 pair with positions 0..3");
 
 // ---- large T*K: tile stream --------------------------------------------------------------
 // With many tokens per expert (T*K >= LT_MIN_PER_EXPERT * E) a unit ("tile")
@@ -202,6 +218,17 @@ enum : int { LARGE_MXF4 = 1, LARGE_F16 = 2, LARGE_MXF8 = 3 };
 __host__ __device__ inline bool use_tiles(int64_t TK, int E) {
   return TK > SMALL_PAIRS && TK >= (int64_t)LT_MIN_PER_EXPERT * E;
 }
+// Whether a launch without tiles and with grid-wide routing takes big units.
+__host__ __device__ inline bool use_big_units(int64_t TK, int E) {
+  return TK > SMALL_PAIRS && !use_tiles(TK, E) && TK >= (int64_t)BIG_MIN_PER_EXPERT * E;
+}
+// The largest T*K up to TKmax that takes big units (0: none), which sizes
+// the per-position x images.
+__host__ __device__ inline int64_t max_big_pairs(int64_t TKmax, int E) {
+  const int64_t below = (int64_t)LT_MIN_PER_EXPERT * E - 1;  // the largest T*K without tiles
+  const int64_t n = TKmax < below ? TKmax : below;
+  return use_big_units(n, E) ? n : 0;
+}
 // Whether its tiles are streamed as tile pairs (two row blocks per job).
 __host__ __device__ inline bool use_tile_pairs(int64_t TK, int E, int H) {
   return use_tiles(TK, E) && H % (LTA_R * JOB_ROWS) == 0 && TK <= (int64_t)LTA_PER_EXPERT * E;
@@ -286,6 +313,7 @@ struct EngineParams {
   int32_t* dunits;            // [Dmax][4] down units (expert, pos0, nt <= ND_MAX, gate/up unit)
   int32_t* n_units;           // [2] gate/up units, down units
   uint8_t* aimg;              // [I/KS][TK][IMG_BYTES] E2M1 term images of the SwiGLU output
+  uint8_t* xp;                // big units: [H/KS][TK][IMG_BYTES] x images per permuted position
   uint8_t* xtl;               // large T*K: [tiles][H/KS][LT_IMG_BYTES] x term images per tile
   uint8_t* atl;               // large T*K: [tiles][I/KS][LT_IMG_BYTES] SwiGLU term images per tile
   uint8_t* xtf;               // bf16 tiles: [tiles][H/FT_HK][FT_TERM_BYTES] x per tile

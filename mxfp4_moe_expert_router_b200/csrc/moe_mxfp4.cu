@@ -27,6 +27,7 @@ struct moe_mxfp4 {
   uint8_t* xt = nullptr;
   uint8_t* aimg = nullptr;
   uint8_t* xtl = nullptr;  // large T*k only
+  uint8_t* xp = nullptr;   // big units only
   uint8_t* atl = nullptr;
   uint8_t *xe = nullptr, *xte = nullptr, *ate = nullptr;  // large T*k only (E4M3 tiles)
   uint8_t* xtf = nullptr;  // large T*k only (bf16 tiles)
@@ -145,7 +146,7 @@ EngineParams base_params(const moe_mxfp4* h, int T) {
   p.idx = h->idx; p.wts = h->wts; p.counts = h->counts; p.offsets = h->offsets;
   p.perm = h->perm; p.inv = h->inv; p.tokpos = h->tokpos; p.wpos = h->wpos;
   p.units = h->units; p.dunits = h->dunits; p.n_units = h->n_units; p.aimg = h->aimg;
-  p.xtl = h->xtl; p.atl = h->atl;
+  p.xtl = h->xtl; p.atl = h->atl; p.xp = h->xp;
   p.xtf = h->xtf; p.atf = h->atf; p.large = h->large;
   p.xe = h->xe; p.xte = h->xte; p.ate = h->ate;
   p.ypair = h->ypair;
@@ -251,6 +252,8 @@ int32_t moe_mxfp4_create(const moe_config_t* cfg, const uint8_t* const* gate_cod
        dalloc(h, &h->stamps, (size_t)(1 + MAX_LAYERS * STAMPS_PER_LAYER) * 8) &&
        dalloc(h, &h->prof, (size_t)PROF_COUNTERS * 8) &&
        dalloc(h, &h->x_stage, (size_t)Tm * H * 2) && dalloc(h, &h->y_stage, (size_t)Tm * H * 2);
+  if (ok && max_big_pairs(TKm, E) > 0)  // per-position x images of the big units
+    ok = dalloc(h, &h->xp, (size_t)(H / KS) * max_big_pairs(TKm, E) * IMG_BYTES);
   if (ok && use_tiles(TKm, E)) {  // tile images of the large-T*k stream
     const size_t tiles = (size_t)max_tiles(E, TKm);
     ok = dalloc(h, &h->xtl, tiles * (H / KS) * LT_IMG_BYTES) && dalloc(h, &h->atl, tiles * (I / KS) * LT_IMG_BYTES);

@@ -78,6 +78,12 @@ SHAPES = {
     "many_tokens_one_expert": (256, 128, 2, 1, 40),
     # H % 256 == 0 and T*k / E <= 24: tile pairs (two row blocks per job)
     "pairs": (512, 256, 16, 4, 80),
+    # grid-wide routing without tiles, >= 4 positions per expert: units of up
+    # to 8 positions (5 and 4.4 per expert on average; ragged units)
+    "big_units": (384, 256, 64, 4, 80),
+    "big_units_ragged": (256, 128, 64, 4, 70),
+    # grid-wide routing without tiles, < 4 positions per expert: units of <= 4
+    "grid_routed": (256, 128, 128, 4, 80),
 }
 
 
@@ -129,9 +135,10 @@ def test_large_t_kinds_match_oracle(m, kind, name, tokens):
     check_forward(y, x_values(xb), lw, w.top_k)
 
 
-@pytest.mark.parametrize("name", ["ragged_large", "pairs"])
+@pytest.mark.parametrize("name", ["ragged_large", "pairs", "big_units"])
 def test_forward_with_router_bias(m, name):
-    """Zipf-biased routing: a few experts hold many positions (several tiles each)."""
+    """Zipf-biased routing: a few experts hold many positions (several tiles or
+    units of 8 each)."""
     from tests.gpu_helpers import bf16_dev, check_forward, make_moe
     w = _workload(name, zipf=1.2)
     xb, lw, _ = quantized_layer_np(w, seed=13)
@@ -200,30 +207,34 @@ def test_forward_host_matches_device(m):
     assert (bf16_host_bits(yh) == y).all()
 
 
-def test_chain_teacher_forced(m):
-    """3 chained layers in one launch; each layer checked on the GPU's own bf16 input."""
+@pytest.mark.parametrize("shape", [(512, 256, 16, 4, 9, 3), (384, 256, 64, 4, 80, 2)])
+def test_chain_teacher_forced(m, shape):
+    """Chained layers in one launch; each layer checked on the GPU's own bf16
+    input.  Per-CTA routing (T*k = 36), and grid-wide routing with units of up
+    to 8 positions (T*k = 320, E = 64)."""
     import torch
     from tests.gpu_helpers import bf16_dev, bf16_host_bits, make_moe
     from tests.helpers import tolerance_ok
-    w = synth.Workload("chain", 512, 256, 16, 4, 9, layers=3, zipf_alpha=1.2, device_draw=False)
+    H, I, E, k, T, L = shape
+    w = synth.Workload("chain", H, I, E, k, T, layers=L, zipf_alpha=1.2, device_draw=False)
     lws, xb = [], None
-    for l in range(3):
+    for l in range(L):
         xl, lw, _ = quantized_layer_np(w, layer=l, seed=19)
         lws.append(lw)
         xb = xl if l == 0 else xb
     mo = make_moe(w, lws)
-    io = torch.empty((4, w.tokens, w.hidden), dtype=torch.bfloat16, device="cuda")
+    io = torch.empty((L + 1, w.tokens, w.hidden), dtype=torch.bfloat16, device="cuda")
     y = mo.moe_forward(bf16_dev(xb), layer_io=io)
     mo.moe_status()
     io_h = x_values(bf16_host_bits(io))
     assert (bf16_host_bits(io[0]) == xb).all()
-    assert (bf16_host_bits(io[3]) == bf16_host_bits(y)).all()
-    for l in range(3):
+    assert (bf16_host_bits(io[L]) == bf16_host_bits(y)).all()
+    for l in range(L):
         ref_y = moe.moe_layer(io_h[l], lws[l], w.top_k)["y"]
-        if l < 2:
+        if l < L - 1:
             ok, ratio = tolerance_ok(io_h[l + 1], moe.rmsnorm(ref_y))
         else:
-            ok, ratio = tolerance_ok(io_h[3], ref_y)
+            ok, ratio = tolerance_ok(io_h[L], ref_y)
         assert ok, (l, ratio)
 
 

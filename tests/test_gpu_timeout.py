@@ -22,9 +22,11 @@ pytestmark = pytest.mark.gpu
 
 DEFAULT_NS = 2_000_000_000
 # (H, I, E, k, T): per-CTA routing (T*k <= 256), the grid-wide routing with the
-# pipeline stream, and the grid-wide routing with the tile stream (T*k >= 8 E):
-# tile pairs (H % 256 == 0, T*k <= 24 E) and single row blocks
-SHAPES = [(512, 256, 16, 4, 37), (384, 256, 64, 4, 80), (256, 256, 16, 4, 80), (384, 256, 16, 4, 80)]
+# pipeline stream (units of up to 8 positions, then of up to 4), and the
+# grid-wide routing with the tile stream (T*k >= 8 E): tile pairs (H % 256 ==
+# 0, T*k <= 24 E) and single row blocks
+SHAPES = [(512, 256, 16, 4, 37), (384, 256, 64, 4, 80), (256, 128, 128, 4, 80), (256, 256, 16, 4, 80),
+          (384, 256, 16, 4, 80)]
 
 
 def _case(shape, seed=41):
