@@ -82,6 +82,7 @@ struct alignas(16) CtaTables {
   float red[WARPS];
   int32_t n_units, n_dunits;
   int32_t last, gen;  // route barrier: this CTA arrived last; barrier generation
+  int32_t claim;      // x image tasks claimed by this CTA (small T*K)
 };
 
 constexpr size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
@@ -362,34 +363,62 @@ __device__ __noinline__ void router_chunk(const double* xd, const float* wsm, co
 // scale-factor rows of the image): all NTERM, or the first NT (the tile
 // streams read only LT_NTERM; term rows past NT get zero codes).  Also the
 // layer-input copy of the optional per-layer output.
-template <int NT = NTERM>
-__device__ void phase_images(const EngineParams& p, const __nv_bfloat16* x, int layer) {
-  const int T = p.T, H = p.H;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// One warp: the image of 32-element block gb of token t.
+template <int NT>
+__device__ __forceinline__ void image_task(const EngineParams& p, const __nv_bfloat16* x, int t, int gb) {
+  const int lane = threadIdx.x & 31;
+  const float v = __bfloat162float(__ldcg(x + (int64_t)t * p.H + gb * 32 + lane));
+  float am = fabsf(v);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(FULL, am, o));
+  const int s0 = term0_exp(am);
+  const uint32_t word = term_word<32>(e2m1_terms<NT>(v, s0), lane);
+  const int b = gb % KB, kk = b >> 1, kc = b & 1;
+  uint8_t* img = p.xt + ((int64_t)(gb / KB) * p.T + t) * IMG_BYTES;
+  *reinterpret_cast<uint32_t*>(img + kk * 256 + kc * 128 + (lane >> 2) * 16 + (lane & 3) * 4) = word;
+  if (lane < NTERM) img[IMG_CODE_BYTES + lane * 16 + b] = (uint8_t)(term_exp(s0, lane) + 127);
+}
+
+// The layer-input copy of the optional per-layer output (grid-stride).
+__device__ __forceinline__ void layer_input_copy(const EngineParams& p, const __nv_bfloat16* x, int layer) {
+  if (!p.layer_io) return;
   const int64_t gt = (int64_t)blockIdx.x * THREADS + threadIdx.x;
   const int64_t gs = (int64_t)gridDim.x * THREADS;
+  const int64_t n8 = (int64_t)p.T * p.H / 8;
+  const uint4* s8 = reinterpret_cast<const uint4*>(x);
+  uint4* d8 = reinterpret_cast<uint4*>(p.layer_io + (int64_t)layer * p.T * p.H);
+  for (int64_t i = gt; i < n8; i += gs) d8[i] = __ldcg(s8 + i);
+}
+
+template <int NT = NTERM>
+__device__ void phase_images(const EngineParams& p, const __nv_bfloat16* x, int layer) {
+  const int warp = threadIdx.x >> 5;
   const int64_t wg = (int64_t)blockIdx.x * WARPS + warp, ws = (int64_t)gridDim.x * WARPS;
-  const int nblk = H / 32;
-  const int64_t ntask = p.route_only ? 0 : (int64_t)T * nblk;  // routing alone needs no images
-  for (int64_t task = wg; task < ntask; task += ws) {
-    const int t = (int)(task / nblk), gb = (int)(task % nblk);
-    const float v = __bfloat162float(__ldcg(x + (int64_t)t * H + gb * 32 + lane));
-    float am = fabsf(v);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(FULL, am, o));
-    const int s0 = term0_exp(am);
-    const uint32_t word = term_word<32>(e2m1_terms<NT>(v, s0), lane);
-    const int b = gb % KB, kk = b >> 1, kc = b & 1;
-    uint8_t* img = p.xt + ((int64_t)(gb / KB) * T + t) * IMG_BYTES;
-    *reinterpret_cast<uint32_t*>(img + kk * 256 + kc * 128 + (lane >> 2) * 16 + (lane & 3) * 4) = word;
-    if (lane < NTERM) img[IMG_CODE_BYTES + lane * 16 + b] = (uint8_t)(term_exp(s0, lane) + 127);
+  const int nblk = p.H / 32;
+  const int64_t ntask = p.route_only ? 0 : (int64_t)p.T * nblk;  // routing alone needs no images
+  for (int64_t task = wg; task < ntask; task += ws) image_task<NT>(p, x, (int)(task / nblk), (int)(task % nblk));
+  layer_input_copy(p, x, layer);
+}
+
+// The same images for the per-CTA routing, where one CTA (the last to arrive)
+// computes the routing while the others write the images: tasks are claimed
+// from sync[SY_IMGQ], one per warp of the claiming CTA, so that the CTA busy
+// with the routing takes none of them late (the stream's producers wait for
+// every image before their first gate/up stage).
+__device__ void phase_images_claimed(const EngineParams& p, const __nv_bfloat16* x, int layer, uint8_t* smem) {
+  CtaTables& tb = tables(smem);
+  const int warp = threadIdx.x >> 5;
+  const int nblk = p.H / 32, ntask = p.T * nblk;  // T*K <= SMALL_PAIRS: far below 2^31
+  for (;;) {
+    if (threadIdx.x == 0) tb.claim = (int32_t)atomicAdd(p.sync + SY_IMGQ, (uint32_t)WARPS);
+    __syncthreads();
+    const int base = tb.claim;
+    __syncthreads();  // every warp has read the claim before the next one replaces it
+    if (base >= ntask) break;
+    const int task = base + warp;
+    if (task < ntask) image_task<NTERM>(p, x, task / nblk, task % nblk);
   }
-  if (p.layer_io) {
-    const int64_t n8 = (int64_t)T * H / 8;
-    const uint4* s8 = reinterpret_cast<const uint4*>(x);
-    uint4* d8 = reinterpret_cast<uint4*>(p.layer_io + (int64_t)layer * T * H);
-    for (int64_t i = gt; i < n8; i += gs) d8[i] = __ldcg(s8 + i);
-  }
+  layer_input_copy(p, x, layer);
 }
 
 // ---- E4M3 term expansion (kind::mxf8f6f4 tiles) -------------------------------------------
@@ -960,10 +989,11 @@ __device__ void phase_route_small(const EngineParams& p, const LayerPtrs& lp, ui
 // publishes it before releasing the barrier; every other CTA then copies the
 // stream's tables (a few KB) into shared memory.  One CTA reading all partial
 // logits is much faster than every CTA reading them at once.  While the
-// routing runs, every CTA writes its share of the x term images and counts
-// itself in sync[SY_XDONE]; the stream's producers wait for the full count
-// before their first gate/up stage.  Bounded like grid_barrier; false on
-// timeout or a recorded error.
+// routing runs, the other CTAs write the x term images (tasks claimed from a
+// counter, so that the routing CTA, which claims after it, finds them taken)
+// and every CTA counts itself in sync[SY_XDONE]; the stream's producers wait
+// for the full count before their first gate/up stage.  Bounded like
+// grid_barrier; false on timeout or a recorded error.
 __device__ bool route_barrier(const EngineParams& p, const LayerPtrs& lp, const __nv_bfloat16* x,
                               int layer, uint8_t* smem, uint32_t where, uint64_t* stamp) {
   CtaTables& tb = tables(smem);
@@ -991,7 +1021,7 @@ __device__ bool route_barrier(const EngineParams& p, const LayerPtrs& lp, const 
     }
   }
   if (!p.route_only) {
-    phase_images(p, x, layer);
+    phase_images_claimed(p, x, layer, smem);
     __syncthreads();
     if (threadIdx.x == 0) {
       __threadfence();
@@ -2962,7 +2992,7 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
     if (st) st[5] = globaltimer_ns();
     // every producer has passed its image wait and every CTA has counted
     // itself: the count restarts for the next layer or launch
-    if (blockIdx.x == 0 && threadIdx.x == 0) p.sync[SY_XDONE] = 0u;
+    if (blockIdx.x == 0 && threadIdx.x == 0) { p.sync[SY_XDONE] = 0u; p.sync[SY_IMGQ] = 0u; }
     // MODE 0 runs single layers without the all-reduce (launch rule), so the
     // decode kernel carries neither the RMSNorm nor the all-reduce code
     if (MODE != 0 && layer + 1 < p.L) {

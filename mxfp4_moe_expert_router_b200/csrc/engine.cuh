@@ -240,6 +240,7 @@ enum : int {
   SY_BAR_COUNT = 0, SY_BAR_GEN = 1, SY_JOBS = 2, SY_ERROR = 3, SY_ERRINFO = 4,
   SY_XDONE = 5,  // CTAs whose x term images of this layer are written (small T*K)
   SY_JOBS2 = 6,  // down-job counter of the operator-by-operator launches
+  SY_IMGQ = 7,   // x image tasks claimed (small T*K)
   SY_READY = 8,  // ready[unit] from here
 };
 // device-side error codes (status word)
