@@ -343,11 +343,53 @@ __device__ __forceinline__ void router_dots(const double* xd, const float* wsm, 
   }
 }
 
-// One token chunk: nt rounded up to 1, 2, 4, 8, 9, 12 or 16.
+// The same dot products, two experts per warp pass.
+template <int NT>
+__device__ __forceinline__ void router_dots2(const double* xd, const float* wsm, const float* router_w,
+                                         int nexp, int e0, int estep, int H, int hpart, int hs,
+                                         double* logits, int T, int t0, int nt, int E) {
+  constexpr int P = pow2_at_least(NT);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // experts 2 k2 and 2 k2 + 1 per pass: each x value read from shared memory
+  // serves both (the reads of x, not the FMAs, bound this loop); each
+  // expert's sums keep the order of a single-expert pass
+  for (int k2 = warp; 2 * k2 < nexp; k2 += WARPS) {
+    const int ka = 2 * k2, kb = min(ka + 1, nexp - 1);
+    const int ea = e0 + ka * estep, eb = e0 + kb * estep;
+    const float* wa = wsm ? wsm + (size_t)ka * hpart : router_w + (int64_t)ea * H + hs * hpart;
+    const float* wb = wsm ? wsm + (size_t)kb * hpart : router_w + (int64_t)eb * H + hs * hpart;
+    double acc[P], bcc[P];
+#pragma unroll
+    for (int j = 0; j < P; ++j) acc[j] = bcc[j] = 0.0;
+#pragma unroll 2
+    for (int h = lane; h < hpart; h += 32) {
+      const double w = (double)wa[h], u = (double)wb[h];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        const double xv = xd[j * hpart + h];
+        acc[j] = fma(xv, w, acc[j]);
+        bcc[j] = fma(xv, u, bcc[j]);
+      }
+    }
+    const double va = warp_sum_rs<P>(acc, lane);  // lane l (< nt <= NT) holds token t0 + l
+    const double vb = warp_sum_rs<P>(bcc, lane);
+    if (lane < nt) {
+      logits[((int64_t)hs * T + t0 + lane) * E + ea] = va;
+      if (kb != ka) logits[((int64_t)hs * T + t0 + lane) * E + eb] = vb;
+    }
+  }
+}
+
+// One token chunk: nt rounded up to 1, 2, 4, 8, 9, 12 or 16; PAIR: two
+// experts per warp pass (the chained instance; the decode instance keeps the
+// single-expert pass and its code generation).
+template <bool PAIR>
 __device__ __noinline__ void router_chunk(const double* xd, const float* wsm, const float* router_w,
                                           int nexp, int e0, int estep, int H, int hpart, int hs,
                                           double* logits, int T, int t0, int nt, int E) {
-#define MOE_ROUTER_DOTS(NT) router_dots<NT>(xd, wsm, router_w, nexp, e0, estep, H, hpart, hs, logits, T, t0, nt, E)
+#define MOE_ROUTER_DOTS(NT)                                                                                 \
+  if constexpr (PAIR) router_dots2<NT>(xd, wsm, router_w, nexp, e0, estep, H, hpart, hs, logits, T, t0, nt, E); \
+  else router_dots<NT>(xd, wsm, router_w, nexp, e0, estep, H, hpart, hs, logits, T, t0, nt, E)
   if (nt == 1) MOE_ROUTER_DOTS(1);
   else if (nt == 2) MOE_ROUTER_DOTS(2);
   else if (nt <= 4) MOE_ROUTER_DOTS(4);
@@ -358,12 +400,10 @@ __device__ __noinline__ void router_chunk(const double* xd, const float* wsm, co
 #undef MOE_ROUTER_DOTS
 }
 
-// x[t] (bf16) -> xt[stage][t]: per 32-element block one warp expands the values
-// into E2M1 terms (codes at the MMA's B-operand rows, scales at the
-// scale-factor rows of the image): all NTERM, or the first NT (the tile
-// streams read only LT_NTERM; term rows past NT get zero codes).  Also the
-// layer-input copy of the optional per-layer output.
-// One warp: the image of 32-element block gb of token t.
+// One warp: the image of 32-element block gb of token t in xt[stage][t], its
+// values expanded into E2M1 terms (codes at the MMA's B-operand rows, scales
+// at the scale-factor rows of the image): all NTERM, or the first NT (the
+// tile streams read only LT_NTERM; term rows past NT get zero codes).
 template <int NT>
 __device__ __forceinline__ void image_task(const EngineParams& p, const __nv_bfloat16* x, int t, int gb) {
   const int lane = threadIdx.x & 31;
@@ -390,6 +430,8 @@ __device__ __forceinline__ void layer_input_copy(const EngineParams& p, const __
   for (int64_t i = gt; i < n8; i += gs) d8[i] = __ldcg(s8 + i);
 }
 
+// x[t] (bf16) -> xt[stage][t], one warp per 32-element block (grid-stride
+// over the warps), then the layer-input copy of the optional per-layer output.
 template <int NT = NTERM>
 __device__ void phase_images(const EngineParams& p, const __nv_bfloat16* x, int layer) {
   const int warp = threadIdx.x >> 5;
@@ -475,8 +517,9 @@ __device__ void phase_images_e4m3(const EngineParams& p, const __nv_bfloat16* x,
 // Router partial logits (and the per-layer resets of the stream's counters).
 // RB: 16-byte loads in flight per thread while staging (the chained-layer
 // instance stages a few thousand per CTA in one or two round trips; the
-// single-layer decode instance keeps its register budget with 2).
-template <int RB = 2>
+// single-layer decode instance keeps its register budget with 2).  PAIR: two
+// experts per warp pass in the dot products (the chained-layer instance).
+template <int RB = 2, bool PAIR = false>
 __device__ void phase_router(const EngineParams& p, const LayerPtrs& lp, const __nv_bfloat16* x,
                              uint8_t* smem) {
   const int T = p.T, H = p.H, E = p.E;
@@ -541,7 +584,7 @@ __device__ void phase_router(const EngineParams& p, const LayerPtrs& lp, const _
         }
       }
       __syncthreads();
-      router_chunk(xd, wstaged ? wsm : nullptr, lp.router_w, nexp, rw.e0, rw.estep, H, hpart, hs, p.logits,
+      router_chunk<PAIR>(xd, wstaged ? wsm : nullptr, lp.router_w, nexp, rw.e0, rw.estep, H, hpart, hs, p.logits,
                    T, t0, nt, E);
     }
   }
@@ -2895,7 +2938,7 @@ __device__ void run_layers(const EngineParams& p, uint8_t* smem, uint32_t tmem, 
     // from a few dozen tokens its 8-token tiles are full enough to pay
     if constexpr (!PIPE) phase_router_tiles(x, lp.router_w, p.logits, p.sync, p.T, p.H, p.E, p.TK, p.HS, smem);
     else if (MODE != 0 && !small) phase_router_tiles(x, lp.router_w, p.logits, p.sync, p.T, p.H, p.E, p.TK, p.HS, smem);
-    else phase_router<MODE == 5 ? 10 : 2>(p, lp, x, smem);
+    else phase_router<MODE == 5 ? 10 : 2, MODE == 5>(p, lp, x, smem);
     if (st) st[0] = globaltimer_ns();
     StreamCtx cx;
     const int32_t* inv;
