@@ -106,17 +106,13 @@ static_assert((size_t)WARPS * MAX_EXPERTS * 8 <= RING_BYTES, "routing scratch in
 static_assert((size_t)16 * (8192 / MAX_HSPLIT) * 8 <= RING_BYTES, "router x slice in ring");
 static_assert((size_t)LT_NSLOT * LT_SLOT_BYTES <= RING_BYTES && LT_SLOT_BYTES % 16 == 0, "tile ring");
 static_assert(SLOT_BYTES % 16 == 0 && STAGE_A_BYTES % 16 == 0 && IMG_BYTES % 16 == 0, "bulk-copy alignment");
-// tensor memory: pipeline p's accumulators, then its scale-factor buffers
-__host__ __device__ constexpr uint32_t tm_acc(int pipe, int b) { return (uint32_t)(pipe * NACC + b) * ACC_COLS; }
-__host__ __device__ constexpr uint32_t tm_sf(int pipe, int i) {
-  return (uint32_t)(NPIPE * NACC * ACC_COLS + (pipe * NSF + i) * SF_COLS);
-}
 
 __device__ __forceinline__ uint8_t* ring_slot(uint8_t* smem, int pipe, int s) {
   return smem + OFF_RING + ((size_t)pipe * NSLOT + s) * SLOT_BYTES;
 }
 // The pipeline stream for units of at most U positions (NT_MAX, or NT_BIG
-// for big units): ring slots and tensor-memory accumulators.
+// for big units): ring slots and, in tensor memory, pipeline p's
+// accumulators, then its scale-factor buffers.
 template <int U> struct PipeCfg;
 template <> struct PipeCfg<NT_MAX> {
   static constexpr int NS = NSLOT, SLOTB = SLOT_BYTES, ACCW = ACC_COLS;
@@ -148,8 +144,9 @@ __device__ __forceinline__ float* xch_buf(uint8_t* smem, int pipe, int i, int u 
 }
 __device__ __forceinline__ CtaTables& tables(uint8_t* smem) { return *reinterpret_cast<CtaTables*>(smem + OFF_TABLES); }
 
-// Stream modes: 0 = pipeline stream (units of <= NT_MAX positions, two
-// pipelines per CTA), 1 = tiles (<= LT_MAX positions, one row block per job),
+// Stream modes: 0 = pipeline stream (units of <= NT_MAX positions, or of
+// <= NT_BIG for big units; two pipelines per CTA), 1 = tiles (<= LT_MAX
+// positions, one row block per job),
 // 4 = tile pairs (<= LTA_MAX positions, LTA_R row blocks per job sharing each
 // B stage).  The tile modes run one pipeline per CTA.
 template <int TM> struct TileCfg;
@@ -905,9 +902,9 @@ __device__ __noinline__ void warp_exclusive_scan(int32_t* a, int n, int32_t* tot
   if (lane == 31) *total = incl;
 }
 
-// Unit tables from per-expert counts/offsets: gate/up units of <= NT_MAX
-// consecutive positions of one expert's segment, down units of <= ND_MAX
-// (each inside one gate/up unit).  scratch: 2*E ints.
+// Unit tables from per-expert counts/offsets: gate/up units of <= us
+// consecutive positions of one expert's segment; the down units are the same
+// ranges, each naming its gate/up unit.  scratch: 2*E ints.
 __device__ __noinline__ void build_units(const int32_t* counts, const int32_t* offsets, int E, int32_t* scratch,
                             int32_t* units, int32_t* dunits, int32_t* n_units, int32_t* n_dunits, int us) {
   const int warp = threadIdx.x >> 5;
@@ -1455,7 +1452,8 @@ __device__ bool wait_entry(const EngineParams& p, JobEntry* en, int32_t qk) {
 // (unit, 64-row block of I) come first in unit order, then down jobs (down
 // unit, 128-row block of H); a down job waits until its gate/up unit's SwiGLU
 // term images are complete.  A stage is the job's weight stage plus one term
-// image per token (gate/up, from xt) or the unit's consecutive pair images
+// image per token (gate/up, from xt), the unit's gathered position images
+// (gate/up of big units, from xp) or the unit's consecutive pair images
 // (down, from aimg).
 // SPLIT (operator-by-operator launches only): 1 runs the gate/up jobs alone, 2
 // the down jobs alone (their gate/up units are then complete).

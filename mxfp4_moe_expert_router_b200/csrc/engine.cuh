@@ -310,8 +310,8 @@ struct EngineParams {
   int32_t* inv;               // [TK]
   int32_t* tokpos;            // [TK] token of each permuted position
   float* wpos;                // [TK] routing weight of each permuted position
-  int32_t* units;             // [Umax][4] gate/up units (expert, pos0, nt <= NT_MAX, 0)
-  int32_t* dunits;            // [Dmax][4] down units (expert, pos0, nt <= ND_MAX, gate/up unit)
+  int32_t* units;             // [Umax][4] gate/up units (expert, pos0, nt <= NT_MAX or NT_BIG, 0)
+  int32_t* dunits;            // [Dmax][4] down units (expert, pos0, nt, gate/up unit): the gate/up ranges
   int32_t* n_units;           // [2] gate/up units, down units
   uint8_t* aimg;              // [I/KS][TK][IMG_BYTES] E2M1 term images of the SwiGLU output
   uint8_t* xp;                // big units: [H/KS][TK][IMG_BYTES] x images per permuted position

@@ -93,8 +93,10 @@ def _virtual_ranks(mx, w, lw, world):
 
 
 @pytest.mark.parametrize("world", [2, 4])
-@pytest.mark.parametrize("T", [37, 80])  # T*k = 148 (verify-block path), 320 (tile path)
-def test_fused_allreduce_virtual_ranks(mx, world, T):
+# T*k = 148 (per-CTA routing), 320 over 16 experts (tile path), 320 over 64
+# experts (grid-wide routing with units of up to 8 positions)
+@pytest.mark.parametrize("E,T", [(16, 37), (16, 80), (64, 80)])
+def test_fused_allreduce_virtual_ranks(mx, world, E, T):
     """The fused all-reduce of moe_forward_ishard, one virtual rank at a time on one GPU.
 
     Before rank r's call of epoch e, every other rank's partial is put in its slot
@@ -105,7 +107,7 @@ def test_fused_allreduce_virtual_ranks(mx, world, T):
     (epochs 1 and 2)."""
     import torch
     from tests.gpu_helpers import bf16_dev, bf16_host_bits
-    w = synth.Workload("s4", 512, 512, 16, 4, T, device_draw=False)
+    w = synth.Workload("s4", 512, 512, E, 4, T, device_draw=False)
     xb, lw, _ = quantized_layer_np(w, seed=60 + T)
     x = bf16_dev(xb)
     ms, views = _virtual_ranks(mx, w, lw, world)
