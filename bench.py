@@ -95,6 +95,18 @@ def source_digest() -> str:
     return h.hexdigest()[:16]
 
 
+PROFILED_WORKLOAD = "decode_t9_h4096_e128"
+
+
+def traffic_for(name: str, T: int):
+    """The committed capture's DRAM bytes per launch, for the launch it was taken of:
+    the decode workload at its own token count (another token count takes another
+    kernel instance and other bytes), else None."""
+    if name != PROFILED_WORKLOAD or T != synth.WORKLOADS[PROFILED_WORKLOAD].tokens:
+        return None
+    return profile_traffic()
+
+
 def profile_traffic():
     """DRAM bytes per launch from the committed ncu summary, if it matches the current source."""
     try:
@@ -565,7 +577,7 @@ def main():
     peak, peak_kind = measured_peaks()
     achieved = alg_bytes / (ms_step * 1e-3) / 1e9
     # the committed capture is of the decode workload's engine launch
-    traffic = profile_traffic() if (w.name == "decode_t9_h4096_e128" and T == w.tokens) else None
+    traffic = traffic_for(w.name, T)
 
     # the pages' baseline execution model: one launch per operator
     ops = None

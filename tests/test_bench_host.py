@@ -30,6 +30,16 @@ def test_committed_profile_matches_the_engine_sources():
     assert bench.profile_traffic() > bench.algorithmic_bytes(synth.WORKLOADS["decode_t9_h4096_e128"], 9, 50)
 
 
+def test_traffic_only_for_the_profiled_launch():
+    """The capture is of the decode workload at its own token count: another token count
+    (another kernel instance, other bytes) or another workload reports no traffic."""
+    assert bench.traffic_for("decode_t9_h4096_e128", 9) == bench.profile_traffic()
+    assert bench.traffic_for("decode_t9_h4096_e128", 72) is None
+    assert bench.traffic_for("decode_t9_h4096_e128", 384) is None
+    assert bench.traffic_for("batched_t144_h6144_e256", 144) is None
+    assert bench.traffic_for("sweep_h7168_e256", 9) is None
+
+
 def test_verify_reference_arm_prints_one_json_line():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
                           "--workload", "verify_tiny_v1000_g8", "--steps", "3", "--warmup", "1"],
